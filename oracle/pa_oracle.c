@@ -1,0 +1,338 @@
+/*
+ * Paged KV cache oracle: plain, slow, fp64 CPU reference.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may link, load or call this
+ * file; only the test suite, the smoke check and the benchmark's CPU-baseline leg do.
+ * It shares no code, header, table or constant generator with the CUDA library.
+ *
+ * What it computes, and where the pages define it:
+ *   - slot mapping: slot = block_table[pos / block_size] * block_size + pos % block_size
+ *     ("vLLM: from KV Cache to high-throughput serving", article 3 outline: logical block,
+ *     physical block, offset and slot, with hand-computed boundaries; the block table is a
+ *     plain int32 array looked up per logical block, "vLLM architecture overview" section 2);
+ *   - the cache write (reshape_and_cache in the kernel layer, "vLLM architecture overview"
+ *     section 3): each new token's K and V are stored at its slot; for an FP8 E4M3 cache the
+ *     value is divided by a per-kv-head fp32 scale and encoded with round-to-nearest-even and
+ *     saturation to +-448 (encoder written from the OCP 8-bit floating point specification);
+ *   - attention: exact softmax attention (the FlashAttention outline in article 7 of the
+ *     first page stresses that it is exact), with every request's queries seeing only its own
+ *     keys (flattened super-sequence, "Inside vLLM" notes core point 2) and, inside a chunk,
+ *     only keys at or before their own position (chunked prefill, article 5 outline).
+ *
+ * Cache layout, read only through elem_index(): [num_blocks][2 (K, V)][num_kv_heads]
+ * [block_size][head_size].  One physical block therefore spans exactly
+ * 2 * block_size * num_kv_heads * head_size * dtype_bytes bytes ("Inside vLLM" notes,
+ * core point 1).
+ *
+ * Deliberately naive: K/V are gathered per (request, kv head) into contiguous fp64 arrays and
+ * a two-pass softmax is run per query row.  No tiling, no online rescaling, no splits.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+enum { OR_OK = 0, OR_BAD_META = 6, OR_NOMEM = 3, OR_BAD_ARG = 1 };
+enum { OR_BF16 = 0, OR_FP8_E4M3 = 1 };
+
+/* ------------------------------------------------------------------ layout */
+static int64_t elem_index(int64_t block, int kv, int head, int tok, int d,
+                          int num_kv_heads, int block_size, int head_size) {
+    return (((block * 2 + kv) * num_kv_heads + head) * (int64_t)block_size + tok)
+           * head_size + d;
+}
+
+int64_t oracle_cache_elems(int num_blocks, int block_size, int num_kv_heads, int head_size) {
+    return (int64_t)num_blocks * 2 * block_size * num_kv_heads * head_size;
+}
+
+/* Bytes of one physical block: 2 * block_size * num_kv_heads * head_size * dtype_bytes. */
+int64_t oracle_block_bytes(int block_size, int num_kv_heads, int head_size, int dtype_bytes) {
+    return 2LL * block_size * num_kv_heads * head_size * dtype_bytes;
+}
+
+/* Blocks needed to hold n tokens: ceil(n / block_size) (17 tokens at 16 -> 2 blocks). */
+int64_t oracle_blocks_needed(int64_t n_tokens, int block_size) {
+    int64_t q = n_tokens / block_size;
+    return (n_tokens % block_size) ? q + 1 : q;
+}
+
+/* ------------------------------------------------------------------ number formats */
+static float bf16_to_float(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+double oracle_bf16_to_double(uint16_t b) { return (double)bf16_to_float(b); }
+
+/* E4M3 decode from its definition: 1 sign bit, 4 exponent bits with bias 7, 3 mantissa
+ * bits; exponent field 0 is subnormal (m/8 * 2^-6); S.1111.111 is NaN; no infinities. */
+double oracle_e4m3_decode(uint8_t code) {
+    int s = code >> 7, e = (code >> 3) & 0xF, m = code & 0x7;
+    double mag;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0)
+        mag = ldexp((double)m / 8.0, 1 - 7);
+    else
+        mag = ldexp(1.0 + (double)m / 8.0, e - 7);
+    return s ? -mag : mag;
+}
+
+/* E4M3 encode: the finite code nearest to y; a tie goes to the code with an even mantissa;
+ * anything beyond the largest finite value (448, infinities included) saturates to it; NaN
+ * stays NaN; the sign of zero is kept.  Done by direct search over the 127 non-negative
+ * finite codes, which are increasing in value. */
+uint8_t oracle_e4m3_encode(float y) {
+    uint8_t sign = signbit(y) ? 0x80 : 0x00;
+    double a, best_err = INFINITY;
+    int best = 0, c;
+    if (isnan(y)) return sign | 0x7F;
+    if (isinf(y)) return sign | 0x7E;
+    a = fabs((double)y);
+    for (c = 0; c <= 0x7E; ++c) {
+        double err = fabs(oracle_e4m3_decode((uint8_t)c) - a);
+        if (err < best_err || (err == best_err && (c & 1) == 0)) {
+            best = c;
+            best_err = err;
+        }
+    }
+    return sign | (uint8_t)best;
+}
+
+/* The value an FP8 cache holds for x under scale s: divide in fp32 (IEEE, round to
+ * nearest), encode, decode, multiply back in fp64. */
+static double fp8_roundtrip(uint16_t x_bf16, float s) {
+    float y = bf16_to_float(x_bf16) / s;
+    return oracle_e4m3_decode(oracle_e4m3_encode(y)) * (double)s;
+}
+
+void oracle_e4m3_encode_array(const float* y, int64_t n, uint8_t* out) {
+    int64_t i;
+    for (i = 0; i < n; ++i) out[i] = oracle_e4m3_encode(y[i]);
+}
+
+void oracle_e4m3_decode_array(const uint8_t* c, int64_t n, double* out) {
+    int64_t i;
+    for (i = 0; i < n; ++i) out[i] = oracle_e4m3_decode(c[i]);
+}
+
+/* ------------------------------------------------------------------ slot mapping */
+/* For request r with q_len = qsl[r+1]-qsl[r] new tokens and total length seq_lens[r]
+ * (this step's tokens included), new token i sits at position p = seq_lens[r] - q_len + i
+ * and goes to slot block_table[r][p / bs] * bs + p % bs. */
+int oracle_slot_mapping(const int32_t* block_table, int max_blocks_per_seq,
+                        const int32_t* seq_lens, const int32_t* qsl, int num_seqs,
+                        int block_size, int32_t* slot_mapping) {
+    int r, i;
+    for (r = 0; r < num_seqs; ++r) {
+        int q_len = qsl[r + 1] - qsl[r];
+        int ctx = seq_lens[r];
+        if (q_len < 0 || q_len > ctx) return OR_BAD_META;
+        for (i = 0; i < q_len; ++i) {
+            int p = ctx - q_len + i;
+            int logical = p / block_size;
+            if (logical >= max_blocks_per_seq) return OR_BAD_META;
+            slot_mapping[qsl[r] + i] =
+                block_table[(int64_t)r * max_blocks_per_seq + logical] * block_size
+                + p % block_size;
+        }
+    }
+    return OR_OK;
+}
+
+/* ------------------------------------------------------------------ cache write */
+/* k, v: bf16 [num_tokens][num_kv_heads][head_size].  A negative slot means "no write". */
+void oracle_write_kv_bf16(uint16_t* cache, int num_blocks, int block_size, int num_kv_heads,
+                          int head_size, const uint16_t* k, const uint16_t* v,
+                          const int32_t* slot_mapping, int num_tokens) {
+    int t, h, d;
+    (void)num_blocks;
+    for (t = 0; t < num_tokens; ++t) {
+        int slot = slot_mapping[t];
+        int b, o;
+        if (slot < 0) continue;
+        b = slot / block_size;
+        o = slot % block_size;
+        for (h = 0; h < num_kv_heads; ++h)
+            for (d = 0; d < head_size; ++d) {
+                int64_t src = ((int64_t)t * num_kv_heads + h) * head_size + d;
+                cache[elem_index(b, 0, h, o, d, num_kv_heads, block_size, head_size)] = k[src];
+                cache[elem_index(b, 1, h, o, d, num_kv_heads, block_size, head_size)] = v[src];
+            }
+    }
+}
+
+void oracle_write_kv_fp8(uint8_t* cache, int num_blocks, int block_size, int num_kv_heads,
+                         int head_size, const uint16_t* k, const uint16_t* v,
+                         const float* k_scale, const float* v_scale,
+                         const int32_t* slot_mapping, int num_tokens) {
+    int t, h, d;
+    (void)num_blocks;
+    for (t = 0; t < num_tokens; ++t) {
+        int slot = slot_mapping[t];
+        int b, o;
+        if (slot < 0) continue;
+        b = slot / block_size;
+        o = slot % block_size;
+        for (h = 0; h < num_kv_heads; ++h)
+            for (d = 0; d < head_size; ++d) {
+                int64_t src = ((int64_t)t * num_kv_heads + h) * head_size + d;
+                float yk = bf16_to_float(k[src]) / k_scale[h];
+                float yv = bf16_to_float(v[src]) / v_scale[h];
+                cache[elem_index(b, 0, h, o, d, num_kv_heads, block_size, head_size)] =
+                    oracle_e4m3_encode(yk);
+                cache[elem_index(b, 1, h, o, d, num_kv_heads, block_size, head_size)] =
+                    oracle_e4m3_encode(yv);
+            }
+    }
+}
+
+/* ------------------------------------------------------------------ attention core */
+/* One query row against keys 0..limit of contiguous fp64 K, V [*, head_size].
+ * Two-pass softmax; writes out[head_size] and returns the natural-log LSE. */
+static double attend_row(const double* qrow, const double* K, const double* V, int limit,
+                         int head_size, double scale, double* s, double* out) {
+    int p, d;
+    double mx = -INFINITY, sum = 0.0;
+    for (p = 0; p <= limit; ++p) {
+        double acc = 0.0;
+        for (d = 0; d < head_size; ++d) acc += qrow[d] * K[(int64_t)p * head_size + d];
+        s[p] = scale * acc;
+        if (s[p] > mx) mx = s[p];
+    }
+    for (p = 0; p <= limit; ++p) sum += exp(s[p] - mx);
+    for (d = 0; d < head_size; ++d) out[d] = 0.0;
+    for (p = 0; p <= limit; ++p) {
+        double w = exp(s[p] - mx) / sum;
+        for (d = 0; d < head_size; ++d) out[d] += w * V[(int64_t)p * head_size + d];
+    }
+    return mx + log(sum);
+}
+
+static double cache_value(const void* cache, int kv_dtype, int64_t idx, double scale) {
+    if (kv_dtype == OR_BF16) return oracle_bf16_to_double(((const uint16_t*)cache)[idx]);
+    return oracle_e4m3_decode(((const uint8_t*)cache)[idx]) * scale;
+}
+
+/* Paged attention over the cache.
+ * q: bf16 [num_tokens][num_q_heads][head_size]; block_table int32 [num_seqs][max_blocks];
+ * seq_lens [num_seqs]; qsl [num_seqs + 1].  Query head h reads kv head h / (Hq / Hkv).
+ * out: fp64 [num_tokens][num_q_heads][head_size]; lse: fp64 [num_tokens][num_q_heads]. */
+int oracle_attention_paged(const void* cache, int kv_dtype, int num_blocks, int block_size,
+                           int num_kv_heads, int head_size, const float* k_scale,
+                           const float* v_scale, const uint16_t* q, int num_q_heads,
+                           const int32_t* block_table, int max_blocks_per_seq,
+                           const int32_t* seq_lens, const int32_t* qsl, int num_seqs,
+                           double scale, double* out, double* lse) {
+    int r, g, i, hh, d, p;
+    int group = num_q_heads / num_kv_heads;
+    if (group * num_kv_heads != num_q_heads) return OR_BAD_ARG;
+    for (r = 0; r < num_seqs; ++r) {
+        int q_len = qsl[r + 1] - qsl[r];
+        int ctx = seq_lens[r];
+        double *K, *V, *s, *qrow;
+        if (q_len == 0) continue;
+        if (q_len < 0 || ctx < q_len || ctx <= 0) return OR_BAD_META;
+        if ((ctx - 1) / block_size >= max_blocks_per_seq) return OR_BAD_META;
+        K = (double*)malloc(sizeof(double) * (size_t)ctx * head_size);
+        V = (double*)malloc(sizeof(double) * (size_t)ctx * head_size);
+        s = (double*)malloc(sizeof(double) * (size_t)ctx);
+        qrow = (double*)malloc(sizeof(double) * (size_t)head_size);
+        if (!K || !V || !s || !qrow) {
+            free(K); free(V); free(s); free(qrow);
+            return OR_NOMEM;
+        }
+        for (g = 0; g < num_kv_heads; ++g) {
+            double ks = k_scale ? (double)k_scale[g] : 1.0;
+            double vs = v_scale ? (double)v_scale[g] : 1.0;
+            /* gather this request's keys and values through its block table */
+            for (p = 0; p < ctx; ++p) {
+                int64_t b = block_table[(int64_t)r * max_blocks_per_seq + p / block_size];
+                int o = p % block_size;
+                if (b < 0 || b >= num_blocks) {
+                    free(K); free(V); free(s); free(qrow);
+                    return OR_BAD_META;
+                }
+                for (d = 0; d < head_size; ++d) {
+                    K[(int64_t)p * head_size + d] = cache_value(
+                        cache, kv_dtype,
+                        elem_index(b, 0, g, o, d, num_kv_heads, block_size, head_size), ks);
+                    V[(int64_t)p * head_size + d] = cache_value(
+                        cache, kv_dtype,
+                        elem_index(b, 1, g, o, d, num_kv_heads, block_size, head_size), vs);
+                }
+            }
+            for (i = 0; i < q_len; ++i) {
+                int t = qsl[r] + i;
+                int limit = ctx - q_len + i; /* last key this query may see */
+                for (hh = 0; hh < group; ++hh) {
+                    int h = g * group + hh;
+                    int64_t row = (int64_t)t * num_q_heads + h;
+                    for (d = 0; d < head_size; ++d)
+                        qrow[d] = oracle_bf16_to_double(q[row * head_size + d]);
+                    lse[row] = attend_row(qrow, K, V, limit, head_size, scale, s,
+                                          out + row * head_size);
+                }
+            }
+        }
+        free(K); free(V); free(s); free(qrow);
+    }
+    return OR_OK;
+}
+
+/* Unpaged attention on selected rows, straight from per-position source K/V.
+ * k_src, v_src: bf16 [rows][num_kv_heads][head_size]; request r's position p reads source
+ * row pos_rows[pos_start[r] + p].  With kv_dtype == FP8 every K/V value is taken through the
+ * FP8 round trip (fp32 divide, encode, decode, times scale), i.e. what an FP8 cache holds.
+ * Selected (token, q head) pairs: sel_tokens[j], sel_heads[j]; out [nsel][head_size]. */
+int oracle_attention_rows(const uint16_t* k_src, const uint16_t* v_src, int num_kv_heads,
+                          int head_size, const int64_t* pos_rows, const int64_t* pos_start,
+                          int kv_dtype, const float* k_scale, const float* v_scale,
+                          const uint16_t* q, int num_q_heads, const int32_t* seq_lens,
+                          const int32_t* qsl, int num_seqs, double scale,
+                          const int32_t* sel_tokens, const int32_t* sel_heads, int nsel,
+                          double* out, double* lse) {
+    int j, r, d, p;
+    int group = num_q_heads / num_kv_heads;
+    if (group * num_kv_heads != num_q_heads) return OR_BAD_ARG;
+    for (j = 0; j < nsel; ++j) {
+        int t = sel_tokens[j], h = sel_heads[j], g, q_len, ctx, limit;
+        double *K, *V, *s, *qrow;
+        for (r = 0; r < num_seqs; ++r)
+            if (qsl[r] <= t && t < qsl[r + 1]) break;
+        if (r == num_seqs || h < 0 || h >= num_q_heads) return OR_BAD_ARG;
+        g = h / group;
+        q_len = qsl[r + 1] - qsl[r];
+        ctx = seq_lens[r];
+        if (ctx < q_len) return OR_BAD_META;
+        limit = ctx - q_len + (t - qsl[r]);
+        K = (double*)malloc(sizeof(double) * (size_t)(limit + 1) * head_size);
+        V = (double*)malloc(sizeof(double) * (size_t)(limit + 1) * head_size);
+        s = (double*)malloc(sizeof(double) * (size_t)(limit + 1));
+        qrow = (double*)malloc(sizeof(double) * (size_t)head_size);
+        if (!K || !V || !s || !qrow) {
+            free(K); free(V); free(s); free(qrow);
+            return OR_NOMEM;
+        }
+        for (p = 0; p <= limit; ++p) {
+            int64_t src_row = pos_rows[pos_start[r] + p];
+            for (d = 0; d < head_size; ++d) {
+                int64_t idx = (src_row * num_kv_heads + g) * head_size + d;
+                if (kv_dtype == OR_BF16) {
+                    K[(int64_t)p * head_size + d] = oracle_bf16_to_double(k_src[idx]);
+                    V[(int64_t)p * head_size + d] = oracle_bf16_to_double(v_src[idx]);
+                } else {
+                    K[(int64_t)p * head_size + d] = fp8_roundtrip(k_src[idx], k_scale[g]);
+                    V[(int64_t)p * head_size + d] = fp8_roundtrip(v_src[idx], v_scale[g]);
+                }
+            }
+        }
+        for (d = 0; d < head_size; ++d)
+            qrow[d] = oracle_bf16_to_double(q[((int64_t)t * num_q_heads + h) * head_size + d]);
+        lse[j] = attend_row(qrow, K, V, limit, head_size, scale, s, out + (int64_t)j * head_size);
+        free(K); free(V); free(s); free(qrow);
+    }
+    return OR_OK;
+}
