@@ -1,0 +1,206 @@
+/*
+ * pa.h — C ABI of the paged KV cache library (libpa.so), B200 / sm_100a.
+ *
+ * The library implements the data-parallel hot path of a vLLM-style paged KV cache:
+ *   - the slot mapping of a step's new tokens and the cache write (reshape_and_cache),
+ *   - varlen paged attention over the flattened continuous-batching step: decode rows,
+ *     causal prefill chunks, mixed batches, GQA head groups, split-KV with an LSE reduce,
+ *     bf16 or FP8 E4M3 cache storage.
+ *
+ * Sources, by page title and section:
+ *   [P1] "vLLM: from KV Cache to high-throughput serving" (liujiyu20000308.github.io/vllm):
+ *        article 3 outline (logical/physical block, offset, slot with boundary arithmetic),
+ *        article 5 outline (chunked prefill), article 6 outline (FP8 E4M3 KV cache),
+ *        article 7 outline (FlashAttention tiling, online softmax, LSE, split of K vs Q).
+ *   [P2] "vLLM architecture overview" (blog.chen3feng.top/vllm-analysis), section 2
+ *        (PagedAttention: fixed-size blocks, int32 block table, shared prefix blocks),
+ *        section 3 (kernel layer: PagedAttention V1/V2 kernels, reshape_and_cache).
+ *   [P3] "Inside vLLM" reading notes (kb.wilsonhandbook.online), core point 1 (16-token
+ *        blocks, per-block bytes, allocate_slots' ceil(n/16)), core point 2 (all requests of
+ *        a step flattened into one super-sequence, separated by positions and masks).
+ *
+ * Conventions for every call:
+ *   - Pointers documented as "device" are CUDA device pointers owned by the caller unless a
+ *     call says otherwise; "host" pointers are ordinary host memory read during the call.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  Calls are
+ *     stream-ordered and asynchronous; none synchronises unless its comment says so.
+ *   - Every call returns a pa_status.  Argument errors are detected on the host before any
+ *     launch and launch nothing.  Faults inside an already launched kernel surface at the
+ *     caller's next synchronisation; kernels never trap: bounded waits and metadata checks
+ *     record a code in a device error word read by pa_device_error().
+ *   - No C++ exception crosses this interface.
+ */
+#ifndef PA_H_
+#define PA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    PA_OK = 0,
+    PA_ERR_INVALID_ARG = 1,   /* null pointer, non-positive size, inconsistent shapes */
+    PA_ERR_UNSUPPORTED = 2,   /* a valid configuration this build has no kernel for */
+    PA_ERR_OOM = 3,           /* device allocation failed */
+    PA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed; see pa_last_cuda_error */
+    PA_ERR_WORKSPACE = 5,     /* workspace smaller than the plan needs */
+    PA_ERR_METADATA = 6,      /* host metadata mirrors are inconsistent (see pa_attention) */
+    PA_ERR_DEVICE = 7         /* a kernel recorded an error in the device error word */
+} pa_status;
+
+typedef enum { PA_BF16 = 0, PA_FP8_E4M3 = 1 } pa_kv_dtype;
+
+typedef struct pa_cache pa_cache; /* opaque handle to one layer's paged K/V pool */
+
+/* Bytes of a pool of num_blocks physical blocks.  One block holds block_size tokens of K and
+ * V for every kv head: 2 * block_size * num_kv_heads * head_size * dtype_bytes bytes ([P3]
+ * core point 1).  Returns 0 for invalid arguments. */
+size_t pa_cache_bytes(int num_blocks, int block_size, int num_kv_heads, int head_size,
+                      int kv_dtype);
+
+/* Create a pool ([P2] section 2: the physical block pool).
+ * Layout in device memory: [num_blocks][2 (K, V)][num_kv_heads][block_size][head_size] in
+ * the cache dtype, so one physical block is one contiguous span of pa_cache_bytes(1, ...)
+ * bytes and each (block, K|V, kv head) tile is block_size * head_size elements contiguous.
+ * Supported: block_size 16; head_size 64 or 128 (bf16), 128 (FP8 E4M3); any num_kv_heads.
+ * k_scale, v_scale: device fp32 [num_kv_heads], required for FP8 (the stored code is
+ *   e4m3(x / scale[head])), ignored for bf16; caller-owned, read by later calls.
+ * external_buf: NULL to let the library cudaMalloc the pool (freed by pa_free_cache), or a
+ *   caller-owned device buffer of at least pa_cache_bytes(...) bytes, 256-byte aligned.
+ * The pool contents are not initialised.  Must be called with the device current that will
+ * run the kernels.  Errors: INVALID_ARG, UNSUPPORTED, OOM, CUDA. */
+int pa_alloc_cache(int num_blocks, int block_size, int num_kv_heads, int head_size,
+                   int kv_dtype, const float* k_scale, const float* v_scale,
+                   void* external_buf, pa_cache** out);
+
+/* Release the handle (and the pool if the library allocated it).  Synchronises the device
+ * before freeing.  NULL is accepted. */
+int pa_free_cache(pa_cache* cache);
+
+/* Device pointer to the pool (for inspection and tests). */
+void* pa_cache_data(const pa_cache* cache);
+
+/* Slot mapping of a step's new tokens ([P1] article 3 outline; [P3] core point 2).
+ * For request r with q_len = query_start_loc[r+1] - query_start_loc[r] new tokens and total
+ * length seq_lens[r] (this step's tokens included), new token i sits at position
+ * p = seq_lens[r] - q_len + i and gets
+ *     slot_mapping[query_start_loc[r] + i] = block_table[r][p / block_size] * block_size
+ *                                           + p % block_size.
+ * block_table: device int32 [num_seqs][max_blocks_per_seq] (row-major); seq_lens: device int32
+ * [num_seqs]; query_start_loc: device int32 [num_seqs + 1], non-decreasing, starting at 0;
+ * slot_mapping: device int32 [num_tokens] output, num_tokens = query_start_loc[num_seqs].
+ * A position whose logical block is >= max_blocks_per_seq gets slot -1 and records a device
+ * error.  Errors: INVALID_ARG, CUDA. */
+int pa_slot_mapping(const int32_t* block_table, int max_blocks_per_seq, const int32_t* seq_lens,
+                    const int32_t* query_start_loc, int num_seqs, int num_tokens,
+                    int block_size, int32_t* slot_mapping, void* stream);
+
+/* Cache write, reshape_and_cache ([P2] section 3): for every token t with slot s =
+ * slot_mapping[t] >= 0 and every kv head h, K and V rows are stored at token s % block_size of
+ * block s / block_size.  bf16 pools store the bits unchanged; FP8 pools store
+ * e4m3_rn_satfinite(x / scale[h]) with an IEEE fp32 divide.  A negative slot skips the token.
+ * k, v: device bf16 [num_tokens][num_kv_heads][head_size], dense.  slot_mapping: device int32
+ * [num_tokens].  Slots must lie inside the pool and be distinct within one call (duplicates
+ * leave an unspecified one of the rows).  Errors: INVALID_ARG, CUDA. */
+int pa_write_kv(pa_cache* cache, const void* k, const void* v, const int32_t* slot_mapping,
+                int num_tokens, void* stream);
+
+/* Workspace for pa_attention's split-KV partials when any request may be split into at most
+ * max_splits parts: max_splits * num_tokens * num_q_heads * (head_size + 1) * 4 bytes plus
+ * alignment.  0 when max_splits <= 1 (no splitting). */
+size_t pa_attention_workspace_bytes(int num_tokens, int num_q_heads, int head_size,
+                                    int max_splits);
+
+/* Paged attention over one flattened step ([P3] core point 2; [P1] articles 5 and 7).
+ * q: device bf16 [num_tokens][num_q_heads][head_size]; query head h reads kv head
+ *   h / (num_q_heads / num_kv_heads) (GQA groups of consecutive heads).
+ * block_table, seq_lens, query_start_loc: device, as in pa_slot_mapping.  seq_lens[r] counts
+ *   this step's tokens, whose K/V must already be in the cache (pa_write_kv first).
+ * seq_lens_host, query_start_loc_host: host copies of the same arrays, used only to plan the
+ *   launch (kernel choice, split count, grid size); they must equal the device contents.
+ * Query i of request r attends to positions 0 .. seq_lens[r] - q_len + i (causal within a
+ *   chunk; a decode row sees the whole context), with the softmax scale `scale`.
+ * out: device fp32 [num_tokens][num_q_heads][head_size].
+ * workspace: device scratch of workspace_bytes for split-KV partials (may be NULL/0: then no
+ *   request is split).  Its contents are opaque; it must not be shared by calls that
+ *   overlap on the GPU.
+ * Host checks (-> PA_ERR_METADATA): query_start_loc_host non-decreasing from 0 to num_tokens,
+ *   0 <= q_len <= seq_len, seq_len > 0 when q_len > 0, ceil(seq_len / block_size) <=
+ *   max_blocks_per_seq.  Errors: INVALID_ARG, UNSUPPORTED, METADATA, CUDA. */
+int pa_attention(const pa_cache* cache, const void* q, int num_q_heads,
+                 const int32_t* block_table, int max_blocks_per_seq, const int32_t* seq_lens,
+                 const int32_t* query_start_loc, const int32_t* seq_lens_host,
+                 const int32_t* query_start_loc_host, int num_seqs, int num_tokens,
+                 float scale, float* out, void* workspace, size_t workspace_bytes,
+                 void* stream);
+
+/* Launch plan chosen for one pa_attention call (pure host computation, exposed for tests
+ * and tools).  Decode-kind requests (q_len * group <= 8) run on the GQA decode kernel,
+ * the others on the chunk kernel.  KV is partitioned in units of split_blocks blocks. */
+typedef struct {
+    int num_decode_seqs;      /* requests served by the decode kernel */
+    int num_chunk_seqs;       /* requests served by the chunk kernel */
+    int decode_split_blocks;  /* blocks per KV split for decode-kind requests */
+    int decode_max_splits;    /* largest split count among decode-kind requests */
+    int chunk_split_blocks;   /* blocks per KV split for chunk-kind requests */
+    int chunk_max_splits;
+    int chunk_max_qtiles;     /* largest number of 64-row query tiles of one (request, kv head) */
+    int64_t decode_ctas;      /* CTAs that do work in the decode kernel */
+    int64_t chunk_ctas;       /* CTAs that do work in the chunk kernel */
+    int any_split;            /* a reduce launch is needed */
+    size_t workspace_needed;  /* bytes of workspace this plan uses */
+} pa_plan;
+
+/* Options for pa_attention_ex (zero-initialise for defaults). */
+typedef struct {
+    int kv_split_tokens;   /* > 0: force this many keys (multiple of block_size) per split
+                              for every request; 0: planner's choice */
+    int num_sms;           /* > 0: plan for this many SMs instead of the device's count */
+    void* events[6];       /* optional cudaEvent_t handles recorded on the call's stream:
+                              [0]/[1] before/after the decode kernel, [2]/[3] around the chunk
+                              kernel, [4]/[5] around the split reduce; an entry is recorded
+                              only when that kernel is launched; NULL entries are skipped */
+} pa_attention_opts;
+
+/* The planner alone: fills *plan for the given host metadata without touching the GPU.
+ * num_sms must be > 0.  Errors: INVALID_ARG, METADATA, UNSUPPORTED. */
+int pa_plan_attention(const int32_t* seq_lens_host, const int32_t* query_start_loc_host,
+                      int num_seqs, int num_tokens, int num_q_heads, int num_kv_heads,
+                      int head_size, int block_size, int max_blocks_per_seq, int num_sms,
+                      size_t workspace_bytes, const pa_attention_opts* opts, pa_plan* plan);
+
+/* pa_attention with options (opts may be NULL). */
+int pa_attention_ex(const pa_cache* cache, const void* q, int num_q_heads,
+                    const int32_t* block_table, int max_blocks_per_seq, const int32_t* seq_lens,
+                    const int32_t* query_start_loc, const int32_t* seq_lens_host,
+                    const int32_t* query_start_loc_host, int num_seqs, int num_tokens,
+                    float scale, float* out, void* workspace, size_t workspace_bytes,
+                    const pa_attention_opts* opts, void* stream);
+
+/* Opt-in device check of the metadata a step will read: every block id that
+ * attention would read (logical blocks 0 .. ceil(seq_len / block_size) - 1 of each request)
+ * lies in [0, num_blocks).  Synchronises `stream`.  Writes the number of bad entries to
+ * *num_bad.  Never traps.  Errors: INVALID_ARG, CUDA. */
+int pa_validate_block_table(const pa_cache* cache, const int32_t* block_table,
+                            int max_blocks_per_seq, const int32_t* seq_lens, int num_seqs,
+                            int* num_bad, void* stream);
+
+/* Read (and, if reset != 0, clear) the device error word of the current device: 0 = none,
+ * 1 = a bounded wait timed out, 2 = a slot position beyond the block table, 3 = a block id
+ * outside the pool.  Synchronises the device.  Returns PA_OK or PA_ERR_CUDA. */
+int pa_device_error(int* code, int reset);
+
+/* Human-readable name of a pa_status value. */
+const char* pa_status_string(int status);
+
+/* The cudaError_t of the last failed CUDA call made by this library in this thread. */
+int pa_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PA_H_ */

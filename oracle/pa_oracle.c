@@ -82,23 +82,35 @@ double oracle_e4m3_decode(uint8_t code) {
 
 /* E4M3 encode: the finite code nearest to y; a tie goes to the code with an even mantissa;
  * anything beyond the largest finite value (448, infinities included) saturates to it; NaN
- * stays NaN; the sign of zero is kept.  Done by direct search over the 127 non-negative
- * finite codes, which are increasing in value. */
+ * stays NaN; the sign of zero is kept.  The 127 non-negative finite codes 0x00..0x7E are
+ * increasing in value, so the nearest one is found by bisection over their decoded values
+ * followed by a comparison of the two neighbours. */
+static double e4m3_value[0x7F];
+static int e4m3_value_ready = 0;
+
 uint8_t oracle_e4m3_encode(float y) {
     uint8_t sign = signbit(y) ? 0x80 : 0x00;
-    double a, best_err = INFINITY;
-    int best = 0, c;
-    if (isnan(y)) return sign | 0x7F;
-    if (isinf(y)) return sign | 0x7E;
-    a = fabs((double)y);
-    for (c = 0; c <= 0x7E; ++c) {
-        double err = fabs(oracle_e4m3_decode((uint8_t)c) - a);
-        if (err < best_err || (err == best_err && (c & 1) == 0)) {
-            best = c;
-            best_err = err;
-        }
+    double a, el, eh;
+    int lo, hi, c;
+    if (!e4m3_value_ready) {
+        for (c = 0; c < 0x7F; ++c) e4m3_value[c] = oracle_e4m3_decode((uint8_t)c);
+        e4m3_value_ready = 1;
     }
-    return sign | (uint8_t)best;
+    if (isnan(y)) return sign | 0x7F;
+    a = fabs((double)y);
+    if (a >= e4m3_value[0x7E]) return sign | 0x7E;
+    /* invariant: value[lo] <= a < value[hi] */
+    lo = 0;
+    hi = 0x7E;
+    while (hi - lo > 1) {
+        int mid = (lo + hi) / 2;
+        if (e4m3_value[mid] <= a) lo = mid; else hi = mid;
+    }
+    el = a - e4m3_value[lo];
+    eh = e4m3_value[hi] - a;
+    if (el < eh) return sign | (uint8_t)lo;
+    if (eh < el) return sign | (uint8_t)hi;
+    return sign | (uint8_t)((lo & 1) == 0 ? lo : hi);
 }
 
 /* The value an FP8 cache holds for x under scale s: divide in fp32 (IEEE, round to

@@ -1,0 +1,492 @@
+// Host side of the C ABI declared in include/pa.h: argument checks, the pool handle with
+// its TMA tensor map, the launch planner, and the launch sequences.
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+
+#include "pa_internal.h"
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+// Device error word (one per device context): kernels record the first problem they meet.
+__device__ int g_device_error_word = 0;
+
+constexpr int kMaxDevices = 64;
+int* g_err_ptr[kMaxDevices] = {nullptr};
+int g_num_sms[kMaxDevices] = {0};
+
+int fail_cuda(cudaError_t e) {
+    g_last_cuda_error = static_cast<int>(e);
+    return PA_ERR_CUDA;
+}
+
+int current_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+    return dev;
+}
+
+// Device address of the error word of the current device (resolved once per device).
+int* device_error_ptr() {
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return nullptr;
+    if (!g_err_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_error_word) != cudaSuccess) return nullptr;
+        g_err_ptr[dev] = static_cast<int*>(p);
+    }
+    return g_err_ptr[dev];
+}
+
+int device_num_sms() {
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return 0;
+    if (!g_num_sms[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        g_num_sms[dev] = n;
+    }
+    return g_num_sms[dev];
+}
+
+int dtype_bytes(int kv_dtype) { return kv_dtype == PA_BF16 ? 2 : (kv_dtype == PA_FP8_E4M3 ? 1 : 0); }
+
+bool supported_shape(int block_size, int head_size, int kv_dtype) {
+    if (block_size != pa::kBlockSize) return false;
+    if (kv_dtype == PA_BF16) return head_size == 64 || head_size == 128;
+    if (kv_dtype == PA_FP8_E4M3) return head_size == 128;
+    return false;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000,
+                                             cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// 2-D view of the pool: rows of head_size elements (one token of one (block, K|V, kv head)
+// tile per row), boxes of 128 bytes x 16 rows, 128-byte swizzle.
+int make_tensor_map(pa_cache* c) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return fail_cuda(cudaErrorNotSupported);
+    const int esz = dtype_bytes(c->kv_dtype);
+    const cuuint64_t rows = static_cast<cuuint64_t>(c->num_blocks) * 2 * c->num_kv_heads * c->block_size;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(c->head_size), rows};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(c->head_size) * esz};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / esz), static_cast<cuuint32_t>(c->block_size)};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(&c->tmap,
+                     c->kv_dtype == PA_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                            : CU_TENSOR_MAP_DATA_TYPE_UINT8,
+                     2, c->data, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                     CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail_cuda(cudaErrorInvalidValue);
+    return PA_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+size_t workspace_for(int num_tokens, int num_q_heads, int head_size, int max_splits) {
+    if (max_splits <= 1) return 0;
+    const size_t rows = static_cast<size_t>(max_splits) * num_tokens * num_q_heads;
+    return align256(rows * head_size * sizeof(float)) + align256(rows * sizeof(float));
+}
+
+int max_splits_for(size_t ws, int num_tokens, int num_q_heads, int head_size) {
+    if (num_tokens <= 0) return 0;
+    const size_t per = static_cast<size_t>(num_tokens) * num_q_heads * (head_size + 1) * 4;
+    long long s = static_cast<long long>(ws / per);
+    if (s > (1 << 20)) s = 1 << 20;
+    while (s > 1 && workspace_for(num_tokens, num_q_heads, head_size, static_cast<int>(s)) > ws) --s;
+    return static_cast<int>(s);
+}
+
+int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+// Planner constants.
+constexpr int kDecodeCtasPerSm = 2;    // decode kernel residency (96 KB of stages per CTA)
+constexpr int kDecodeWaves = 8;        // target waves of decode CTAs over the GPU
+constexpr int kMinDecodeSplitBlocks = 32;  // >= 512 keys per split keeps CTA overheads small
+constexpr int kMinChunkSplitBlocks = 16;
+
+int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int Hkv, int D,
+              int bs, int maxb, int num_sms, size_t ws, const pa_attention_opts* opts,
+              pa_plan* pl) {
+    std::memset(pl, 0, sizeof(*pl));
+    if (B < 0 || T < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || num_sms <= 0 || maxb <= 0)
+        return PA_ERR_INVALID_ARG;
+    if (bs != pa::kBlockSize) return PA_ERR_UNSUPPORTED;
+    if (B > 65535 || Hkv > 65535) return PA_ERR_UNSUPPORTED;
+    if (B > 0 && (!sl || !qsl)) return PA_ERR_INVALID_ARG;
+    const int G = Hq / Hkv;
+    const int forced = opts ? opts->kv_split_tokens : 0;
+    if (forced < 0 || forced % bs) return PA_ERR_INVALID_ARG;
+    if (B > 0 && qsl[0] != 0) return PA_ERR_METADATA;
+    long long dec_units = 0;
+    int dec_max_blocks = 0, chunk_max_blocks = 0, chunk_max_qtiles = 0;
+    long long chunk_tiles = 0;
+    for (int r = 0; r < B; ++r) {
+        const int ql = qsl[r + 1] - qsl[r];
+        const int ctx = sl[r];
+        if (ql < 0 || ctx < ql || (ql > 0 && ctx <= 0)) return PA_ERR_METADATA;
+        if (ql == 0) continue;
+        const int blocks = pa::ceil_div(ctx, bs);
+        if (blocks > maxb) return PA_ERR_METADATA;
+        if (pa::is_decode_kind(ql, G)) {
+            pl->num_decode_seqs++;
+            dec_units += static_cast<long long>(blocks) * Hkv;
+            if (blocks > dec_max_blocks) dec_max_blocks = blocks;
+        } else {
+            pl->num_chunk_seqs++;
+            const int qt = pa::ceil_div(ql * G, pa::kChunkRows);
+            if (qt > chunk_max_qtiles) chunk_max_qtiles = qt;
+            chunk_tiles += static_cast<long long>(qt) * Hkv;
+            if (blocks > chunk_max_blocks) chunk_max_blocks = blocks;
+        }
+    }
+    if (B > 0 && qsl[B] != T) return PA_ERR_METADATA;
+    const int allowed = max_splits_for(ws, T, Hq, D);
+
+    // decode partition
+    int dsb = 1;
+    if (pl->num_decode_seqs) {
+        if (forced) {
+            dsb = forced / bs;
+        } else {
+            const long long target = static_cast<long long>(num_sms) * kDecodeCtasPerSm * kDecodeWaves;
+            long long sb = (dec_units + target - 1) / target;
+            if (sb < kMinDecodeSplitBlocks) sb = kMinDecodeSplitBlocks;
+            dsb = round_up(static_cast<int>(sb < dec_max_blocks ? sb : dec_max_blocks), 4);
+        }
+        int ns = pa::ceil_div(dec_max_blocks, dsb);
+        if (ns > 1 && ns > allowed) {
+            if (forced) return PA_ERR_WORKSPACE;
+            dsb = allowed <= 1 ? dec_max_blocks : pa::ceil_div(dec_max_blocks, allowed);
+            ns = pa::ceil_div(dec_max_blocks, dsb);
+        }
+        pl->decode_split_blocks = dsb;
+        pl->decode_max_splits = ns;
+    }
+    // chunk partition
+    if (pl->num_chunk_seqs) {
+        int csb;
+        if (forced) {
+            csb = forced / bs;
+        } else {
+            csb = round_up(chunk_max_blocks, 4);
+            if (chunk_tiles < num_sms && chunk_max_blocks >= 2 * kMinChunkSplitBlocks) {
+                const long long want = (2LL * num_sms + chunk_tiles - 1) / chunk_tiles;
+                int sb = pa::ceil_div(chunk_max_blocks, static_cast<int>(want));
+                if (sb < kMinChunkSplitBlocks) sb = kMinChunkSplitBlocks;
+                csb = round_up(sb, 4);
+            }
+        }
+        int ns = pa::ceil_div(chunk_max_blocks, csb);
+        if (ns > 1 && ns > allowed) {
+            if (forced) return PA_ERR_WORKSPACE;
+            csb = allowed <= 1 ? round_up(chunk_max_blocks, 4)
+                               : round_up(pa::ceil_div(chunk_max_blocks, allowed), 4);
+            ns = pa::ceil_div(chunk_max_blocks, csb);
+        }
+        pl->chunk_split_blocks = csb;
+        pl->chunk_max_splits = ns;
+        pl->chunk_max_qtiles = chunk_max_qtiles;
+    }
+    // working CTA counts
+    for (int r = 0; r < B; ++r) {
+        const int ql = qsl[r + 1] - qsl[r];
+        if (ql == 0) continue;
+        if (pa::is_decode_kind(ql, G)) {
+            pl->decode_ctas += static_cast<int64_t>(pa::num_splits(sl[r], pl->decode_split_blocks)) * Hkv;
+        } else {
+            pl->chunk_ctas += static_cast<int64_t>(pa::num_splits(sl[r], pl->chunk_split_blocks)) *
+                              Hkv * pa::ceil_div(ql * G, pa::kChunkRows);
+        }
+    }
+    const int smax = pl->decode_max_splits > pl->chunk_max_splits ? pl->decode_max_splits
+                                                                   : pl->chunk_max_splits;
+    pl->any_split = smax > 1;
+    pl->workspace_needed = workspace_for(T, Hq, D, smax);
+    return PA_OK;
+}
+
+void record(void* ev, cudaStream_t s) {
+    if (ev) cudaEventRecord(static_cast<cudaEvent_t>(ev), s);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pa_status_string(int status) {
+    switch (status) {
+        case PA_OK: return "PA_OK";
+        case PA_ERR_INVALID_ARG: return "PA_ERR_INVALID_ARG";
+        case PA_ERR_UNSUPPORTED: return "PA_ERR_UNSUPPORTED";
+        case PA_ERR_OOM: return "PA_ERR_OOM";
+        case PA_ERR_CUDA: return "PA_ERR_CUDA";
+        case PA_ERR_WORKSPACE: return "PA_ERR_WORKSPACE";
+        case PA_ERR_METADATA: return "PA_ERR_METADATA";
+        case PA_ERR_DEVICE: return "PA_ERR_DEVICE";
+        default: return "PA_ERR_UNKNOWN";
+    }
+}
+
+int pa_last_cuda_error(void) { return g_last_cuda_error; }
+
+size_t pa_cache_bytes(int num_blocks, int block_size, int num_kv_heads, int head_size,
+                      int kv_dtype) {
+    const int eb = dtype_bytes(kv_dtype);
+    if (num_blocks <= 0 || block_size <= 0 || num_kv_heads <= 0 || head_size <= 0 || !eb) return 0;
+    return static_cast<size_t>(num_blocks) * 2 * block_size * num_kv_heads * head_size * eb;
+}
+
+int pa_alloc_cache(int num_blocks, int block_size, int num_kv_heads, int head_size,
+                   int kv_dtype, const float* k_scale, const float* v_scale,
+                   void* external_buf, pa_cache** out) {
+    if (!out) return PA_ERR_INVALID_ARG;
+    *out = nullptr;
+    const size_t bytes = pa_cache_bytes(num_blocks, block_size, num_kv_heads, head_size, kv_dtype);
+    if (!bytes) return PA_ERR_INVALID_ARG;
+    if (!supported_shape(block_size, head_size, kv_dtype)) return PA_ERR_UNSUPPORTED;
+    if (kv_dtype == PA_FP8_E4M3 && (!k_scale || !v_scale)) return PA_ERR_INVALID_ARG;
+    if (static_cast<unsigned long long>(num_blocks) * 2 * num_kv_heads * block_size >= (1ull << 31))
+        return PA_ERR_UNSUPPORTED;  // TMA row coordinates are 32-bit signed
+    if (external_buf && (reinterpret_cast<uintptr_t>(external_buf) & 255)) return PA_ERR_INVALID_ARG;
+    pa_cache* c = new (std::nothrow) pa_cache();
+    if (!c) return PA_ERR_OOM;
+    c->num_blocks = num_blocks;
+    c->block_size = block_size;
+    c->num_kv_heads = num_kv_heads;
+    c->head_size = head_size;
+    c->kv_dtype = kv_dtype;
+    c->k_scale = kv_dtype == PA_FP8_E4M3 ? k_scale : nullptr;
+    c->v_scale = kv_dtype == PA_FP8_E4M3 ? v_scale : nullptr;
+    c->bytes = bytes;
+    c->device = current_device();
+    if (external_buf) {
+        c->data = external_buf;
+        c->owns = false;
+    } else {
+        cudaError_t e = cudaMalloc(&c->data, bytes);
+        if (e != cudaSuccess) {
+            g_last_cuda_error = static_cast<int>(e);
+            cudaGetLastError();
+            delete c;
+            return e == cudaErrorMemoryAllocation ? PA_ERR_OOM : PA_ERR_CUDA;
+        }
+        c->owns = true;
+    }
+    const int st = make_tensor_map(c);
+    if (st != PA_OK) {
+        if (c->owns) cudaFree(c->data);
+        delete c;
+        return st;
+    }
+    *out = c;
+    return PA_OK;
+}
+
+int pa_free_cache(pa_cache* cache) {
+    if (!cache) return PA_OK;
+    int st = PA_OK;
+    if (cache->owns) {
+        cudaError_t e = cudaDeviceSynchronize();
+        if (e == cudaSuccess) e = cudaFree(cache->data);
+        if (e != cudaSuccess) st = fail_cuda(e);
+    }
+    delete cache;
+    return st;
+}
+
+void* pa_cache_data(const pa_cache* cache) { return cache ? cache->data : nullptr; }
+
+int pa_slot_mapping(const int32_t* block_table, int max_blocks_per_seq, const int32_t* seq_lens,
+                    const int32_t* query_start_loc, int num_seqs, int num_tokens,
+                    int block_size, int32_t* slot_mapping, void* stream) {
+    if (num_seqs < 0 || num_tokens < 0 || block_size <= 0 || max_blocks_per_seq <= 0)
+        return PA_ERR_INVALID_ARG;
+    if (num_seqs == 0 || num_tokens == 0) return PA_OK;
+    if (!block_table || !seq_lens || !query_start_loc || !slot_mapping) return PA_ERR_INVALID_ARG;
+    if (num_seqs > (1 << 30)) return PA_ERR_UNSUPPORTED;
+    cudaError_t e = pa::launch_slot_mapping(block_table, max_blocks_per_seq, seq_lens,
+                                            query_start_loc, num_seqs, num_tokens, block_size,
+                                            slot_mapping,
+                                            device_error_ptr(), static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PA_OK : fail_cuda(e);
+}
+
+int pa_write_kv(pa_cache* cache, const void* k, const void* v, const int32_t* slot_mapping,
+                int num_tokens, void* stream) {
+    if (!cache || num_tokens < 0) return PA_ERR_INVALID_ARG;
+    if (num_tokens == 0) return PA_OK;
+    if (!k || !v || !slot_mapping) return PA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(k) | reinterpret_cast<uintptr_t>(v)) & 15)
+        return PA_ERR_INVALID_ARG;  // rows are moved as 16-byte vectors
+    cudaError_t e = pa::launch_write_kv(*cache, k, v, slot_mapping, num_tokens, device_error_ptr(),
+                                        static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PA_OK : fail_cuda(e);
+}
+
+size_t pa_attention_workspace_bytes(int num_tokens, int num_q_heads, int head_size,
+                                    int max_splits) {
+    if (num_tokens <= 0 || num_q_heads <= 0 || head_size <= 0) return 0;
+    return workspace_for(num_tokens, num_q_heads, head_size, max_splits);
+}
+
+int pa_plan_attention(const int32_t* seq_lens_host, const int32_t* query_start_loc_host,
+                      int num_seqs, int num_tokens, int num_q_heads, int num_kv_heads,
+                      int head_size, int block_size, int max_blocks_per_seq, int num_sms,
+                      size_t workspace_bytes, const pa_attention_opts* opts, pa_plan* plan) {
+    if (!plan) return PA_ERR_INVALID_ARG;
+    if (head_size != 64 && head_size != 128) return PA_ERR_UNSUPPORTED;
+    return plan_impl(seq_lens_host, query_start_loc_host, num_seqs, num_tokens, num_q_heads,
+                     num_kv_heads, head_size, block_size, max_blocks_per_seq, num_sms,
+                     workspace_bytes, opts, plan);
+}
+
+int pa_attention_ex(const pa_cache* cache, const void* q, int num_q_heads,
+                    const int32_t* block_table, int max_blocks_per_seq, const int32_t* seq_lens,
+                    const int32_t* query_start_loc, const int32_t* seq_lens_host,
+                    const int32_t* query_start_loc_host, int num_seqs, int num_tokens,
+                    float scale, float* out, void* workspace, size_t workspace_bytes,
+                    const pa_attention_opts* opts, void* stream) {
+    if (!cache || num_seqs < 0 || num_tokens < 0 || num_q_heads <= 0) return PA_ERR_INVALID_ARG;
+    if (num_q_heads % cache->num_kv_heads) return PA_ERR_INVALID_ARG;
+    if (num_tokens == 0) return PA_OK;
+    if (!q || !block_table || !seq_lens || !query_start_loc || !seq_lens_host ||
+        !query_start_loc_host || !out)
+        return PA_ERR_INVALID_ARG;
+    if (!(scale > 0.f) || scale != scale) return PA_ERR_INVALID_ARG;
+    if (workspace_bytes && !workspace) return PA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(q) & 15) || (reinterpret_cast<uintptr_t>(out) & 15) ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255))
+        return PA_ERR_INVALID_ARG;
+    const int num_sms = (opts && opts->num_sms > 0) ? opts->num_sms : device_num_sms();
+    if (num_sms <= 0) return fail_cuda(cudaErrorNoDevice);
+    pa_plan pl;
+    int st = plan_impl(seq_lens_host, query_start_loc_host, num_seqs, num_tokens, num_q_heads,
+                       cache->num_kv_heads, cache->head_size, cache->block_size,
+                       max_blocks_per_seq, num_sms, workspace_bytes, opts, &pl);
+    if (st != PA_OK) return st;
+    if (pl.num_chunk_seqs && cache->kv_dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+    if (pl.workspace_needed > workspace_bytes) return PA_ERR_WORKSPACE;
+
+    pa::AttnParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.block_table = block_table;
+    p.seq_lens = seq_lens;
+    p.qsl = query_start_loc;
+    p.out = out;
+    if (pl.any_split) {
+        const int smax = pl.decode_max_splits > pl.chunk_max_splits ? pl.decode_max_splits
+                                                                     : pl.chunk_max_splits;
+        p.max_splits = smax;
+        const size_t rows = static_cast<size_t>(smax) * num_tokens * num_q_heads;
+        p.part_o = static_cast<float*>(workspace);
+        p.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                              align256(rows * cache->head_size * sizeof(float)));
+    }
+    p.k_scale = cache->k_scale;
+    p.v_scale = cache->v_scale;
+    p.max_blocks_per_seq = max_blocks_per_seq;
+    p.num_seqs = num_seqs;
+    p.num_tokens = num_tokens;
+    p.num_q_heads = num_q_heads;
+    p.num_kv_heads = cache->num_kv_heads;
+    p.group = num_q_heads / cache->num_kv_heads;
+    p.num_blocks = cache->num_blocks;
+    p.decode_split_blocks = pl.decode_split_blocks > 0 ? pl.decode_split_blocks : 1;
+    p.chunk_split_blocks = pl.chunk_split_blocks > 0 ? pl.chunk_split_blocks : 4;
+    p.chunk_max_qtiles = pl.chunk_max_qtiles > 0 ? pl.chunk_max_qtiles : 1;
+    p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    p.err = device_error_ptr();
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    void* const* ev = opts ? opts->events : nullptr;
+    cudaError_t e = cudaSuccess;
+    if (pl.num_decode_seqs) {
+        if (ev) record(ev[0], s);
+        e = pa::launch_decode(cache->tmap, p, cache->head_size, cache->kv_dtype,
+                              pl.decode_max_splits, s);
+        if (e != cudaSuccess) return fail_cuda(e);
+        if (ev) record(ev[1], s);
+    }
+    if (pl.num_chunk_seqs) {
+        if (ev) record(ev[2], s);
+        e = pa::launch_chunk(cache->tmap, p, cache->head_size, cache->kv_dtype,
+                             pl.chunk_max_splits, s);
+        if (e != cudaSuccess) return fail_cuda(e);
+        if (ev) record(ev[3], s);
+    }
+    if (pl.any_split) {
+        if (ev) record(ev[4], s);
+        e = pa::launch_reduce(p, cache->head_size, s);
+        if (e != cudaSuccess) return fail_cuda(e);
+        if (ev) record(ev[5], s);
+    }
+    return PA_OK;
+}
+
+int pa_attention(const pa_cache* cache, const void* q, int num_q_heads,
+                 const int32_t* block_table, int max_blocks_per_seq, const int32_t* seq_lens,
+                 const int32_t* query_start_loc, const int32_t* seq_lens_host,
+                 const int32_t* query_start_loc_host, int num_seqs, int num_tokens,
+                 float scale, float* out, void* workspace, size_t workspace_bytes,
+                 void* stream) {
+    return pa_attention_ex(cache, q, num_q_heads, block_table, max_blocks_per_seq, seq_lens,
+                           query_start_loc, seq_lens_host, query_start_loc_host, num_seqs,
+                           num_tokens, scale, out, workspace, workspace_bytes, nullptr, stream);
+}
+
+int pa_validate_block_table(const pa_cache* cache, const int32_t* block_table,
+                            int max_blocks_per_seq, const int32_t* seq_lens, int num_seqs,
+                            int* num_bad, void* stream) {
+    if (!cache || !num_bad || num_seqs < 0 || max_blocks_per_seq <= 0) return PA_ERR_INVALID_ARG;
+    *num_bad = 0;
+    if (num_seqs == 0) return PA_OK;
+    if (!block_table || !seq_lens) return PA_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    int* counter = nullptr;
+    cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&counter), sizeof(int), s);
+    if (e != cudaSuccess) return fail_cuda(e);
+    e = cudaMemsetAsync(counter, 0, sizeof(int), s);
+    if (e == cudaSuccess)
+        e = pa::launch_validate(block_table, max_blocks_per_seq, seq_lens, num_seqs,
+                                cache->block_size, cache->num_blocks, counter, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(num_bad, counter, sizeof(int), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    cudaFreeAsync(counter, s);
+    return e == cudaSuccess ? PA_OK : fail_cuda(e);
+}
+
+int pa_device_error(int* code, int reset) {
+    if (!code) return PA_ERR_INVALID_ARG;
+    *code = 0;
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e == cudaSuccess) e = cudaMemcpyFromSymbol(code, g_device_error_word, sizeof(int));
+    if (e == cudaSuccess && reset) {
+        const int zero = 0;
+        e = cudaMemcpyToSymbol(g_device_error_word, &zero, sizeof(int));
+    }
+    return e == cudaSuccess ? PA_OK : fail_cuda(e);
+}
+
+}  // extern "C"

@@ -1,0 +1,402 @@
+// GQA-grouped paged decode attention (sm_100a).
+//
+// One CTA owns (KV split, kv head, request) of a decode-kind request (q_len * group <= 8
+// query rows sharing one kv head; a plain decode step has q_len = 1).  It streams the
+// split's physical blocks, looked up through the request's block table ("vLLM
+// architecture overview", section 2: the block table is an int32 array indexed by logical
+// block), and runs the online-softmax recurrence of FlashAttention ("vLLM: from KV Cache to
+// high-throughput serving", article 7 outline) over them.  The split-KV partition with an
+// LSE merge is the "V2" partitioned PagedAttention kernel of the kernel layer (architecture
+// overview, section 3).
+//
+// Data movement.  Each (physical block, K|V, kv head) tile is 16 tokens x head_size
+// contiguous in the pool and arrives in shared memory by one or two 2-D TMA loads with
+// 128-byte swizzling, completing on an mbarrier.  Every warp owns a private ring of
+// NS stages and the blocks j = warp, warp + NW, ... of the split, so warps never wait for
+// one another inside the stream; the CTA merges its warps' (m, l, O) at the end.
+//
+// Math.  The MMA runs transposed: S^T = K Q^T with the 16 keys of a block on M and the
+// query rows (GQA group x q_len, padded to 8) on N of an m16n8k16 tile, so a group of 8
+// fills the tile with no padding.  P^T is brought into B-operand layout with movmatrix,
+// and O^T += V^T P^T reads V through ldmatrix.trans.  Softmax runs in the log2 domain.
+// FP8 E4M3 caches are decoded to f16 (exact) in registers; the K scale folds into the score
+// scale and the V scale into the epilogue.
+#include "pa_internal.h"
+
+namespace pa {
+namespace {
+
+constexpr uint32_t kFull = 0xffffffffu;
+constexpr int kIdsPerRound = 1024;  // block ids staged in shared memory per round
+
+template <int D, int NW, int NS, bool FP8>
+struct DecodeCfg {
+    static constexpr int kEsz = FP8 ? 1 : 2;
+    static constexpr int kBoxes = D * kEsz / 128;          // 128-byte column slabs per row
+    static constexpr int kBoxElems = 128 / kEsz;
+    static constexpr int kTileBytes = kBlockSize * D * kEsz;  // one (block, K|V, head) tile
+    static constexpr int kStageBytes = 2 * kTileBytes;
+    static constexpr int kRingBytes = NW * NS * kStageBytes;
+    static constexpr int kMergeBytes = NW * (kDecodeRows * D + 2 * kDecodeRows) * 4;
+    static constexpr int kSmemBytes =
+        (kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes) + 1024;  // + alignment slack
+    static constexpr int kKSteps = D / 16;
+};
+
+template <int D, int NW, int NS, bool FP8>
+__global__ void __launch_bounds__(NW * 32)
+decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
+    using C = DecodeCfg<D, NW, NS, FP8>;
+    const int split = blockIdx.x, g = blockIdx.y, r = blockIdx.z;
+    const int q0 = p.qsl[r];
+    const int q_len = p.qsl[r + 1] - q0;
+    if (!is_decode_kind(q_len, p.group)) return;
+    if (q0 < 0 || q0 + q_len > p.num_tokens) {  // never index q/out past num_tokens
+        if (split == 0 && threadIdx.x == 0) raise_error(p.err, kErrMetadata);
+        return;
+    }
+    int ctx = p.seq_lens[r];
+    if (ctx > p.max_blocks_per_seq * kBlockSize) {  // never read past the table row
+        if (split == 0 && threadIdx.x == 0) raise_error(p.err, kErrMetadata);
+        ctx = p.max_blocks_per_seq * kBlockSize;
+    }
+    const int nblocks = ceil_div(ctx, kBlockSize);
+    const int nsplit = ceil_div(nblocks, p.decode_split_blocks);
+    if (split >= nsplit) return;
+    const int jb = split * p.decode_split_blocks;
+    const int je = min(nblocks, jb + p.decode_split_blocks);
+
+    extern __shared__ uint8_t smem_raw[];
+    __shared__ uint64_t bars[NW * NS];
+    __shared__ int ids[kIdsPerRound];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int gq = lane >> 2, tq = lane & 3;
+    const int rows = q_len * p.group;
+
+    if (tid == 0) prefetch_tensor_map(&tmap);
+    if (lane == 0)
+        for (int s = 0; s < NS; ++s) mbar_init(smem_u32(&bars[warp * NS + s]), 1);
+    fence_barrier_init();
+
+    // ---- Q^T as B fragments: row n = gq is (token n / group, head g * group + n % group)
+    uint32_t qb[C::kKSteps][2];
+    {
+        const int n = gq;
+        const bool valid = n < rows;
+        const __nv_bfloat16* qrow =
+            p.q + (static_cast<int64_t>(q0 + (valid ? n / p.group : 0)) * p.num_q_heads +
+                   g * p.group + (valid ? n % p.group : 0)) * D;
+#pragma unroll
+        for (int ks = 0; ks < C::kKSteps; ++ks) {
+            if (!valid) {
+                qb[ks][0] = qb[ks][1] = 0u;
+            } else if constexpr (!FP8) {
+                qb[ks][0] = *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * tq);
+                qb[ks][1] = *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * tq + 8);
+            } else {
+                // k-step ks covers dims 16ks..16ks+15 permuted to match the FP8 K fragments:
+                // logical k = 2t+e <-> dim 16ks+4t+e, k = 8+2t+e <-> dim 16ks+4t+2+e.
+                const uint2 raw = *reinterpret_cast<const uint2*>(qrow + 16 * ks + 4 * tq);
+                const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
+                const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
+                qb[ks][0] = pack_f16(__low2float(lo), __high2float(lo));
+                qb[ks][1] = pack_f16(__low2float(hi), __high2float(hi));
+            }
+        }
+    }
+    // last visible key of the two rows this thread's S/O columns belong to
+    const int row0 = 2 * tq, row1 = 2 * tq + 1;
+    const int lim0 = row0 < rows ? ctx - q_len + row0 / p.group : ctx - 1;
+    const int lim1 = row1 < rows ? ctx - q_len + row1 / p.group : ctx - 1;
+    float sl = p.scale_log2;
+    if constexpr (FP8) sl *= p.k_scale[g];
+
+    float o[C::kKSteps][4];
+#pragma unroll
+    for (int i = 0; i < C::kKSteps; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+
+    const uint32_t ring = smem_u32(smem) + warp * NS * C::kStageBytes;
+    const int kv_rows_per_block = 2 * p.num_kv_heads * kBlockSize;
+    uint32_t loads = 0;  // loads issued by this warp so far (stage = n % NS, phase = n / NS)
+    bool ok = true;
+
+    for (int rb = jb; rb < je; rb += kIdsPerRound) {
+        const int rn = min(kIdsPerRound, je - rb);
+        __syncthreads();  // every warp reaches this once per round, even after an error
+        for (int k = tid; k < rn; k += NW * 32) {
+            int b = p.block_table[static_cast<int64_t>(r) * p.max_blocks_per_seq + rb + k];
+            if (b < 0 || b >= p.num_blocks) {
+                raise_error(p.err, kErrBadBlockId);
+                b = 0;
+            }
+            ids[k] = b;
+        }
+        __syncthreads();
+        const int mine = (ok && rn > warp) ? (rn - warp + NW - 1) / NW : 0;
+
+        auto issue = [&](int i, uint32_t n) {
+            const int blk = ids[warp + i * NW];
+            const uint32_t st = n % NS;
+            const uint32_t bar = smem_u32(&bars[warp * NS + st]);
+            const uint32_t dst = ring + st * C::kStageBytes;
+            const int rowk = blk * kv_rows_per_block + g * kBlockSize;
+            const int rowv = rowk + p.num_kv_heads * kBlockSize;
+            mbar_arrive_expect_tx(bar, C::kStageBytes);
+#pragma unroll
+            for (int b = 0; b < C::kBoxes; ++b) {
+                tma_load_2d(dst + b * 2048, &tmap, bar, b * C::kBoxElems, rowk);
+                tma_load_2d(dst + C::kTileBytes + b * 2048, &tmap, bar, b * C::kBoxElems, rowv);
+            }
+        };
+
+        if (lane == 0)
+            for (int i = 0; i < min(NS, mine); ++i) issue(i, loads + i);
+        __syncwarp();
+
+        int fail_i = -1;
+        for (int i = 0; i < mine; ++i) {
+            const uint32_t n = loads + i;
+            const uint32_t st = n % NS;
+            if (!mbar_wait(smem_u32(&bars[warp * NS + st]), (n / NS) & 1u, kWaitLimitNs, p.err)) {
+                ok = false;
+                fail_i = i;
+                break;
+            }
+            const uint32_t kt = ring + st * C::kStageBytes;
+            const uint32_t vt = kt + C::kTileBytes;
+            const int kb = (rb + warp + i * NW) * kBlockSize;  // position of the block's key 0
+
+            if (kb + kBlockSize > ctx) {
+                // last, partly filled block: clear V rows past the context so that stale
+                // cache bytes (possibly NaN patterns) cannot reach P.V
+                const int nz = ctx - kb;
+                uint8_t* vg = smem + (vt - smem_u32(smem));
+                for (int idx = lane; idx < (kBlockSize - nz) * C::kBoxes * 8; idx += 32) {
+                    const int row = nz + idx / (C::kBoxes * 8);
+                    const int c = idx % (C::kBoxes * 8);
+                    *reinterpret_cast<uint4*>(vg + (c >> 3) * 2048 + row * 128 + (c & 7) * 16) =
+                        make_uint4(0, 0, 0, 0);
+                }
+                fence_proxy_async();  // order these writes before the stage's next TMA fill
+                __syncwarp();
+            }
+
+            // ---- S^T (16 keys x 8 rows) = K Q^T
+            float s[4] = {0.f, 0.f, 0.f, 0.f};
+            if constexpr (!FP8) {
+#pragma unroll
+                for (int ks = 0; ks < C::kKSteps; ++ks) {
+                    const int mi = lane >> 3, rr = lane & 7;
+                    const int key = rr + ((mi & 1) << 3);
+                    const int chunk = 2 * ks + (mi >> 1);
+                    uint32_t a0, a1, a2, a3;
+                    ldsm_x4(kt + (chunk >> 3) * 2048 + sw128(key, chunk & 7), a0, a1, a2, a3);
+                    mma_bf16(s, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
+                }
+            } else {
+#pragma unroll
+                for (int cp = 0; cp < C::kKSteps / 2; ++cp) {
+                    // matrices: (keys 0-7, chunk 2cp), (keys 8-15, 2cp), (0-7, 2cp+1), (8-15, 2cp+1)
+                    const int mi = lane >> 3, rr = lane & 7;
+                    const int key = rr + ((mi & 1) << 3);
+                    const int chunk = 2 * cp + (mi >> 1);
+                    uint32_t r0, r1, r2, r3;
+                    ldsm_x4(kt + sw128(key, chunk), r0, r1, r2, r3);
+                    mma_f16(s, e4m3x2_to_f16x2(r0 & 0xffff), e4m3x2_to_f16x2(r1 & 0xffff),
+                            e4m3x2_to_f16x2(r0 >> 16), e4m3x2_to_f16x2(r1 >> 16),
+                            qb[2 * cp][0], qb[2 * cp][1]);
+                    mma_f16(s, e4m3x2_to_f16x2(r2 & 0xffff), e4m3x2_to_f16x2(r3 & 0xffff),
+                            e4m3x2_to_f16x2(r2 >> 16), e4m3x2_to_f16x2(r3 >> 16),
+                            qb[2 * cp + 1][0], qb[2 * cp + 1][1]);
+                }
+            }
+
+            // ---- online softmax over the block's keys (log2 domain)
+            const int p0 = kb + gq, p1 = kb + gq + 8;
+            float x0 = p0 <= lim0 ? s[0] * sl : -INFINITY;
+            float x1 = p0 <= lim1 ? s[1] * sl : -INFINITY;
+            float x2 = p1 <= lim0 ? s[2] * sl : -INFINITY;
+            float x3 = p1 <= lim1 ? s[3] * sl : -INFINITY;
+            float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) {
+                mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, off));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(kFull, mx1, off));
+            }
+            const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+            const float ref0 = mn0 == -INFINITY ? 0.f : mn0;
+            const float ref1 = mn1 == -INFINITY ? 0.f : mn1;
+            const float al0 = fast_exp2(m0 - ref0), al1 = fast_exp2(m1 - ref1);
+            x0 = fast_exp2(x0 - ref0);
+            x2 = fast_exp2(x2 - ref0);
+            x1 = fast_exp2(x1 - ref1);
+            x3 = fast_exp2(x3 - ref1);
+            l0 = l0 * al0 + x0 + x2;
+            l1 = l1 * al1 + x1 + x3;
+            m0 = mn0;
+            m1 = mn1;
+            if (__any_sync(kFull, al0 != 1.f || al1 != 1.f)) {
+#pragma unroll
+                for (int mt = 0; mt < C::kKSteps; ++mt) {
+                    o[mt][0] *= al0;
+                    o[mt][1] *= al1;
+                    o[mt][2] *= al0;
+                    o[mt][3] *= al1;
+                }
+            }
+
+            // ---- O^T (D x 8) += V^T P^T
+            if constexpr (!FP8) {
+                const uint32_t pb0 = movmatrix_t(pack_bf16(x0, x1));
+                const uint32_t pb1 = movmatrix_t(pack_bf16(x2, x3));
+#pragma unroll
+                for (int mt = 0; mt < C::kKSteps; ++mt) {
+                    const int mi = lane >> 3, rr = lane & 7;
+                    const int key = rr + ((mi >> 1) << 3);
+                    const int chunk = 2 * mt + (mi & 1);
+                    uint32_t a0, a1, a2, a3;
+                    ldsm_x4_t(vt + (chunk >> 3) * 2048 + sw128(key, chunk & 7), a0, a1, a2, a3);
+                    mma_bf16(o[mt], a0, a1, a2, a3, pb0, pb1);
+                }
+            } else {
+                const uint32_t pb0 = movmatrix_t(pack_f16(x0, x1));
+                const uint32_t pb1 = movmatrix_t(pack_f16(x2, x3));
+                const uint8_t* vs = smem + (vt - smem_u32(smem));
+#pragma unroll
+                for (int j = 0; j < D / 32; ++j) {
+                    // word w = 8j + gq of key rows 2t, 2t+1, 2t+8, 2t+9 (dims 32j + 4gq .. +3)
+                    const int w = 8 * j + gq;
+                    const int c = w >> 2, wb = (w & 3) * 4;
+                    const uint32_t k0 = *reinterpret_cast<const uint32_t*>(vs + sw128(2 * tq, c) + wb);
+                    const uint32_t k1 = *reinterpret_cast<const uint32_t*>(vs + sw128(2 * tq + 1, c) + wb);
+                    const uint32_t k2 = *reinterpret_cast<const uint32_t*>(vs + sw128(2 * tq + 8, c) + wb);
+                    const uint32_t k3 = *reinterpret_cast<const uint32_t*>(vs + sw128(2 * tq + 9, c) + wb);
+                    // byte pairs (key 2t, key 2t+1) for dims +0,+1 and +2,+3
+                    const uint32_t lo01 = __byte_perm(k0, k1, 0x5140);
+                    const uint32_t hi01 = __byte_perm(k0, k1, 0x7362);
+                    const uint32_t lo23 = __byte_perm(k2, k3, 0x5140);
+                    const uint32_t hi23 = __byte_perm(k2, k3, 0x7362);
+                    // m-tile (j, 0): rows m=g <-> dim +0, m=g+8 <-> dim +1
+                    mma_f16(o[2 * j], e4m3x2_to_f16x2(lo01 & 0xffff), e4m3x2_to_f16x2(lo01 >> 16),
+                            e4m3x2_to_f16x2(lo23 & 0xffff), e4m3x2_to_f16x2(lo23 >> 16), pb0, pb1);
+                    // m-tile (j, 1): m=g <-> dim +2, m=g+8 <-> dim +3
+                    mma_f16(o[2 * j + 1], e4m3x2_to_f16x2(hi01 & 0xffff), e4m3x2_to_f16x2(hi01 >> 16),
+                            e4m3x2_to_f16x2(hi23 & 0xffff), e4m3x2_to_f16x2(hi23 >> 16), pb0, pb1);
+                }
+            }
+            __syncwarp();
+            if (lane == 0 && i + NS < mine) issue(i + NS, n + NS);
+            __syncwarp();
+        }
+        if (fail_i >= 0) {
+            // wind down: wait (bounded, 0.1 s each) for this warp's loads still in flight
+            for (int i = fail_i; i < min(fail_i + NS, mine); ++i) {
+                const uint32_t n = loads + i;
+                mbar_wait(smem_u32(&bars[warp * NS + n % NS]), (n / NS) & 1u, kWindDownLimitNs,
+                          p.err);
+            }
+        }
+        loads += mine;
+    }
+    if (!__all_sync(kFull, ok)) ok = false;
+
+    // ---- merge the warps: (m, l, O^T) per warp through shared memory
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+        l0 += __shfl_xor_sync(kFull, l0, off);
+        l1 += __shfl_xor_sync(kFull, l1, off);
+    }
+    __syncthreads();
+    float* red_o = reinterpret_cast<float*>(smem);            // [NW][D][8]
+    float* red_m = red_o + NW * D * kDecodeRows;              // [NW][8]
+    float* red_l = red_m + NW * kDecodeRows;                  // [NW][8]
+    if (gq == 0) {
+        red_m[warp * 8 + row0] = m0;
+        red_m[warp * 8 + row1] = m1;
+        red_l[warp * 8 + row0] = l0;
+        red_l[warp * 8 + row1] = l1;
+    }
+#pragma unroll
+    for (int mt = 0; mt < C::kKSteps; ++mt) {
+        int d0, d1;
+        if constexpr (!FP8) {
+            d0 = 16 * mt + gq;
+            d1 = d0 + 8;
+        } else {
+            d0 = 32 * (mt >> 1) + 4 * gq + 2 * (mt & 1);
+            d1 = d0 + 1;
+        }
+        float* base = red_o + warp * D * 8;
+        base[d0 * 8 + row0] = o[mt][0];
+        base[d0 * 8 + row1] = o[mt][1];
+        base[d1 * 8 + row0] = o[mt][2];
+        base[d1 * 8 + row1] = o[mt][3];
+    }
+    __syncthreads();
+    if (!ok) return;
+
+    const float vscale = FP8 ? p.v_scale[g] : 1.f;
+    const bool direct = nsplit == 1;
+    if (!direct && split >= p.max_splits) return;  // workspace bound (planned launch ensures it)
+    for (int idx = tid; idx < rows * D; idx += NW * 32) {
+        const int n = idx / D, d = idx % D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) M = fmaxf(M, red_m[w * 8 + n]);
+        float L = 0.f, acc = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < NW; ++w) {
+                const float e = fast_exp2(red_m[w * 8 + n] - M);
+                L += red_l[w * 8 + n] * e;
+                acc += red_o[(w * D + d) * 8 + n] * e;
+            }
+        }
+        const float val = L > 0.f ? acc / L * vscale : 0.f;
+        const int t = q0 + n / p.group;
+        const int h = g * p.group + n % p.group;
+        if (direct) {
+            p.out[(static_cast<int64_t>(t) * p.num_q_heads + h) * D + d] = val;
+        } else {
+            const int64_t prow = (static_cast<int64_t>(split) * p.num_tokens + t) * p.num_q_heads + h;
+            p.part_o[prow * D + d] = val;
+            if (d == 0) p.part_lse[prow] = L > 0.f ? M + __log2f(L) : -INFINITY;
+        }
+    }
+}
+
+template <int D, int NW, int NS, bool FP8>
+cudaError_t launch_decode_t(const CUtensorMap& tmap, const AttnParams& p, int max_splits,
+                            cudaStream_t stream) {
+    using C = DecodeCfg<D, NW, NS, FP8>;
+    auto kern = decode_kernel<D, NW, NS, FP8>;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             C::kSmemBytes);
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    dim3 grid(max_splits, p.num_kv_heads, p.num_seqs);
+    kern<<<grid, NW * 32, C::kSmemBytes, stream>>>(tmap, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const CUtensorMap& tmap, const AttnParams& p, int head_size,
+                          int kv_dtype, int max_splits, cudaStream_t stream) {
+    if (kv_dtype == PA_BF16 && head_size == 128)
+        return launch_decode_t<128, 4, 3, false>(tmap, p, max_splits, stream);
+    if (kv_dtype == PA_BF16 && head_size == 64)
+        return launch_decode_t<64, 4, 6, false>(tmap, p, max_splits, stream);
+    if (kv_dtype == PA_FP8_E4M3 && head_size == 128)
+        return launch_decode_t<128, 4, 6, true>(tmap, p, max_splits, stream);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace pa

@@ -1,0 +1,66 @@
+// Internal declarations shared by the host API and the kernel translation units.
+#pragma once
+
+#include "../../include/pa.h"
+#include "pa_common.cuh"
+
+struct pa_cache {
+    int num_blocks;
+    int block_size;
+    int num_kv_heads;
+    int head_size;
+    int kv_dtype;
+    const float* k_scale;  // device [num_kv_heads] (FP8 only)
+    const float* v_scale;
+    void* data;            // device pool
+    size_t bytes;
+    bool owns;
+    int device;
+    CUtensorMap tmap;      // 2-D view of the pool: rows of head_size elements
+};
+
+namespace pa {
+
+// Arguments of one attention launch (kernels read them from the parameter space).
+struct AttnParams {
+    const __nv_bfloat16* q;     // [T][Hq][D]
+    const int32_t* block_table; // [B][max_blocks_per_seq]
+    const int32_t* seq_lens;    // [B]
+    const int32_t* qsl;         // [B+1]
+    float* out;                 // [T][Hq][D]
+    float* part_o;              // [S][T][Hq][D] split partials (normalised)
+    float* part_lse;            // [S][T][Hq]   split log2-sum-exp2 of scaled scores
+    const float* k_scale;       // FP8 per-kv-head scales, else null
+    const float* v_scale;
+    int max_blocks_per_seq;
+    int num_seqs;
+    int num_tokens;
+    int num_q_heads;
+    int num_kv_heads;
+    int group;                  // num_q_heads / num_kv_heads
+    int num_blocks;             // pool size, for block id checks
+    int decode_split_blocks;    // KV partition of decode-kind requests (blocks)
+    int chunk_split_blocks;     // KV partition of chunk-kind requests (blocks, multiple of 4)
+    int chunk_max_qtiles;       // grid.x stride of the chunk kernel
+    int max_splits;             // splits the workspace holds (bounds every partial index)
+    float scale_log2;           // softmax scale * log2(e)
+    int* err;                   // device error word
+};
+
+cudaError_t launch_decode(const CUtensorMap& tmap, const AttnParams& p, int head_size,
+                          int kv_dtype, int max_splits, cudaStream_t stream);
+cudaError_t launch_chunk(const CUtensorMap& tmap, const AttnParams& p, int head_size,
+                         int kv_dtype, int max_splits, cudaStream_t stream);
+cudaError_t launch_reduce(const AttnParams& p, int head_size, cudaStream_t stream);
+cudaError_t launch_slot_mapping(const int32_t* block_table, int max_blocks_per_seq,
+                                const int32_t* seq_lens, const int32_t* qsl, int num_seqs,
+                                int num_tokens, int block_size, int32_t* slot_mapping, int* err,
+                                cudaStream_t stream);
+cudaError_t launch_write_kv(const pa_cache& c, const void* k, const void* v,
+                            const int32_t* slot_mapping, int num_tokens, int* err,
+                            cudaStream_t stream);
+cudaError_t launch_validate(const int32_t* block_table, int max_blocks_per_seq,
+                            const int32_t* seq_lens, int num_seqs, int block_size,
+                            int num_blocks, int* counter, cudaStream_t stream);
+
+}  // namespace pa

@@ -1,0 +1,152 @@
+// Slot mapping, cache write (reshape_and_cache) and the opt-in block-table validator.
+//
+// Slot of a new token ("vLLM: from KV Cache to high-throughput serving", article 3 outline;
+// "Inside vLLM" notes, core point 2): token i of request r sits at position
+// p = seq_len - q_len + i and lands in slot block_table[r][p / bs] * bs + p % bs.
+//
+// The write ("vLLM architecture overview", section 3, reshape_and_cache) moves each
+// (token, kv head) row of K and V into its slot of the pool [block][K|V][kv head][16][D].
+// One thread moves 16 bytes of bf16 input; consecutive threads cover consecutive bytes of a
+// row, so both the reads of k/v and the writes into the pool are coalesced.  An FP8 pool
+// stores e4m3(x / scale[head]) with an IEEE-rounded fp32 divide and saturating conversion.
+#include "pa_internal.h"
+
+namespace pa {
+namespace {
+
+__global__ void slot_mapping_kernel(const int32_t* __restrict__ bt, int maxb,
+                                    const int32_t* __restrict__ seq_lens,
+                                    const int32_t* __restrict__ qsl, int bs, int num_tokens,
+                                    int32_t* __restrict__ slots, int* err) {
+    const int r = blockIdx.x;
+    const int q0 = qsl[r];
+    const int q_len = qsl[r + 1] - q0;
+    const int ctx = seq_lens[r];
+    if (q0 < 0 || q0 + q_len > num_tokens) {  // never write past the slot array
+        if (threadIdx.x == 0) raise_error(err, kErrBadSlotMeta);
+        return;
+    }
+    for (int i = threadIdx.x; i < q_len; i += blockDim.x) {
+        const int pos = ctx - q_len + i;
+        const int logical = pos / bs;
+        if (pos < 0 || logical >= maxb) {
+            raise_error(err, kErrBadSlotMeta);
+            slots[q0 + i] = -1;
+            continue;
+        }
+        slots[q0 + i] = bt[static_cast<int64_t>(r) * maxb + logical] * bs + pos % bs;
+    }
+}
+
+template <int D, bool FP8>
+__global__ void __launch_bounds__(256)
+write_kv_kernel(uint8_t* __restrict__ cache, const uint16_t* __restrict__ k,
+                const uint16_t* __restrict__ v, const int32_t* __restrict__ slots,
+                int num_tokens, int num_kv_heads, int64_t num_slots,
+                const float* __restrict__ k_scale, const float* __restrict__ v_scale,
+                int* err) {
+    constexpr int kChunks = D / 8;  // 16-byte pieces of one bf16 row
+    const int64_t total = static_cast<int64_t>(num_tokens) * num_kv_heads * 2 * kChunks;
+    for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+         idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int c = static_cast<int>(idx % kChunks);
+        int64_t rest = idx / kChunks;
+        const int kv = static_cast<int>(rest % 2);
+        rest /= 2;
+        const int h = static_cast<int>(rest % num_kv_heads);
+        const int64_t t = rest / num_kv_heads;
+        const int slot = slots[t];
+        if (slot < 0) continue;
+        if (slot >= num_slots) {
+            raise_error(err, kErrBadSlotMeta);
+            continue;
+        }
+        const uint16_t* src = (kv ? v : k) + (t * num_kv_heads + h) * D + c * 8;
+        const uint4 x = __ldg(reinterpret_cast<const uint4*>(src));
+        const int64_t dst =
+            (((static_cast<int64_t>(slot / kBlockSize) * 2 + kv) * num_kv_heads + h) * kBlockSize +
+             slot % kBlockSize) * D + c * 8;
+        if constexpr (!FP8) {
+            *reinterpret_cast<uint4*>(cache + dst * 2) = x;
+        } else {
+            const float s = (kv ? v_scale : k_scale)[h];
+            const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+            uint16_t out[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float lo = __uint_as_float(w[j] << 16);
+                const float hi = __uint_as_float(w[j] & 0xffff0000u);
+                float2 y = make_float2(__fdiv_rn(lo, s), __fdiv_rn(hi, s));
+                out[j] = static_cast<uint16_t>(__nv_cvt_float2_to_fp8x2(y, __NV_SATFINITE, __NV_E4M3));
+            }
+            uint2 packed;
+            packed.x = static_cast<uint32_t>(out[0]) | (static_cast<uint32_t>(out[1]) << 16);
+            packed.y = static_cast<uint32_t>(out[2]) | (static_cast<uint32_t>(out[3]) << 16);
+            *reinterpret_cast<uint2*>(cache + dst) = packed;
+        }
+    }
+}
+
+__global__ void validate_kernel(const int32_t* __restrict__ bt, int maxb,
+                                const int32_t* __restrict__ seq_lens, int bs, int num_blocks,
+                                int* counter) {
+    const int r = blockIdx.x;
+    const int need = ceil_div(seq_lens[r], bs);
+    int bad = 0;
+    if (threadIdx.x == 0 && need > maxb) bad += need - maxb;
+    for (int j = threadIdx.x; j < min(need, maxb); j += blockDim.x) {
+        const int b = bt[static_cast<int64_t>(r) * maxb + j];
+        bad += (b < 0 || b >= num_blocks);
+    }
+    for (int off = 16; off > 0; off >>= 1) bad += __shfl_xor_sync(0xffffffffu, bad, off);
+    if ((threadIdx.x & 31) == 0 && bad) atomicAdd(counter, bad);
+}
+
+template <int D, bool FP8>
+cudaError_t launch_write_t(const pa_cache& c, const void* k, const void* v, const int32_t* slots,
+                           int num_tokens, int* err, cudaStream_t stream) {
+    const int64_t total = static_cast<int64_t>(num_tokens) * c.num_kv_heads * 2 * (D / 8);
+    const int threads = 256;
+    const int64_t blocks = (total + threads - 1) / threads;
+    const int grid = static_cast<int>(blocks < 148 * 32 ? blocks : 148 * 32);
+    write_kv_kernel<D, FP8><<<grid, threads, 0, stream>>>(
+        static_cast<uint8_t*>(c.data), static_cast<const uint16_t*>(k),
+        static_cast<const uint16_t*>(v), slots, num_tokens, c.num_kv_heads,
+        static_cast<int64_t>(c.num_blocks) * c.block_size, c.k_scale, c.v_scale, err);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_slot_mapping(const int32_t* block_table, int max_blocks_per_seq,
+                                const int32_t* seq_lens, const int32_t* qsl, int num_seqs,
+                                int num_tokens, int block_size, int32_t* slot_mapping, int* err,
+                                cudaStream_t stream) {
+    slot_mapping_kernel<<<num_seqs, 128, 0, stream>>>(block_table, max_blocks_per_seq, seq_lens,
+                                                      qsl, block_size, num_tokens, slot_mapping,
+                                                      err);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_write_kv(const pa_cache& c, const void* k, const void* v,
+                            const int32_t* slot_mapping, int num_tokens, int* err,
+                            cudaStream_t stream) {
+    if (num_tokens == 0) return cudaSuccess;
+    if (c.kv_dtype == PA_BF16 && c.head_size == 128)
+        return launch_write_t<128, false>(c, k, v, slot_mapping, num_tokens, err, stream);
+    if (c.kv_dtype == PA_BF16 && c.head_size == 64)
+        return launch_write_t<64, false>(c, k, v, slot_mapping, num_tokens, err, stream);
+    if (c.kv_dtype == PA_FP8_E4M3 && c.head_size == 128)
+        return launch_write_t<128, true>(c, k, v, slot_mapping, num_tokens, err, stream);
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_validate(const int32_t* block_table, int max_blocks_per_seq,
+                            const int32_t* seq_lens, int num_seqs, int block_size,
+                            int num_blocks, int* counter, cudaStream_t stream) {
+    validate_kernel<<<num_seqs, 128, 0, stream>>>(block_table, max_blocks_per_seq, seq_lens,
+                                                  block_size, num_blocks, counter);
+    return cudaGetLastError();
+}
+
+}  // namespace pa

@@ -1,0 +1,165 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports every entry point
+its header declares, sizes pools by the pages' block formula, plans launches consistently
+and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+from conftest import ROOT, golden_lines
+from paged_kv_cache_421_b200 import _binding as B
+from paged_kv_cache_421_b200 import build as pa_build
+from paged_kv_cache_421_b200 import workloads as W
+
+
+@pytest.fixture(scope="module")
+def lib():
+    pa_build.build()
+    return B.load()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "pa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\**\s*(pa_[a-z_0-9]+)\s*\(",
+                       src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ["pa_alloc_cache", "pa_write_kv", "pa_attention", "pa_slot_mapping",
+                     "pa_cache_bytes", "pa_free_cache", "pa_attention_workspace_bytes"]:
+        assert required in names
+    assert sorted(B.EXPORTED) == names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_cache_bytes_follow_block_formula(lib):
+    for row in golden_lines("block_sizing.txt"):
+        if row[0] != "block_bytes":
+            continue
+        bs, hkv, d, eb, want = map(int, row[1:])
+        dtype = B.PA_BF16 if eb == 2 else B.PA_FP8_E4M3
+        assert B.pa_cache_bytes(1, bs, hkv, d, dtype) == want
+        assert B.pa_cache_bytes(1000, bs, hkv, d, dtype) == 1000 * want
+    assert B.pa_cache_bytes(0, 16, 8, 128, B.PA_BF16) == 0
+    assert B.pa_cache_bytes(4, 16, 8, 128, 7) == 0
+
+
+def test_workspace_formula(lib):
+    assert B.pa_attention_workspace_bytes(8, 64, 128, 1) == 0
+    ws = B.pa_attention_workspace_bytes(8, 64, 128, 10)
+    assert ws >= 10 * 8 * 64 * 129 * 4 and ws < 10 * 8 * 64 * 129 * 4 + 512
+
+
+def _plan(wl, num_sms=148, ws=None, split=0):
+    if ws is None:
+        ws = B.pa_attention_workspace_bytes(max(wl.num_tokens, 1), wl.num_q_heads, wl.head_size,
+                                            1 << 16)
+    return B.pa_plan_attention(wl.seq_lens, wl.qsl, wl.num_q_heads, wl.num_kv_heads,
+                               wl.head_size, wl.max_blocks_per_seq, num_sms, ws,
+                               kv_split_tokens=split)
+
+
+@pytest.mark.parametrize("name", ["tiny_decode", "llama8b_decode", "mixed_step",
+                                  "prefix_share_decode", "long70b_decode"])
+def test_plan_invariants(lib, name):
+    wl = W.CONFIGS[name]()
+    p = _plan(wl)
+    G = wl.num_q_heads // wl.num_kv_heads
+    ql = wl.q_lens
+    dec = (ql > 0) & (ql * G <= 8)
+    assert p["num_decode_seqs"] == int(dec.sum())
+    assert p["num_chunk_seqs"] == int(((ql > 0) & ~dec).sum())
+    blocks = -(-wl.seq_lens.astype(np.int64) // 16)
+    if p["num_decode_seqs"]:
+        sb = p["decode_split_blocks"]
+        ns = -(-blocks[dec] // sb)
+        assert p["decode_max_splits"] == ns.max()
+        assert p["decode_ctas"] == int(ns.sum()) * wl.num_kv_heads
+        assert sb % 4 == 0 or sb == blocks[dec].max()
+    if p["num_chunk_seqs"]:
+        assert p["chunk_max_qtiles"] == int(np.max(-(-(ql[~dec & (ql > 0)] * G) // 64)))
+    smax = max(p["decode_max_splits"], p["chunk_max_splits"])
+    assert p["any_split"] == int(smax > 1)
+    assert p["workspace_needed"] == B.pa_attention_workspace_bytes(wl.num_tokens, wl.num_q_heads,
+                                                                    wl.head_size, smax)
+
+
+def test_plan_long_context_is_split_for_occupancy(lib):
+    wl = W.long70b_decode()
+    p = _plan(wl)
+    assert p["decode_max_splits"] > 1
+    assert p["decode_ctas"] >= 148 * 4  # several waves of CTAs on 148 SMs
+    # without workspace nothing is split
+    p0 = _plan(wl, ws=0)
+    assert p0["decode_max_splits"] == 1 and p0["workspace_needed"] == 0
+    # a small workspace caps the split count
+    ws3 = B.pa_attention_workspace_bytes(wl.num_tokens, wl.num_q_heads, wl.head_size, 3)
+    p3 = _plan(wl, ws=ws3)
+    assert p3["decode_max_splits"] <= 3 and p3["workspace_needed"] <= ws3
+
+
+def test_plan_forced_split(lib):
+    wl = W.tiny_decode()
+    p = _plan(wl, split=16)
+    assert p["decode_split_blocks"] == 1 and p["decode_max_splits"] == 4
+    with pytest.raises(B.PaError) as e:
+        _plan(wl, ws=0, split=16)
+    assert e.value.status == B.PA_ERR_WORKSPACE
+    with pytest.raises(B.PaError) as e:
+        _plan(wl, split=24)  # not a multiple of the block size
+    assert e.value.status == B.PA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("sl,qsl", [
+    ([5, 6], [0, 7, 8]),     # q_len > seq_len
+    ([5, 6], [1, 2, 3]),     # does not start at 0
+    ([5, 6], [0, 2, 1]),     # decreasing
+    ([0, 6], [0, 1, 2]),     # a query with no context
+    ([5, 2000], [0, 1, 2]),  # more blocks than the table holds
+])
+def test_plan_rejects_bad_metadata(lib, sl, qsl):
+    with pytest.raises(B.PaError) as e:
+        B.pa_plan_attention(np.array(sl), np.array(qsl), 8, 2, 128, 16, 148, 1 << 20)
+    assert e.value.status == B.PA_ERR_METADATA
+
+
+def test_plan_rejects_unsupported(lib):
+    with pytest.raises(B.PaError) as e:
+        B.pa_plan_attention(np.array([5]), np.array([0, 1]), 8, 2, 96, 16, 148, 0)
+    assert e.value.status == B.PA_ERR_UNSUPPORTED
+    with pytest.raises(B.PaError) as e:
+        B.pa_plan_attention(np.array([5]), np.array([0, 1]), 8, 3, 128, 16, 148, 0)
+    assert e.value.status == B.PA_ERR_INVALID_ARG
+
+
+def test_argument_errors_without_device(lib):
+    h = ctypes.c_void_p()
+    # unsupported shapes and missing FP8 scales fail before any allocation
+    assert lib.pa_alloc_cache(16, 16, 2, 96, B.PA_BF16, None, None, None, ctypes.byref(h)) == \
+        B.PA_ERR_UNSUPPORTED
+    assert lib.pa_alloc_cache(16, 8, 2, 128, B.PA_BF16, None, None, None, ctypes.byref(h)) == \
+        B.PA_ERR_UNSUPPORTED
+    assert lib.pa_alloc_cache(16, 16, 2, 64, B.PA_FP8_E4M3, None, None, None, ctypes.byref(h)) == \
+        B.PA_ERR_UNSUPPORTED
+    assert lib.pa_alloc_cache(16, 16, 2, 128, B.PA_FP8_E4M3, None, None, None, ctypes.byref(h)) == \
+        B.PA_ERR_INVALID_ARG
+    assert lib.pa_alloc_cache(0, 16, 2, 128, B.PA_BF16, None, None, None, ctypes.byref(h)) == \
+        B.PA_ERR_INVALID_ARG
+    assert lib.pa_alloc_cache(16, 16, 2, 128, B.PA_BF16, None, None, ctypes.c_void_p(0x1001),
+                              ctypes.byref(h)) == B.PA_ERR_INVALID_ARG
+    assert lib.pa_write_kv(None, None, None, None, 4, None) == B.PA_ERR_INVALID_ARG
+    assert lib.pa_attention(None, None, 8, None, 4, None, None, None, None, 1, 1, 0.1, None, None,
+                            0, None) == B.PA_ERR_INVALID_ARG
+    assert lib.pa_slot_mapping(None, 4, None, None, 1, 1, 16, None, None) == B.PA_ERR_INVALID_ARG
+    assert lib.pa_free_cache(None) == B.PA_OK
+    assert B.pa_status_string(B.PA_ERR_METADATA) == "PA_ERR_METADATA"

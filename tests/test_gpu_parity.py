@@ -1,0 +1,307 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle.
+
+Bit-exact for slot mapping and the cache contents; attention within the stated tolerance
+(bf16 KV: max abs 2e-2, mean abs 2e-3 against fp64; FP8 E4M3 KV: 4e-2 / 4e-3)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_common import (GpuStep, assert_close, oracle_attention_all, oracle_attention_rows,
+                        oracle_cache, sample_rows)
+from paged_kv_cache_421_b200 import _binding as B
+from paged_kv_cache_421_b200 import ops
+from paged_kv_cache_421_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+FULL_CACHE_CONFIGS = ["tiny_decode", "llama8b_decode", "mixed_step", "prefix_share_decode"]
+ALL_CONFIGS = FULL_CACHE_CONFIGS + ["long70b_decode", "long70b_decode_fp8"]
+
+
+@pytest.fixture(autouse=True)
+def _clean_error_word():
+    B.pa_device_error(reset=True)
+    yield
+    assert B.pa_device_error(reset=True) == 0, "a kernel recorded a device error"
+
+
+_steps = {}
+
+
+def step_of(name):
+    if name not in _steps:
+        _steps.clear()
+        torch.cuda.empty_cache()
+        wl = W.CONFIGS[name]()
+        _steps[name] = GpuStep(wl)
+    return _steps[name]
+
+
+# ------------------------------------------------------------------ slot mapping + write
+@pytest.mark.parametrize("name", ALL_CONFIGS)
+def test_slot_mapping_bit_exact(name):
+    st = step_of(name)
+    wl = st.wl
+    want_h = oracle.slot_mapping(wl.hist_block_table, wl.hist_seq_lens, wl.hist_qsl, 16)
+    want = oracle.slot_mapping(wl.block_table, wl.seq_lens, wl.qsl, 16)
+    assert np.array_equal(st.hist_slots.cpu().numpy(), want_h)
+    assert np.array_equal(st.slots.cpu().numpy(), want)
+
+
+@pytest.mark.parametrize("name", FULL_CACHE_CONFIGS)
+def test_cache_write_bit_exact_full_buffer(name):
+    st = step_of(name)
+    want = oracle_cache(st.wl)
+    got = st.cache_host()
+    assert got.nbytes == want.nbytes
+    assert np.array_equal(got, want.view(np.uint8)), "cache bytes differ from the oracle"
+
+
+@pytest.mark.parametrize("name", ["long70b_decode", "long70b_decode_fp8"])
+def test_cache_write_bit_exact_sampled(name):
+    # full-size pools: check every new token and 4096 sampled history tokens, each written
+    # by the oracle into a scratch pool and compared with the GPU's bytes at its slot
+    st = step_of(name)
+    wl = st.wl
+    rng = np.random.default_rng(1)
+    Th = int(wl.hist_qsl[-1])
+    hs = st.hist_slots.cpu().numpy()
+    ns = st.slots.cpu().numpy()
+    pick_h = rng.choice(Th, 4096, replace=False)
+    rows_k = torch.cat([wl.k_hist[torch.from_numpy(pick_h)], wl.k_new])
+    rows_v = torch.cat([wl.v_hist[torch.from_numpy(pick_h)], wl.v_new])
+    slots = np.concatenate([hs[pick_h], ns])
+    n = slots.size
+    nb = -(-n // 16)
+    scratch_n = oracle.cache_elems(nb, 16, wl.num_kv_heads, wl.head_size)
+    dt = np.uint16 if wl.kv_dtype == W.BF16 else np.uint8
+    scratch = np.zeros(scratch_n, dt)
+    ks = None if wl.k_scale is None else wl.k_scale.numpy()
+    vs = None if wl.v_scale is None else wl.v_scale.numpy()
+    oracle.write_kv(scratch, wl.kv_dtype, nb, 16, wl.num_kv_heads, wl.head_size, W.bits(rows_k),
+                    W.bits(rows_v), np.arange(n, dtype=np.int32), ks, vs)
+    scratch = scratch.reshape(nb, 2, wl.num_kv_heads, 16, wl.head_size)
+    view = st.cache.view()
+    got = view.view(torch.int16) if wl.kv_dtype == W.BF16 else view
+    idx_b = torch.from_numpy(slots // 16).cuda()
+    idx_o = torch.from_numpy(slots % 16).cuda()
+    gathered = got[idx_b, :, :, idx_o, :].cpu().numpy().view(dt)  # [n, 2, Hkv, D]
+    want = scratch.transpose(0, 3, 1, 2, 4).reshape(nb * 16, 2, wl.num_kv_heads, wl.head_size)[:n]
+    assert np.array_equal(gathered, want)
+
+
+def test_fp8_write_divides_at_ties():
+    # x / 7 lands exactly on an E4M3 midpoint; the GPU must divide (not multiply by 1/7)
+    xs = torch.tensor([0.0888671875, 0.1708984375, 0.1982421875, -0.0888671875])
+    want = [0x06, 0x0C, 0x0E, 0x86]
+    n = xs.numel()
+    scale = torch.full((1,), 7.0, device="cuda")
+    cache = ops.PagedKVCache(1, 1, 128, B.PA_FP8_E4M3, k_scale=scale, v_scale=scale)
+    k = torch.zeros(n, 1, 128, dtype=torch.bfloat16, device="cuda")
+    k[:, 0, 0] = xs.to(torch.bfloat16).cuda()
+    slots = torch.arange(n, dtype=torch.int32, device="cuda")
+    ops.write_kv(cache, k, k, slots)
+    got = cache.view()[0, 0, 0, :n, 0].cpu().tolist()
+    assert got == want
+
+
+# ------------------------------------------------------------------ attention
+@pytest.mark.parametrize("name", ["tiny_decode", "llama8b_decode"])
+def test_attention_all_rows(name):
+    st = step_of(name)
+    want, _ = oracle_attention_all(st.wl, oracle_cache(st.wl))
+    stats = assert_close(st.out.cpu().numpy(), want, st.wl.kv_dtype, name)
+    print(name, stats)
+
+
+@pytest.mark.parametrize("name", ["mixed_step", "prefix_share_decode", "long70b_decode",
+                                  "long70b_decode_fp8"])
+def test_attention_sampled_rows(name):
+    st = step_of(name)
+    wl = st.wl
+    n = {"mixed_step": 40, "prefix_share_decode": 40, "long70b_decode": 8,
+         "long70b_decode_fp8": 4}[name]
+    tokens, heads = sample_rows(wl, n)
+    want, _ = oracle_attention_rows(wl, tokens, heads)
+    got = st.out.cpu().numpy()[tokens, heads]
+    stats = assert_close(got, want, wl.kv_dtype, name)
+    print(name, stats, len(tokens), "rows")
+
+
+def test_mixed_step_chunks_all_rows():
+    # every row of both prefill chunks (the chunk kernel's causal diagonal tiles included)
+    st = step_of("mixed_step")
+    wl = st.wl
+    t0 = int(wl.qsl[48])
+    T = wl.num_tokens
+    tok = np.repeat(np.arange(t0, T), 2).astype(np.int32)
+    hed = np.tile(np.array([0, 31], np.int32), T - t0)
+    want, _ = oracle_attention_rows(wl, tok, hed)
+    assert_close(st.out.cpu().numpy()[tok, hed], want, wl.kv_dtype, "chunks")
+
+
+@pytest.mark.parametrize("name", ["tiny_decode", "llama8b_decode", "prefix_share_decode"])
+def test_split_invariance(name):
+    st = step_of(name)
+    base = st.attend(kv_split_tokens=1 << 20).cpu().numpy()  # one split per request
+    want, _ = oracle_attention_all(st.wl, oracle_cache(st.wl)) if name != "prefix_share_decode" \
+        else (None, None)
+    for kv_split in [16, 48, 112, 512]:
+        got = st.attend(kv_split_tokens=kv_split).cpu().numpy()
+        assert np.max(np.abs(got - base)) < 2e-3, kv_split
+        if want is not None:
+            assert_close(got, want, st.wl.kv_dtype, f"split {kv_split}")
+
+
+def test_split_invariance_fp8_long():
+    st = step_of("long70b_decode_fp8")
+    a = st.attend(kv_split_tokens=4096).cpu().numpy()
+    b = st.attend(kv_split_tokens=1 << 17).cpu().numpy()
+    assert np.max(np.abs(a - b)) < 4e-3
+
+
+# ------------------------------------------------------------------ edge cases
+def _small(ctx, ql, hq, hkv, d, seed, kv_dtype=W.BF16, shared=0, nb=None):
+    need = sum(-(-c // 16) for c in ctx)
+    return W.make_workload("edge", ctx, ql, hq, hkv, d, 16, nb or need + 8, seed,
+                           kv_dtype=kv_dtype, shared_prefix_tokens=shared)
+
+
+EDGE_CASES = {
+    "ctx1": ([1], [1], 8, 1, 128),
+    "one_block_exact": ([16, 32], [1, 1], 4, 2, 128),
+    "ragged_tail": ([17, 33, 63, 15], [1, 1, 1, 1], 32, 8, 128),
+    "mha_group1": ([40, 77], [1, 1], 4, 4, 128),
+    "spec_decode_qlen2_g4": ([50, 300], [2, 2], 8, 2, 128),
+    "qlen3_g4_chunk_kind": ([50, 300], [3, 3], 8, 2, 128),
+    "first_chunk_no_history": ([70], [70], 8, 2, 128),
+    "chunk_d64": ([130, 64], [100, 64], 8, 2, 64),
+    "decode_d64_g2": ([1, 17, 33, 64], [1, 1, 1, 1], 4, 2, 64),
+    "zero_query_mixed": ([10, 20, 5, 40], [0, 2, 0, 1], 8, 2, 128),
+    "long_chunk_tail": ([1000], [333], 16, 2, 128),
+    "many_requests": ([int(x) for x in np.random.default_rng(3).integers(1, 200, 300)],
+                      [1] * 300, 8, 2, 128),
+    "g16_chunk": ([90, 40], [1, 1], 32, 2, 128),
+}
+
+
+@pytest.mark.parametrize("case", sorted(EDGE_CASES))
+def test_edge_case(case):
+    ctx, ql, hq, hkv, d = EDGE_CASES[case]
+    wl = _small(ctx, ql, hq, hkv, d, seed=hash(case) % 1000)
+    st = GpuStep(wl)
+    assert np.array_equal(st.cache_host(), oracle_cache(wl).view(np.uint8))
+    want, _ = oracle_attention_all(wl, oracle_cache(wl))
+    assert_close(st.out.cpu().numpy(), want, wl.kv_dtype, case)
+    for split in [16, 64]:
+        assert_close(st.attend(kv_split_tokens=split).cpu().numpy(), want, wl.kv_dtype,
+                     f"{case} split {split}")
+
+
+@pytest.mark.parametrize("kv_dtype", [W.BF16, W.FP8_E4M3])
+def test_nan_garbage_in_unwritten_slots(kv_dtype):
+    # stale NaN patterns in the unused tail of partly filled blocks must not reach the output
+    wl = _small([17, 33, 5, 100], [1, 1, 1, 1], 16, 2, 128, seed=9, kv_dtype=kv_dtype)
+    st = GpuStep(wl, fill=False, garbage_tail=True)
+    tokens = np.repeat(np.arange(wl.num_tokens), wl.num_q_heads)
+    heads = np.tile(np.arange(wl.num_q_heads), wl.num_tokens)
+    want, _ = oracle_attention_rows(wl, tokens, heads)
+    assert_close(st.out.cpu().numpy().reshape(-1, 128), want, kv_dtype, "garbage tail")
+
+
+@pytest.mark.parametrize("seed", range(10))
+def test_random_small_steps(seed):
+    rng = np.random.default_rng(1000 + seed)
+    B_ = int(rng.integers(1, 12))
+    hkv = int(rng.choice([1, 2, 4]))
+    G = int(rng.choice([1, 2, 4, 8]))
+    d = int(rng.choice([64, 128]))
+    ctx = rng.integers(1, 700, size=B_)
+    ql = np.array([int(rng.choice([0, 1, 1, 1, 2, int(rng.integers(1, c + 1))])) for c in ctx])
+    ql = np.minimum(ql, ctx)
+    if ql.sum() == 0:
+        ql[0] = 1
+    wl = _small(ctx, ql, hkv * G, hkv, d, seed=seed)
+    st = GpuStep(wl)
+    assert np.array_equal(st.cache_host(), oracle_cache(wl).view(np.uint8))
+    want, _ = oracle_attention_all(wl, oracle_cache(wl))
+    assert_close(st.out.cpu().numpy(), want, wl.kv_dtype, f"seed {seed}")
+
+
+def test_random_small_steps_fp8():
+    for seed in range(4):
+        rng = np.random.default_rng(2000 + seed)
+        ctx = rng.integers(1, 900, size=5)
+        wl = _small(ctx, [1] * 5, 16, 2, 128, seed=seed, kv_dtype=W.FP8_E4M3)
+        st = GpuStep(wl)
+        assert np.array_equal(st.cache_host(), oracle_cache(wl))
+        want, _ = oracle_attention_all(wl, oracle_cache(wl))
+        assert_close(st.out.cpu().numpy(), want, W.FP8_E4M3, f"fp8 seed {seed}")
+        for split in [16, 128]:
+            assert_close(st.attend(kv_split_tokens=split).cpu().numpy(), want, W.FP8_E4M3,
+                         f"fp8 seed {seed} split {split}")
+
+
+def test_empty_step_is_a_no_op():
+    wl = _small([5], [1], 4, 2, 128, seed=1)
+    st = GpuStep(wl)
+    out = torch.full((0, 4, 128), 1.0, device="cuda")
+    B.pa_attention(st.cache.handle, st.wl.q.cuda(), 4, st.step["bt"], st.step["bt"].shape[1],
+                   st.step["sl"], st.step["qsl"], np.array([5], np.int32),
+                   np.array([0, 0], np.int32), 1, 0, 0.1, out)
+    B.pa_write_kv(st.cache.handle, st.wl.k_new.cuda(), st.wl.v_new.cuda(), st.slots, 0)
+
+
+def test_prefix_alias_write_visible_to_all_tables():
+    wl = _small([40, 35, 50], [1, 1, 1], 4, 2, 64, seed=5, shared=32)
+    st = GpuStep(wl)
+    want, _ = oracle_attention_all(wl, oracle_cache(wl))
+    assert_close(st.out.cpu().numpy(), want, W.BF16, "aliased")
+    # overwrite token 3 of the first shared block through request 0's table
+    slot = int(wl.block_table[0, 0]) * 16 + 3
+    k = torch.full((1, 2, 64), 2.5, dtype=torch.bfloat16, device="cuda")
+    ops.write_kv(st.cache, k, k, torch.tensor([slot], dtype=torch.int32, device="cuda"))
+    view = st.cache.view()
+    for r in range(3):
+        assert torch.all(view[int(wl.block_table[r, 0]), :, :, 3, :] == 2.5)
+
+
+# ------------------------------------------------------------------ error paths (no faults)
+def test_bad_block_id_is_reported_not_faulted():
+    wl = _small([40], [1], 4, 2, 128, seed=2)
+    st = GpuStep(wl)
+    bt = st.step["bt"].clone()
+    bt[0, 1] = wl.num_blocks + 1000  # outside the pool: the kernel clamps and records code 3
+    ops.attention(st.cache, wl.q.cuda(), bt, st.step["sl"], st.step["qsl"], wl.seq_lens, wl.qsl,
+                  wl.scale)
+    assert B.pa_device_error(reset=True) == 3
+    assert B.pa_validate_block_table(st.cache.handle, bt, bt.shape[1], st.step["sl"], 1) == 1
+    assert B.pa_validate_block_table(st.cache.handle, st.step["bt"], bt.shape[1],
+                                     st.step["sl"], 1) == 0
+
+
+def test_slot_beyond_table_is_reported():
+    bt = torch.zeros(1, 2, dtype=torch.int32, device="cuda")
+    sl = torch.tensor([40], dtype=torch.int32, device="cuda")
+    qsl = torch.tensor([0, 1], dtype=torch.int32, device="cuda")
+    slots = ops.slot_mapping(bt, sl, qsl, 1)
+    assert slots.item() == -1
+    assert B.pa_device_error(reset=True) == 2
+
+
+def test_host_metadata_errors():
+    wl = _small([40], [1], 4, 2, 128, seed=2)
+    st = GpuStep(wl, run_attention=False)
+    q = wl.q.cuda()
+    out = torch.empty(1, 4, 128, device="cuda")
+    with pytest.raises(B.PaError) as e:  # q_len > seq_len
+        B.pa_attention(st.cache.handle, q, 4, st.step["bt"], st.step["bt"].shape[1],
+                       st.step["sl"], st.step["qsl"], np.array([0], np.int32),
+                       np.array([0, 1], np.int32), 1, 1, 0.1, out)
+    assert e.value.status == B.PA_ERR_METADATA
+    with pytest.raises(B.PaError) as e:  # forced split without workspace
+        B.pa_attention_ex(st.cache.handle, q, 4, st.step["bt"], st.step["bt"].shape[1],
+                          st.step["sl"], st.step["qsl"], wl.seq_lens, wl.qsl, 1, 1, 0.1, out,
+                          kv_split_tokens=16)
+    assert e.value.status == B.PA_ERR_WORKSPACE
