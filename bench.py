@@ -1,0 +1,509 @@
+"""Benchmark of one serving step of the paged KV cache hot path on B200.
+
+A step is the whole hot path over one batch: slot mapping of the step's new tokens, the
+cache write of their K/V, and paged attention of their queries over the cache (decode and
+chunk kernels plus the split-KV reduce).  The request metadata, the step's Q/K/V and the
+earlier tokens' K/V (already written into the pool) are resident in HBM before the timed
+region.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Prints one JSON line (rank 0).  `value` is KV-read GB/s of the whole step (algorithmic KV
+bytes the step's attention reads / step time, summed over ranks); `tokens_per_s` is query
+tokens per second.  Under torchrun every rank runs its own copy of the batch (weak scaling,
+no collective on the data path); times are the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+DEFAULT_WORKLOAD = "llama8b_decode"
+METRIC = "paged-attn KV-read GB/s (% of HBM peak) and query tokens/s per batch step"
+FALLBACK_HBM_GBS = 6650.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ---------------------------------------------------------------- helpers (no GPU needed)
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing")
+    ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    ap.add_argument("--no-flush", action="store_true", help="do not flush L2 between steps")
+    return ap.parse_args(argv)
+
+
+def kv_bytes(wl) -> int:
+    """Algorithmic KV bytes the step's attention reads: every request's full context of K
+    and V once per kv head (the GQA group shares one read)."""
+    return int(np.sum(wl.seq_lens.astype(np.int64))) * 2 * wl.num_kv_heads * wl.head_size * \
+        wl.dtype_bytes
+
+
+def decode_kv_bytes(wl) -> int:
+    G = wl.num_q_heads // wl.num_kv_heads
+    ql = wl.q_lens
+    dec = (ql > 0) & (ql * G <= 8)
+    return int(np.sum(wl.seq_lens[dec].astype(np.int64))) * 2 * wl.num_kv_heads * \
+        wl.head_size * wl.dtype_bytes
+
+
+def unique_kv_bytes(wl) -> int:
+    used = set()
+    for r in range(wl.num_seqs):
+        used.update(wl.block_table[r, :-(-int(wl.seq_lens[r]) // 16)].tolist())
+    return len(used) * 2 * 16 * wl.num_kv_heads * wl.head_size * wl.dtype_bytes
+
+
+def load_peaks() -> tuple:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_digest(*names) -> str:
+    h = hashlib.sha256()
+    for n in names:
+        with open(os.path.join(ROOT, "paged_kv_cache_421_b200", "csrc", n), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` on `workload` from the committed ncu summary, if it
+    was taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    digest = source_digest("pa_decode.cu", "pa_common.cuh")
+    for line in open(path):
+        parts = line.split()
+        if len(parts) == 4 and parts[0] == kernel and parts[1] == workload and parts[2] == digest:
+            return float(parts[3])
+    return None
+
+
+def median_clock(samples):
+    loaded = [s for s in samples if s["util"] is None or s["util"] > 0] or samples
+    mhz = [s["sm"] for s in loaded]
+    return statistics.median(mhz) if mhz else None
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap,"
+              "utilization.gpu")
+
+    def __init__(self, index: int, path: str):
+        self.path, self.index, self.proc = path, index, None
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        samples, reasons = [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            p = [x.strip() for x in line.split(",")]
+            if len(p) < 10:
+                continue
+            try:
+                sm, smax = float(p[1]), float(p[2])
+            except ValueError:
+                continue
+            util = float(p[9]) if p[9].replace(".", "").isdigit() else None
+            samples.append({"sm": sm, "max": smax, "util": util})
+            for n, v in zip(names, p[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        if not samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": median_clock(samples), "sm_max_mhz": max(s["max"] for s in samples),
+                "reasons": sorted(reasons), "samples": len(samples)}
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Max of a per-rank scalar over all ranks (identity on one rank)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sub_workload_rows(wl, n_req: int):
+    """Metadata of the first n_req requests of a step (for bounded CPU samples)."""
+    qsl = wl.qsl[:n_req + 1].copy()
+    return wl.block_table[:n_req], wl.seq_lens[:n_req], qsl
+
+
+def oracle_requests_for_budget(wl, kv_token_heads_budget: int) -> int:
+    """How many leading requests fit a budget of (context tokens x q heads)."""
+    acc, n = 0, 0
+    for r in range(wl.num_seqs):
+        acc += int(wl.seq_lens[r]) * max(int(wl.q_lens[r]), 1) * wl.num_q_heads
+        n += 1
+        if acc >= kv_token_heads_budget:
+            break
+    return max(n, 1)
+
+
+# ---------------------------------------------------------------- CPU oracle timing
+def oracle_step_timer(wl):
+    """Build the oracle's cache (untimed) and return a function that times the oracle over
+    the first n requests of the step: slot mapping, cache write of their new tokens and
+    attention of their queries.  Returns (seconds, kv_bytes_of_those_requests)."""
+    import oracle
+    from paged_kv_cache_421_b200 import workloads as W
+    oracle.build()
+    n_el = oracle.cache_elems(wl.num_blocks, 16, wl.num_kv_heads, wl.head_size)
+    dt = np.uint16 if wl.kv_dtype == W.BF16 else np.uint8
+    cache = np.full(n_el, W.CACHE_FILL_BF16 if dt == np.uint16 else W.CACHE_FILL_FP8, dt)
+    ks = None if wl.k_scale is None else wl.k_scale.cpu().numpy()
+    vs = None if wl.v_scale is None else wl.v_scale.cpu().numpy()
+    hslots = oracle.slot_mapping(wl.hist_block_table, wl.hist_seq_lens, wl.hist_qsl, 16)
+    oracle.write_kv(cache, wl.kv_dtype, wl.num_blocks, 16, wl.num_kv_heads, wl.head_size,
+                    W.bits(wl.k_hist), W.bits(wl.v_hist), hslots, ks, vs)
+    q_bits, k_bits, v_bits = W.bits(wl.q), W.bits(wl.k_new), W.bits(wl.v_new)
+    per_tok = 2 * wl.num_kv_heads * wl.head_size * wl.dtype_bytes
+
+    def run(n_req: int):
+        bt, sl, qsl = sub_workload_rows(wl, n_req)
+        T = int(qsl[-1])
+        t0 = time.perf_counter()
+        slots = oracle.slot_mapping(bt, sl, qsl, 16)
+        oracle.write_kv(cache, wl.kv_dtype, wl.num_blocks, 16, wl.num_kv_heads, wl.head_size,
+                        k_bits[:T], v_bits[:T], slots, ks, vs)
+        oracle.attention_paged(cache, wl.kv_dtype, wl.num_blocks, 16, wl.num_kv_heads,
+                               wl.head_size, q_bits[:T], wl.num_q_heads, bt, sl, qsl, wl.scale,
+                               ks, vs)
+        return time.perf_counter() - t0, int(np.sum(sl.astype(np.int64))) * per_tok
+    return run
+
+
+def cpu_baseline(wl, budget_s: float) -> dict:
+    run = oracle_step_timer(wl)
+    # grow the sample until it takes about budget_s of CPU time
+    n = 1
+    sec, nbytes = run(n)
+    while sec < budget_s and n < wl.num_seqs:
+        est = max(1, int(n * min(8.0, budget_s / max(sec, 1e-3))))
+        n = min(wl.num_seqs, max(n + 1, est))
+        sec, nbytes = run(n)
+    return {"value": round(nbytes / sec / 1e9, 6), "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"first {n} of {wl.num_seqs} requests of the step (slot mapping, cache "
+                      f"write and fp64 attention, {sec:.1f} s, single-threaded C oracle)"}
+
+
+# ---------------------------------------------------------------- device step
+class DeviceStep:
+    def __init__(self, wl, device):
+        import torch
+        from paged_kv_cache_421_b200 import ops
+        from paged_kv_cache_421_b200 import workloads as W
+        self.wl, self.dev, self.ops, self.torch = wl, device, ops, torch
+        self.cache = ops.PagedKVCache(wl.num_blocks, wl.num_kv_heads, wl.head_size, wl.kv_dtype,
+                                      k_scale=wl.k_scale, v_scale=wl.v_scale, device=device)
+        if wl.kv_dtype == W.BF16:
+            self.cache.buffer.view(torch.int16).fill_(W.CACHE_FILL_BF16)
+        else:
+            self.cache.buffer.fill_(W.CACHE_FILL_FP8)
+
+        def i32(a):
+            return torch.from_numpy(np.ascontiguousarray(a, np.int32)).to(device)
+        hb, hs, hq = i32(wl.hist_block_table), i32(wl.hist_seq_lens), i32(wl.hist_qsl)
+        Th = int(wl.hist_qsl[-1])
+        if Th:
+            hslots = ops.slot_mapping(hb, hs, hq, Th)
+            ops.write_kv(self.cache, wl.k_hist.to(device).contiguous(),
+                         wl.v_hist.to(device).contiguous(), hslots)
+        self.bt, self.sl, self.qsl = i32(wl.block_table), i32(wl.seq_lens), i32(wl.qsl)
+        self.q = wl.q.to(device).contiguous()
+        self.k = wl.k_new.to(device).contiguous()
+        self.v = wl.v_new.to(device).contiguous()
+        T = wl.num_tokens
+        self.slots = torch.empty(T, dtype=torch.int32, device=device)
+        self.out = torch.empty(T, wl.num_q_heads, wl.head_size, dtype=torch.float32,
+                               device=device)
+        nb = ops.workspace_bytes_for(self.cache, wl.seq_lens, wl.qsl, wl.num_q_heads,
+                                     wl.max_blocks_per_seq)
+        self.workspace = torch.empty(max(nb, 256), dtype=torch.uint8, device=device)
+        self.plan = ops.B.pa_plan_attention(
+            wl.seq_lens, wl.qsl, wl.num_q_heads, wl.num_kv_heads, wl.head_size,
+            wl.max_blocks_per_seq,
+            torch.cuda.get_device_properties(device).multi_processor_count,
+            self.workspace.numel())
+        torch.cuda.synchronize(device)
+
+    def launches_per_step(self) -> int:
+        p = self.plan
+        return 2 + (p["num_decode_seqs"] > 0) + (p["num_chunk_seqs"] > 0) + int(p["any_split"])
+
+    def run(self, events=None, q=None, k=None, v=None, bt=None, sl=None, qsl=None):
+        B = self.ops.B
+        wl = self.wl
+        bt = self.bt if bt is None else bt
+        sl = self.sl if sl is None else sl
+        qsl = self.qsl if qsl is None else qsl
+        T = wl.num_tokens
+        B.pa_slot_mapping(bt, bt.shape[1], sl, qsl, wl.num_seqs, T, 16, self.slots)
+        B.pa_write_kv(self.cache.handle, self.k if k is None else k, self.v if v is None else v,
+                      self.slots, T)
+        B.pa_attention_ex(self.cache.handle, self.q if q is None else q, wl.num_q_heads, bt,
+                          bt.shape[1], sl, qsl, wl.seq_lens, wl.qsl, wl.num_seqs, T, wl.scale,
+                          self.out, self.workspace, self.workspace.numel(), events=events)
+
+
+def run_device_bench(args, rank, world, local):
+    import torch
+    import torch.distributed as dist
+    from paged_kv_cache_421_b200 import workloads as W
+
+    device = torch.device(f"cuda:{local}")
+    torch.cuda.set_device(device)
+    wl = W.CONFIGS[args.workload](device=device)
+    step = DeviceStep(wl, device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    nbytes = kv_bytes(wl)
+    dec_bytes = decode_kv_bytes(wl)
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    # warm-up (untimed)
+    for _ in range(max(args.warmup, 0)):
+        step.run()
+    torch.cuda.synchronize(device)
+
+    # ---- device-resident timed region
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(args.steps)]
+    st_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(args.steps)]
+    for e in ev:  # torch creates events lazily: record once so the library gets real handles
+        for x in e:
+            x.record()
+    clocks = ClockSampler(local, os.path.join(ROOT, "gpurun_out", f".clocks_{rank}.csv")
+                          if os.path.isdir(os.path.join(ROOT, "gpurun_out"))
+                          else f"/tmp/clocks_{os.getpid()}.csv")
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize(device)
+    stream = torch.cuda.current_stream(device)
+    for i in range(args.steps):
+        if not args.no_flush:
+            flush.zero_()
+        st_ev[i][0].record(stream)
+        step.run(events=ev[i])
+        st_ev[i][1].record(stream)
+    torch.cuda.synchronize(device)
+    barrier()
+    clk = clocks.stop()
+    step_ms = [a.elapsed_time(b) for a, b in st_ev]
+    total_ms = max_over_ranks(sum(step_ms), world, device)
+    ms_per_step = total_ms / args.steps
+    dec_ms = None
+    if step.plan["num_decode_seqs"]:
+        dec_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+        dec_ms = max_over_ranks(dec_ms, world, device)
+    chunk_ms = None
+    if step.plan["num_chunk_seqs"]:
+        chunk_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
+    reduce_ms = None
+    if step.plan["any_split"]:
+        reduce_ms = statistics.mean(e[4].elapsed_time(e[5]) for e in ev)
+
+    # ---- end-to-end: host inputs (pinned) -> device -> step -> output back to the host
+    e2e = None
+    if not args.no_e2e:
+        hq = wl.q.cpu().pin_memory()
+        hk = wl.k_new.cpu().pin_memory()
+        hv = wl.v_new.cpu().pin_memory()
+        hbt = torch.from_numpy(np.ascontiguousarray(wl.block_table, np.int32)).pin_memory()
+        hsl = torch.from_numpy(np.ascontiguousarray(wl.seq_lens, np.int32)).pin_memory()
+        hqsl = torch.from_numpy(np.ascontiguousarray(wl.qsl, np.int32)).pin_memory()
+        hout = torch.empty(step.out.shape, dtype=torch.float32).pin_memory()
+        dq, dk, dv = torch.empty_like(step.q), torch.empty_like(step.k), torch.empty_like(step.v)
+        dbt, dsl, dqsl = (torch.empty_like(step.bt), torch.empty_like(step.sl),
+                          torch.empty_like(step.qsl))
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hbt, hsl, hqsl))
+        d2h = hout.numel() * hout.element_size()
+
+        def e2e_step():
+            for d, h in ((dq, hq), (dk, hk), (dv, hv), (dbt, hbt), (dsl, hsl), (dqsl, hqsl)):
+                d.copy_(h, non_blocking=True)
+            step.run(q=dq, k=dk, v=dv, bt=dbt, sl=dsl, qsl=dqsl)
+            hout.copy_(step.out, non_blocking=True)
+
+        for _ in range(max(args.warmup, 0)):
+            e2e_step()
+        torch.cuda.synchronize(device)
+        barrier()
+        e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(args.steps)]
+        for i in range(args.steps):
+            if not args.no_flush:
+                flush.zero_()
+            e_ev[i][0].record(stream)
+            e2e_step()
+            e_ev[i][1].record(stream)
+        torch.cuda.synchronize(device)
+        barrier()
+        e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e_ev), world, device) / args.steps
+        e2e = {"value": round(world * nbytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+               "ms_per_step": round(e2e_ms, 4)}
+
+    result = None
+    if rank == 0:
+        peak, peak_kind = load_peaks()
+        value = world * nbytes / (ms_per_step * 1e-3) / 1e9
+        roof = None
+        if dec_ms:
+            achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
+            roof = {"bound": "hbm", "kernel": "decode_kernel", "achieved": round(achieved, 1),
+                    "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                    "traffic": recorded_traffic("decode_kernel", args.workload),
+                    "peak_kind": peak_kind, "bytes_per_launch": dec_bytes,
+                    "ms_per_launch": round(dec_ms, 4)}
+        elif chunk_ms:
+            roof = {"bound": "tensor", "kernel": "chunk_kernel", "achieved": None, "peak": None,
+                    "unit": "TFLOP/s", "frac": None, "traffic": None}
+        result = {
+            "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if wl.kv_dtype == W.BF16 else "fp8_e4m3-kv/f16-mma",
+            "data": "synthetic (seeded; random-init Q/K/V ~ N(0,1) in bf16)",
+            "config": {"workload": args.workload, "num_seqs": wl.num_seqs,
+                       "tokens_per_step": wl.num_tokens, "num_q_heads": wl.num_q_heads,
+                       "num_kv_heads": wl.num_kv_heads, "head_size": wl.head_size,
+                       "block_size": 16, "num_blocks": wl.num_blocks,
+                       "kv_bytes_per_step": nbytes, "unique_kv_bytes_per_step": unique_kv_bytes(wl),
+                       "l2": "no flush" if args.no_flush else
+                             "flushed between steps (256 MiB write outside the step events)",
+                       "parallelism": f"replicas x{world} (one batch per GPU)"},
+            "tokens_per_s": round(world * wl.num_tokens / (ms_per_step * 1e-3), 1),
+            "pct_hbm_peak": round(100 * value / world / peak, 2),
+            "roofline": roof,
+            "kernel_ms": {"decode": dec_ms, "chunk": chunk_ms, "reduce": reduce_ms},
+            "e2e": e2e,
+            "gpu_launches": step.launches_per_step() * args.steps,
+            "clocks": clk,
+        }
+    return result, wl
+
+
+def reference_arm(args, rank, world):
+    """The oracle, as it stands, on the host cores: each step a bounded sample (the leading
+    requests of the same workload), slot mapping + cache write + fp64 attention."""
+    if rank != 0:
+        return None
+    from paged_kv_cache_421_b200 import workloads as W
+    wl = W.CONFIGS[args.workload]()
+    run = oracle_step_timer(wl)
+    n = oracle_requests_for_budget(wl, 60_000_000)
+    for _ in range(max(args.warmup, 0)):
+        run(n)
+    secs, nb = [], 0
+    for _ in range(args.steps):
+        s, nb = run(n)
+        secs.append(s)
+    sec = sum(secs) / len(secs)
+    value = nb / sec / 1e9
+    sample = (f"first {n} of {wl.num_seqs} requests per step (slot mapping, cache write, fp64 "
+              f"attention; single-threaded C oracle)")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(sec * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "config": {"workload": args.workload, "num_seqs": wl.num_seqs,
+                   "tokens_per_step": wl.num_tokens, "num_q_heads": wl.num_q_heads,
+                   "num_kv_heads": wl.num_kv_heads, "head_size": wl.head_size, "block_size": 16},
+        "cpu_baseline": {"value": round(value, 6), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        res = reference_arm(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return 0
+    import torch
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device(f"cuda:{local}"))
+    result, wl = run_device_bench(args, rank, world, local)
+    if rank == 0:
+        if not args.no_cpu_baseline:
+            result["cpu_baseline"] = cpu_baseline(wl, args.cpu_budget_s)
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

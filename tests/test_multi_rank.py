@@ -1,0 +1,84 @@
+"""Multi-rank host logic of the benchmark on CPU (gloo, world size 2).
+
+The serving step shards by request batch: every rank runs its own batch with no collective
+on the data path, and only the timing is combined (max over ranks).  These tests run the
+same host code the GPU ranks run, with gloo on CPU."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from conftest import ROOT
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    sys.path.insert(0, ROOT)
+    import bench
+    got = bench.max_over_ranks(1.5 + rank, world, device="cpu")
+    # every rank reports the same max, regardless of its own value
+    q.put((rank, got))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_max_over_ranks_gloo():
+    world = 2
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    res = dict(q.get(timeout=10) for _ in range(world))
+    assert res == {0: 2.5, 1: 2.5}
+
+
+def test_reference_arm_runs_on_rank0_only():
+    # under torchrun the oracle arm runs and prints on rank 0; the other ranks exit quietly
+    port = _free_port()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), "bench.py", "--impl",
+           "reference", "--gpus", "2", "--steps", "1", "--warmup", "0", "--workload",
+           "tiny_decode"]
+    res = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert res.returncode == 0, res.stderr[-2000:]
+    lines = [ln for ln in res.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    rec = json.loads(lines[0])
+    assert rec["impl"] == "reference" and rec["n_gpus"] == 2
+    assert rec["cpu_baseline"]["kind"] == "oracle" and rec["value"] > 0
+    assert rec["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_bench_byte_accounting():
+    sys.path.insert(0, ROOT)
+    import bench
+    from paged_kv_cache_421_b200 import workloads as W
+    wl = W.tiny_decode()
+    assert bench.kv_bytes(wl) == 58880
+    assert bench.decode_kv_bytes(wl) == 58880
+    assert bench.unique_kv_bytes(wl) == 10 * 8192
+    wl = W.mixed_step()
+    assert bench.decode_kv_bytes(wl) == bench.kv_bytes(wl) - (512 + 2560) * 2 * 8 * 128 * 2
+    wl = W.prefix_share_decode()
+    assert bench.unique_kv_bytes(wl) < bench.kv_bytes(wl)
+    args = bench.parse_args([])
+    assert args.gpus == 1 and args.steps > 0 and args.warmup >= 3
