@@ -137,6 +137,33 @@ int pa_attention(const pa_cache* cache, const void* q, int num_q_heads,
                  float scale, float* out, void* workspace, size_t workspace_bytes,
                  void* stream);
 
+/* Size of the fixed scratch used by pa_attention_noalloc: 64 MiB of static device memory,
+ * held by every GPU on which the library's kernels are loaded until the process exits. */
+#define PA_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+/* pa_attention without a workspace argument, for callers that cannot allocate device memory.
+ * The pages describe no such call; it exists for integrators: a host framework that owns all
+ * device memory and gives plugins no allocator, a serving process with a fixed memory budget
+ * that forbids allocation after start-up, or code that may not call cudaMalloc where it runs.
+ * Such callers cannot hand pa_attention a workspace, yet long contexts need split-KV partials.
+ * This call keeps them in a file-scope static device array of PA_NOALLOC_SCRATCH_BYTES and
+ * otherwise behaves exactly like pa_attention (same arguments, results and errors).
+ * It allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ * Set-up: the first call on a device (with that device current) resolves the scratch's
+ *   device address with cudaGetSymbolAddress; make that first call before any stream capture.
+ * Limit: calls whose 2 * num_tokens * num_q_heads * (head_size + 1) * 4 bytes of partials (plus
+ *   alignment) exceed PA_NOALLOC_SCRATCH_BYTES return PA_ERR_WORKSPACE and launch nothing; other
+ *   calls get a split-KV partition fitted to the scratch.
+ * Sharing: all calls on a device share the one scratch, which keeps the last call's contents;
+ *   nothing in it has to start at zero (each call writes every partial it reads).  Calls that
+ *   overlap on the GPU (other streams, or other host threads) race on the scratch: serialise
+ *   them, e.g. on one stream. */
+int pa_attention_noalloc(const pa_cache* cache, const void* q, int num_q_heads,
+                         const int32_t* block_table, int max_blocks_per_seq,
+                         const int32_t* seq_lens, const int32_t* query_start_loc,
+                         const int32_t* seq_lens_host, const int32_t* query_start_loc_host,
+                         int num_seqs, int num_tokens, float scale, float* out, void* stream);
+
 /* Launch plan chosen for one pa_attention call (pure host computation, exposed for tests
  * and tools).  Decode-kind requests (q_len * group <= 8) run on the GQA decode kernel,
  * the others on the chunk kernel.  KV is partitioned in units of split_blocks blocks. */

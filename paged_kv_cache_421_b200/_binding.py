@@ -32,8 +32,9 @@ EXPORTED = [
     "pa_cache_bytes", "pa_alloc_cache", "pa_free_cache", "pa_cache_data", "pa_slot_mapping",
     "pa_write_kv", "pa_attention_workspace_bytes", "pa_attention", "pa_plan_attention",
     "pa_attention_ex", "pa_validate_block_table", "pa_device_error", "pa_status_string",
-    "pa_last_cuda_error",
+    "pa_last_cuda_error", "pa_attention_noalloc",
 ]
+PA_NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 class pa_plan(ctypes.Structure):
@@ -103,6 +104,7 @@ def load() -> ctypes.CDLL:
         "pa_device_error": (I, [ctypes.POINTER(I), I]),
         "pa_status_string": (ctypes.c_char_p, [I]),
         "pa_last_cuda_error": (I, []),
+        "pa_attention_noalloc": (I, [P, P, I, P, I, P, P, P, P, I, I, F, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -227,6 +229,20 @@ def pa_attention_ex(handle, q, num_q_heads, block_table, max_blocks_per_seq, seq
                                   sl.ctypes.data, qs.ctypes.data, num_seqs, num_tokens,
                                   float(scale), _ptr(out), _ptr(workspace), workspace_bytes,
                                   ctypes.byref(opts), _stream(stream)), "pa_attention_ex")
+
+
+def pa_attention_noalloc(handle, q, num_q_heads, block_table, max_blocks_per_seq, seq_lens,
+                         query_start_loc, seq_lens_host, query_start_loc_host, num_seqs,
+                         num_tokens, scale, out, stream=None) -> None:
+    """pa_attention for callers that cannot allocate device memory: the split-KV partials go
+    to the library's fixed static scratch (PA_NOALLOC_SCRATCH_BYTES) instead of a workspace."""
+    sl = _host_i32(seq_lens_host)
+    qs = _host_i32(query_start_loc_host)
+    _check(load().pa_attention_noalloc(handle, _ptr(q), num_q_heads, _ptr(block_table),
+                                       max_blocks_per_seq, _ptr(seq_lens), _ptr(query_start_loc),
+                                       sl.ctypes.data, qs.ctypes.data, num_seqs, num_tokens,
+                                       float(scale), _ptr(out), _stream(stream)),
+           "pa_attention_noalloc")
 
 
 def pa_validate_block_table(handle, block_table, max_blocks_per_seq, seq_lens, num_seqs,
