@@ -34,6 +34,7 @@ DEFAULT_WORKLOAD = "llama8b_decode"
 METRIC = "paged-attn KV-read GB/s (% of HBM peak) and query tokens/s per batch step"
 FALLBACK_HBM_GBS = 6650.0
 L2_FLUSH_BYTES = 256 << 20
+L2_BYTES = 126 << 20
 
 
 # ---------------------------------------------------------------- helpers (no GPU needed)
@@ -47,7 +48,11 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing")
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
-    ap.add_argument("--no-flush", action="store_true", help="do not flush L2 between steps")
+    ap.add_argument("--flush", choices=["auto", "always", "never"], default="auto",
+                    help="L2 flush between timed steps (auto: only when the step's KV bytes "
+                         "are under 4x the 126 MB L2)")
+    ap.add_argument("--kv-split-tokens", type=int, default=0,
+                    help="force the KV partition (keys per split); 0 = planner's choice")
     return ap.parse_args(argv)
 
 
@@ -246,8 +251,9 @@ def cpu_baseline(wl, budget_s: float) -> dict:
 
 # ---------------------------------------------------------------- device step
 class DeviceStep:
-    def __init__(self, wl, device):
+    def __init__(self, wl, device, kv_split_tokens: int = 0):
         import torch
+        self.kv_split_tokens = kv_split_tokens
         from paged_kv_cache_421_b200 import ops
         from paged_kv_cache_421_b200 import workloads as W
         self.wl, self.dev, self.ops, self.torch = wl, device, ops, torch
@@ -275,18 +281,20 @@ class DeviceStep:
         self.out = torch.empty(T, wl.num_q_heads, wl.head_size, dtype=torch.float32,
                                device=device)
         nb = ops.workspace_bytes_for(self.cache, wl.seq_lens, wl.qsl, wl.num_q_heads,
-                                     wl.max_blocks_per_seq)
+                                     wl.max_blocks_per_seq, kv_split_tokens)
         self.workspace = torch.empty(max(nb, 256), dtype=torch.uint8, device=device)
         self.plan = ops.B.pa_plan_attention(
             wl.seq_lens, wl.qsl, wl.num_q_heads, wl.num_kv_heads, wl.head_size,
             wl.max_blocks_per_seq,
             torch.cuda.get_device_properties(device).multi_processor_count,
-            self.workspace.numel())
+            self.workspace.numel(), kv_split_tokens=kv_split_tokens)
         torch.cuda.synchronize(device)
 
     def launches_per_step(self) -> int:
+        """Kernels of ours per step: slot mapping, write, decode and/or chunk, chunk reduce."""
         p = self.plan
-        return 2 + (p["num_decode_seqs"] > 0) + (p["num_chunk_seqs"] > 0) + int(p["any_split"])
+        return 2 + (p["num_decode_seqs"] > 0) + (p["num_chunk_seqs"] > 0) + \
+            int(p["chunk_max_splits"] > 1)
 
     def run(self, events=None, q=None, k=None, v=None, bt=None, sl=None, qsl=None):
         B = self.ops.B
@@ -300,7 +308,8 @@ class DeviceStep:
                       self.slots, T)
         B.pa_attention_ex(self.cache.handle, self.q if q is None else q, wl.num_q_heads, bt,
                           bt.shape[1], sl, qsl, wl.seq_lens, wl.qsl, wl.num_seqs, T, wl.scale,
-                          self.out, self.workspace, self.workspace.numel(), events=events)
+                          self.out, self.workspace, self.workspace.numel(),
+                          kv_split_tokens=self.kv_split_tokens, events=events)
 
 
 def run_device_bench(args, rank, world, local):
@@ -311,10 +320,11 @@ def run_device_bench(args, rank, world, local):
     device = torch.device(f"cuda:{local}")
     torch.cuda.set_device(device)
     wl = W.CONFIGS[args.workload](device=device)
-    step = DeviceStep(wl, device)
+    step = DeviceStep(wl, device, args.kv_split_tokens)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     nbytes = kv_bytes(wl)
     dec_bytes = decode_kv_bytes(wl)
+    flush_l2 = args.flush == "always" or (args.flush == "auto" and nbytes < 4 * L2_BYTES)
 
     def barrier():
         if world > 1:
@@ -341,7 +351,7 @@ def run_device_bench(args, rank, world, local):
     torch.cuda.synchronize(device)
     stream = torch.cuda.current_stream(device)
     for i in range(args.steps):
-        if not args.no_flush:
+        if flush_l2:
             flush.zero_()
         st_ev[i][0].record(stream)
         step.run(events=ev[i])
@@ -359,8 +369,8 @@ def run_device_bench(args, rank, world, local):
     chunk_ms = None
     if step.plan["num_chunk_seqs"]:
         chunk_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
-    reduce_ms = None
-    if step.plan["any_split"]:
+    reduce_ms = None  # decode-kind splits merge inside the decode kernel; only chunk splits reduce
+    if step.plan["chunk_max_splits"] > 1:
         reduce_ms = statistics.mean(e[4].elapsed_time(e[5]) for e in ev)
 
     # ---- end-to-end: host inputs (pinned) -> device -> step -> output back to the host
@@ -392,7 +402,7 @@ def run_device_bench(args, rank, world, local):
         e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                 for _ in range(args.steps)]
         for i in range(args.steps):
-            if not args.no_flush:
+            if flush_l2:
                 flush.zero_()
             e_ev[i][0].record(stream)
             e2e_step()
@@ -430,8 +440,11 @@ def run_device_bench(args, rank, world, local):
                        "num_kv_heads": wl.num_kv_heads, "head_size": wl.head_size,
                        "block_size": 16, "num_blocks": wl.num_blocks,
                        "kv_bytes_per_step": nbytes, "unique_kv_bytes_per_step": unique_kv_bytes(wl),
-                       "l2": "no flush" if args.no_flush else
-                             "flushed between steps (256 MiB write outside the step events)",
+                       "l2": ("flushed between steps (256 MiB write outside the step events)"
+                              if flush_l2 else
+                              f"inputs larger than L2: {nbytes / 1e6:.0f} MB of KV per step vs "
+                              f"126 MB L2, no flush"),
+                       "kv_split_tokens": args.kv_split_tokens or "planner",
                        "parallelism": f"replicas x{world} (one batch per GPU)"},
             "tokens_per_s": round(world * wl.num_tokens / (ms_per_step * 1e-3), 1),
             "pct_hbm_peak": round(100 * value / world / peak, 2),

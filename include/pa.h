@@ -109,8 +109,9 @@ int pa_write_kv(pa_cache* cache, const void* k, const void* v, const int32_t* sl
                 int num_tokens, void* stream);
 
 /* Workspace for pa_attention's split-KV partials when any request may be split into at most
- * max_splits parts: max_splits * num_tokens * num_q_heads * (head_size + 1) * 4 bytes plus
- * alignment.  0 when max_splits <= 1 (no splitting). */
+ * max_splits parts: max_splits * num_tokens * num_q_heads * (head_size + 1) * 4 bytes of
+ * partials plus num_tokens * num_q_heads * 4 bytes of split counters, each part 256-byte
+ * aligned.  0 when max_splits <= 1 (no splitting). */
 size_t pa_attention_workspace_bytes(int num_tokens, int num_q_heads, int head_size,
                                     int max_splits);
 
@@ -151,13 +152,14 @@ int pa_attention(const pa_cache* cache, const void* q, int num_q_heads,
  * It allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
  * Set-up: the first call on a device (with that device current) resolves the scratch's
  *   device address with cudaGetSymbolAddress; make that first call before any stream capture.
- * Limit: calls whose 2 * num_tokens * num_q_heads * (head_size + 1) * 4 bytes of partials (plus
- *   alignment) exceed PA_NOALLOC_SCRATCH_BYTES return PA_ERR_WORKSPACE and launch nothing; other
- *   calls get a split-KV partition fitted to the scratch.
+ * Limit: calls for which pa_attention_workspace_bytes(num_tokens, num_q_heads, head_size, 2)
+ *   (two splits of every row) exceeds PA_NOALLOC_SCRATCH_BYTES return PA_ERR_WORKSPACE and
+ *   launch nothing; other calls get a split-KV partition fitted to the scratch.
  * Sharing: all calls on a device share the one scratch, which keeps the last call's contents;
- *   nothing in it has to start at zero (each call writes every partial it reads).  Calls that
- *   overlap on the GPU (other streams, or other host threads) race on the scratch: serialise
- *   them, e.g. on one stream. */
+ *   each call clears the split counters it uses (the only part that must start at zero) on its
+ *   stream before its kernels run, and writes every partial it reads.  Calls that overlap on
+ *   the GPU (other streams, or other host threads) race on the scratch: serialise them, e.g.
+ *   on one stream. */
 int pa_attention_noalloc(const pa_cache* cache, const void* q, int num_q_heads,
                          const int32_t* block_table, int max_blocks_per_seq,
                          const int32_t* seq_lens, const int32_t* query_start_loc,
@@ -179,6 +181,7 @@ typedef struct {
     int64_t chunk_ctas;       /* CTAs that do work in the chunk kernel */
     int any_split;            /* a reduce launch is needed */
     size_t workspace_needed;  /* bytes of workspace this plan uses */
+    int reduce_rows_max;      /* largest q_len * group among split chunk-kind requests */
 } pa_plan;
 
 /* Options for pa_attention_ex (zero-initialise for defaults). */

@@ -50,6 +50,7 @@ class pa_plan(ctypes.Structure):
         ("chunk_ctas", ctypes.c_int64),
         ("any_split", ctypes.c_int),
         ("workspace_needed", ctypes.c_size_t),
+        ("reduce_rows_max", ctypes.c_int),
     ]
 
     def as_dict(self) -> dict:

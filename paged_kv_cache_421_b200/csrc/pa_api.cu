@@ -102,10 +102,14 @@ int make_tensor_map(pa_cache* c) {
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// Workspace of a plan with up to max_splits splits: partial outputs [S][T][Hq][D], partial
+// LSEs [S][T][Hq], then per-(request, kv head) finished-split counters indexed by the
+// request's first token (at most T x Hkv <= T x Hq of them).
 size_t workspace_for(int num_tokens, int num_q_heads, int head_size, int max_splits) {
     if (max_splits <= 1) return 0;
     const size_t rows = static_cast<size_t>(max_splits) * num_tokens * num_q_heads;
-    return align256(rows * head_size * sizeof(float)) + align256(rows * sizeof(float));
+    return align256(rows * head_size * sizeof(float)) + align256(rows * sizeof(float)) +
+           align256(static_cast<size_t>(num_tokens) * num_q_heads * sizeof(int));
 }
 
 int max_splits_for(size_t ws, int num_tokens, int num_q_heads, int head_size) {
@@ -120,9 +124,14 @@ int max_splits_for(size_t ws, int num_tokens, int num_q_heads, int head_size) {
 int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
 // Planner constants.
-constexpr int kDecodeCtasPerSm = 2;    // decode kernel residency (96 KB of stages per CTA)
-constexpr int kDecodeWaves = 8;        // target waves of decode CTAs over the GPU
-constexpr int kMinDecodeSplitBlocks = 32;  // >= 512 keys per split keeps CTA overheads small
+constexpr int kDecodeCtasPerSm = 3;    // decode kernel residency (64 KB of stages per CTA)
+constexpr int kMaxDecodeSplits = 1024;  // merge weights of one row fit the CTA's shared memory
+int env_int(const char* name, int dflt) {
+    const char* v = std::getenv(name);
+    return v ? std::atoi(v) : dflt;
+}
+const int kDecodeWaves = env_int("PA_TUNE_WAVES", 4);  // target waves of decode CTAs
+const int kMinDecodeSplitBlocks = env_int("PA_TUNE_MIN_SPLIT", 64);  // >= 1024 keys per split
 constexpr int kMinChunkSplitBlocks = 16;
 
 int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int Hkv, int D,
@@ -175,9 +184,10 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
             dsb = round_up(static_cast<int>(sb < dec_max_blocks ? sb : dec_max_blocks), 4);
         }
         int ns = pa::ceil_div(dec_max_blocks, dsb);
-        if (ns > 1 && ns > allowed) {
+        const int cap = allowed < kMaxDecodeSplits ? allowed : kMaxDecodeSplits;
+        if (ns > 1 && ns > cap) {
             if (forced) return PA_ERR_WORKSPACE;
-            dsb = allowed <= 1 ? dec_max_blocks : pa::ceil_div(dec_max_blocks, allowed);
+            dsb = cap <= 1 ? dec_max_blocks : pa::ceil_div(dec_max_blocks, cap);
             ns = pa::ceil_div(dec_max_blocks, dsb);
         }
         pl->decode_split_blocks = dsb;
@@ -208,16 +218,20 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
         pl->chunk_max_splits = ns;
         pl->chunk_max_qtiles = chunk_max_qtiles;
     }
-    // working CTA counts
+    // working CTA counts and the rows the reduce must cover
     for (int r = 0; r < B; ++r) {
         const int ql = qsl[r + 1] - qsl[r];
         if (ql == 0) continue;
+        int ns;
         if (pa::is_decode_kind(ql, G)) {
-            pl->decode_ctas += static_cast<int64_t>(pa::num_splits(sl[r], pl->decode_split_blocks)) * Hkv;
+            ns = pa::num_splits(sl[r], pl->decode_split_blocks);
+            pl->decode_ctas += static_cast<int64_t>(ns) * Hkv;
         } else {
-            pl->chunk_ctas += static_cast<int64_t>(pa::num_splits(sl[r], pl->chunk_split_blocks)) *
-                              Hkv * pa::ceil_div(ql * G, pa::kChunkRows);
+            ns = pa::num_splits(sl[r], pl->chunk_split_blocks);
+            pl->chunk_ctas += static_cast<int64_t>(ns) * Hkv * pa::ceil_div(ql * G, pa::kChunkRows);
         }
+        if (ns > 1 && !pa::is_decode_kind(ql, G) && ql * G > pl->reduce_rows_max)
+            pl->reduce_rows_max = ql * G;
     }
     const int smax = pl->decode_max_splits > pl->chunk_max_splits ? pl->decode_max_splits
                                                                    : pl->chunk_max_splits;
@@ -403,6 +417,8 @@ int pa_attention_ex(const pa_cache* cache, const void* q, int num_q_heads,
         p.part_o = static_cast<float*>(workspace);
         p.part_lse = reinterpret_cast<float*>(static_cast<char*>(workspace) +
                                               align256(rows * cache->head_size * sizeof(float)));
+        p.split_counters = reinterpret_cast<int*>(reinterpret_cast<char*>(p.part_lse) +
+                                                  align256(rows * sizeof(float)));
     }
     p.k_scale = cache->k_scale;
     p.v_scale = cache->v_scale;
@@ -416,12 +432,18 @@ int pa_attention_ex(const pa_cache* cache, const void* q, int num_q_heads,
     p.decode_split_blocks = pl.decode_split_blocks > 0 ? pl.decode_split_blocks : 1;
     p.chunk_split_blocks = pl.chunk_split_blocks > 0 ? pl.chunk_split_blocks : 4;
     p.chunk_max_qtiles = pl.chunk_max_qtiles > 0 ? pl.chunk_max_qtiles : 1;
+    p.reduce_row_tiles = pa::ceil_div(pl.reduce_rows_max > 0 ? pl.reduce_rows_max : 1, 4);
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     p.err = device_error_ptr();
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     void* const* ev = opts ? opts->events : nullptr;
     cudaError_t e = cudaSuccess;
+    if (pl.decode_max_splits > 1) {
+        e = cudaMemsetAsync(p.split_counters, 0,
+                            static_cast<size_t>(num_tokens) * cache->num_kv_heads * sizeof(int), s);
+        if (e != cudaSuccess) return fail_cuda(e);
+    }
     if (pl.num_decode_seqs) {
         if (ev) record(ev[0], s);
         e = pa::launch_decode(cache->tmap, p, cache->head_size, cache->kv_dtype,
@@ -436,7 +458,7 @@ int pa_attention_ex(const pa_cache* cache, const void* q, int num_q_heads,
         if (e != cudaSuccess) return fail_cuda(e);
         if (ev) record(ev[3], s);
     }
-    if (pl.any_split) {
+    if (pl.chunk_max_splits > 1) {
         if (ev) record(ev[4], s);
         e = pa::launch_reduce(p, cache->head_size, s);
         if (e != cudaSuccess) return fail_cuda(e);

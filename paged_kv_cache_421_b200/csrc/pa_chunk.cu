@@ -35,6 +35,8 @@ __global__ void __launch_bounds__(128)
 chunk_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
     int* err = p.err;
     using C = ChunkCfg<D>;
+    pdl_trigger();
+    pdl_wait();
     const int qt = blockIdx.x % p.chunk_max_qtiles;
     const int split = blockIdx.x / p.chunk_max_qtiles;
     const int g = blockIdx.y, r = blockIdx.z;
@@ -302,8 +304,7 @@ cudaError_t launch_chunk_t(const CUtensorMap& tmap, const AttnParams& p, int max
         attr_set = true;
     }
     dim3 grid(p.chunk_max_qtiles * max_splits, p.num_kv_heads, p.num_seqs);
-    chunk_kernel<D><<<grid, 128, C::kSmemBytes, stream>>>(tmap, p);
-    return cudaGetLastError();
+    return launch_pdl(chunk_kernel<D>, grid, dim3(128), C::kSmemBytes, stream, tmap, p);
 }
 
 }  // namespace

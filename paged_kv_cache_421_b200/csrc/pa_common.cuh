@@ -44,6 +44,16 @@ __device__ __forceinline__ void raise_error(int* err, int code) {
     if (err) atomicCAS(err, 0, code);
 }
 
+// ------------------------------------------------------------------ programmatic launch
+// Kernels are launched with programmatic stream serialization: the next kernel in the
+// stream may be scheduled once every CTA of this one has started (pdl_trigger), and every
+// kernel waits for its predecessors to finish and publish their memory (pdl_wait) before it
+// reads global memory.  Without the launch attribute both are no-ops.
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------ smem / barriers
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));

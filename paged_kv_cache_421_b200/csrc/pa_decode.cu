@@ -21,6 +21,8 @@
 // and O^T += V^T P^T reads V through ldmatrix.trans.  Softmax runs in the log2 domain.
 // FP8 E4M3 caches are decoded to f16 (exact) in registers; the K scale folds into the score
 // scale and the V scale into the epilogue.
+#include <cstdlib>
+
 #include "pa_internal.h"
 
 namespace pa {
@@ -47,6 +49,8 @@ template <int D, int NW, int NS, bool FP8>
 __global__ void __launch_bounds__(NW * 32)
 decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
     using C = DecodeCfg<D, NW, NS, FP8>;
+    pdl_trigger();
+    pdl_wait();
     const int split = blockIdx.x, g = blockIdx.y, r = blockIdx.z;
     const int q0 = p.qsl[r];
     const int q_len = p.qsl[r + 1] - q0;
@@ -336,12 +340,15 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
         base[d1 * 8 + row0] = o[mt][2];
         base[d1 * 8 + row1] = o[mt][3];
     }
-    __syncthreads();
-    if (!ok) return;
+    if (!__syncthreads_and(ok)) return;
 
     const float vscale = FP8 ? p.v_scale[g] : 1.f;
     const bool direct = nsplit == 1;
-    if (!direct && split >= p.max_splits) return;  // workspace bound (planned launch ensures it)
+    if (!direct && split >= p.max_splits) {  // workspace bound (a planned launch never hits it)
+        if (tid == 0) raise_error(p.err, kErrMetadata);
+        return;
+    }
+    const int64_t stride = static_cast<int64_t>(p.num_tokens) * p.num_q_heads;  // one split
     for (int idx = tid; idx < rows * D; idx += NW * 32) {
         const int n = idx / D, d = idx % D;
         float M = -INFINITY;
@@ -362,10 +369,64 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
         if (direct) {
             p.out[(static_cast<int64_t>(t) * p.num_q_heads + h) * D + d] = val;
         } else {
-            const int64_t prow = (static_cast<int64_t>(split) * p.num_tokens + t) * p.num_q_heads + h;
+            const int64_t prow = split * stride + static_cast<int64_t>(t) * p.num_q_heads + h;
             p.part_o[prow * D + d] = val;
             if (d == 0) p.part_lse[prow] = L > 0.f ? M + __log2f(L) : -INFINITY;
         }
+    }
+    if (direct) return;
+
+    // ---- split merge: the last CTA of this (request, kv head) to finish merges every split
+    // (out = sum_s 2^(lse_s - L) O_s / sum_s 2^(lse_s - L), L = max_s lse_s).  Each call's
+    // counters start at zero (cleared on the stream before the launch).
+    __shared__ int s_last;
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = atomicAdd(p.split_counters + q0 * p.num_kv_heads + g, 1) == nsplit - 1;
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    float* s_w = reinterpret_cast<float*>(smem);  // [rows][nsplit] merge weights
+    float* s_inv = s_w + rows * nsplit;           // [rows] 1 / sum of weights
+    for (int n = warp; n < rows; n += NW) {
+        const int64_t row = static_cast<int64_t>(q0 + n / p.group) * p.num_q_heads +
+                            g * p.group + n % p.group;
+        float M = -INFINITY;
+        for (int sp = lane; sp < nsplit; sp += 32) M = fmaxf(M, __ldcg(p.part_lse + sp * stride + row));
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, off));
+        float W = 0.f;
+        for (int sp = lane; sp < nsplit; sp += 32) {
+            const float w = M == -INFINITY ? 0.f : fast_exp2(__ldcg(p.part_lse + sp * stride + row) - M);
+            s_w[n * nsplit + sp] = w;
+            W += w;
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) W += __shfl_xor_sync(kFull, W, off);
+        if (lane == 0) s_inv[n] = W > 0.f ? 1.f / W : 0.f;
+    }
+    __syncthreads();
+    constexpr int kV4 = D / 4;
+    for (int item = tid; item < rows * kV4; item += NW * 32) {
+        const int n = item / kV4, c = item % kV4;
+        const int64_t row = static_cast<int64_t>(q0 + n / p.group) * p.num_q_heads +
+                            g * p.group + n % p.group;
+        const float4* src = reinterpret_cast<const float4*>(p.part_o + row * D) + c;
+        const int64_t s4 = stride * D / 4;
+        const float* w = s_w + n * nsplit;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+        for (int sp = 0; sp < nsplit; ++sp) {
+            const float4 v = __ldcg(src + sp * s4);
+            const float ws = w[sp];
+            acc.x += ws * v.x;
+            acc.y += ws * v.y;
+            acc.z += ws * v.z;
+            acc.w += ws * v.w;
+        }
+        const float inv = s_inv[n];
+        reinterpret_cast<float4*>(p.out + row * D)[c] =
+            make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
     }
 }
 
@@ -382,20 +443,32 @@ cudaError_t launch_decode_t(const CUtensorMap& tmap, const AttnParams& p, int ma
         attr_set = true;
     }
     dim3 grid(max_splits, p.num_kv_heads, p.num_seqs);
-    kern<<<grid, NW * 32, C::kSmemBytes, stream>>>(tmap, p);
-    return cudaGetLastError();
+    return launch_pdl(kern, grid, dim3(NW * 32), C::kSmemBytes, stream, tmap, p);
 }
 
 }  // namespace
 
 cudaError_t launch_decode(const CUtensorMap& tmap, const AttnParams& p, int head_size,
                           int kv_dtype, int max_splits, cudaStream_t stream) {
-    if (kv_dtype == PA_BF16 && head_size == 128)
-        return launch_decode_t<128, 4, 3, false>(tmap, p, max_splits, stream);
+    if (kv_dtype == PA_BF16 && head_size == 128) {
+        static const int stages = [] {
+            const char* v = std::getenv("PA_TUNE_STAGES");
+            return v ? std::atoi(v) : 2;
+        }();
+        if (stages == 3) return launch_decode_t<128, 4, 3, false>(tmap, p, max_splits, stream);
+        return launch_decode_t<128, 4, 2, false>(tmap, p, max_splits, stream);
+    }
     if (kv_dtype == PA_BF16 && head_size == 64)
         return launch_decode_t<64, 4, 6, false>(tmap, p, max_splits, stream);
-    if (kv_dtype == PA_FP8_E4M3 && head_size == 128)
+    if (kv_dtype == PA_FP8_E4M3 && head_size == 128) {
+        static const int variant = [] {
+            const char* v = std::getenv("PA_TUNE_FP8");
+            return v ? std::atoi(v) : 0;
+        }();
+        if (variant == 1) return launch_decode_t<128, 4, 4, true>(tmap, p, max_splits, stream);
+        if (variant == 2) return launch_decode_t<128, 8, 3, true>(tmap, p, max_splits, stream);
         return launch_decode_t<128, 4, 6, true>(tmap, p, max_splits, stream);
+    }
     return cudaErrorInvalidValue;
 }
 

@@ -1,6 +1,8 @@
 // Internal declarations shared by the host API and the kernel translation units.
 #pragma once
 
+#include <utility>
+
 #include "../../include/pa.h"
 #include "pa_common.cuh"
 
@@ -21,6 +23,23 @@ struct pa_cache {
 
 namespace pa {
 
+// Launch `kern` with programmatic stream serialization (see pdl_trigger / pdl_wait).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 // Arguments of one attention launch (kernels read them from the parameter space).
 struct AttnParams {
     const __nv_bfloat16* q;     // [T][Hq][D]
@@ -30,6 +49,7 @@ struct AttnParams {
     float* out;                 // [T][Hq][D]
     float* part_o;              // [S][T][Hq][D] split partials (normalised)
     float* part_lse;            // [S][T][Hq]   split log2-sum-exp2 of scaled scores
+    int* split_counters;        // [T][Hkv] finished-split counts (zeroed before each launch)
     const float* k_scale;       // FP8 per-kv-head scales, else null
     const float* v_scale;
     int max_blocks_per_seq;
@@ -43,6 +63,7 @@ struct AttnParams {
     int chunk_split_blocks;     // KV partition of chunk-kind requests (blocks, multiple of 4)
     int chunk_max_qtiles;       // grid.x stride of the chunk kernel
     int max_splits;             // splits the workspace holds (bounds every partial index)
+    int reduce_row_tiles;       // grid.x of the reduce: 4-row tiles of the largest split request
     float scale_log2;           // softmax scale * log2(e)
     int* err;                   // device error word
 };

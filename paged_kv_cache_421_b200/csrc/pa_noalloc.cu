@@ -25,10 +25,7 @@ void* g_noalloc_scratch_addr[kMaxNoallocDevices] = {nullptr};
 // Bytes of split partials that two splits of every (token, q head) row need; a call whose
 // rows do not fit twice in the scratch is beyond this entry point's maximum.
 size_t two_split_bytes(int num_tokens, int num_q_heads, int head_size) {
-    const size_t rows = 2ull * static_cast<size_t>(num_tokens) * num_q_heads;
-    const size_t o = (rows * head_size * sizeof(float) + 255) & ~static_cast<size_t>(255);
-    const size_t l = (rows * sizeof(float) + 255) & ~static_cast<size_t>(255);
-    return o + l;
+    return pa_attention_workspace_bytes(num_tokens, num_q_heads, head_size, 2);
 }
 
 }  // namespace
@@ -55,8 +52,8 @@ extern "C" int pa_attention_noalloc(const pa_cache* cache, const void* q, int nu
         if (e != cudaSuccess || !ptr) return PA_ERR_CUDA;
         g_noalloc_scratch_addr[dev] = ptr;
     }
-    // The partials need no zeroing: every partial the merge reads is written earlier in the
-    // same call.  The planner fits the split-KV partition into the scratch.
+    // pa_attention clears the split counters on the stream before its kernels and writes every
+    // partial the merge reads; the planner fits the split-KV partition into the scratch.
     return pa_attention(cache, q, num_q_heads, block_table, max_blocks_per_seq, seq_lens,
                         query_start_loc, seq_lens_host, query_start_loc_host, num_seqs,
                         num_tokens, scale, out, g_noalloc_scratch_addr[dev],

@@ -18,6 +18,8 @@ __global__ void slot_mapping_kernel(const int32_t* __restrict__ bt, int maxb,
                                     const int32_t* __restrict__ seq_lens,
                                     const int32_t* __restrict__ qsl, int bs, int num_tokens,
                                     int32_t* __restrict__ slots, int* err) {
+    pdl_trigger();
+    pdl_wait();
     const int r = blockIdx.x;
     const int q0 = qsl[r];
     const int q_len = qsl[r + 1] - q0;
@@ -45,6 +47,8 @@ write_kv_kernel(uint8_t* __restrict__ cache, const uint16_t* __restrict__ k,
                 int num_tokens, int num_kv_heads, int64_t num_slots,
                 const float* __restrict__ k_scale, const float* __restrict__ v_scale,
                 int* err) {
+    pdl_trigger();
+    pdl_wait();
     constexpr int kChunks = D / 8;  // 16-byte pieces of one bf16 row
     const int64_t total = static_cast<int64_t>(num_tokens) * num_kv_heads * 2 * kChunks;
     for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
@@ -109,11 +113,11 @@ cudaError_t launch_write_t(const pa_cache& c, const void* k, const void* v, cons
     const int threads = 256;
     const int64_t blocks = (total + threads - 1) / threads;
     const int grid = static_cast<int>(blocks < 148 * 32 ? blocks : 148 * 32);
-    write_kv_kernel<D, FP8><<<grid, threads, 0, stream>>>(
-        static_cast<uint8_t*>(c.data), static_cast<const uint16_t*>(k),
-        static_cast<const uint16_t*>(v), slots, num_tokens, c.num_kv_heads,
-        static_cast<int64_t>(c.num_blocks) * c.block_size, c.k_scale, c.v_scale, err);
-    return cudaGetLastError();
+    return launch_pdl(write_kv_kernel<D, FP8>, dim3(grid), dim3(threads), 0, stream,
+                      static_cast<uint8_t*>(c.data), static_cast<const uint16_t*>(k),
+                      static_cast<const uint16_t*>(v), slots, num_tokens, c.num_kv_heads,
+                      static_cast<int64_t>(c.num_blocks) * c.block_size, c.k_scale, c.v_scale,
+                      err);
 }
 
 }  // namespace
@@ -122,10 +126,9 @@ cudaError_t launch_slot_mapping(const int32_t* block_table, int max_blocks_per_s
                                 const int32_t* seq_lens, const int32_t* qsl, int num_seqs,
                                 int num_tokens, int block_size, int32_t* slot_mapping, int* err,
                                 cudaStream_t stream) {
-    slot_mapping_kernel<<<num_seqs, 128, 0, stream>>>(block_table, max_blocks_per_seq, seq_lens,
-                                                      qsl, block_size, num_tokens, slot_mapping,
-                                                      err);
-    return cudaGetLastError();
+    return launch_pdl(slot_mapping_kernel, dim3(num_seqs), dim3(128), 0, stream, block_table,
+                      max_blocks_per_seq, seq_lens, qsl, block_size, num_tokens, slot_mapping,
+                      err);
 }
 
 cudaError_t launch_write_kv(const pa_cache& c, const void* k, const void* v,
