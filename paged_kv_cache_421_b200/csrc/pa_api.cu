@@ -3,6 +3,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <algorithm>
 #include <new>
 
 #include "pa_internal.h"
@@ -133,6 +134,7 @@ int env_int(const char* name, int dflt) {
 const int kDecodeWaves = env_int("PA_TUNE_WAVES", 4);  // target waves of decode CTAs
 const int kMinDecodeSplitBlocks = env_int("PA_TUNE_MIN_SPLIT", 64);  // >= 1024 keys per split
 constexpr int kMinChunkSplitBlocks = 16;
+constexpr int kMaxChunkSplitBlocks = 1024;  // chunk kernels stage up to 1024 block ids
 
 int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int Hkv, int D,
               int bs, int maxb, int num_sms, size_t ws, const pa_attention_opts* opts,
@@ -163,7 +165,7 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
             if (blocks > dec_max_blocks) dec_max_blocks = blocks;
         } else {
             pl->num_chunk_seqs++;
-            const int qt = pa::ceil_div(ql * G, pa::kChunkRows);
+            const int qt = pa::ceil_div(ql * G, pa::chunk_rows(D, 1));
             if (qt > chunk_max_qtiles) chunk_max_qtiles = qt;
             chunk_tiles += static_cast<long long>(qt) * Hkv;
             if (blocks > chunk_max_blocks) chunk_max_blocks = blocks;
@@ -200,7 +202,11 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
             csb = forced / bs;
         } else {
             csb = round_up(chunk_max_blocks, 4);
-            if (chunk_tiles < num_sms && chunk_max_blocks >= 2 * kMinChunkSplitBlocks) {
+            if (csb > kMaxChunkSplitBlocks && allowed > 1)  // keep block ids in shared memory
+                csb = round_up(pa::ceil_div(chunk_max_blocks,
+                                            pa::ceil_div(chunk_max_blocks, kMaxChunkSplitBlocks)), 4);
+            // split only when the chunk CTAs would leave most of the GPU idle
+            if (2 * chunk_tiles <= num_sms && chunk_max_blocks >= 2 * kMinChunkSplitBlocks) {
                 const long long want = (2LL * num_sms + chunk_tiles - 1) / chunk_tiles;
                 int sb = pa::ceil_div(chunk_max_blocks, static_cast<int>(want));
                 if (sb < kMinChunkSplitBlocks) sb = kMinChunkSplitBlocks;
@@ -228,7 +234,7 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
             pl->decode_ctas += static_cast<int64_t>(ns) * Hkv;
         } else {
             ns = pa::num_splits(sl[r], pl->chunk_split_blocks);
-            pl->chunk_ctas += static_cast<int64_t>(ns) * Hkv * pa::ceil_div(ql * G, pa::kChunkRows);
+            pl->chunk_ctas += static_cast<int64_t>(ns) * Hkv * pa::ceil_div(ql * G, pa::chunk_rows(D, 1));
         }
         if (ns > 1 && !pa::is_decode_kind(ql, G) && ql * G > pl->reduce_rows_max)
             pl->reduce_rows_max = ql * G;
@@ -451,16 +457,29 @@ int pa_attention_ex(const pa_cache* cache, const void* q, int num_q_heads,
         if (e != cudaSuccess) return fail_cuda(e);
         if (ev) record(ev[1], s);
     }
+    // the chunk-kind requests, longest context first; a longer list falls back to a grid over
+    // every request
+    static thread_local pa::ChunkList list;
+    list.count = 0;
     if (pl.num_chunk_seqs) {
+        if (pl.num_chunk_seqs <= pa::kMaxChunkList) {
+            for (int r = 0; r < num_seqs; ++r) {
+                const int ql = query_start_loc_host[r + 1] - query_start_loc_host[r];
+                if (ql > 0 && !pa::is_decode_kind(ql, p.group)) list.req[list.count++] = r;
+            }
+            std::stable_sort(list.req, list.req + list.count, [&](int a, int b) {
+                return seq_lens_host[a] > seq_lens_host[b];
+            });
+        }
         if (ev) record(ev[2], s);
-        e = pa::launch_chunk(cache->tmap, p, cache->head_size, cache->kv_dtype,
+        e = pa::launch_chunk(cache->tmap, p, list, cache->head_size, cache->kv_dtype,
                              pl.chunk_max_splits, s);
         if (e != cudaSuccess) return fail_cuda(e);
         if (ev) record(ev[3], s);
     }
     if (pl.chunk_max_splits > 1) {
         if (ev) record(ev[4], s);
-        e = pa::launch_reduce(p, cache->head_size, s);
+        e = pa::launch_reduce(p, list, cache->head_size, s);
         if (e != cudaSuccess) return fail_cuda(e);
         if (ev) record(ev[5], s);
     }

@@ -18,6 +18,7 @@ namespace {
 constexpr uint32_t kFull = 0xffffffffu;
 constexpr int kTileKeys = 64;
 constexpr int kBlocksPerTile = kTileKeys / kBlockSize;
+constexpr int kMaxIds = 1024;  // block ids staged in shared memory
 
 template <int D>
 struct ChunkCfg {
@@ -32,14 +33,17 @@ struct ChunkCfg {
 
 template <int D>
 __global__ void __launch_bounds__(128)
-chunk_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
+chunk_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
+             const __grid_constant__ ChunkList list) {
     int* err = p.err;
     using C = ChunkCfg<D>;
     pdl_trigger();
     pdl_wait();
-    const int qt = blockIdx.x % p.chunk_max_qtiles;
+    // the last query tiles see the most keys (causal): dispatch them first
+    const int qt = p.chunk_max_qtiles - 1 - static_cast<int>(blockIdx.x % p.chunk_max_qtiles);
     const int split = blockIdx.x / p.chunk_max_qtiles;
-    const int g = blockIdx.y, r = blockIdx.z;
+    const int g = blockIdx.y;
+    const int r = list.count > 0 ? list.req[blockIdx.z] : static_cast<int>(blockIdx.z);
     const int q0 = p.qsl[r];
     const int q_len = p.qsl[r + 1] - q0;
     if (q_len <= 0 || is_decode_kind(q_len, p.group)) return;
@@ -71,6 +75,7 @@ chunk_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
 
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t bars[2];
+    __shared__ int ids[kMaxIds];  // physical ids of the split's first kMaxIds logical blocks
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const uint32_t sbase = smem_u32(smem);
@@ -109,6 +114,14 @@ chunk_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
         mbar_init(smem_u32(&bars[0]), 1);
         mbar_init(smem_u32(&bars[1]), 1);
     }
+    for (int k = tid; k < min(je - jb, kMaxIds); k += 128) {
+        int blk = p.block_table[static_cast<int64_t>(r) * p.max_blocks_per_seq + jb + k];
+        if (blk < 0 || blk >= p.num_blocks) {
+            raise_error(err, kErrBadBlockId);
+            blk = 0;
+        }
+        ids[k] = blk;
+    }
     fence_barrier_init();
     __syncthreads();
 
@@ -121,10 +134,15 @@ chunk_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
         const int nload = min(kBlocksPerTile, je - j0);
         mbar_arrive_expect_tx(bar, nload * 2 * C::kTileBytes);
         for (int b = 0; b < nload; ++b) {
-            int blk = p.block_table[static_cast<int64_t>(r) * p.max_blocks_per_seq + j0 + b];
-            if (blk < 0 || blk >= p.num_blocks) {
-                raise_error(err, kErrBadBlockId);
-                blk = 0;
+            int blk;
+            if (j0 + b - jb < kMaxIds) {
+                blk = ids[j0 + b - jb];
+            } else {
+                blk = p.block_table[static_cast<int64_t>(r) * p.max_blocks_per_seq + j0 + b];
+                if (blk < 0 || blk >= p.num_blocks) {
+                    raise_error(err, kErrBadBlockId);
+                    blk = 0;
+                }
             }
             const int rowk = blk * kv_rows_per_block + g * kBlockSize;
             const int rowv = rowk + p.num_kv_heads * kBlockSize;
@@ -292,8 +310,8 @@ chunk_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
 }
 
 template <int D>
-cudaError_t launch_chunk_t(const CUtensorMap& tmap, const AttnParams& p, int max_splits,
-                           cudaStream_t stream) {
+cudaError_t launch_chunk_t(const CUtensorMap& tmap, const AttnParams& p, const ChunkList& list,
+                           int max_splits, cudaStream_t stream) {
     using C = ChunkCfg<D>;
     static bool attr_set = false;
     if (!attr_set) {
@@ -303,17 +321,18 @@ cudaError_t launch_chunk_t(const CUtensorMap& tmap, const AttnParams& p, int max
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    dim3 grid(p.chunk_max_qtiles * max_splits, p.num_kv_heads, p.num_seqs);
-    return launch_pdl(chunk_kernel<D>, grid, dim3(128), C::kSmemBytes, stream, tmap, p);
+    dim3 grid(p.chunk_max_qtiles * max_splits, p.num_kv_heads,
+              list.count > 0 ? list.count : p.num_seqs);
+    return launch_pdl(chunk_kernel<D>, grid, dim3(128), C::kSmemBytes, stream, tmap, p, list);
 }
 
 }  // namespace
 
-cudaError_t launch_chunk(const CUtensorMap& tmap, const AttnParams& p, int head_size,
-                         int kv_dtype, int max_splits, cudaStream_t stream) {
+cudaError_t launch_chunk(const CUtensorMap& tmap, const AttnParams& p, const ChunkList& list,
+                         int head_size, int kv_dtype, int max_splits, cudaStream_t stream) {
     if (kv_dtype != PA_BF16) return cudaErrorInvalidValue;
-    if (head_size == 128) return launch_chunk_t<128>(tmap, p, max_splits, stream);
-    if (head_size == 64) return launch_chunk_t<64>(tmap, p, max_splits, stream);
+    if (head_size == 128) return launch_chunk_tc(tmap, p, list, max_splits, stream);
+    if (head_size == 64) return launch_chunk_t<64>(tmap, p, list, max_splits, stream);
     return cudaErrorInvalidValue;
 }
 

@@ -17,7 +17,8 @@ namespace pa {
 // ------------------------------------------------------------------ shared rules
 constexpr int kBlockSize = 16;      // tokens per physical block (the pages' default)
 constexpr int kDecodeRows = 8;      // decode tile: q_len * group <= 8 rows share one kv head
-constexpr int kChunkRows = 64;      // chunk tile: 64 (token, q head) rows per CTA
+constexpr int kChunkRows = 64;      // mma.sync chunk tile: 64 (token, q head) rows per CTA
+constexpr int kChunkRowsTc = 256;   // tcgen05 chunk CTA: two 128-row q-tiles (TMEM lanes)
 
 // Error codes written to the device error word.
 constexpr int kErrWaitTimeout = 1;
@@ -31,6 +32,10 @@ __host__ __device__ inline bool is_decode_kind(int q_len, int group) {
     return q_len > 0 && q_len * group <= kDecodeRows;
 }
 __host__ __device__ inline int ceil_div(int a, int b) { return (a + b - 1) / b; }
+// Query rows per chunk-kernel CTA: the tcgen05 kernel serves bf16 caches with head_size 128.
+__host__ __device__ inline int chunk_rows(int head_size, int kv_dtype_is_bf16) {
+    return (head_size == 128 && kv_dtype_is_bf16) ? kChunkRowsTc : kChunkRows;
+}
 // Number of KV splits of a request with ctx tokens under a partition of split_blocks blocks.
 __host__ __device__ inline int num_splits(int ctx, int split_blocks) {
     int blocks = ceil_div(ctx, kBlockSize);

@@ -68,11 +68,22 @@ struct AttnParams {
     int* err;                   // device error word
 };
 
+// The chunk-kind requests of a launch, longest context first (passed by value, so the chunk
+// grid covers only them); count == 0 means "every request, in order".
+constexpr int kMaxChunkList = 512;
+struct ChunkList {
+    int count;
+    int req[kMaxChunkList];
+};
+
 cudaError_t launch_decode(const CUtensorMap& tmap, const AttnParams& p, int head_size,
                           int kv_dtype, int max_splits, cudaStream_t stream);
-cudaError_t launch_chunk(const CUtensorMap& tmap, const AttnParams& p, int head_size,
-                         int kv_dtype, int max_splits, cudaStream_t stream);
-cudaError_t launch_reduce(const AttnParams& p, int head_size, cudaStream_t stream);
+cudaError_t launch_chunk(const CUtensorMap& tmap, const AttnParams& p, const ChunkList& list,
+                         int head_size, int kv_dtype, int max_splits, cudaStream_t stream);
+cudaError_t launch_chunk_tc(const CUtensorMap& tmap, const AttnParams& p, const ChunkList& list,
+                            int max_splits, cudaStream_t stream);
+cudaError_t launch_reduce(const AttnParams& p, const ChunkList& list, int head_size,
+                          cudaStream_t stream);
 cudaError_t launch_slot_mapping(const int32_t* block_table, int max_blocks_per_seq,
                                 const int32_t* seq_lens, const int32_t* qsl, int num_seqs,
                                 int num_tokens, int block_size, int32_t* slot_mapping, int* err,

@@ -15,10 +15,12 @@ namespace pa {
 namespace {
 
 template <int D>
-__global__ void __launch_bounds__(128) reduce_kernel(const AttnParams p) {
+__global__ void __launch_bounds__(128) reduce_kernel(const AttnParams p,
+                                                     const __grid_constant__ ChunkList list) {
     pdl_trigger();
     pdl_wait();
-    const int r = blockIdx.z, g = blockIdx.y;
+    const int r = list.count > 0 ? list.req[blockIdx.z] : static_cast<int>(blockIdx.z);
+    const int g = blockIdx.y;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int row = blockIdx.x * 4 + warp;  // one warp per (token, q head) row
     const int q0 = p.qsl[r];
@@ -79,10 +81,13 @@ __global__ void __launch_bounds__(128) reduce_kernel(const AttnParams p) {
 
 }  // namespace
 
-cudaError_t launch_reduce(const AttnParams& p, int head_size, cudaStream_t stream) {
-    dim3 grid(p.reduce_row_tiles, p.num_kv_heads, p.num_seqs);
-    if (head_size == 128) return launch_pdl(reduce_kernel<128>, grid, dim3(128), 0, stream, p);
-    if (head_size == 64) return launch_pdl(reduce_kernel<64>, grid, dim3(128), 0, stream, p);
+cudaError_t launch_reduce(const AttnParams& p, const ChunkList& list, int head_size,
+                          cudaStream_t stream) {
+    dim3 grid(p.reduce_row_tiles, p.num_kv_heads, list.count > 0 ? list.count : p.num_seqs);
+    if (head_size == 128)
+        return launch_pdl(reduce_kernel<128>, grid, dim3(128), 0, stream, p, list);
+    if (head_size == 64)
+        return launch_pdl(reduce_kernel<64>, grid, dim3(128), 0, stream, p, list);
     return cudaErrorInvalidValue;
 }
 

@@ -89,7 +89,8 @@ def test_plan_invariants(lib, name):
         assert p["decode_ctas"] == int(ns.sum()) * wl.num_kv_heads
         assert sb % 4 == 0 or sb == blocks[dec].max()
     if p["num_chunk_seqs"]:
-        assert p["chunk_max_qtiles"] == int(np.max(-(-(ql[~dec & (ql > 0)] * G) // 64)))
+        rows_per_cta = 256 if wl.head_size == 128 else 64  # tcgen05 CTA / mma.sync CTA
+        assert p["chunk_max_qtiles"] == int(np.max(-(-(ql[~dec & (ql > 0)] * G) // rows_per_cta)))
     smax = max(p["decode_max_splits"], p["chunk_max_splits"])
     assert p["any_split"] == int(smax > 1)
     assert p["workspace_needed"] == B.pa_attention_workspace_bytes(wl.num_tokens, wl.num_q_heads,
