@@ -62,9 +62,11 @@ size_t pa_cache_bytes(int num_blocks, int block_size, int num_kv_heads, int head
                       int kv_dtype);
 
 /* Create a pool ([P2] section 2: the physical block pool).
- * Layout in device memory: [num_blocks][2 (K, V)][num_kv_heads][block_size][head_size] in
- * the cache dtype, so one physical block is one contiguous span of pa_cache_bytes(1, ...)
- * bytes and each (block, K|V, kv head) tile is block_size * head_size elements contiguous.
+ * Layout in device memory: [num_blocks][2 (K, V)][num_kv_heads] tiles of block_size *
+ * head_size elements in the cache dtype, so one physical block is one contiguous span of
+ * pa_cache_bytes(1, ...) bytes and each (block, K|V, kv head) tile is contiguous.  Inside a
+ * tile, K and bf16 V are token-major ([block_size][head_size]); FP8 V tiles are dim-major
+ * ([head_size][block_size]), so attention reads consecutive tokens of one dim together.
  * Supported: block_size 16; head_size 64 or 128 (bf16), 128 (FP8 E4M3); any num_kv_heads.
  * k_scale, v_scale: device fp32 [num_kv_heads], required for FP8 (the stored code is
  *   e4m3(x / scale[head])), ignored for bf16; caller-owned, read by later calls.

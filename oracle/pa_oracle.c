@@ -19,8 +19,9 @@
  *     keys (flattened super-sequence, "Inside vLLM" notes core point 2) and, inside a chunk,
  *     only keys at or before their own position (chunked prefill, article 5 outline).
  *
- * Cache layout, read only through elem_index(): [num_blocks][2 (K, V)][num_kv_heads]
- * [block_size][head_size].  One physical block therefore spans exactly
+ * Cache layout, read only through elem_index_dt(): [num_blocks][2 (K, V)][num_kv_heads] tiles
+ * of [block_size][head_size] elements (FP8 pools store V tiles as [head_size][block_size]).
+ * One physical block therefore spans exactly
  * 2 * block_size * num_kv_heads * head_size * dtype_bytes bytes ("Inside vLLM" notes,
  * core point 1).
  *
@@ -36,10 +37,19 @@ enum { OR_OK = 0, OR_BAD_META = 6, OR_NOMEM = 3, OR_BAD_ARG = 1 };
 enum { OR_BF16 = 0, OR_FP8_E4M3 = 1 };
 
 /* ------------------------------------------------------------------ layout */
+/* Element (token tok, dim d) of the K (kv = 0) or V (kv = 1) tile of (block, head).  Tiles
+ * are [block][K|V][head] of block_size * head_size elements; inside a tile the layout is
+ * token-major ([tok][d]) except for V tiles of an FP8 pool, which are dim-major ([d][tok]). */
+static int64_t elem_index_dt(int64_t block, int kv, int head, int tok, int d,
+                             int num_kv_heads, int block_size, int head_size, int kv_dtype) {
+    int64_t tile = ((block * 2 + kv) * num_kv_heads + head) * (int64_t)block_size * head_size;
+    if (kv == 1 && kv_dtype == OR_FP8_E4M3) return tile + (int64_t)d * block_size + tok;
+    return tile + (int64_t)tok * head_size + d;
+}
+
 static int64_t elem_index(int64_t block, int kv, int head, int tok, int d,
                           int num_kv_heads, int block_size, int head_size) {
-    return (((block * 2 + kv) * num_kv_heads + head) * (int64_t)block_size + tok)
-           * head_size + d;
+    return elem_index_dt(block, kv, head, tok, d, num_kv_heads, block_size, head_size, OR_BF16);
 }
 
 int64_t oracle_cache_elems(int num_blocks, int block_size, int num_kv_heads, int head_size) {
@@ -193,10 +203,10 @@ void oracle_write_kv_fp8(uint8_t* cache, int num_blocks, int block_size, int num
                 int64_t src = ((int64_t)t * num_kv_heads + h) * head_size + d;
                 float yk = bf16_to_float(k[src]) / k_scale[h];
                 float yv = bf16_to_float(v[src]) / v_scale[h];
-                cache[elem_index(b, 0, h, o, d, num_kv_heads, block_size, head_size)] =
-                    oracle_e4m3_encode(yk);
-                cache[elem_index(b, 1, h, o, d, num_kv_heads, block_size, head_size)] =
-                    oracle_e4m3_encode(yv);
+                cache[elem_index_dt(b, 0, h, o, d, num_kv_heads, block_size, head_size,
+                                    OR_FP8_E4M3)] = oracle_e4m3_encode(yk);
+                cache[elem_index_dt(b, 1, h, o, d, num_kv_heads, block_size, head_size,
+                                    OR_FP8_E4M3)] = oracle_e4m3_encode(yv);
             }
     }
 }
@@ -270,10 +280,12 @@ int oracle_attention_paged(const void* cache, int kv_dtype, int num_blocks, int 
                 for (d = 0; d < head_size; ++d) {
                     K[(int64_t)p * head_size + d] = cache_value(
                         cache, kv_dtype,
-                        elem_index(b, 0, g, o, d, num_kv_heads, block_size, head_size), ks);
+                        elem_index_dt(b, 0, g, o, d, num_kv_heads, block_size, head_size,
+                                      kv_dtype), ks);
                     V[(int64_t)p * head_size + d] = cache_value(
                         cache, kv_dtype,
-                        elem_index(b, 1, g, o, d, num_kv_heads, block_size, head_size), vs);
+                        elem_index_dt(b, 1, g, o, d, num_kv_heads, block_size, head_size,
+                                      kv_dtype), vs);
                 }
             }
             for (i = 0; i < q_len; ++i) {

@@ -127,12 +127,8 @@ int round_up(int x, int m) { return (x + m - 1) / m * m; }
 // Planner constants.
 constexpr int kDecodeCtasPerSm = 3;    // decode kernel residency (64 KB of stages per CTA)
 constexpr int kMaxDecodeSplits = 1024;  // merge weights of one row fit the CTA's shared memory
-int env_int(const char* name, int dflt) {
-    const char* v = std::getenv(name);
-    return v ? std::atoi(v) : dflt;
-}
-const int kDecodeWaves = env_int("PA_TUNE_WAVES", 4);  // target waves of decode CTAs
-const int kMinDecodeSplitBlocks = env_int("PA_TUNE_MIN_SPLIT", 64);  // >= 1024 keys per split
+constexpr int kDecodeWaves = 4;             // target waves of decode CTAs
+constexpr int kMinDecodeSplitBlocks = 64;   // >= 1024 keys per split
 constexpr int kMinChunkSplitBlocks = 16;
 constexpr int kMaxChunkSplitBlocks = 1024;  // chunk kernels stage up to 1024 block ids
 
@@ -446,8 +442,7 @@ int pa_attention_ex(const pa_cache* cache, const void* q, int num_q_heads,
     void* const* ev = opts ? opts->events : nullptr;
     cudaError_t e = cudaSuccess;
     if (pl.decode_max_splits > 1) {
-        e = cudaMemsetAsync(p.split_counters, 0,
-                            static_cast<size_t>(num_tokens) * cache->num_kv_heads * sizeof(int), s);
+        e = pa::launch_zero_counters(p.split_counters, num_tokens * cache->num_kv_heads, s);
         if (e != cudaSuccess) return fail_cuda(e);
     }
     if (pl.num_decode_seqs) {

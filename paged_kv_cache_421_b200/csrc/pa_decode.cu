@@ -19,8 +19,10 @@
 // query rows (GQA group x q_len, padded to 8) on N of an m16n8k16 tile, so a group of 8
 // fills the tile with no padding.  P^T is brought into B-operand layout with movmatrix,
 // and O^T += V^T P^T reads V through ldmatrix.trans.  Softmax runs in the log2 domain.
-// FP8 E4M3 caches are decoded to f16 (exact) in registers; the K scale folds into the score
-// scale and the V scale into the epilogue.
+// FP8 E4M3 caches: S^T = K Q^T runs on FP8 tensor cores from the cache bytes (Q split
+// exactly into two E4M3 terms), and V tiles are stored dim-major so that ldmatrix hands out
+// four consecutive keys per word, decoded to f16 (exact) for O^T += V^T P^T; the K scale
+// folds into the score scale and the V scale into the epilogue.
 #include <cstdlib>
 
 #include "pa_internal.h"
@@ -30,6 +32,16 @@ namespace {
 
 constexpr uint32_t kFull = 0xffffffffu;
 constexpr int kIdsPerRound = 1024;  // block ids staged in shared memory per round
+
+// Key of the block held by row m (0..15) of the S^T = K Q^T tile.  With a bf16 cache rows are
+// keys in order.  With an FP8 cache the rows are permuted so that, after movmatrix, each
+// thread's P^T B fragments hold keys 4t..4t+3 -- the keys that one 32-bit ldmatrix word of a
+// dim-major V tile holds -- so P V needs no byte shuffling.
+template <bool FP8>
+__device__ __forceinline__ int key_of_row(int m) {
+    if constexpr (!FP8) return m;
+    return m < 8 ? 4 * (m >> 1) + (m & 1) : 4 * ((m - 8) >> 1) + 2 + (m & 1);
+}
 
 template <int D, int NW, int NS, bool FP8>
 struct DecodeCfg {
@@ -86,37 +98,81 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
     fence_barrier_init();
 
     // ---- Q^T as B fragments: row n = gq is (token n / group, head g * group + n % group)
+    // bf16 cache: bf16 pairs for m16n8k16.  FP8 cache: S^T = K Q^T runs on FP8 tensor cores
+    // (m16n8k32 E4M3) straight from the cache bytes; each Q row is scaled by a power of two
+    // 2^e and split exactly into two E4M3 terms q1 + q2 (q1 = e4m3(q 2^e), q2 = e4m3 of the
+    // fp32-exact remainder), so the product keeps bf16-level precision; qb[0..3] hold q1 and
+    // qb[4..7] q2 (k-steps of 32 dims).  The row's 2^-e, the K scale and the softmax scale
+    // multiply its scores.
     uint32_t qb[C::kKSteps][2];
+    float sl0 = p.scale_log2, sl1 = p.scale_log2;  // score multipliers of rows 2tq, 2tq+1
     {
         const int n = gq;
         const bool valid = n < rows;
         const __nv_bfloat16* qrow =
             p.q + (static_cast<int64_t>(q0 + (valid ? n / p.group : 0)) * p.num_q_heads +
                    g * p.group + (valid ? n % p.group : 0)) * D;
+        if constexpr (!FP8) {
 #pragma unroll
-        for (int ks = 0; ks < C::kKSteps; ++ks) {
-            if (!valid) {
-                qb[ks][0] = qb[ks][1] = 0u;
-            } else if constexpr (!FP8) {
-                qb[ks][0] = *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * tq);
-                qb[ks][1] = *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * tq + 8);
-            } else {
-                // k-step ks covers dims 16ks..16ks+15 permuted to match the FP8 K fragments:
-                // logical k = 2t+e <-> dim 16ks+4t+e, k = 8+2t+e <-> dim 16ks+4t+2+e.
-                const uint2 raw = *reinterpret_cast<const uint2*>(qrow + 16 * ks + 4 * tq);
-                const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
-                const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
-                qb[ks][0] = pack_f16(__low2float(lo), __high2float(lo));
-                qb[ks][1] = pack_f16(__low2float(hi), __high2float(hi));
+            for (int ks = 0; ks < C::kKSteps; ++ks) {
+                qb[ks][0] = valid ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * tq) : 0u;
+                qb[ks][1] = valid ? *reinterpret_cast<const uint32_t*>(qrow + 16 * ks + 2 * tq + 8) : 0u;
             }
+        } else {
+            constexpr int kSteps32 = D / 32;
+            float qv[kSteps32][8];  // dims 32ks + 16h + 4tq + i, h < 2, i < 4
+            float mx = 0.f;
+#pragma unroll
+            for (int ks = 0; ks < kSteps32; ++ks) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    uint2 raw = make_uint2(0, 0);
+                    if (valid)
+                        raw = *reinterpret_cast<const uint2*>(qrow + 32 * ks + 16 * h + 4 * tq);
+                    const uint32_t w[2] = {raw.x, raw.y};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const uint32_t bits = (i & 1) ? (w[i >> 1] & 0xffff0000u) : (w[i >> 1] << 16);
+                        qv[ks][4 * h + i] = __uint_as_float(bits);
+                        mx = fmaxf(mx, fabsf(qv[ks][4 * h + i]));
+                    }
+                }
+            }
+            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, 2));
+            // largest power of two keeping the row's max |q| at or below 224 (one bit below 448)
+            int e = 0;
+            if (mx > 0.f) e = min(max(static_cast<int>(floorf(log2f(448.f / mx))) - 1, -120), 120);
+            const float up = ldexpf(1.f, e);
+#pragma unroll
+            for (int ks = 0; ks < kSteps32; ++ks) {
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    uint32_t w1 = 0, w2 = 0;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const float x = qv[ks][4 * h + i] * up;
+                        const __nv_fp8_storage_t c1 = __nv_cvt_float_to_fp8(x, __NV_SATFINITE, __NV_E4M3);
+                        const float x1 = __half2float(__half(__nv_cvt_fp8_to_halfraw(c1, __NV_E4M3)));
+                        const __nv_fp8_storage_t c2 =
+                            __nv_cvt_float_to_fp8(x - x1, __NV_SATFINITE, __NV_E4M3);
+                        w1 |= static_cast<uint32_t>(c1) << (8 * i);
+                        w2 |= static_cast<uint32_t>(c2) << (8 * i);
+                    }
+                    qb[ks][h] = w1;
+                    qb[kSteps32 + ks][h] = w2;
+                }
+            }
+            const float rm = ldexpf(1.f, -e) * p.k_scale[g] * p.scale_log2;
+            sl0 = __shfl_sync(kFull, rm, (2 * tq) * 4);      // lanes 4n..4n+3 hold row n
+            sl1 = __shfl_sync(kFull, rm, (2 * tq + 1) * 4);
         }
     }
     // last visible key of the two rows this thread's S/O columns belong to
     const int row0 = 2 * tq, row1 = 2 * tq + 1;
     const int lim0 = row0 < rows ? ctx - q_len + row0 / p.group : ctx - 1;
     const int lim1 = row1 < rows ? ctx - q_len + row1 / p.group : ctx - 1;
-    float sl = p.scale_log2;
-    if constexpr (FP8) sl *= p.k_scale[g];
+    const int lim_min = min(lim0, lim1);
 
     float o[C::kKSteps][4];
 #pragma unroll
@@ -175,15 +231,28 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
             const int kb = (rb + warp + i * NW) * kBlockSize;  // position of the block's key 0
 
             if (kb + kBlockSize > ctx) {
-                // last, partly filled block: clear V rows past the context so that stale
-                // cache bytes (possibly NaN patterns) cannot reach P.V
+                // last, partly filled block: clear V past the context so that stale cache
+                // bytes (possibly NaN patterns) cannot reach P.V
                 const int nz = ctx - kb;
                 uint8_t* vg = smem + (vt - smem_u32(smem));
-                for (int idx = lane; idx < (kBlockSize - nz) * C::kBoxes * 8; idx += 32) {
-                    const int row = nz + idx / (C::kBoxes * 8);
-                    const int c = idx % (C::kBoxes * 8);
-                    *reinterpret_cast<uint4*>(vg + (c >> 3) * 2048 + row * 128 + (c & 7) * 16) =
-                        make_uint4(0, 0, 0, 0);
+                if constexpr (!FP8) {
+                    for (int idx = lane; idx < (kBlockSize - nz) * C::kBoxes * 8; idx += 32) {
+                        const int row = nz + idx / (C::kBoxes * 8);
+                        const int c = idx % (C::kBoxes * 8);
+                        *reinterpret_cast<uint4*>(vg + (c >> 3) * 2048 + row * 128 + (c & 7) * 16) =
+                            make_uint4(0, 0, 0, 0);
+                    }
+                } else {
+                    // dim-major tile: clear bytes nz..15 of every dim's 16-byte row
+                    for (int d = lane; d < D; d += 32) {
+                        uint32_t* row = reinterpret_cast<uint32_t*>(vg + sw128(d >> 3, d & 7));
+#pragma unroll
+                        for (int w = 0; w < 4; ++w) {
+                            const int keep = min(max(nz - 4 * w, 0), 4);  // bytes to keep
+                            const uint32_t mask = keep == 4 ? 0xffffffffu : ((1u << (8 * keep)) - 1u);
+                            row[w] &= mask;
+                        }
+                    }
                 }
                 fence_proxy_async();  // order these writes before the stage's next TMA fill
                 __syncwarp();
@@ -203,28 +272,29 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
                 }
             } else {
 #pragma unroll
-                for (int cp = 0; cp < C::kKSteps / 2; ++cp) {
-                    // matrices: (keys 0-7, chunk 2cp), (keys 8-15, 2cp), (0-7, 2cp+1), (8-15, 2cp+1)
+                for (int ks = 0; ks < D / 32; ++ks) {
+                    // K tile rows are keys with 4 dims per byte group: ldmatrix yields the E4M3
+                    // A fragments directly -- (keys 0-7 | 8-15) x (dims 32ks.. | 32ks+16..)
                     const int mi = lane >> 3, rr = lane & 7;
-                    const int key = rr + ((mi & 1) << 3);
-                    const int chunk = 2 * cp + (mi >> 1);
-                    uint32_t r0, r1, r2, r3;
-                    ldsm_x4(kt + sw128(key, chunk), r0, r1, r2, r3);
-                    mma_f16(s, e4m3x2_to_f16x2(r0 & 0xffff), e4m3x2_to_f16x2(r1 & 0xffff),
-                            e4m3x2_to_f16x2(r0 >> 16), e4m3x2_to_f16x2(r1 >> 16),
-                            qb[2 * cp][0], qb[2 * cp][1]);
-                    mma_f16(s, e4m3x2_to_f16x2(r2 & 0xffff), e4m3x2_to_f16x2(r3 & 0xffff),
-                            e4m3x2_to_f16x2(r2 >> 16), e4m3x2_to_f16x2(r3 >> 16),
-                            qb[2 * cp + 1][0], qb[2 * cp + 1][1]);
+                    const int key = key_of_row<true>(rr + ((mi & 1) << 3));
+                    const int chunk = 2 * ks + (mi >> 1);
+                    uint32_t a0, a1, a2, a3;
+                    ldsm_x4(kt + sw128(key, chunk), a0, a1, a2, a3);
+                    mma_e4m3(s, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
+                    mma_e4m3(s, a0, a1, a2, a3, qb[D / 32 + ks][0], qb[D / 32 + ks][1]);
                 }
             }
 
-            // ---- online softmax over the block's keys (log2 domain)
-            const int p0 = kb + gq, p1 = kb + gq + 8;
-            float x0 = p0 <= lim0 ? s[0] * sl : -INFINITY;
-            float x1 = p0 <= lim1 ? s[1] * sl : -INFINITY;
-            float x2 = p1 <= lim0 ? s[2] * sl : -INFINITY;
-            float x3 = p1 <= lim1 ? s[3] * sl : -INFINITY;
+            // ---- online softmax over the block's keys (log2 domain); blocks whose 16 keys
+            // every row may see skip the mask
+            float x0 = s[0] * sl0, x1 = s[1] * sl1, x2 = s[2] * sl0, x3 = s[3] * sl1;
+            if (kb + kBlockSize - 1 > lim_min) {
+                const int p0 = kb + key_of_row<FP8>(gq), p1 = kb + key_of_row<FP8>(gq + 8);
+                if (p0 > lim0) x0 = -INFINITY;
+                if (p0 > lim1) x1 = -INFINITY;
+                if (p1 > lim0) x2 = -INFINITY;
+                if (p1 > lim1) x3 = -INFINITY;
+            }
             float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
 #pragma unroll
             for (int off = 4; off < 32; off <<= 1) {
@@ -267,29 +337,21 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
                     mma_bf16(o[mt], a0, a1, a2, a3, pb0, pb1);
                 }
             } else {
+                // P^T for keys 4t..4t+3 (the row permutation of S^T) against the dim-major V
+                // tile: one ldmatrix word per dim row holds exactly those four keys
                 const uint32_t pb0 = movmatrix_t(pack_f16(x0, x1));
                 const uint32_t pb1 = movmatrix_t(pack_f16(x2, x3));
-                const uint8_t* vs = smem + (vt - smem_u32(smem));
 #pragma unroll
-                for (int j = 0; j < D / 32; ++j) {
-                    // word w = 8j + gq of key rows 2t, 2t+1, 2t+8, 2t+9 (dims 32j + 4gq .. +3)
-                    const int w = 8 * j + gq;
-                    const int c = w >> 2, wb = (w & 3) * 4;
-                    const uint32_t k0 = *reinterpret_cast<const uint32_t*>(vs + sw128(2 * tq, c) + wb);
-                    const uint32_t k1 = *reinterpret_cast<const uint32_t*>(vs + sw128(2 * tq + 1, c) + wb);
-                    const uint32_t k2 = *reinterpret_cast<const uint32_t*>(vs + sw128(2 * tq + 8, c) + wb);
-                    const uint32_t k3 = *reinterpret_cast<const uint32_t*>(vs + sw128(2 * tq + 9, c) + wb);
-                    // byte pairs (key 2t, key 2t+1) for dims +0,+1 and +2,+3
-                    const uint32_t lo01 = __byte_perm(k0, k1, 0x5140);
-                    const uint32_t hi01 = __byte_perm(k0, k1, 0x7362);
-                    const uint32_t lo23 = __byte_perm(k2, k3, 0x5140);
-                    const uint32_t hi23 = __byte_perm(k2, k3, 0x7362);
-                    // m-tile (j, 0): rows m=g <-> dim +0, m=g+8 <-> dim +1
-                    mma_f16(o[2 * j], e4m3x2_to_f16x2(lo01 & 0xffff), e4m3x2_to_f16x2(lo01 >> 16),
-                            e4m3x2_to_f16x2(lo23 & 0xffff), e4m3x2_to_f16x2(lo23 >> 16), pb0, pb1);
-                    // m-tile (j, 1): m=g <-> dim +2, m=g+8 <-> dim +3
-                    mma_f16(o[2 * j + 1], e4m3x2_to_f16x2(hi01 & 0xffff), e4m3x2_to_f16x2(hi01 >> 16),
-                            e4m3x2_to_f16x2(hi23 & 0xffff), e4m3x2_to_f16x2(hi23 >> 16), pb0, pb1);
+                for (int mp = 0; mp < D / 32; ++mp) {
+                    // matrices: dims 32mp + 8mi .. +7 (16-byte rows = 16 keys each)
+                    const int mi = lane >> 3, rr = lane & 7;
+                    const int d = 32 * mp + 8 * mi + rr;
+                    uint32_t r0, r1, r2, r3;
+                    ldsm_x4(vt + sw128(d >> 3, d & 7), r0, r1, r2, r3);
+                    mma_f16(o[2 * mp], e4m3x2_to_f16x2(r0 & 0xffff), e4m3x2_to_f16x2(r1 & 0xffff),
+                            e4m3x2_to_f16x2(r0 >> 16), e4m3x2_to_f16x2(r1 >> 16), pb0, pb1);
+                    mma_f16(o[2 * mp + 1], e4m3x2_to_f16x2(r2 & 0xffff), e4m3x2_to_f16x2(r3 & 0xffff),
+                            e4m3x2_to_f16x2(r2 >> 16), e4m3x2_to_f16x2(r3 >> 16), pb0, pb1);
                 }
             }
             __syncwarp();
@@ -326,14 +388,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
     }
 #pragma unroll
     for (int mt = 0; mt < C::kKSteps; ++mt) {
-        int d0, d1;
-        if constexpr (!FP8) {
-            d0 = 16 * mt + gq;
-            d1 = d0 + 8;
-        } else {
-            d0 = 32 * (mt >> 1) + 4 * gq + 2 * (mt & 1);
-            d1 = d0 + 1;
-        }
+        const int d0 = 16 * mt + gq, d1 = d0 + 8;
         float* base = red_o + warp * D * 8;
         base[d0 * 8 + row0] = o[mt][0];
         base[d0 * 8 + row1] = o[mt][1];
@@ -450,25 +505,15 @@ cudaError_t launch_decode_t(const CUtensorMap& tmap, const AttnParams& p, int ma
 
 cudaError_t launch_decode(const CUtensorMap& tmap, const AttnParams& p, int head_size,
                           int kv_dtype, int max_splits, cudaStream_t stream) {
-    if (kv_dtype == PA_BF16 && head_size == 128) {
-        static const int stages = [] {
-            const char* v = std::getenv("PA_TUNE_STAGES");
-            return v ? std::atoi(v) : 2;
-        }();
-        if (stages == 3) return launch_decode_t<128, 4, 3, false>(tmap, p, max_splits, stream);
-        return launch_decode_t<128, 4, 2, false>(tmap, p, max_splits, stream);
-    }
+    // 4 warps with a 2-deep ring each (3 CTAs per SM for bf16 by shared memory, for FP8 by
+    // registers) measured fastest at head_size 128: deeper rings cost residency, and capping
+    // FP8 registers for 6 CTAs per SM spilled and ran no faster.
+    if (head_size == 128)
+        return kv_dtype == PA_BF16
+                   ? launch_decode_t<128, 4, 2, false>(tmap, p, max_splits, stream)
+                   : launch_decode_t<128, 4, 2, true>(tmap, p, max_splits, stream);
     if (kv_dtype == PA_BF16 && head_size == 64)
         return launch_decode_t<64, 4, 6, false>(tmap, p, max_splits, stream);
-    if (kv_dtype == PA_FP8_E4M3 && head_size == 128) {
-        static const int variant = [] {
-            const char* v = std::getenv("PA_TUNE_FP8");
-            return v ? std::atoi(v) : 0;
-        }();
-        if (variant == 1) return launch_decode_t<128, 4, 4, true>(tmap, p, max_splits, stream);
-        if (variant == 2) return launch_decode_t<128, 8, 3, true>(tmap, p, max_splits, stream);
-        return launch_decode_t<128, 4, 6, true>(tmap, p, max_splits, stream);
-    }
     return cudaErrorInvalidValue;
 }
 

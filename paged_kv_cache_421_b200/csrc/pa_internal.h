@@ -84,6 +84,7 @@ cudaError_t launch_chunk_tc(const CUtensorMap& tmap, const AttnParams& p, const 
                             int max_splits, cudaStream_t stream);
 cudaError_t launch_reduce(const AttnParams& p, const ChunkList& list, int head_size,
                           cudaStream_t stream);
+cudaError_t launch_zero_counters(int* counters, int n, cudaStream_t stream);
 cudaError_t launch_slot_mapping(const int32_t* block_table, int max_blocks_per_seq,
                                 const int32_t* seq_lens, const int32_t* qsl, int num_seqs,
                                 int num_tokens, int block_size, int32_t* slot_mapping, int* err,

@@ -79,7 +79,20 @@ __global__ void __launch_bounds__(128) reduce_kernel(const AttnParams p,
     }
 }
 
+// Zero the finished-split counters of a launch (part of the same programmatic launch chain).
+__global__ void __launch_bounds__(256) zero_counters_kernel(int* __restrict__ c, int n) {
+    pdl_trigger();
+    pdl_wait();
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += gridDim.x * blockDim.x) c[i] = 0;
+}
+
 }  // namespace
+
+cudaError_t launch_zero_counters(int* counters, int n, cudaStream_t stream) {
+    const int blocks = n < 256 * 148 ? (n + 255) / 256 : 148;
+    return launch_pdl(zero_counters_kernel, dim3(blocks > 0 ? blocks : 1), dim3(256), 0, stream,
+                      counters, n);
+}
 
 cudaError_t launch_reduce(const AttnParams& p, const ChunkList& list, int head_size,
                           cudaStream_t stream) {

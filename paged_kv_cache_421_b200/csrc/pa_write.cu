@@ -8,7 +8,8 @@
 // (token, kv head) row of K and V into its slot of the pool [block][K|V][kv head][16][D].
 // One thread moves 16 bytes of bf16 input; consecutive threads cover consecutive bytes of a
 // row, so both the reads of k/v and the writes into the pool are coalesced.  An FP8 pool
-// stores e4m3(x / scale[head]) with an IEEE-rounded fp32 divide and saturating conversion.
+// stores e4m3(x / scale[head]) with an IEEE-rounded fp32 divide and saturating conversion;
+// its V tiles are dim-major, so V bytes are scattered with a 16-byte stride.
 #include "pa_internal.h"
 
 namespace pa {
@@ -83,10 +84,19 @@ write_kv_kernel(uint8_t* __restrict__ cache, const uint16_t* __restrict__ k,
                 float2 y = make_float2(__fdiv_rn(lo, s), __fdiv_rn(hi, s));
                 out[j] = static_cast<uint16_t>(__nv_cvt_float2_to_fp8x2(y, __NV_SATFINITE, __NV_E4M3));
             }
-            uint2 packed;
-            packed.x = static_cast<uint32_t>(out[0]) | (static_cast<uint32_t>(out[1]) << 16);
-            packed.y = static_cast<uint32_t>(out[2]) | (static_cast<uint32_t>(out[3]) << 16);
-            *reinterpret_cast<uint2*>(cache + dst) = packed;
+            if (kv == 0) {
+                uint2 packed;
+                packed.x = static_cast<uint32_t>(out[0]) | (static_cast<uint32_t>(out[1]) << 16);
+                packed.y = static_cast<uint32_t>(out[2]) | (static_cast<uint32_t>(out[3]) << 16);
+                *reinterpret_cast<uint2*>(cache + dst) = packed;
+            } else {
+                // FP8 V tiles are dim-major: dim d of token o sits at byte d * 16 + o of the tile
+                uint8_t* tile = cache + (dst - (slot % kBlockSize) * D - c * 8);
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    tile[(c * 8 + j) * kBlockSize + slot % kBlockSize] =
+                        static_cast<uint8_t>(out[j >> 1] >> (8 * (j & 1)));
+            }
         }
     }
 }

@@ -37,7 +37,9 @@ class PagedKVCache:
         return self.buffer.numel()
 
     def view(self) -> torch.Tensor:
-        """The pool as [num_blocks, 2, num_kv_heads, block_size, head_size] (bf16 or uint8)."""
+        """The pool as [num_blocks, 2, num_kv_heads, block_size, head_size] (bf16 or uint8).
+        For an FP8 pool the V tiles ([:, 1]) are dim-major: read them as
+        ``view()[:, 1].reshape(num_blocks, num_kv_heads, head_size, block_size)``."""
         dt = torch.bfloat16 if self.kv_dtype == B.PA_BF16 else torch.uint8
         return self.buffer.view(dt).view(self.num_blocks, 2, self.num_kv_heads, self.block_size,
                                          self.head_size)

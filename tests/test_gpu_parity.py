@@ -81,14 +81,27 @@ def test_cache_write_bit_exact_sampled(name):
     vs = None if wl.v_scale is None else wl.v_scale.numpy()
     oracle.write_kv(scratch, wl.kv_dtype, nb, 16, wl.num_kv_heads, wl.head_size, W.bits(rows_k),
                     W.bits(rows_v), np.arange(n, dtype=np.int32), ks, vs)
-    scratch = scratch.reshape(nb, 2, wl.num_kv_heads, 16, wl.head_size)
-    view = st.cache.view()
-    got = view.view(torch.int16) if wl.kv_dtype == W.BF16 else view
+    def rows_of(tiles, n_tok):
+        """[blocks][2][Hkv][tile] -> per slot [2][Hkv][D] (K token-major; FP8 V dim-major)."""
+        k = tiles[:, 0].reshape(-1, wl.num_kv_heads, 16, wl.head_size)
+        if wl.kv_dtype == W.BF16:
+            v = tiles[:, 1].reshape(-1, wl.num_kv_heads, 16, wl.head_size)
+        else:
+            v = tiles[:, 1].reshape(-1, wl.num_kv_heads, wl.head_size, 16).transpose(0, 1, 3, 2)
+        return k, v
+
+    ks_, vs_ = rows_of(scratch.reshape(nb, 2, wl.num_kv_heads, 16 * wl.head_size), n)
+    want_k = ks_.transpose(0, 2, 1, 3).reshape(nb * 16, wl.num_kv_heads, wl.head_size)[:n]
+    want_v = vs_.transpose(0, 2, 1, 3).reshape(nb * 16, wl.num_kv_heads, wl.head_size)[:n]
+    raw = st.cache.buffer.view(torch.int16 if wl.kv_dtype == W.BF16 else torch.uint8)
+    tiles = raw.view(wl.num_blocks, 2, wl.num_kv_heads, 16 * wl.head_size)
     idx_b = torch.from_numpy(slots // 16).cuda()
-    idx_o = torch.from_numpy(slots % 16).cuda()
-    gathered = got[idx_b, :, :, idx_o, :].cpu().numpy().view(dt)  # [n, 2, Hkv, D]
-    want = scratch.transpose(0, 3, 1, 2, 4).reshape(nb * 16, 2, wl.num_kv_heads, wl.head_size)[:n]
-    assert np.array_equal(gathered, want)
+    idx_o = slots % 16
+    sel = tiles[idx_b].cpu().numpy().view(dt)  # [n, 2, Hkv, tile]
+    gk, gv = rows_of(sel, n)
+    ar = np.arange(n)
+    assert np.array_equal(gk[ar, :, idx_o, :], want_k)
+    assert np.array_equal(gv[ar, :, idx_o, :], want_v)
 
 
 def test_fp8_write_divides_at_ties():

@@ -220,8 +220,9 @@ def test_write_skips_negative_slots(oracle_mod):
 
 
 def test_write_fp8_vs_torch_codec(oracle_mod):
+    # FP8 pools keep K tiles token-major ([tok][d]) and V tiles dim-major ([d][tok])
     wl = W.make_workload("t", [9, 30], [9, 4], 4, 2, 8, 4, 32, 5, kv_dtype=W.FP8_E4M3)
-    cache = _oracle_cache(oracle_mod, wl).reshape(32, 2, 2, 4, 8)
+    tiles = _oracle_cache(oracle_mod, wl).reshape(32, 2, 2, 4 * 8)
     k_src, v_src = wl.kv_src()
     for r in range(wl.num_seqs):
         for p in range(int(wl.seq_lens[r])):
@@ -231,7 +232,9 @@ def test_write_fp8_vs_torch_codec(oracle_mod):
             for kv, src, sc in [(0, k_src, wl.k_scale), (1, v_src, wl.v_scale)]:
                 y = (src[row].float() / sc[:, None])  # fp32 IEEE division, per kv head
                 ref = y.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
-                assert np.array_equal(cache[b, kv, :, o, :], ref)
+                got = tiles[b, 0].reshape(2, 4, 8)[:, o, :] if kv == 0 else \
+                    tiles[b, 1].reshape(2, 8, 4)[:, :, o]
+                assert np.array_equal(got, ref)
 
 
 # ------------------------------------------------------------------ attention
