@@ -93,6 +93,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t phase) {
     return ok != 0;
 }
 
+// As mbar_try_wait, but the thread may stay suspended inside the instruction for up to
+// `hint_ns` until the phase completes, so a waiting warp issues almost nothing.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint32_t bar, uint32_t phase,
+                                                    uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(phase), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 __device__ __forceinline__ uint64_t global_timer_ns() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -106,7 +121,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t phase, uint64_t
                                           int* err) {
     if (mbar_try_wait(bar, phase)) return true;
     const uint64_t t0 = global_timer_ns();
-    while (!mbar_try_wait(bar, phase)) {
+    while (!mbar_try_wait_sleep(bar, phase, 1000000u)) {
         if (global_timer_ns() - t0 > limit_ns) {
             raise_error(err, kErrWaitTimeout);
             return false;
@@ -204,6 +219,17 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t two) {
     __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two), __NV_E4M3);
     return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+}
+
+// Four E4M3 codes (bytes b0..b3 of r) -> two f16x2 words holding 2^-8 times their values,
+// exactly: an E4M3 code's sign goes to bit 15 and its 4 exponent + 3 mantissa bits to bits
+// 7..13 of an f16, which reads the same exponent field with bias 15 instead of 7 (subnormals
+// line up the same way).  even = (b0, b2), odd = (b1, b3).  The NaN codes 0x7f / 0xff come
+// out as the finite 2^-8 * 480; cache writes saturate, so they never hold them.
+__device__ __forceinline__ void e4m3x4_to_f16x2_scaled(uint32_t r, uint32_t& even,
+                                                       uint32_t& odd) {
+    even = ((r << 7) & 0x3f803f80u) | ((r << 8) & 0x80008000u);
+    odd = ((r >> 1) & 0x3f803f80u) | (r & 0x80008000u);
 }
 
 __device__ __forceinline__ float fast_exp2(float x) { return exp2f(x); }

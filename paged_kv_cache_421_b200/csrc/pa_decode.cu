@@ -34,13 +34,14 @@ constexpr uint32_t kFull = 0xffffffffu;
 constexpr int kIdsPerRound = 1024;  // block ids staged in shared memory per round
 
 // Key of the block held by row m (0..15) of the S^T = K Q^T tile.  With a bf16 cache rows are
-// keys in order.  With an FP8 cache the rows are permuted so that, after movmatrix, each
-// thread's P^T B fragments hold keys 4t..4t+3 -- the keys that one 32-bit ldmatrix word of a
-// dim-major V tile holds -- so P V needs no byte shuffling.
+// keys in order.  With an FP8 cache the rows are permuted so that, after movmatrix, thread
+// t's P^T B fragments hold keys (4t, 4t+2) and (4t+1, 4t+3): one 32-bit ldmatrix word of a
+// dim-major V tile holds keys 4t..4t+3, and widening it to f16 splits it into the even and
+// the odd bytes, so P V needs no byte shuffling.
 template <bool FP8>
 __device__ __forceinline__ int key_of_row(int m) {
     if constexpr (!FP8) return m;
-    return m < 8 ? 4 * (m >> 1) + (m & 1) : 4 * ((m - 8) >> 1) + 2 + (m & 1);
+    return m < 8 ? 4 * (m >> 1) + 2 * (m & 1) : 4 * ((m - 8) >> 1) + 1 + 2 * (m & 1);
 }
 
 template <int D, int NW, int NS, bool FP8>
@@ -348,10 +349,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
                     const int d = 32 * mp + 8 * mi + rr;
                     uint32_t r0, r1, r2, r3;
                     ldsm_x4(vt + sw128(d >> 3, d & 7), r0, r1, r2, r3);
-                    mma_f16(o[2 * mp], e4m3x2_to_f16x2(r0 & 0xffff), e4m3x2_to_f16x2(r1 & 0xffff),
-                            e4m3x2_to_f16x2(r0 >> 16), e4m3x2_to_f16x2(r1 >> 16), pb0, pb1);
-                    mma_f16(o[2 * mp + 1], e4m3x2_to_f16x2(r2 & 0xffff), e4m3x2_to_f16x2(r3 & 0xffff),
-                            e4m3x2_to_f16x2(r2 >> 16), e4m3x2_to_f16x2(r3 >> 16), pb0, pb1);
+                    uint32_t e0, d0, e1, d1, e2, d2, e3, d3;  // (even, odd) byte pairs, 2^-8 V
+                    e4m3x4_to_f16x2_scaled(r0, e0, d0);
+                    e4m3x4_to_f16x2_scaled(r1, e1, d1);
+                    e4m3x4_to_f16x2_scaled(r2, e2, d2);
+                    e4m3x4_to_f16x2_scaled(r3, e3, d3);
+                    mma_f16(o[2 * mp], e0, e1, d0, d1, pb0, pb1);
+                    mma_f16(o[2 * mp + 1], e2, e3, d2, d3, pb0, pb1);
                 }
             }
             __syncwarp();
@@ -397,7 +401,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
     }
     if (!__syncthreads_and(ok)) return;
 
-    const float vscale = FP8 ? p.v_scale[g] : 1.f;
+    const float vscale = FP8 ? 256.f * p.v_scale[g] : 1.f;  // FP8 V was widened as 2^-8 V
     const bool direct = nsplit == 1;
     if (!direct && split >= p.max_splits) {  // workspace bound (a planned launch never hits it)
         if (tid == 0) raise_error(p.err, kErrMetadata);
