@@ -215,17 +215,11 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
-// Two E4M3 codes (low byte first) -> f16x2, exact.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t two) {
-    __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two), __NV_E4M3);
-    return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
-}
-
 // Four E4M3 codes (bytes b0..b3 of r) -> two f16x2 words holding 2^-8 times their values,
 // exactly: an E4M3 code's sign goes to bit 15 and its 4 exponent + 3 mantissa bits to bits
 // 7..13 of an f16, which reads the same exponent field with bias 15 instead of 7 (subnormals
-// line up the same way).  even = (b0, b2), odd = (b1, b3).  The NaN codes 0x7f / 0xff come
-// out as the finite 2^-8 * 480; cache writes saturate, so they never hold them.
+// line up the same way).  even = (b0, b2), odd = (b1, b3).  Every byte widens to a finite
+// value (the NaN codes 0x7f / 0xff give 2^-8 * 480), so stale bytes times P = 0 stay 0.
 __device__ __forceinline__ void e4m3x4_to_f16x2_scaled(uint32_t r, uint32_t& even,
                                                        uint32_t& odd) {
     even = ((r << 7) & 0x3f803f80u) | ((r << 8) & 0x80008000u);

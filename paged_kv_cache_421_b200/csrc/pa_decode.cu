@@ -50,7 +50,10 @@ struct DecodeCfg {
     static constexpr int kBoxes = D * kEsz / 128;          // 128-byte column slabs per row
     static constexpr int kBoxElems = 128 / kEsz;
     static constexpr int kTileBytes = kBlockSize * D * kEsz;  // one (block, K|V, head) tile
-    static constexpr int kStageBytes = 2 * kTileBytes;
+    // Blocks a warp takes per softmax step: two for FP8, so that a step moves as many bytes
+    // as one bf16 block and the per-step softmax cost is spread over 32 keys.
+    static constexpr int kBpu = FP8 ? 2 : 1;
+    static constexpr int kStageBytes = kBpu * 2 * kTileBytes;
     static constexpr int kRingBytes = NW * NS * kStageBytes;
     static constexpr int kMergeBytes = NW * (kDecodeRows * D + 2 * kDecodeRows) * 4;
     static constexpr int kSmemBytes =
@@ -59,7 +62,7 @@ struct DecodeCfg {
 };
 
 template <int D, int NW, int NS, bool FP8>
-__global__ void __launch_bounds__(NW * 32)
+__global__ void __launch_bounds__(NW * 32, 3)
 decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
     using C = DecodeCfg<D, NW, NS, FP8>;
     pdl_trigger();
@@ -197,20 +200,28 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
             ids[k] = b;
         }
         __syncthreads();
-        const int mine = (ok && rn > warp) ? (rn - warp + NW - 1) / NW : 0;
+        // a unit is kBpu consecutive blocks of the round; warp w takes units w, w + NW, ...
+        constexpr int BPU = C::kBpu;
+        const int units = (rn + BPU - 1) / BPU;
+        const int mine = (ok && units > warp) ? (units - warp + NW - 1) / NW : 0;
+        const int kend = (rb + rn) * kBlockSize;  // first position past this round's blocks
 
         auto issue = [&](int i, uint32_t n) {
-            const int blk = ids[warp + i * NW];
+            const int u0 = (warp + i * NW) * BPU;  // round index of the unit's first block
+            const int nb = min(BPU, rn - u0);
             const uint32_t st = n % NS;
             const uint32_t bar = smem_u32(&bars[warp * NS + st]);
             const uint32_t dst = ring + st * C::kStageBytes;
-            const int rowk = blk * kv_rows_per_block + g * kBlockSize;
-            const int rowv = rowk + p.num_kv_heads * kBlockSize;
-            mbar_arrive_expect_tx(bar, C::kStageBytes);
+            mbar_arrive_expect_tx(bar, nb * 2 * C::kTileBytes);
+            for (int h = 0; h < nb; ++h) {
+                const int rowk = ids[u0 + h] * kv_rows_per_block + g * kBlockSize;
+                const int rowv = rowk + p.num_kv_heads * kBlockSize;
+                const uint32_t dk = dst + h * 2 * C::kTileBytes;
 #pragma unroll
-            for (int b = 0; b < C::kBoxes; ++b) {
-                tma_load_2d(dst + b * 2048, &tmap, bar, b * C::kBoxElems, rowk);
-                tma_load_2d(dst + C::kTileBytes + b * 2048, &tmap, bar, b * C::kBoxElems, rowv);
+                for (int b = 0; b < C::kBoxes; ++b) {
+                    tma_load_2d(dk + b * 2048, &tmap, bar, b * C::kBoxElems, rowk);
+                    tma_load_2d(dk + C::kTileBytes + b * 2048, &tmap, bar, b * C::kBoxElems, rowv);
+                }
             }
         };
 
@@ -227,76 +238,83 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
                 fail_i = i;
                 break;
             }
-            const uint32_t kt = ring + st * C::kStageBytes;
-            const uint32_t vt = kt + C::kTileBytes;
-            const int kb = (rb + warp + i * NW) * kBlockSize;  // position of the block's key 0
+            const uint32_t stage = ring + st * C::kStageBytes;
+            const int kb = (rb + (warp + i * NW) * BPU) * kBlockSize;  // position of key 0
 
-            if (kb + kBlockSize > ctx) {
-                // last, partly filled block: clear V past the context so that stale cache
-                // bytes (possibly NaN patterns) cannot reach P.V
-                const int nz = ctx - kb;
-                uint8_t* vg = smem + (vt - smem_u32(smem));
-                if constexpr (!FP8) {
+            if constexpr (!FP8) {
+                if (kb + kBlockSize > ctx) {
+                    // last, partly filled block: clear V past the context so that stale cache
+                    // bytes (possibly NaN patterns) cannot reach P.V.  FP8 V needs no clearing:
+                    // its f16 widening is finite for every byte, and masked keys get P = 0.
+                    const int nz = ctx - kb;
+                    uint8_t* vg = smem + (stage + C::kTileBytes - smem_u32(smem));
                     for (int idx = lane; idx < (kBlockSize - nz) * C::kBoxes * 8; idx += 32) {
                         const int row = nz + idx / (C::kBoxes * 8);
                         const int c = idx % (C::kBoxes * 8);
                         *reinterpret_cast<uint4*>(vg + (c >> 3) * 2048 + row * 128 + (c & 7) * 16) =
                             make_uint4(0, 0, 0, 0);
                     }
-                } else {
-                    // dim-major tile: clear bytes nz..15 of every dim's 16-byte row
-                    for (int d = lane; d < D; d += 32) {
-                        uint32_t* row = reinterpret_cast<uint32_t*>(vg + sw128(d >> 3, d & 7));
+                    fence_proxy_async();  // order these writes before the stage's next TMA fill
+                    __syncwarp();
+                }
+            }
+
+            // ---- S^T (16 keys x 8 rows per block) = K Q^T
+            float x[BPU][4];
 #pragma unroll
-                        for (int w = 0; w < 4; ++w) {
-                            const int keep = min(max(nz - 4 * w, 0), 4);  // bytes to keep
-                            const uint32_t mask = keep == 4 ? 0xffffffffu : ((1u << (8 * keep)) - 1u);
-                            row[w] &= mask;
-                        }
+            for (int h = 0; h < BPU; ++h) {
+                const uint32_t kt = stage + h * 2 * C::kTileBytes;
+                float s[4] = {0.f, 0.f, 0.f, 0.f};
+                if constexpr (!FP8) {
+#pragma unroll
+                    for (int ks = 0; ks < C::kKSteps; ++ks) {
+                        const int mi = lane >> 3, rr = lane & 7;
+                        const int key = rr + ((mi & 1) << 3);
+                        const int chunk = 2 * ks + (mi >> 1);
+                        uint32_t a0, a1, a2, a3;
+                        ldsm_x4(kt + (chunk >> 3) * 2048 + sw128(key, chunk & 7), a0, a1, a2, a3);
+                        mma_bf16(s, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
+                    }
+                } else {
+#pragma unroll
+                    for (int ks = 0; ks < D / 32; ++ks) {
+                        // K tile rows are keys with 4 dims per byte group: ldmatrix yields the
+                        // E4M3 A fragments directly -- (keys 0-7 | 8-15) x (dims 32ks.. | +16..)
+                        const int mi = lane >> 3, rr = lane & 7;
+                        const int key = key_of_row<true>(rr + ((mi & 1) << 3));
+                        const int chunk = 2 * ks + (mi >> 1);
+                        uint32_t a0, a1, a2, a3;
+                        ldsm_x4(kt + sw128(key, chunk), a0, a1, a2, a3);
+                        mma_e4m3(s, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
+                        mma_e4m3(s, a0, a1, a2, a3, qb[D / 32 + ks][0], qb[D / 32 + ks][1]);
                     }
                 }
-                fence_proxy_async();  // order these writes before the stage's next TMA fill
-                __syncwarp();
+                x[h][0] = s[0] * sl0;
+                x[h][1] = s[1] * sl1;
+                x[h][2] = s[2] * sl0;
+                x[h][3] = s[3] * sl1;
             }
 
-            // ---- S^T (16 keys x 8 rows) = K Q^T
-            float s[4] = {0.f, 0.f, 0.f, 0.f};
-            if constexpr (!FP8) {
+            // ---- online softmax over the unit's keys (log2 domain).  Units whose keys every
+            // row may see skip the mask; a key past the round's blocks (the missing second
+            // block of a unit) is masked like a future key.
+            if (kb + BPU * kBlockSize - 1 > min(lim_min, kend - 1)) {
 #pragma unroll
-                for (int ks = 0; ks < C::kKSteps; ++ks) {
-                    const int mi = lane >> 3, rr = lane & 7;
-                    const int key = rr + ((mi & 1) << 3);
-                    const int chunk = 2 * ks + (mi >> 1);
-                    uint32_t a0, a1, a2, a3;
-                    ldsm_x4(kt + (chunk >> 3) * 2048 + sw128(key, chunk & 7), a0, a1, a2, a3);
-                    mma_bf16(s, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
-                }
-            } else {
-#pragma unroll
-                for (int ks = 0; ks < D / 32; ++ks) {
-                    // K tile rows are keys with 4 dims per byte group: ldmatrix yields the E4M3
-                    // A fragments directly -- (keys 0-7 | 8-15) x (dims 32ks.. | 32ks+16..)
-                    const int mi = lane >> 3, rr = lane & 7;
-                    const int key = key_of_row<true>(rr + ((mi & 1) << 3));
-                    const int chunk = 2 * ks + (mi >> 1);
-                    uint32_t a0, a1, a2, a3;
-                    ldsm_x4(kt + sw128(key, chunk), a0, a1, a2, a3);
-                    mma_e4m3(s, a0, a1, a2, a3, qb[ks][0], qb[ks][1]);
-                    mma_e4m3(s, a0, a1, a2, a3, qb[D / 32 + ks][0], qb[D / 32 + ks][1]);
+                for (int h = 0; h < BPU; ++h) {
+                    const int p0 = kb + h * kBlockSize + key_of_row<FP8>(gq);
+                    const int p1 = kb + h * kBlockSize + key_of_row<FP8>(gq + 8);
+                    if (p0 > lim0 || p0 >= kend) x[h][0] = -INFINITY;
+                    if (p0 > lim1 || p0 >= kend) x[h][1] = -INFINITY;
+                    if (p1 > lim0 || p1 >= kend) x[h][2] = -INFINITY;
+                    if (p1 > lim1 || p1 >= kend) x[h][3] = -INFINITY;
                 }
             }
-
-            // ---- online softmax over the block's keys (log2 domain); blocks whose 16 keys
-            // every row may see skip the mask
-            float x0 = s[0] * sl0, x1 = s[1] * sl1, x2 = s[2] * sl0, x3 = s[3] * sl1;
-            if (kb + kBlockSize - 1 > lim_min) {
-                const int p0 = kb + key_of_row<FP8>(gq), p1 = kb + key_of_row<FP8>(gq + 8);
-                if (p0 > lim0) x0 = -INFINITY;
-                if (p0 > lim1) x1 = -INFINITY;
-                if (p1 > lim0) x2 = -INFINITY;
-                if (p1 > lim1) x3 = -INFINITY;
+            float mx0 = fmaxf(x[0][0], x[0][2]), mx1 = fmaxf(x[0][1], x[0][3]);
+#pragma unroll
+            for (int h = 1; h < BPU; ++h) {
+                mx0 = fmaxf(mx0, fmaxf(x[h][0], x[h][2]));
+                mx1 = fmaxf(mx1, fmaxf(x[h][1], x[h][3]));
             }
-            float mx0 = fmaxf(x0, x2), mx1 = fmaxf(x1, x3);
 #pragma unroll
             for (int off = 4; off < 32; off <<= 1) {
                 mx0 = fmaxf(mx0, __shfl_xor_sync(kFull, mx0, off));
@@ -306,12 +324,18 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
             const float ref0 = mn0 == -INFINITY ? 0.f : mn0;
             const float ref1 = mn1 == -INFINITY ? 0.f : mn1;
             const float al0 = fast_exp2(m0 - ref0), al1 = fast_exp2(m1 - ref1);
-            x0 = fast_exp2(x0 - ref0);
-            x2 = fast_exp2(x2 - ref0);
-            x1 = fast_exp2(x1 - ref1);
-            x3 = fast_exp2(x3 - ref1);
-            l0 = l0 * al0 + x0 + x2;
-            l1 = l1 * al1 + x1 + x3;
+            float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+            for (int h = 0; h < BPU; ++h) {
+                x[h][0] = fast_exp2(x[h][0] - ref0);
+                x[h][2] = fast_exp2(x[h][2] - ref0);
+                x[h][1] = fast_exp2(x[h][1] - ref1);
+                x[h][3] = fast_exp2(x[h][3] - ref1);
+                sum0 += x[h][0] + x[h][2];
+                sum1 += x[h][1] + x[h][3];
+            }
+            l0 = l0 * al0 + sum0;
+            l1 = l1 * al1 + sum1;
             m0 = mn0;
             m1 = mn1;
             if (__any_sync(kFull, al0 != 1.f || al1 != 1.f)) {
@@ -326,8 +350,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
 
             // ---- O^T (D x 8) += V^T P^T
             if constexpr (!FP8) {
-                const uint32_t pb0 = movmatrix_t(pack_bf16(x0, x1));
-                const uint32_t pb1 = movmatrix_t(pack_bf16(x2, x3));
+                const uint32_t vt = stage + C::kTileBytes;
+                const uint32_t pb0 = movmatrix_t(pack_bf16(x[0][0], x[0][1]));
+                const uint32_t pb1 = movmatrix_t(pack_bf16(x[0][2], x[0][3]));
 #pragma unroll
                 for (int mt = 0; mt < C::kKSteps; ++mt) {
                     const int mi = lane >> 3, rr = lane & 7;
@@ -338,24 +363,28 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
                     mma_bf16(o[mt], a0, a1, a2, a3, pb0, pb1);
                 }
             } else {
-                // P^T for keys 4t..4t+3 (the row permutation of S^T) against the dim-major V
-                // tile: one ldmatrix word per dim row holds exactly those four keys
-                const uint32_t pb0 = movmatrix_t(pack_f16(x0, x1));
-                const uint32_t pb1 = movmatrix_t(pack_f16(x2, x3));
+                // P^T for keys (4t, 4t+2 | 4t+1, 4t+3) (the row permutation of S^T) against the
+                // dim-major V tile: one ldmatrix word per dim row holds keys 4t..4t+3, widened
+                // exactly to f16 (as 2^-8 V) in an even and an odd half
 #pragma unroll
-                for (int mp = 0; mp < D / 32; ++mp) {
-                    // matrices: dims 32mp + 8mi .. +7 (16-byte rows = 16 keys each)
-                    const int mi = lane >> 3, rr = lane & 7;
-                    const int d = 32 * mp + 8 * mi + rr;
-                    uint32_t r0, r1, r2, r3;
-                    ldsm_x4(vt + sw128(d >> 3, d & 7), r0, r1, r2, r3);
-                    uint32_t e0, d0, e1, d1, e2, d2, e3, d3;  // (even, odd) byte pairs, 2^-8 V
-                    e4m3x4_to_f16x2_scaled(r0, e0, d0);
-                    e4m3x4_to_f16x2_scaled(r1, e1, d1);
-                    e4m3x4_to_f16x2_scaled(r2, e2, d2);
-                    e4m3x4_to_f16x2_scaled(r3, e3, d3);
-                    mma_f16(o[2 * mp], e0, e1, d0, d1, pb0, pb1);
-                    mma_f16(o[2 * mp + 1], e2, e3, d2, d3, pb0, pb1);
+                for (int h = 0; h < BPU; ++h) {
+                    const uint32_t vt = stage + (2 * h + 1) * C::kTileBytes;
+                    const uint32_t pb0 = movmatrix_t(pack_f16(x[h][0], x[h][1]));
+                    const uint32_t pb1 = movmatrix_t(pack_f16(x[h][2], x[h][3]));
+#pragma unroll
+                    for (int mp = 0; mp < D / 32; ++mp) {
+                        const int mi = lane >> 3, rr = lane & 7;
+                        const int d = 32 * mp + 8 * mi + rr;
+                        uint32_t r0, r1, r2, r3;
+                        ldsm_x4(vt + sw128(d >> 3, d & 7), r0, r1, r2, r3);
+                        uint32_t e0, d0, e1, d1, e2, d2, e3, d3;
+                        e4m3x4_to_f16x2_scaled(r0, e0, d0);
+                        e4m3x4_to_f16x2_scaled(r1, e1, d1);
+                        e4m3x4_to_f16x2_scaled(r2, e2, d2);
+                        e4m3x4_to_f16x2_scaled(r3, e3, d3);
+                        mma_f16(o[2 * mp], e0, e1, d0, d1, pb0, pb1);
+                        mma_f16(o[2 * mp + 1], e2, e3, d2, d3, pb0, pb1);
+                    }
                 }
             }
             __syncwarp();
