@@ -291,10 +291,11 @@ class DeviceStep:
         torch.cuda.synchronize(device)
 
     def launches_per_step(self) -> int:
-        """Kernels of ours per step: slot mapping, write, decode and/or chunk, chunk reduce."""
+        """Kernels of ours per step: slot mapping, write, the split-counter clear (split
+        decode), decode and/or chunk, chunk reduce."""
         p = self.plan
-        return 2 + (p["num_decode_seqs"] > 0) + (p["num_chunk_seqs"] > 0) + \
-            int(p["chunk_max_splits"] > 1)
+        return 2 + int(p["decode_max_splits"] > 1) + (p["num_decode_seqs"] > 0) + \
+            (p["num_chunk_seqs"] > 0) + int(p["chunk_max_splits"] > 1)
 
     def run(self, events=None, q=None, k=None, v=None, bt=None, sl=None, qsl=None):
         B = self.ops.B
