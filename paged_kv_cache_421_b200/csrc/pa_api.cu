@@ -4,6 +4,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <algorithm>
+#include <vector>
 #include <new>
 
 #include "pa_internal.h"
@@ -98,6 +99,18 @@ int make_tensor_map(pa_cache* c) {
                      CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail_cuda(cudaErrorInvalidValue);
+    if (c->kv_dtype == PA_BF16 && c->head_size == 128) {
+        // 4-D view for whole-tile loads: (64 elements, 8 rows, 2 halves, 8-row groups), so
+        // that one 4 KB box lands a 16-token tile as [group][half][8 rows][128 B]
+        cuuint64_t dims4[4] = {64, 8, 2, rows / 8};
+        cuuint64_t strides4[3] = {256, 128, 2048};
+        cuuint32_t box4[4] = {64, 8, 2, 2};
+        cuuint32_t estr4[4] = {1, 1, 1, 1};
+        r = enc(&c->tmap_blk, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, c->data, dims4, strides4, box4,
+                estr4, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) return fail_cuda(cudaErrorInvalidValue);
+    }
     return PA_OK;
 }
 
@@ -130,6 +143,7 @@ constexpr int kMaxDecodeSplits = 1024;  // merge weights of one row fit the CTA'
 constexpr int kDecodeWaves = 4;             // target waves of decode CTAs
 constexpr int kMinDecodeSplitBlocks = 64;   // >= 1024 keys per split
 constexpr int kMinChunkSplitBlocks = 16;
+constexpr int kMinChunkSplitTiles = 4;      // a chunk split walks at least four key tiles
 constexpr int kMaxChunkSplitBlocks = 1024;  // chunk kernels stage up to 1024 block ids
 
 int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int Hkv, int D,
@@ -147,7 +161,10 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
     if (B > 0 && qsl[0] != 0) return PA_ERR_METADATA;
     long long dec_units = 0;
     int dec_max_blocks = 0, chunk_max_blocks = 0, chunk_max_qtiles = 0;
-    long long chunk_tiles = 0;
+    // chunk work in key tiles: the CTA of each q-tile walks the keys its last row may see
+    const int chunk_cta_rows = pa::chunk_rows(D, 1);
+    const int chunk_tile_keys = D == 128 ? 128 : 64;
+    long long chunk_work = 0, chunk_work_max = 0;
     for (int r = 0; r < B; ++r) {
         const int ql = qsl[r + 1] - qsl[r];
         const int ctx = sl[r];
@@ -161,10 +178,15 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
             if (blocks > dec_max_blocks) dec_max_blocks = blocks;
         } else {
             pl->num_chunk_seqs++;
-            const int qt = pa::ceil_div(ql * G, pa::chunk_rows(D, 1));
+            const int qt = pa::ceil_div(ql * G, chunk_cta_rows);
             if (qt > chunk_max_qtiles) chunk_max_qtiles = qt;
-            chunk_tiles += static_cast<long long>(qt) * Hkv;
             if (blocks > chunk_max_blocks) chunk_max_blocks = blocks;
+            for (int i = 0; i < qt; ++i) {
+                const int last_row = std::min((i + 1) * chunk_cta_rows, ql * G) - 1;
+                const long long w = pa::ceil_div(ctx - ql + last_row / G + 1, chunk_tile_keys);
+                chunk_work += w * Hkv;
+                if (w > chunk_work_max) chunk_work_max = w;
+            }
         }
     }
     if (B > 0 && qsl[B] != T) return PA_ERR_METADATA;
@@ -201,12 +223,14 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
             if (csb > kMaxChunkSplitBlocks && allowed > 1)  // keep block ids in shared memory
                 csb = round_up(pa::ceil_div(chunk_max_blocks,
                                             pa::ceil_div(chunk_max_blocks, kMaxChunkSplitBlocks)), 4);
-            // split only when the chunk CTAs would leave most of the GPU idle
-            if (2 * chunk_tiles <= num_sms && chunk_max_blocks >= 2 * kMinChunkSplitBlocks) {
-                const long long want = (2LL * num_sms + chunk_tiles - 1) / chunk_tiles;
-                int sb = pa::ceil_div(chunk_max_blocks, static_cast<int>(want));
-                if (sb < kMinChunkSplitBlocks) sb = kMinChunkSplitBlocks;
-                csb = round_up(sb, 4);
+            // one CTA per SM: split the KV walk when the longest CTA would walk well past the
+            // average work per SM, so that no SM is left with most of the step
+            const long long per_sm = (chunk_work + num_sms - 1) / num_sms;
+            const long long target = std::max<long long>(per_sm, kMinChunkSplitTiles);
+            if (chunk_work_max > target + target / 2) {
+                const int tile_blocks = chunk_tile_keys / bs;
+                const int sb = static_cast<int>(target) * tile_blocks;
+                if (sb < csb) csb = round_up(std::max(sb, kMinChunkSplitBlocks), 4);
             }
         }
         int ns = pa::ceil_div(chunk_max_blocks, csb);
@@ -466,9 +490,49 @@ int pa_attention_ex(const pa_cache* cache, const void* q, int num_q_heads,
                 return seq_lens_host[a] > seq_lens_host[b];
             });
         }
+        // the chunk CTAs, most key tiles first; a list that does not fit falls back to the grid
+        static thread_local pa::ChunkWork work;
+        static thread_local std::vector<std::pair<int, uint32_t>> items;
+        work.count = 0;
+        items.clear();
+        const int cta_rows = pa::chunk_rows(cache->head_size, 1);
+        const int tile_keys = cache->head_size == 128 ? 128 : 64;
+        const int csb = p.chunk_split_blocks;
+        bool fits = list.count > 0;
+        for (int i = 0; i < list.count && fits; ++i) {
+            const int r = list.req[i];
+            const int ql = query_start_loc_host[r + 1] - query_start_loc_host[r];
+            const int ctx = seq_lens_host[r];
+            const int nsplit = pa::ceil_div(pa::ceil_div(ctx, cache->block_size), csb);
+            const int nqt = pa::ceil_div(ql * p.group, cta_rows);
+            if (r >= pa::kChunkWorkMaxReq || nqt > pa::kChunkWorkMaxQt ||
+                nsplit > pa::kChunkWorkMaxSplit ||
+                items.size() + static_cast<size_t>(nqt) * nsplit > pa::kMaxChunkWork) {
+                fits = false;
+                break;
+            }
+            for (int qt = 0; qt < nqt; ++qt) {
+                const int last_row = std::min((qt + 1) * cta_rows, ql * p.group) - 1;
+                const int kmax = ctx - ql + last_row / p.group;
+                for (int sp = 0; sp < nsplit; ++sp) {
+                    const int key_lo = sp * csb * cache->block_size;
+                    const int key_hi = std::min(std::min((sp + 1) * csb * cache->block_size, ctx), kmax + 1);
+                    const int tiles = key_hi > key_lo ? pa::ceil_div(key_hi - key_lo, tile_keys) : 0;
+                    items.emplace_back(tiles, static_cast<uint32_t>(r) | (static_cast<uint32_t>(qt) << 10) |
+                                                  (static_cast<uint32_t>(sp) << 22));
+                }
+            }
+        }
+        if (fits) {
+            std::stable_sort(items.begin(), items.end(),
+                             [](const std::pair<int, uint32_t>& a, const std::pair<int, uint32_t>& b) {
+                                 return a.first > b.first;
+                             });
+            for (const auto& it : items) work.item[work.count++] = it.second;
+        }
         if (ev) record(ev[2], s);
-        e = pa::launch_chunk(cache->tmap, p, list, cache->head_size, cache->kv_dtype,
-                             pl.chunk_max_splits, s);
+        e = pa::launch_chunk(cache->tmap, cache->tmap_blk, p, work, cache->head_size,
+                             cache->kv_dtype, pl.chunk_max_splits, s);
         if (e != cudaSuccess) return fail_cuda(e);
         if (ev) record(ev[3], s);
     }

@@ -34,16 +34,25 @@ struct ChunkCfg {
 template <int D>
 __global__ void __launch_bounds__(128)
 chunk_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
-             const __grid_constant__ ChunkList list) {
+             const __grid_constant__ ChunkWork work) {
     int* err = p.err;
     using C = ChunkCfg<D>;
     pdl_trigger();
     pdl_wait();
-    // the last query tiles see the most keys (causal): dispatch them first
-    const int qt = p.chunk_max_qtiles - 1 - static_cast<int>(blockIdx.x % p.chunk_max_qtiles);
-    const int split = blockIdx.x / p.chunk_max_qtiles;
+    int qt, split, r;
+    if (work.count > 0) {
+        const uint32_t item = work.item[blockIdx.x];
+        r = static_cast<int>(item & (kChunkWorkMaxReq - 1));
+        qt = static_cast<int>((item >> 10) & (kChunkWorkMaxQt - 1));
+        split = static_cast<int>(item >> 22);
+    } else {
+        // the last query tiles see the most keys (causal): dispatch them first
+        qt = p.chunk_max_qtiles - 1 - static_cast<int>(blockIdx.x % p.chunk_max_qtiles);
+        split = blockIdx.x / p.chunk_max_qtiles;
+        r = static_cast<int>(blockIdx.z);
+    }
+    if (r >= p.num_seqs) return;
     const int g = blockIdx.y;
-    const int r = list.count > 0 ? list.req[blockIdx.z] : static_cast<int>(blockIdx.z);
     const int q0 = p.qsl[r];
     const int q_len = p.qsl[r + 1] - q0;
     if (q_len <= 0 || is_decode_kind(q_len, p.group)) return;
@@ -310,7 +319,7 @@ chunk_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
 }
 
 template <int D>
-cudaError_t launch_chunk_t(const CUtensorMap& tmap, const AttnParams& p, const ChunkList& list,
+cudaError_t launch_chunk_t(const CUtensorMap& tmap, const AttnParams& p, const ChunkWork& work,
                            int max_splits, cudaStream_t stream) {
     using C = ChunkCfg<D>;
     static bool attr_set = false;
@@ -321,18 +330,19 @@ cudaError_t launch_chunk_t(const CUtensorMap& tmap, const AttnParams& p, const C
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    dim3 grid(p.chunk_max_qtiles * max_splits, p.num_kv_heads,
-              list.count > 0 ? list.count : p.num_seqs);
-    return launch_pdl(chunk_kernel<D>, grid, dim3(128), C::kSmemBytes, stream, tmap, p, list);
+    const dim3 grid = work.count > 0 ? dim3(work.count, p.num_kv_heads, 1)
+                                     : dim3(p.chunk_max_qtiles * max_splits, p.num_kv_heads, p.num_seqs);
+    return launch_pdl(chunk_kernel<D>, grid, dim3(128), C::kSmemBytes, stream, tmap, p, work);
 }
 
 }  // namespace
 
-cudaError_t launch_chunk(const CUtensorMap& tmap, const AttnParams& p, const ChunkList& list,
-                         int head_size, int kv_dtype, int max_splits, cudaStream_t stream) {
+cudaError_t launch_chunk(const CUtensorMap& tmap, const CUtensorMap& tmap_blk, const AttnParams& p,
+                         const ChunkWork& work, int head_size, int kv_dtype, int max_splits,
+                         cudaStream_t stream) {
     if (kv_dtype != PA_BF16) return cudaErrorInvalidValue;
-    if (head_size == 128) return launch_chunk_tc(tmap, p, list, max_splits, stream);
-    if (head_size == 64) return launch_chunk_t<64>(tmap, p, list, max_splits, stream);
+    if (head_size == 128) return launch_chunk_tc(tmap_blk, p, work, max_splits, stream);
+    if (head_size == 64) return launch_chunk_t<64>(tmap, p, work, max_splits, stream);
     return cudaErrorInvalidValue;
 }
 

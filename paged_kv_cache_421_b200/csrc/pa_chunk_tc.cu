@@ -6,24 +6,24 @@
 // bottom-right causal mask of chunked prefill ("vLLM: from KV Cache to high-throughput
 // serving", article 5 outline) and the online softmax of FlashAttention (article 7 outline).
 //
-// How.  One CTA owns 128 query rows of one (request, kv head) and optionally one KV split;
-// two CTAs share an SM.  Its warps specialise: warps 0-3 run the softmax (thread i owns row
-// i, which is TMEM lane i), warp 4 issues the tensor-core MMAs, warp 5 issues the TMA loads.
-// Keys are walked in tiles of 64 (four physical blocks from the block table); each block's K
-// and V tiles arrive by TMA (2-D loads, 128-byte swizzle) into two-slot K and V rings laid
-// out [64-dim half][key][128 B], so that one layout serves as the K-major B operand of
-// S = Q K^T and as the MN-major B operand of O += P V.  Per tile j:
-//   * the MMA warp issues S_j = Q K_j^T (8 tcgen05.mma, M 128, N 64, K 16, bf16 -> fp32, two
-//     shared-memory descriptors) into one of two TMEM S buffers as soon as the P V that last
-//     read that buffer has finished -- so S_{j+1} is computed during the softmax of tile j;
-//   * the softmax warps load their rows of S_j, mask (only tiles that cross a causal limit or
-//     the split end) and update a running max; O is rescaled only when the max grows by more
-//     than 2^8 (a stale max keeps every probability <= 256; numerator and denominator share
-//     it, so results are exact), and P_j (bf16) is stored over S_j's columns;
-//   * the MMA warp then issues O += P_j V_j (4 tcgen05.mma, A from TMEM, V from shared
-//     memory) into TMEM columns [128, 256).
-// Full/empty mbarriers between the roles replace CTA-wide barriers inside the loop; MMA
-// completion is signalled by tcgen05.commit.  Every wait is bounded: on a timeout each role
+// How.  One CTA owns two 128-row query tiles (256 rows of one (request, kv head)) and
+// optionally one KV split; one CTA per SM.  Its warps specialise: warps 0-7 run the softmax
+// (warps 4q..4q+3 serve q-tile q; thread i of the q-tile owns row i, which is TMEM lane i),
+// warp 8 issues the tensor-core MMAs, warp 9 the TMA loads.  Keys are walked in tiles of 128
+// (eight physical blocks from the block table); each block's K and V tiles arrive by TMA (2-D
+// loads, 128-byte swizzle) into two-slot K and V rings laid out [64-dim half][key][128 B], so
+// one layout is the K-major B operand of S = Q K^T and the MN-major B operand of O += P V.
+// TMEM (512 columns): per q-tile an S buffer of 128 columns, in whose first 64 columns the
+// softmax stores P (bf16 pairs), and O (128 columns).  Per tile j the MMA warp issues
+//     O_0 += P_0 V_j,  S_0 = Q_0 K_{j+1}^T,  O_1 += P_1 V_j,  S_1 = Q_1 K_{j+1}^T
+// (8 tcgen05.mma each: M 128, N 128, K 16, fp32 accumulate), so the tensor core computes one
+// q-tile's products while the other q-tile's softmax runs.  S_q of tile j+1 overwrites P_q of
+// tile j only after the P V that reads it: tcgen05.mma instructions of one thread execute in
+// issue order.  For the same reason the commit that signals S_q(j+1) also covers O_q += P_q
+// V_j, so the softmax may rescale O as soon as it sees S.  O is rescaled lazily, only when a
+// row's max grows by more than 2^8 (a stale max keeps every probability <= 256; numerator and
+// denominator share it, so results are exact).  Full/empty mbarriers and tcgen05.commit
+// replace CTA barriers inside the loop.  Every wait is bounded: on a timeout each role
 // records the error and stops, and the CTA frees its TMEM and returns.
 #include "pa_internal.h"
 
@@ -33,24 +33,26 @@ namespace {
 constexpr int kD = 128;
 constexpr int kRows = 128;                       // query rows per q-tile = TMEM lanes
 constexpr int kQTiles = 2;                       // q-tiles per CTA, sharing every K/V tile
-constexpr int kKeys = 64;                        // keys per tile
-constexpr int kTileBlocks = kKeys / kBlockSize;  // 4 physical blocks
+constexpr int kKeys = 128;                       // keys per tile
+constexpr int kTileBlocks = kKeys / kBlockSize;  // 8 physical blocks
 constexpr int kHalfRows = 128;                   // bytes per swizzled row (64 bf16)
 constexpr int kQHalf = kRows * kHalfRows;        // 16 KB: one 64-dim half of a q-tile
 constexpr int kQBytes = 2 * kQHalf;              // 32 KB per q-tile
-constexpr int kKVHalf = kKeys * kHalfRows;       // 8 KB: one 64-dim half of a K or V tile
-constexpr int kKBytes = 2 * kKVHalf;             // 16 KB per K or V tile
-constexpr int kKSlots = 4, kVSlots = 3;          // K runs two tiles ahead of V
-constexpr int kSmemBytes = kQTiles * kQBytes + (kKSlots + kVSlots) * kKBytes + 1024;  // 177 KB
+// A K or V tile (128 keys x 128 dims, 32 KB) is eight 4 KB block tiles, each laid out as
+// [8-row group][64-dim half][8 rows][128 B]: 8-key groups are kGroupStride apart for every key
+// of the tile, the two halves of a group kAtom apart (one 128-byte swizzle atom each).
+constexpr int kAtom = 8 * kHalfRows;             // 1 KB: 8 rows x 128 B
+constexpr int kGroupStride = 2 * kAtom;          // 2 KB between consecutive 8-key groups
+constexpr int kBlockTile = kBlockSize * 2 * kHalfRows;  // 4 KB: one block's 16 x 128 tile
+constexpr int kKBytes = kTileBlocks * kBlockTile;       // 32 KB per K or V tile
+constexpr int kKSlots = 2, kVSlots = 2;
+constexpr int kSmemBytes = kQTiles * kQBytes + (kKSlots + kVSlots) * kKBytes + 1024;  // 193 KB
 constexpr uint32_t kTmemCols = 512;
-// TMEM columns of q-tile q: S of even tiles [256q, 256q + 64), of odd tiles [256q + 64, 256q + 128)
-// (P overwrites the first half of its own tile's S once that S is in registers); O
-// [256q + 128, 256q + 256).
-constexpr uint32_t kColO = 128;
+constexpr uint32_t kColO = 128;                  // q-tile q: S/P [256q, 256q+128), O after it
 constexpr int kMaxIds = 1024;                    // block ids staged in shared memory
 
 // Instruction descriptors (kind::f16): fp32 accumulate, bf16 A and B, M = 128.
-// S = Q K^T: A and B K-major, N = 64 keys.  O = P V: B (V) MN-major, N = 128 dims.
+// S = Q K^T: A and B K-major, N = 128 keys.  O = P V: B (V) MN-major, N = 128 dims.
 constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) |
                               (static_cast<uint32_t>(kKeys >> 3) << 17) |
                               (static_cast<uint32_t>(kRows >> 4) << 24);
@@ -132,23 +134,60 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         : "memory");
 }
 
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+        "r"(r[15])
+        : "memory");
+}
+
+// One (block, K|V, kv head) tile through the 4-D view: box (64, 8, 2, 2) at 8-row group `grp`.
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int grp) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(0), "r"(0), "r"(0), "r"(grp)
+        : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
-constexpr int kThreads = 320;  // warps 0-7 softmax (q-tile = warp / 4), 8 MMA, 9 TMA
+// Warpgroups: 0 and 1 run the softmax of q-tiles 0 and 1; in warpgroup 2, warp 8 issues the
+// MMAs, warp 9 the TMA loads, warps 10-11 only hand back registers.  The launch gives every
+// thread 168 registers (3 warps per SM sub-partition); warpgroup 2 drops to 40 and the softmax
+// warpgroups rise to 232: 8 x 32 x 232 + 4 x 32 x 40 = 64512 = 12 x 32 x 168, the launch's
+// total, and each sub-partition holds 2 x 232 + 40 registers per lane (16128 <= 16384).
+constexpr int kThreads = 384;
+constexpr uint32_t kRegsSoftmax = 232, kRegsProducer = 40;
+static_assert(8 * 32 * kRegsSoftmax + 4 * 32 * kRegsProducer <= kThreads * 168,
+              "register split exceeds the launch's registers");
 
 __global__ void __launch_bounds__(kThreads, 1)
-chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
-                const __grid_constant__ ChunkList list) {
+chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p,
+                const __grid_constant__ ChunkWork work) {
     pdl_trigger();
     pdl_wait();
     int* err = p.err;
-    // the last query tiles see the most keys (causal): dispatch them first
-    const int qt = p.chunk_max_qtiles - 1 - static_cast<int>(blockIdx.x % p.chunk_max_qtiles);
-    const int split = blockIdx.x / p.chunk_max_qtiles;
+    int qt, split, r;
+    if (work.count > 0) {
+        const uint32_t item = work.item[blockIdx.x];
+        r = static_cast<int>(item & (kChunkWorkMaxReq - 1));
+        qt = static_cast<int>((item >> 10) & (kChunkWorkMaxQt - 1));
+        split = static_cast<int>(item >> 22);
+    } else {
+        // the last query tiles see the most keys (causal): dispatch them first
+        qt = p.chunk_max_qtiles - 1 - static_cast<int>(blockIdx.x % p.chunk_max_qtiles);
+        split = blockIdx.x / p.chunk_max_qtiles;
+        r = static_cast<int>(blockIdx.z);
+    }
+    if (r >= p.num_seqs) return;
     const int g = blockIdx.y;
-    const int r = list.count > 0 ? list.req[blockIdx.z] : static_cast<int>(blockIdx.z);
     const int q0 = p.qsl[r];
     const int q_len = p.qsl[r + 1] - q0;
     if (q_len <= 0 || is_decode_kind(q_len, p.group)) return;
@@ -182,15 +221,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
 
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t bar_kf[kKSlots], bar_ke[kKSlots], bar_vf[kVSlots], bar_ve[kVSlots];
-    __shared__ uint64_t bar_sf[kQTiles][2], bar_pf[kQTiles][2];  // S computed / P stored
-    __shared__ uint64_t bar_o[kQTiles];                          // a P V of the q-tile done
+    __shared__ uint64_t bar_sf[kQTiles], bar_pf[kQTiles];  // S computed / P stored
+    __shared__ uint64_t bar_o[kQTiles];                    // a P V of the q-tile done
     __shared__ uint32_t tmem_holder;
     __shared__ int ids[kMaxIds];  // physical ids of the split's first kMaxIds logical blocks
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const uint32_t q_s = smem_u32(smem);                      // [q-tile][32 KB]
-    const uint32_t k_s = q_s + kQTiles * kQBytes;             // [K slot][16 KB]
-    const uint32_t v_s = k_s + kKSlots * kKBytes;             // [V slot][16 KB]
+    const uint32_t k_s = q_s + kQTiles * kQBytes;             // [K slot][32 KB]
+    const uint32_t v_s = k_s + kKSlots * kKBytes;             // [V slot][32 KB]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -202,7 +241,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     if (tid == 0) {
-        prefetch_tensor_map(&tmap);
+        prefetch_tensor_map(&tmap_blk);
         for (int i = 0; i < kKSlots; ++i) {
             mbar_init(smem_u32(&bar_kf[i]), 1);
             mbar_init(smem_u32(&bar_ke[i]), 1);
@@ -212,10 +251,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
             mbar_init(smem_u32(&bar_ve[i]), 1);
         }
         for (int q = 0; q < kQTiles; ++q) {
-            for (int i = 0; i < 2; ++i) {
-                mbar_init(smem_u32(&bar_sf[q][i]), 1);
-                mbar_init(smem_u32(&bar_pf[q][i]), kRows);
-            }
+            mbar_init(smem_u32(&bar_sf[q]), 1);
+            mbar_init(smem_u32(&bar_pf[q]), kRows);
             mbar_init(smem_u32(&bar_o[q]), 1);
         }
         fence_barrier_init();
@@ -228,16 +265,29 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
         }
         ids[k] = blk;
     }
-    // Q tiles -> shared memory in the swizzled K-major layout [q-tile][half][row][128 B]
-    for (int idx = tid; idx < kQTiles * kRows * (kD / 8); idx += kThreads) {
-        const int rr = idx >> 4, c = idx & 15;  // rr over both q-tiles
-        const int Rr = R0 + rr;
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (Rr < rows_total)
-            v = *reinterpret_cast<const uint4*>(
-                p.q + (static_cast<int64_t>(q0 + Rr / G) * p.num_q_heads + g * G + Rr % G) * kD + c * 8);
-        *reinterpret_cast<uint4*>(smem + (rr >> 7) * kQBytes + (c >> 3) * kQHalf +
-                                  sw128(rr & (kRows - 1), c & 7)) = v;
+    // Q tiles -> shared memory in the swizzled K-major layout [q-tile][half][row][128 B]; every
+    // load of a thread is issued before its first store, so their latencies overlap
+    {
+        constexpr int kVecs = kQTiles * kRows * (kD / 8), kPer = (kVecs + kThreads - 1) / kThreads;
+        uint4 v[kPer];
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            const int idx = tid + i * kThreads;
+            const int Rr = R0 + (idx >> 4), c = idx & 15;
+            v[i] = make_uint4(0, 0, 0, 0);
+            if (idx < kVecs && Rr < rows_total)
+                v[i] = __ldg(reinterpret_cast<const uint4*>(
+                    p.q + (static_cast<int64_t>(q0 + Rr / G) * p.num_q_heads + g * G + Rr % G) * kD +
+                    c * 8));
+        }
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            const int idx = tid + i * kThreads;
+            const int rr = idx >> 4, c = idx & 15;  // rr over both q-tiles
+            if (idx < kVecs)
+                *reinterpret_cast<uint4*>(smem + (rr >> 7) * kQBytes + (c >> 3) * kQHalf +
+                                          sw128(rr & (kRows - 1), c & 7)) = v[i];
+        }
     }
     fence_proxy_async();  // Q's generic-proxy stores, before the tensor core reads them
     tc_fence_before();
@@ -246,18 +296,23 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
     const uint32_t tmem = tmem_holder;
     bool ok = true;
 
-    if (warp == 9) {
-        // ================= TMA producer: K runs two tiles ahead of V
-        if (lane == 0) {
+    if (warp >= 8) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsProducer));
+        if (warp == 9) {
+            // ================= TMA producer: K one tile ahead of V.  The expected bytes are
+            // posted first, then lane i issues block i's whole 4 KB tile, so the per-copy
+            // issue latency overlaps across the warp.
             const int kv_rows_per_block = 2 * p.num_kv_heads * kBlockSize;
             auto load = [&](int t, int which) {
-                const int st = which ? t % kVSlots : t % kKSlots;
+                const int st = t & 1;
                 const uint32_t bar = smem_u32(which ? &bar_vf[st] : &bar_kf[st]);
                 const uint32_t dst = (which ? v_s : k_s) + st * kKBytes;
                 const int j0 = key_lo / kBlockSize + t * kTileBlocks;
                 const int nload = min(kTileBlocks, je - j0);
-                mbar_arrive_expect_tx(bar, nload * 2 * (kBlockSize * kHalfRows));
-                for (int b2 = 0; b2 < nload; ++b2) {
+                if (lane == 0) mbar_arrive_expect_tx(bar, nload * kBlockTile);
+                __syncwarp();
+                if (lane < nload) {
+                    const int b2 = lane;
                     int blk;
                     if (j0 + b2 - jb < kMaxIds) {
                         blk = ids[j0 + b2 - jb];
@@ -269,229 +324,230 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
                         }
                     }
                     const int row = blk * kv_rows_per_block + (which * p.num_kv_heads + g) * kBlockSize;
-#pragma unroll
-                    for (int x = 0; x < 2; ++x)
-                        tma_load_2d(dst + x * kKVHalf + b2 * (kBlockSize * kHalfRows), &tmap, bar,
-                                    x * 64, row);
+                    tma_load_4d(dst + b2 * kBlockTile, &tmap_blk, bar, row / 8);
                 }
+                __syncwarp();
             };
-            // step t issues K(t) and V(t - 2); a slot is free once the MMAs that read its
+            // step t issues K(t) and V(t - 1); a slot is free once the MMAs that read its
             // previous tile have completed (their commit arrives on the slot's empty barrier)
-            for (int t = 0; t < ntiles + 2 && ok; ++t) {
+            for (int t = 0; t < ntiles + 1 && ok; ++t) {
                 if (t < ntiles) {
                     if (t >= kKSlots &&
-                        !mbar_wait(smem_u32(&bar_ke[t % kKSlots]), ((t / kKSlots) + 1) & 1,
-                                   kWaitLimitNs, err))
+                        !__all_sync(0xffffffffu, mbar_wait(smem_u32(&bar_ke[t & 1]), ((t >> 1) + 1) & 1,
+                                                           kWaitLimitNs, err)))
                         ok = false;
                     if (ok) load(t, 0);
                 }
-                const int tv = t - 2;
-                if (ok && tv >= 0 && tv < ntiles) {
+                const int tv = t - 1;
+                if (ok && tv >= 0) {
                     if (tv >= kVSlots &&
-                        !mbar_wait(smem_u32(&bar_ve[tv % kVSlots]), ((tv / kVSlots) + 1) & 1,
-                                   kWaitLimitNs, err))
+                        !__all_sync(0xffffffffu, mbar_wait(smem_u32(&bar_ve[tv & 1]), ((tv >> 1) + 1) & 1,
+                                                           kWaitLimitNs, err)))
                         ok = false;
                     if (ok) load(tv, 1);
                 }
             }
-        }
-    } else if (warp == 8) {
-        // ================= MMA issuer: S one tile ahead, O += P V when P is stored
-        if (lane == 0 && ntiles > 0) {
-            auto qk = [&](int t) {  // S of tile t for every q-tile, then free its K slot
-                const uint32_t ks = k_s + (t % kKSlots) * kKBytes;
-                tc_fence_after();
-                for (int q = 0; q < nq; ++q) {
-#pragma unroll
+        } else if (warp == 8) {
+            // ================= MMA issuer
+            if (lane == 0 && ntiles > 0) {
+                auto qk = [&](int q, int t) {  // S_q = Q_q K_t^T
+                    const uint32_t ks = k_s + (t & 1) * kKBytes;
+    #pragma unroll
                     for (int k = 0; k < kD / 16; ++k) {
                         const uint32_t off = q * kQBytes + (k >> 2) * kQHalf + (k & 3) * 32;
-                        const uint32_t koff = (k >> 2) * kKVHalf + (k & 3) * 32;
-                        mma_ss(tmem + q * 256 + (t & 1) * kKeys, smem_desc(q_s + off, 16, 1024),
-                               smem_desc(ks + koff, 16, 1024), kIdescQK, k > 0);
+                        const uint32_t koff = (k >> 2) * kAtom + (k & 3) * 32;
+                        mma_ss(tmem + q * 256, smem_desc(q_s + off, 16, 1024),
+                               smem_desc(ks + koff, 16, kGroupStride), kIdescQK, k > 0);
                     }
-                    mma_commit(smem_u32(&bar_sf[q][t & 1]));
-                }
-                mma_commit(smem_u32(&bar_ke[t % kKSlots]));
-            };
-            if (mbar_wait(smem_u32(&bar_kf[0]), 0, kWaitLimitNs, err)) qk(0); else ok = false;
-            for (int kt = 0; kt < ntiles && ok; ++kt) {
-                const int st = kt & 1;
-                if (kt + 1 < ntiles) {
-                    // the other S buffers are free once each q-tile's P V of tile kt-1 is done
-                    if (kt >= 1) {
-                        bool w = true;
-                        for (int q = 0; q < nq && w; ++q)
-                            w = mbar_wait(smem_u32(&bar_o[q]), (kt - 1) & 1, kWaitLimitNs, err);
-                        if (!w) break;
-                    }
-                    if (!mbar_wait(smem_u32(&bar_kf[(kt + 1) % kKSlots]), ((kt + 1) / kKSlots) & 1,
-                                   kWaitLimitNs, err))
-                        break;
-                    qk(kt + 1);
-                }
-                if (!mbar_wait(smem_u32(&bar_vf[kt % kVSlots]), (kt / kVSlots) & 1, kWaitLimitNs, err))
-                    break;
-                const uint32_t vs = v_s + (kt % kVSlots) * kKBytes;
-                bool w = true;
-                for (int q = 0; q < nq; ++q) {
-                    if (!mbar_wait(smem_u32(&bar_pf[q][st]), (kt >> 1) & 1, kWaitLimitNs, err)) {
-                        w = false;
-                        break;
-                    }
-                    tc_fence_after();
-#pragma unroll
+                    mma_commit(smem_u32(&bar_sf[q]));
+                };
+                auto pv = [&](int q, int t) {  // O_q += P_q V_t (P from TMEM)
+                    const uint32_t vs = v_s + (t & 1) * kKBytes;
+    #pragma unroll
                     for (int j = 0; j < kKeys / 16; ++j)
-                        mma_ts(tmem + q * 256 + kColO, tmem + q * 256 + st * kKeys + 8 * j,
-                               smem_desc(vs + j * (kBlockSize * kHalfRows), kKVHalf, 1024), kIdescPV,
-                               (kt > 0 || j > 0) ? 1u : 0u);
+                        mma_ts(tmem + q * 256 + kColO, tmem + q * 256 + 8 * j,
+                               smem_desc(vs + j * kBlockTile, kAtom, kGroupStride), kIdescPV,
+                               (t > 0 || j > 0) ? 1u : 0u);
                     mma_commit(smem_u32(&bar_o[q]));
+                };
+                if (mbar_wait(smem_u32(&bar_kf[0]), 0, kWaitLimitNs, err)) {
+                    tc_fence_after();
+                    for (int q = 0; q < nq; ++q) qk(q, 0);
+                    mma_commit(smem_u32(&bar_ke[0]));
+                } else {
+                    ok = false;
                 }
-                if (!w) break;
-                mma_commit(smem_u32(&bar_ve[kt % kVSlots]));
+                for (int kt = 0; kt < ntiles && ok; ++kt) {
+                    const bool more = kt + 1 < ntiles;
+                    if (!mbar_wait(smem_u32(&bar_vf[kt & 1]), (kt >> 1) & 1, kWaitLimitNs, err)) break;
+                    if (more && !mbar_wait(smem_u32(&bar_kf[(kt + 1) & 1]), ((kt + 1) >> 1) & 1,
+                                           kWaitLimitNs, err))
+                        break;
+                    bool w = true;
+                    for (int q = 0; q < nq; ++q) {
+                        if (!mbar_wait(smem_u32(&bar_pf[q]), kt & 1, kWaitLimitNs, err)) {
+                            w = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        pv(q, kt);
+                        if (more) qk(q, kt + 1);  // overwrites P_q(kt) after the P V above
+                    }
+                    if (!w) break;
+                    mma_commit(smem_u32(&bar_ve[kt & 1]));
+                    if (more) mma_commit(smem_u32(&bar_ke[(kt + 1) & 1]));
+                }
             }
         }
-    } else if (warp / 4 < nq) {
-        // ================= softmax: thread = row = TMEM lane of its q-tile
-        const int q = warp / 4;
-        const int row = tid & (kRows - 1);
-        const int R = R0 + q * kRows + row;
-        const bool valid = R < rows_total;
-        const int lim = valid ? ctx - q_len + R / G : kmax;
-        const int first_lim = ctx - q_len + (R0 + q * kRows) / G;  // smallest limit of the q-tile
-        const uint32_t tq = tmem + q * 256;
-        const uint32_t tmem_lane = tq + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-        const float sl = p.scale_log2;
-        float m_used = -INFINITY, l = 0.f;
-        for (int kt = 0; kt < ntiles; ++kt) {
-            const int st = kt & 1;
-            const int key0 = key_lo + kt * kKeys;
-            if (!mbar_wait(smem_u32(&bar_sf[q][st]), (kt >> 1) & 1, kWaitLimitNs, err)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            float s[kKeys];
-#pragma unroll
-            for (int c = 0; c < kKeys / 32; ++c) {
-                uint32_t raw[32];
-                tmem_ld32(tmem_lane + st * kKeys + c * 32, raw);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(raw[i]);
-            }
-            tmem_wait_ld();
-            // only tiles crossing a causal limit or the split end need masking
-            if (!(key0 + kKeys - 1 <= first_lim && key0 + kKeys <= kend)) {
-#pragma unroll
-                for (int c = 0; c < kKeys; ++c) {
-                    const int pos = key0 + c;
-                    if (pos > lim || pos >= kend) s[c] = -INFINITY;
-                }
-            }
-            // max with independent partial maxima (short dependency chains)
-            float mp[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) mp[i] = s[i];
-#pragma unroll
-            for (int c = 8; c < kKeys; ++c) mp[c & 7] = fmaxf(mp[c & 7], s[c]);
-            float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
-            mx *= sl;  // scores stay unscaled: max(s) * sl is the scaled max (sl > 0)
-            const float m_new = fmaxf(m_used, mx);
-            float alpha = 1.f;
-            if (m_used == -INFINITY) {
-                m_used = m_new;
-            } else if (m_new > m_used + 8.f) {
-                alpha = ex2(m_used - m_new);
-                m_used = m_new;
-            }
-            if (__any_sync(0xffffffffu, alpha != 1.f) && kt > 0) {
-                // rescale O (this warp's 32 rows) once the q-tile's previous P V has landed
-                if (!mbar_wait(smem_u32(&bar_o[q]), (kt - 1) & 1, kWaitLimitNs, err)) {
+    } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
+        if (warp / 4 < nq) {
+            // ================= softmax: thread = row = TMEM lane of its q-tile
+            const int q = warp / 4;
+            const int row = tid & (kRows - 1);
+            const int R = R0 + q * kRows + row;
+            const bool valid = R < rows_total;
+            const int lim = valid ? ctx - q_len + R / G : kmax;
+            const int first_lim = ctx - q_len + (R0 + q * kRows) / G;  // smallest limit of the q-tile
+            const uint32_t tq = tmem + q * 256;
+            const uint32_t tmem_lane = tq + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+            const float sl = p.scale_log2;
+            float m_used = -INFINITY, l = 0.f;
+            for (int kt = 0; kt < ntiles; ++kt) {
+                const int key0 = key_lo + kt * kKeys;
+                // waits end warp-uniformly: the tcgen05 loads below are warp-collective
+                if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&bar_sf[q]), kt & 1, kWaitLimitNs, err))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                l *= alpha;
-#pragma unroll
-                for (int c = 0; c < kD / 32; ++c) {
+                // only tiles crossing a causal limit or the split end need masking
+                const bool masked = !(key0 + kKeys - 1 <= first_lim && key0 + kKeys <= kend);
+                // S of this row: all four loads in flight, one wait (TMEM load latency is long)
+                float sv[kKeys];
+    #pragma unroll
+                for (int c = 0; c < kKeys / 32; ++c) {
                     uint32_t raw[32];
-                    tmem_ld32(tmem_lane + kColO + c * 32, raw);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        raw[i] = __float_as_uint(__uint_as_float(raw[i]) * alpha);
-                    tmem_st32(tmem_lane + kColO + c * 32, raw);
+                    tmem_ld32(tmem_lane + c * 32, raw);
+    #pragma unroll
+                    for (int i = 0; i < 32; ++i) sv[c * 32 + i] = __uint_as_float(raw[i]);
                 }
-            }
-            const float neg_ref = m_used == -INFINITY ? 0.f : -m_used;
-            float sp[4] = {0.f, 0.f, 0.f, 0.f};
-            uint32_t packed[32];
-#pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const float a0 = ex2(fmaf(s[2 * i], sl, neg_ref));
-                const float a1 = ex2(fmaf(s[2 * i + 1], sl, neg_ref));
-                sp[i & 3] += a0 + a1;
-                packed[i] = pack_bf16(a0, a1);
-            }
-            tmem_st32(tmem_lane + st * kKeys, packed);  // P over this tile's S columns
-            l += (sp[0] + sp[1]) + (sp[2] + sp[3]);
-            tmem_wait_st();
-            if (q == 0 && key0 + kKeys > kend) {
-                // keys past the split / context: clear their V rows once V has landed (q-tile 0
-                // does it; its P V is issued before q-tile 1's)
-                const int vslot = kt % kVSlots;
-                if (!mbar_wait(smem_u32(&bar_vf[vslot]), (kt / kVSlots) & 1, kWaitLimitNs, err)) {
-                    ok = false;
-                    break;
+                tmem_wait_ld();
+                if (masked) {
+    #pragma unroll
+                    for (int c = 0; c < kKeys; ++c) {
+                        const int pos = key0 + c;
+                        if (pos > lim || pos >= kend) sv[c] = -INFINITY;
+                    }
                 }
-                uint8_t* vg = smem + kQTiles * kQBytes + (kKSlots + vslot) * kKBytes;
-                const int nvalid = kend - key0;
-                for (int idx = row; idx < (kKeys - nvalid) * 2 * 8; idx += kRows) {
-                    const int kk = nvalid + idx / 16, c = idx % 16;
-                    *reinterpret_cast<uint4*>(vg + (c >> 3) * kKVHalf + kk * kHalfRows + (c & 7) * 16) =
-                        make_uint4(0, 0, 0, 0);
+                // the row max with independent partial maxima (short dependency chains)
+                float mp[8];
+    #pragma unroll
+                for (int i = 0; i < 8; ++i) mp[i] = sv[i];
+    #pragma unroll
+                for (int c = 8; c < kKeys; ++c) mp[c & 7] = fmaxf(mp[c & 7], sv[c]);
+                float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                                 fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+                mx *= sl;  // scores stay unscaled: max(s) * sl is the scaled max (sl > 0)
+                const float m_new = fmaxf(m_used, mx);
+                float alpha = 1.f;
+                if (m_used == -INFINITY) {
+                    m_used = m_new;
+                } else if (m_new > m_used + 8.f) {
+                    alpha = ex2(m_used - m_new);
+                    m_used = m_new;
                 }
-                fence_proxy_async();
+                if (__any_sync(0xffffffffu, alpha != 1.f) && kt > 0) {
+                    // rescale O (this warp's 32 rows): the commit that signalled S of this tile
+                    // also covers the q-tile's previous P V
+                    l *= alpha;
+    #pragma unroll
+                    for (int c = 0; c < kD / 32; ++c) {
+                        uint32_t raw[32];
+                        tmem_ld32(tmem_lane + kColO + c * 32, raw);
+                        tmem_wait_ld();
+    #pragma unroll
+                        for (int i = 0; i < 32; ++i)
+                            raw[i] = __float_as_uint(__uint_as_float(raw[i]) * alpha);
+                        tmem_st32(tmem_lane + kColO + c * 32, raw);
+                    }
+                }
+                // P = 2^(s sl - m) as bf16 pairs over the first 64 S columns, 32 keys at a time
+                const float neg_ref = m_used == -INFINITY ? 0.f : -m_used;
+                float sp[4] = {0.f, 0.f, 0.f, 0.f};
+    #pragma unroll
+                for (int c = 0; c < kKeys / 32; ++c) {
+                    uint32_t packed[16];
+    #pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const float a0 = ex2(fmaf(sv[32 * c + 2 * i], sl, neg_ref));
+                        const float a1 = ex2(fmaf(sv[32 * c + 2 * i + 1], sl, neg_ref));
+                        sp[i & 3] += a0 + a1;
+                        packed[i] = pack_bf16(a0, a1);
+                    }
+                    tmem_st16(tmem_lane + 16 * c, packed);
+                }
+                l += (sp[0] + sp[1]) + (sp[2] + sp[3]);
+                tmem_wait_st();
+                if (q == 0 && key0 + kKeys > kend) {
+                    // keys past the split / context: clear their V rows once V has landed (q-tile 0
+                    // does it; its P V is issued before q-tile 1's)
+                    const int vslot = kt & 1;
+                    if (!__all_sync(0xffffffffu,
+                                    mbar_wait(smem_u32(&bar_vf[vslot]), (kt >> 1) & 1, kWaitLimitNs, err))) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* vg = smem + kQTiles * kQBytes + (kKSlots + vslot) * kKBytes;
+                    const int nvalid = kend - key0;
+                    for (int idx = row; idx < (kKeys - nvalid) * 2 * 8; idx += kRows) {
+                        const int kk = nvalid + idx / 16, c = idx % 16;
+                        *reinterpret_cast<uint4*>(vg + (kk >> 3) * kGroupStride + (c >> 3) * kAtom +
+                                              (kk & 7) * kHalfRows + (c & 7) * 16) =
+                            make_uint4(0, 0, 0, 0);
+                    }
+                    fence_proxy_async();
+                }
+                tc_fence_before();
+                mbar_arrive(smem_u32(&bar_pf[q]));
             }
-            tc_fence_before();
-            mbar_arrive(smem_u32(&bar_pf[q][st]));
-        }
-        // ---- epilogue: O / l for this row.  Wait for the q-tile's last two P V in order (a
-        // parity wait is unambiguous only with one phase outstanding; the last P V is issued
-        // without waiting for the one before it).
-        float o[kD];
-        if (ok && ntiles > 1 && !mbar_wait(smem_u32(&bar_o[q]), (ntiles - 2) & 1, kWaitLimitNs, err))
-            ok = false;
-        if (ok && ntiles > 0 && mbar_wait(smem_u32(&bar_o[q]), (ntiles - 1) & 1, kWaitLimitNs, err)) {
-            tc_fence_after();
-#pragma unroll
-            for (int c = 0; c < kD / 32; ++c) {
-                uint32_t raw[32];
-                tmem_ld32(tmem_lane + kColO + c * 32, raw);
-#pragma unroll
-                for (int i = 0; i < 32; ++i) o[c * 32 + i] = __uint_as_float(raw[i]);
-            }
-            tmem_wait_ld();
-        } else {
-            if (ntiles > 0) ok = false;
-#pragma unroll
-            for (int i = 0; i < kD; ++i) o[i] = 0.f;
-        }
-        if (ok && valid) {
+            // ---- epilogue: O / l for this row.  S of the last tile covers every P V before the
+            // last one, so one phase of the q-tile's P V barrier is outstanding here.
+            if (ok && ntiles > 0 && !mbar_wait(smem_u32(&bar_o[q]), (ntiles - 1) & 1, kWaitLimitNs, err))
+                ok = false;
+            // tcgen05.ld is warp-collective: the whole warp loads (or none of it), rows store
+            const bool have = __all_sync(0xffffffffu, ok) && ntiles > 0;
             const int t = q0 + R / G, h = g * G + R % G;
             const float inv = l > 0.f ? 1.f / l : 0.f;
-            float* dst;
-            if (nsplit == 1) {
-                dst = p.out + (static_cast<int64_t>(t) * p.num_q_heads + h) * kD;
-            } else {
-                const int64_t prow = (static_cast<int64_t>(split) * p.num_tokens + t) * p.num_q_heads + h;
-                dst = p.part_o + prow * kD;
-                p.part_lse[prow] = l > 0.f ? m_used + __log2f(l) : -INFINITY;
+            float* dst = nullptr;
+            if (ok && valid) {
+                if (nsplit == 1) {
+                    dst = p.out + (static_cast<int64_t>(t) * p.num_q_heads + h) * kD;
+                } else {
+                    const int64_t prow = (static_cast<int64_t>(split) * p.num_tokens + t) * p.num_q_heads + h;
+                    dst = p.part_o + prow * kD;
+                    p.part_lse[prow] = l > 0.f ? m_used + __log2f(l) : -INFINITY;
+                }
             }
-#pragma unroll
-            for (int i = 0; i < kD; i += 4)
-                *reinterpret_cast<float4*>(dst + i) =
-                    make_float4(o[i] * inv, o[i + 1] * inv, o[i + 2] * inv, o[i + 3] * inv);
+            if (have) tc_fence_after();
+    #pragma unroll
+            for (int c = 0; c < kD / 32; ++c) {
+                uint32_t raw[32];
+                if (have) {
+                    tmem_ld32(tmem_lane + kColO + c * 32, raw);
+                    tmem_wait_ld();
+                } else {
+    #pragma unroll
+                    for (int i = 0; i < 32; ++i) raw[i] = 0u;
+                }
+                if (dst) {
+    #pragma unroll
+                    for (int i = 0; i < 32; i += 4)
+                        *reinterpret_cast<float4*>(dst + c * 32 + i) = make_float4(
+                            __uint_as_float(raw[i]) * inv, __uint_as_float(raw[i + 1]) * inv,
+                            __uint_as_float(raw[i + 2]) * inv, __uint_as_float(raw[i + 3]) * inv);
+                }
+            }
         }
     }
     // all roles end here; after an error every role has given up its bounded waits
@@ -505,7 +561,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
 
 }  // namespace
 
-cudaError_t launch_chunk_tc(const CUtensorMap& tmap, const AttnParams& p, const ChunkList& list,
+cudaError_t launch_chunk_tc(const CUtensorMap& tmap_blk, const AttnParams& p, const ChunkWork& work,
                             int max_splits, cudaStream_t stream) {
     static bool attr_set = false;
     if (!attr_set) {
@@ -514,9 +570,9 @@ cudaError_t launch_chunk_tc(const CUtensorMap& tmap, const AttnParams& p, const 
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    dim3 grid(p.chunk_max_qtiles * max_splits, p.num_kv_heads,
-              list.count > 0 ? list.count : p.num_seqs);
-    return launch_pdl(chunk_tc_kernel, grid, dim3(kThreads), kSmemBytes, stream, tmap, p, list);
+    const dim3 grid = work.count > 0 ? dim3(work.count, p.num_kv_heads, 1)
+                                     : dim3(p.chunk_max_qtiles * max_splits, p.num_kv_heads, p.num_seqs);
+    return launch_pdl(chunk_tc_kernel, grid, dim3(kThreads), kSmemBytes, stream, tmap_blk, p, work);
 }
 
 }  // namespace pa

@@ -19,6 +19,8 @@ struct pa_cache {
     bool owns;
     int device;
     CUtensorMap tmap;      // 2-D view of the pool: rows of head_size elements
+    CUtensorMap tmap_blk;  // bf16 head_size 128 only: 4-D view, one box = one (block, K|V,
+                           // kv head) tile as [8-row group][64-dim half][8 rows][128 B]
 };
 
 namespace pa {
@@ -76,11 +78,22 @@ struct ChunkList {
     int req[kMaxChunkList];
 };
 
+// The CTAs of a chunk launch, most key tiles first (longest-processing-time order, so the
+// short CTAs fill in behind the long ones): item = request | q-tile << 10 | split << 22.
+// count == 0 means "derive them from the grid" (x: q-tile and split, z: request).
+constexpr int kMaxChunkWork = 3072;
+constexpr int kChunkWorkMaxReq = 1 << 10, kChunkWorkMaxQt = 1 << 12, kChunkWorkMaxSplit = 1 << 10;
+struct ChunkWork {
+    int count;
+    uint32_t item[kMaxChunkWork];
+};
+
 cudaError_t launch_decode(const CUtensorMap& tmap, const AttnParams& p, int head_size,
                           int kv_dtype, int max_splits, cudaStream_t stream);
-cudaError_t launch_chunk(const CUtensorMap& tmap, const AttnParams& p, const ChunkList& list,
-                         int head_size, int kv_dtype, int max_splits, cudaStream_t stream);
-cudaError_t launch_chunk_tc(const CUtensorMap& tmap, const AttnParams& p, const ChunkList& list,
+cudaError_t launch_chunk(const CUtensorMap& tmap, const CUtensorMap& tmap_blk, const AttnParams& p,
+                         const ChunkWork& work, int head_size, int kv_dtype, int max_splits,
+                         cudaStream_t stream);
+cudaError_t launch_chunk_tc(const CUtensorMap& tmap_blk, const AttnParams& p, const ChunkWork& work,
                             int max_splits, cudaStream_t stream);
 cudaError_t launch_reduce(const AttnParams& p, const ChunkList& list, int head_size,
                           cudaStream_t stream);

@@ -212,10 +212,12 @@ def test_edge_case(case):
                      f"{case} split {split}")
 
 
-@pytest.mark.parametrize("kv_dtype", [W.BF16, W.FP8_E4M3])
-def test_nan_garbage_in_unwritten_slots(kv_dtype):
+@pytest.mark.parametrize("kv_dtype,q_lens", [(W.BF16, [1, 1, 1, 1]), (W.FP8_E4M3, [1, 1, 1, 1]),
+                                             (W.BF16, [17, 9, 5, 60])])
+def test_nan_garbage_in_unwritten_slots(kv_dtype, q_lens):
     # stale NaN patterns in the unused tail of partly filled blocks must not reach the output
-    wl = _small([17, 33, 5, 100], [1, 1, 1, 1], 16, 2, 128, seed=9, kv_dtype=kv_dtype)
+    # (decode rows, and prefill chunks whose last key tile ends inside a block)
+    wl = _small([17, 33, 5, 100], q_lens, 16, 2, 128, seed=9, kv_dtype=kv_dtype)
     st = GpuStep(wl, fill=False, garbage_tail=True)
     tokens = np.repeat(np.arange(wl.num_tokens), wl.num_q_heads)
     heads = np.tile(np.arange(wl.num_q_heads), wl.num_tokens)
