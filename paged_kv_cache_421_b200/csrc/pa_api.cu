@@ -465,7 +465,10 @@ int pa_attention_ex(const pa_cache* cache, const void* q, int num_q_heads,
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     void* const* ev = opts ? opts->events : nullptr;
     cudaError_t e = cudaSuccess;
-    if (pl.decode_max_splits > 1) {
+    // split counters: decode splits, and tcgen05 chunk splits merged inside the chunk kernel
+    const bool chunk_merge_fused = cache->head_size == 128 && pl.chunk_max_splits <= pa::kMaxFusedSplits;
+    p.chunk_fused_merge = chunk_merge_fused ? 1 : 0;
+    if (pl.decode_max_splits > 1 || (pl.chunk_max_splits > 1 && chunk_merge_fused)) {
         e = pa::launch_zero_counters(p.split_counters, num_tokens * cache->num_kv_heads, s);
         if (e != cudaSuccess) return fail_cuda(e);
     }
@@ -536,7 +539,7 @@ int pa_attention_ex(const pa_cache* cache, const void* q, int num_q_heads,
         if (e != cudaSuccess) return fail_cuda(e);
         if (ev) record(ev[3], s);
     }
-    if (pl.chunk_max_splits > 1) {
+    if (pl.chunk_max_splits > 1 && !chunk_merge_fused) {
         if (ev) record(ev[4], s);
         e = pa::launch_reduce(p, list, cache->head_size, s);
         if (e != cudaSuccess) return fail_cuda(e);

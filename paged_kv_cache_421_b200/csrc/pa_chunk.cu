@@ -39,20 +39,22 @@ chunk_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
     using C = ChunkCfg<D>;
     pdl_trigger();
     pdl_wait();
-    int qt, split, r;
+    int qt, split, r, g;
     if (work.count > 0) {
-        const uint32_t item = work.item[blockIdx.x];
+        // grid (kv heads, items): the kv head varies fastest, so CTAs dispatch item by item
+        const uint32_t item = work.item[blockIdx.y];
         r = static_cast<int>(item & (kChunkWorkMaxReq - 1));
         qt = static_cast<int>((item >> 10) & (kChunkWorkMaxQt - 1));
         split = static_cast<int>(item >> 22);
+        g = blockIdx.x;
     } else {
         // the last query tiles see the most keys (causal): dispatch them first
         qt = p.chunk_max_qtiles - 1 - static_cast<int>(blockIdx.x % p.chunk_max_qtiles);
         split = blockIdx.x / p.chunk_max_qtiles;
         r = static_cast<int>(blockIdx.z);
+        g = blockIdx.y;
     }
-    if (r >= p.num_seqs) return;
-    const int g = blockIdx.y;
+    if (r >= p.num_seqs || g >= p.num_kv_heads) return;
     const int q0 = p.qsl[r];
     const int q_len = p.qsl[r + 1] - q0;
     if (q_len <= 0 || is_decode_kind(q_len, p.group)) return;
@@ -330,7 +332,7 @@ cudaError_t launch_chunk_t(const CUtensorMap& tmap, const AttnParams& p, const C
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    const dim3 grid = work.count > 0 ? dim3(work.count, p.num_kv_heads, 1)
+    const dim3 grid = work.count > 0 ? dim3(p.num_kv_heads, work.count, 1)
                                      : dim3(p.chunk_max_qtiles * max_splits, p.num_kv_heads, p.num_seqs);
     return launch_pdl(chunk_kernel<D>, grid, dim3(128), C::kSmemBytes, stream, tmap, p, work);
 }

@@ -154,6 +154,11 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map
         : "memory");
 }
 
+// Barrier `id` among the first `count` threads of the CTA (whole warps).
+__device__ __forceinline__ void named_barrier_sync(int id, int count) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
@@ -165,6 +170,10 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 // total, and each sub-partition holds 2 x 232 + 40 registers per lane (16128 <= 16384).
 constexpr int kThreads = 384;
 constexpr uint32_t kRegsSoftmax = 232, kRegsProducer = 40;
+constexpr int kQLoaders = 256;           // the softmax warps stage Q
+constexpr int kEpiRowBytes = 32 * 4 + 16;  // epilogue staging row: 32 floats + 16 B (no conflicts)
+constexpr int kEpiWarpBytes = 32 * kEpiRowBytes;
+constexpr int kMergeRows = 8;            // rows a warp merges with all loads in flight
 static_assert(8 * 32 * kRegsSoftmax + 4 * 32 * kRegsProducer <= kThreads * 168,
               "register split exceeds the launch's registers");
 
@@ -174,20 +183,22 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
     pdl_trigger();
     pdl_wait();
     int* err = p.err;
-    int qt, split, r;
+    int qt, split, r, g;
     if (work.count > 0) {
-        const uint32_t item = work.item[blockIdx.x];
+        // grid (kv heads, items): the kv head varies fastest, so CTAs dispatch item by item
+        const uint32_t item = work.item[blockIdx.y];
         r = static_cast<int>(item & (kChunkWorkMaxReq - 1));
         qt = static_cast<int>((item >> 10) & (kChunkWorkMaxQt - 1));
         split = static_cast<int>(item >> 22);
+        g = blockIdx.x;
     } else {
         // the last query tiles see the most keys (causal): dispatch them first
         qt = p.chunk_max_qtiles - 1 - static_cast<int>(blockIdx.x % p.chunk_max_qtiles);
         split = blockIdx.x / p.chunk_max_qtiles;
         r = static_cast<int>(blockIdx.z);
+        g = blockIdx.y;
     }
-    if (r >= p.num_seqs) return;
-    const int g = blockIdx.y;
+    if (r >= p.num_seqs || g >= p.num_kv_heads) return;
     const int q0 = p.qsl[r];
     const int q_len = p.qsl[r + 1] - q0;
     if (q_len <= 0 || is_decode_kind(q_len, p.group)) return;
@@ -223,6 +234,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
     __shared__ uint64_t bar_kf[kKSlots], bar_ke[kKSlots], bar_vf[kVSlots], bar_ve[kVSlots];
     __shared__ uint64_t bar_sf[kQTiles], bar_pf[kQTiles];  // S computed / P stored
     __shared__ uint64_t bar_o[kQTiles];                    // a P V of the q-tile done
+    __shared__ uint64_t bar_q;                             // Q staged by the softmax warps
     __shared__ uint32_t tmem_holder;
     __shared__ int ids[kMaxIds];  // physical ids of the split's first kMaxIds logical blocks
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -255,6 +267,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
             mbar_init(smem_u32(&bar_pf[q]), kRows);
             mbar_init(smem_u32(&bar_o[q]), 1);
         }
+        mbar_init(smem_u32(&bar_q), kQLoaders);
         fence_barrier_init();
     }
     for (int k = tid; k < min(je - jb, kMaxIds); k += kThreads) {
@@ -265,31 +278,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
         }
         ids[k] = blk;
     }
-    // Q tiles -> shared memory in the swizzled K-major layout [q-tile][half][row][128 B]; every
-    // load of a thread is issued before its first store, so their latencies overlap
-    {
-        constexpr int kVecs = kQTiles * kRows * (kD / 8), kPer = (kVecs + kThreads - 1) / kThreads;
-        uint4 v[kPer];
-#pragma unroll
-        for (int i = 0; i < kPer; ++i) {
-            const int idx = tid + i * kThreads;
-            const int Rr = R0 + (idx >> 4), c = idx & 15;
-            v[i] = make_uint4(0, 0, 0, 0);
-            if (idx < kVecs && Rr < rows_total)
-                v[i] = __ldg(reinterpret_cast<const uint4*>(
-                    p.q + (static_cast<int64_t>(q0 + Rr / G) * p.num_q_heads + g * G + Rr % G) * kD +
-                    c * 8));
-        }
-#pragma unroll
-        for (int i = 0; i < kPer; ++i) {
-            const int idx = tid + i * kThreads;
-            const int rr = idx >> 4, c = idx & 15;  // rr over both q-tiles
-            if (idx < kVecs)
-                *reinterpret_cast<uint4*>(smem + (rr >> 7) * kQBytes + (c >> 3) * kQHalf +
-                                          sw128(rr & (kRows - 1), c & 7)) = v[i];
-        }
-    }
-    fence_proxy_async();  // Q's generic-proxy stores, before the tensor core reads them
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -370,7 +358,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
                                (t > 0 || j > 0) ? 1u : 0u);
                     mma_commit(smem_u32(&bar_o[q]));
                 };
-                if (mbar_wait(smem_u32(&bar_kf[0]), 0, kWaitLimitNs, err)) {
+                if (mbar_wait(smem_u32(&bar_q), 0, kWaitLimitNs, err) &&
+                    mbar_wait(smem_u32(&bar_kf[0]), 0, kWaitLimitNs, err)) {
                     tc_fence_after();
                     for (int q = 0; q < nq; ++q) qk(q, 0);
                     mma_commit(smem_u32(&bar_ke[0]));
@@ -400,6 +389,32 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
             }
         }
     } else {
+        // Q tiles -> shared memory in the swizzled K-major layout [q-tile][half][row][128 B],
+        // by the softmax warps while the producer already fetches the first K / V tiles; every
+        // load of a thread is issued before its first store, so their latencies overlap
+        {
+            constexpr int kVecs = kQTiles * kRows * (kD / 8), kPer = kVecs / kQLoaders;
+            uint4 v[kPer];
+#pragma unroll
+            for (int i = 0; i < kPer; ++i) {
+                const int idx = tid + i * kQLoaders;
+                const int Rr = R0 + (idx >> 4), c = idx & 15;
+                v[i] = make_uint4(0, 0, 0, 0);
+                if (Rr < rows_total)
+                    v[i] = __ldg(reinterpret_cast<const uint4*>(
+                        p.q + (static_cast<int64_t>(q0 + Rr / G) * p.num_q_heads + g * G + Rr % G) * kD +
+                        c * 8));
+            }
+#pragma unroll
+            for (int i = 0; i < kPer; ++i) {
+                const int idx = tid + i * kQLoaders;
+                const int rr = idx >> 4, c = idx & 15;  // rr over both q-tiles
+                *reinterpret_cast<uint4*>(smem + (rr >> 7) * kQBytes + (c >> 3) * kQHalf +
+                                          sw128(rr & (kRows - 1), c & 7)) = v[i];
+            }
+            fence_proxy_async();  // generic-proxy stores, before the tensor core reads them
+            mbar_arrive(smem_u32(&bar_q));
+        }
         asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoftmax));
         if (warp / 4 < nq) {
             // ================= softmax: thread = row = TMEM lane of its q-tile
@@ -515,37 +530,130 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
             // last one, so one phase of the q-tile's P V barrier is outstanding here.
             if (ok && ntiles > 0 && !mbar_wait(smem_u32(&bar_o[q]), (ntiles - 1) & 1, kWaitLimitNs, err))
                 ok = false;
-            // tcgen05.ld is warp-collective: the whole warp loads (or none of it), rows store
-            const bool have = __all_sync(0xffffffffu, ok) && ntiles > 0;
-            const int t = q0 + R / G, h = g * G + R % G;
+            // tcgen05.ld is warp-collective: the whole warp loads (or none of it)
+            const bool all_ok = __all_sync(0xffffffffu, ok);
+            const bool have = all_ok && ntiles > 0;
             const float inv = l > 0.f ? 1.f / l : 0.f;
-            float* dst = nullptr;
-            if (ok && valid) {
-                if (nsplit == 1) {
-                    dst = p.out + (static_cast<int64_t>(t) * p.num_q_heads + h) * kD;
-                } else {
-                    const int64_t prow = (static_cast<int64_t>(split) * p.num_tokens + t) * p.num_q_heads + h;
-                    dst = p.part_o + prow * kD;
-                    p.part_lse[prow] = l > 0.f ? m_used + __log2f(l) : -INFINITY;
+            if (all_ok && valid && nsplit > 1) {
+                const int t = q0 + R / G, h = g * G + R % G;
+                p.part_lse[(static_cast<int64_t>(split) * p.num_tokens + t) * p.num_q_heads + h] =
+                    l > 0.f ? m_used + __log2f(l) : -INFINITY;
+            }
+            if (all_ok) {
+                // O / l through shared memory (this q-tile's Q region: its last MMA has
+                // completed), 32 columns at a time, so that each store instruction of the warp
+                // writes four whole 128-byte row segments instead of 32 scattered pieces
+                uint8_t* stage = smem + q * kQBytes + (warp & 3) * kEpiWarpBytes;
+                const int row_base = R0 + q * kRows + (warp & 3) * 32;
+                if (have) tc_fence_after();
+#pragma unroll
+                for (int c = 0; c < kD / 32; ++c) {
+                    uint32_t raw[32];
+                    if (have) {
+                        tmem_ld32(tmem_lane + kColO + c * 32, raw);
+                        tmem_wait_ld();
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) raw[i] = 0u;
+                    }
+                    float4* srow = reinterpret_cast<float4*>(stage + lane * kEpiRowBytes);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        srow[i] = make_float4(__uint_as_float(raw[4 * i]) * inv,
+                                              __uint_as_float(raw[4 * i + 1]) * inv,
+                                              __uint_as_float(raw[4 * i + 2]) * inv,
+                                              __uint_as_float(raw[4 * i + 3]) * inv);
+                    __syncwarp();
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const int rl = 4 * k + (lane >> 3), ch = lane & 7;
+                        const int Rr = row_base + rl;
+                        if (Rr < rows_total) {
+                            const int t = q0 + Rr / G, h = g * G + Rr % G;
+                            float* dst = nsplit == 1
+                                             ? p.out + (static_cast<int64_t>(t) * p.num_q_heads + h) * kD
+                                             : p.part_o + ((static_cast<int64_t>(split) * p.num_tokens + t) *
+                                                               p.num_q_heads + h) * kD;
+                            *reinterpret_cast<float4*>(dst + 32 * c + 4 * ch) =
+                                *reinterpret_cast<const float4*>(stage + rl * kEpiRowBytes + ch * 16);
+                        }
+                    }
+                    __syncwarp();
                 }
             }
-            if (have) tc_fence_after();
-    #pragma unroll
-            for (int c = 0; c < kD / 32; ++c) {
-                uint32_t raw[32];
-                if (have) {
-                    tmem_ld32(tmem_lane + kColO + c * 32, raw);
-                    tmem_wait_ld();
-                } else {
-    #pragma unroll
-                    for (int i = 0; i < 32; ++i) raw[i] = 0u;
+        }
+        if (nsplit > 1 && p.chunk_fused_merge) {
+            // ---- split merge: the last CTA of this (q-tile pair, kv head) to finish merges
+            // every split's (O_s, lse_s): out = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M),
+            // M = max_s lse_s (at most kMaxFusedSplits splits; the host launches the reduce
+            // kernel otherwise).  Counters start at zero on every call (cleared on the stream
+            // before the launch); decode requests use other tokens' counters.
+            __shared__ int s_last;
+            __threadfence();
+            named_barrier_sync(1, kQLoaders);  // every partial of this CTA is written
+            if (tid == 0) {
+                const int ctr = (q0 + R0 / G) * p.num_kv_heads + g;
+                s_last = atomicAdd(p.split_counters + ctr, 1) == nsplit - 1;
+            }
+            named_barrier_sync(1, kQLoaders);
+            if (s_last) {
+                __threadfence();
+                const int64_t stride = static_cast<int64_t>(p.num_tokens) * p.num_q_heads;
+                auto row_of = [&](int Rr) {
+                    return static_cast<int64_t>(q0 + Rr / G) * p.num_q_heads + g * G + Rr % G;
+                };
+                // phase 1: thread t turns row R0 + t's LSEs into normalised split weights
+                float* wsm = reinterpret_cast<float*>(smem);  // [256 rows][kMaxFusedSplits]
+                {
+                    const int Rr = R0 + tid;
+                    float w[kMaxFusedSplits];
+                    float M = -INFINITY;
+#pragma unroll
+                    for (int sp = 0; sp < kMaxFusedSplits; ++sp) {
+                        w[sp] = (Rr < rows_total && sp < nsplit)
+                                    ? __ldcg(p.part_lse + sp * stride + row_of(Rr)) : -INFINITY;
+                        M = fmaxf(M, w[sp]);
+                    }
+                    float W = 0.f;
+#pragma unroll
+                    for (int sp = 0; sp < kMaxFusedSplits; ++sp) {
+                        w[sp] = M == -INFINITY ? 0.f : ex2(w[sp] - M);
+                        W += w[sp];
+                    }
+                    const float inv = W > 0.f ? 1.f / W : 0.f;
+#pragma unroll
+                    for (int sp = 0; sp < kMaxFusedSplits; ++sp) wsm[tid * kMaxFusedSplits + sp] = w[sp] * inv;
                 }
-                if (dst) {
-    #pragma unroll
-                    for (int i = 0; i < 32; i += 4)
-                        *reinterpret_cast<float4*>(dst + c * 32 + i) = make_float4(
-                            __uint_as_float(raw[i]) * inv, __uint_as_float(raw[i + 1]) * inv,
-                            __uint_as_float(raw[i + 2]) * inv, __uint_as_float(raw[i + 3]) * inv);
+                named_barrier_sync(1, kQLoaders);
+                // phase 2: warp w merges rows w, w + 8, ..., lane l the 16 bytes at 4l of each
+                // row (coalesced), kMergeRows rows with all their loads in flight at once
+                for (int i0 = 0; i0 < 32; i0 += kMergeRows) {
+                    float4 v[kMergeRows][kMaxFusedSplits];
+#pragma unroll
+                    for (int b2 = 0; b2 < kMergeRows; ++b2) {
+                        const int Rr = R0 + warp + 8 * (i0 + b2);
+#pragma unroll
+                        for (int sp = 0; sp < kMaxFusedSplits; ++sp)
+                            v[b2][sp] = (Rr < rows_total && sp < nsplit)
+                                            ? __ldcg(reinterpret_cast<const float4*>(
+                                                         p.part_o + (sp * stride + row_of(Rr)) * kD) + lane)
+                                            : make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+#pragma unroll
+                    for (int b2 = 0; b2 < kMergeRows; ++b2) {
+                        const int rl = warp + 8 * (i0 + b2), Rr = R0 + rl;
+                        if (Rr >= rows_total) continue;
+                        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                        for (int sp = 0; sp < kMaxFusedSplits; ++sp) {
+                            const float w = wsm[rl * kMaxFusedSplits + sp];
+                            acc.x += w * v[b2][sp].x;
+                            acc.y += w * v[b2][sp].y;
+                            acc.z += w * v[b2][sp].z;
+                            acc.w += w * v[b2][sp].w;
+                        }
+                        reinterpret_cast<float4*>(p.out + row_of(Rr) * kD)[lane] = acc;
+                    }
                 }
             }
         }
@@ -570,7 +678,7 @@ cudaError_t launch_chunk_tc(const CUtensorMap& tmap_blk, const AttnParams& p, co
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    const dim3 grid = work.count > 0 ? dim3(work.count, p.num_kv_heads, 1)
+    const dim3 grid = work.count > 0 ? dim3(p.num_kv_heads, work.count, 1)
                                      : dim3(p.chunk_max_qtiles * max_splits, p.num_kv_heads, p.num_seqs);
     return launch_pdl(chunk_tc_kernel, grid, dim3(kThreads), kSmemBytes, stream, tmap_blk, p, work);
 }

@@ -18,6 +18,7 @@ namespace pa {
 constexpr int kBlockSize = 16;      // tokens per physical block (the pages' default)
 constexpr int kDecodeRows = 8;      // decode tile: q_len * group <= 8 rows share one kv head
 constexpr int kChunkRows = 64;      // mma.sync chunk tile: 64 (token, q head) rows per CTA
+constexpr int kMaxFusedSplits = 4;    // tcgen05 chunk kernel: splits it merges itself
 constexpr int kChunkRowsTc = 256;   // tcgen05 chunk CTA: two 128-row q-tiles (TMEM lanes)
 
 // Error codes written to the device error word.

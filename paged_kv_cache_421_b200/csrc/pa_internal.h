@@ -68,6 +68,7 @@ struct AttnParams {
     int reduce_row_tiles;       // grid.x of the reduce: 4-row tiles of the largest split request
     float scale_log2;           // softmax scale * log2(e)
     int* err;                   // device error word
+    int chunk_fused_merge;      // tcgen05 chunk kernel merges its own splits (<= kMaxFusedSplits)
 };
 
 // The chunk-kind requests of a launch, longest context first (passed by value, so the chunk
