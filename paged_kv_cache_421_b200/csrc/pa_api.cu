@@ -223,11 +223,12 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
             if (csb > kMaxChunkSplitBlocks && allowed > 1)  // keep block ids in shared memory
                 csb = round_up(pa::ceil_div(chunk_max_blocks,
                                             pa::ceil_div(chunk_max_blocks, kMaxChunkSplitBlocks)), 4);
-            // one CTA per SM: split the KV walk when the longest CTA would walk well past the
-            // average work per SM, so that no SM is left with most of the step
+            // one CTA per SM: split the KV walk only when the longest CTA would walk more than
+            // three times the average work per SM.  A split writes fp32 partials of every row
+            // and merges them, which costs more than a 2x imbalance (measured on the mixed step).
             const long long per_sm = (chunk_work + num_sms - 1) / num_sms;
             const long long target = std::max<long long>(per_sm, kMinChunkSplitTiles);
-            if (chunk_work_max > target + target / 2) {
+            if (chunk_work_max > 3 * target) {
                 const int tile_blocks = chunk_tile_keys / bs;
                 const int sb = static_cast<int>(target) * tile_blocks;
                 if (sb < csb) csb = round_up(std::max(sb, kMinChunkSplitBlocks), 4);

@@ -106,6 +106,29 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
+// Packed two-wide fp32 arithmetic and three-input max (sm_100): half the instructions for the
+// softmax's per-score scale, sum and max.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;"
+        : "=l"(d)
+        : "l"(*reinterpret_cast<uint64_t*>(&a)), "l"(*reinterpret_cast<uint64_t*>(&b)),
+          "l"(*reinterpret_cast<uint64_t*>(&c)));
+    return *reinterpret_cast<float2*>(&d);
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;"
+        : "=l"(d)
+        : "l"(*reinterpret_cast<uint64_t*>(&a)), "l"(*reinterpret_cast<uint64_t*>(&b)));
+    return *reinterpret_cast<float2*>(&d);
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
 // 32 consecutive 32-bit columns of this thread's TMEM lane.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile(
@@ -340,7 +363,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
             if (lane == 0 && ntiles > 0) {
                 auto qk = [&](int q, int t) {  // S_q = Q_q K_t^T
                     const uint32_t ks = k_s + (t & 1) * kKBytes;
-    #pragma unroll
+#pragma unroll
                     for (int k = 0; k < kD / 16; ++k) {
                         const uint32_t off = q * kQBytes + (k >> 2) * kQHalf + (k & 3) * 32;
                         const uint32_t koff = (k >> 2) * kAtom + (k & 3) * 32;
@@ -351,7 +374,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
                 };
                 auto pv = [&](int q, int t) {  // O_q += P_q V_t (P from TMEM)
                     const uint32_t vs = v_s + (t & 1) * kKBytes;
-    #pragma unroll
+#pragma unroll
                     for (int j = 0; j < kKeys / 16; ++j)
                         mma_ts(tmem + q * 256 + kColO, tmem + q * 256 + 8 * j,
                                smem_desc(vs + j * kBlockTile, kAtom, kGroupStride), kIdescPV,
@@ -440,16 +463,16 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
                 const bool masked = !(key0 + kKeys - 1 <= first_lim && key0 + kKeys <= kend);
                 // S of this row: all four loads in flight, one wait (TMEM load latency is long)
                 float sv[kKeys];
-    #pragma unroll
+#pragma unroll
                 for (int c = 0; c < kKeys / 32; ++c) {
                     uint32_t raw[32];
                     tmem_ld32(tmem_lane + c * 32, raw);
-    #pragma unroll
+#pragma unroll
                     for (int i = 0; i < 32; ++i) sv[c * 32 + i] = __uint_as_float(raw[i]);
                 }
                 tmem_wait_ld();
                 if (masked) {
-    #pragma unroll
+#pragma unroll
                     for (int c = 0; c < kKeys; ++c) {
                         const int pos = key0 + c;
                         if (pos > lim || pos >= kend) sv[c] = -INFINITY;
@@ -457,12 +480,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
                 }
                 // the row max with independent partial maxima (short dependency chains)
                 float mp[8];
-    #pragma unroll
+#pragma unroll
                 for (int i = 0; i < 8; ++i) mp[i] = sv[i];
-    #pragma unroll
-                for (int c = 8; c < kKeys; ++c) mp[c & 7] = fmaxf(mp[c & 7], sv[c]);
-                float mx = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                                 fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+#pragma unroll
+                for (int c = 8; c < kKeys; c += 2) mp[(c >> 1) & 7] = fmax3(mp[(c >> 1) & 7], sv[c], sv[c + 1]);
+                float mx = fmaxf(fmax3(mp[0], mp[1], mp[2]), fmax3(mp[3], mp[4], fmax3(mp[5], mp[6], mp[7])));
                 mx *= sl;  // scores stay unscaled: max(s) * sl is the scaled max (sl > 0)
                 const float m_new = fmaxf(m_used, mx);
                 float alpha = 1.f;
@@ -476,12 +498,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
                     // rescale O (this warp's 32 rows): the commit that signalled S of this tile
                     // also covers the q-tile's previous P V
                     l *= alpha;
-    #pragma unroll
+#pragma unroll
                     for (int c = 0; c < kD / 32; ++c) {
                         uint32_t raw[32];
                         tmem_ld32(tmem_lane + kColO + c * 32, raw);
                         tmem_wait_ld();
-    #pragma unroll
+#pragma unroll
                         for (int i = 0; i < 32; ++i)
                             raw[i] = __float_as_uint(__uint_as_float(raw[i]) * alpha);
                         tmem_st32(tmem_lane + kColO + c * 32, raw);
@@ -489,20 +511,21 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
                 }
                 // P = 2^(s sl - m) as bf16 pairs over the first 64 S columns, 32 keys at a time
                 const float neg_ref = m_used == -INFINITY ? 0.f : -m_used;
-                float sp[4] = {0.f, 0.f, 0.f, 0.f};
-    #pragma unroll
+                const float2 sl2 = make_float2(sl, sl), nr2 = make_float2(neg_ref, neg_ref);
+                float2 sp[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll
                 for (int c = 0; c < kKeys / 32; ++c) {
                     uint32_t packed[16];
-    #pragma unroll
+#pragma unroll
                     for (int i = 0; i < 16; ++i) {
-                        const float a0 = ex2(fmaf(sv[32 * c + 2 * i], sl, neg_ref));
-                        const float a1 = ex2(fmaf(sv[32 * c + 2 * i + 1], sl, neg_ref));
-                        sp[i & 3] += a0 + a1;
-                        packed[i] = pack_bf16(a0, a1);
+                        const float2 x = ffma2(make_float2(sv[32 * c + 2 * i], sv[32 * c + 2 * i + 1]), sl2, nr2);
+                        const float2 a = make_float2(ex2(x.x), ex2(x.y));
+                        sp[i & 1] = fadd2(sp[i & 1], a);
+                        packed[i] = pack_bf16(a.x, a.y);
                     }
                     tmem_st16(tmem_lane + 16 * c, packed);
                 }
-                l += (sp[0] + sp[1]) + (sp[2] + sp[3]);
+                l += (sp[0].x + sp[0].y) + (sp[1].x + sp[1].y);
                 tmem_wait_st();
                 if (q == 0 && key0 + kKeys > kend) {
                     // keys past the split / context: clear their V rows once V has landed (q-tile 0
