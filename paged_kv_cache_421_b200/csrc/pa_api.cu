@@ -140,7 +140,7 @@ int round_up(int x, int m) { return (x + m - 1) / m * m; }
 // Planner constants.
 constexpr int kDecodeCtasPerSm = 3;    // decode kernel residency (64 KB of stages per CTA)
 constexpr int kMaxDecodeSplits = 1024;  // merge weights of one row fit the CTA's shared memory
-constexpr int kDecodeWaves = 4;             // target waves of decode CTAs
+constexpr int kDecodeWaves = 2;             // target waves of decode CTAs (2 measured best)
 constexpr int kMinDecodeSplitBlocks = 64;   // >= 1024 keys per split
 constexpr int kMinChunkSplitBlocks = 16;
 constexpr int kMinChunkSplitTiles = 4;      // a chunk split walks at least four key tiles
