@@ -77,6 +77,10 @@ def _load():
     lib.oracle_e4m3_decode_array.argtypes = [P, i64, P]
     lib.oracle_slot_mapping.restype = i32
     lib.oracle_slot_mapping.argtypes = [P, i32, P, P, i32, i32, P]
+    lib.oracle_allocate_slots.restype = i32
+    lib.oracle_allocate_slots.argtypes = [P, i32, P, P, i32, i32, P, i32, P, P]
+    lib.oracle_free_blocks.restype = i32
+    lib.oracle_free_blocks.argtypes = [P, i32, P, i32, P]
     lib.oracle_write_kv_bf16.restype = None
     lib.oracle_write_kv_bf16.argtypes = [P, i32, i32, i32, i32, P, P, P, i32]
     lib.oracle_write_kv_fp8.restype = None
@@ -149,6 +153,30 @@ def slot_mapping(block_table: np.ndarray, seq_lens: np.ndarray, qsl: np.ndarray,
     _check(_load().oracle_slot_mapping(_p(bt), bt.shape[1], _p(sl), _p(q), sl.size,
                                        block_size, _p(out)), "oracle_slot_mapping")
     return out
+
+
+def allocate_slots(block_table: np.ndarray, num_computed, num_new, block_size: int,
+                   queue: np.ndarray, state: np.ndarray) -> np.ndarray:
+    """In place on block_table (int32 [B][max_blocks]) and state (int32 [head, count]); returns
+    num_allocated (int32 [B], -1 for a request not served).  See oracle_allocate_slots."""
+    assert block_table.dtype == np.int32 and block_table.flags.c_contiguous
+    assert state.dtype == np.int32 and state.size == 2
+    c = _c(np.asarray(num_computed), np.int32)
+    n = _c(np.asarray(num_new), np.int32)
+    q = _c(queue, np.int32)
+    out = np.zeros(c.size, np.int32)
+    _check(_load().oracle_allocate_slots(_p(block_table), block_table.shape[1], _p(c), _p(n),
+                                         c.size, block_size, _p(q), q.size, _p(state), _p(out)),
+           "oracle_allocate_slots")
+    return out
+
+
+def free_blocks(ids, queue: np.ndarray, state: np.ndarray) -> None:
+    """In place on queue (int32 ring) and state (int32 [head, count])."""
+    assert queue.dtype == np.int32 and state.dtype == np.int32
+    i = _c(np.asarray(ids), np.int32)
+    _check(_load().oracle_free_blocks(_p(i), i.size, _p(queue), queue.size, _p(state)),
+           "oracle_free_blocks")
 
 
 def write_kv(cache: np.ndarray, kv_dtype: int, num_blocks: int, block_size: int,

@@ -164,6 +164,61 @@ int oracle_slot_mapping(const int32_t* block_table, int max_blocks_per_seq,
     return OR_OK;
 }
 
+/* ------------------------------------------------------------------ block allocation */
+/* The pages' allocate_slots ("Inside vLLM" reading notes, core point 1; the free-block queue of
+   the "vLLM architecture overview", section 2): for each request, in scheduling order,
+     1. count the new blocks it needs: ceil((computed + new) / bs) - ceil(computed / bs)
+        (a fresh request with 17 new tokens needs ceil(17/16) = 2);
+     2. check that the free-block queue holds that many;
+     3. take them from the head of the queue, in queue order, and append them to the request's
+        block-table row.
+   Batched reading (the pages describe one request at a time): requests are served in order and
+   service stops at the first request that cannot be placed -- too few free blocks, or a row
+   that would exceed max_blocks_per_seq -- so that request and every later one get nothing.
+   The queue is a ring of `capacity` ids; state[0] = head index, state[1] = free count.
+   num_allocated[r] = blocks taken by request r, or -1 when it was not served. */
+int oracle_allocate_slots(int32_t* block_table, int max_blocks_per_seq,
+                          const int32_t* num_computed, const int32_t* num_new, int num_seqs,
+                          int block_size, const int32_t* queue, int capacity, int32_t* state,
+                          int32_t* num_allocated) {
+    int r, j, stopped = 0;
+    int64_t head = state[0], count = state[1];
+    if (capacity <= 0 || head < 0 || head >= capacity || count < 0 || count > capacity)
+        return OR_BAD_ARG;
+    for (r = 0; r < num_seqs; ++r) {
+        int64_t c = num_computed[r], n = num_new[r], have, total, need;
+        if (c < 0 || n < 0) return OR_BAD_META;
+        have = oracle_blocks_needed(c, block_size);
+        total = oracle_blocks_needed(c + n, block_size);
+        need = total - have;
+        if (stopped || total > max_blocks_per_seq || need > count) {
+            stopped = 1;
+            num_allocated[r] = -1;
+            continue;
+        }
+        for (j = 0; j < need; ++j)
+            block_table[(int64_t)r * max_blocks_per_seq + have + j] = queue[(head + j) % capacity];
+        head = (head + need) % capacity;
+        count -= need;
+        num_allocated[r] = (int32_t)need;
+    }
+    state[0] = (int32_t)head;
+    state[1] = (int32_t)count;
+    return OR_OK;
+}
+
+/* Freed blocks go back to the tail of the queue, in the order given. */
+int oracle_free_blocks(const int32_t* ids, int num_ids, int32_t* queue, int capacity,
+                       int32_t* state) {
+    int i;
+    int64_t tail;
+    if (num_ids < 0 || (int64_t)state[1] + num_ids > capacity) return OR_BAD_ARG;
+    tail = ((int64_t)state[0] + state[1]) % capacity;
+    for (i = 0; i < num_ids; ++i) queue[(tail + i) % capacity] = ids[i];
+    state[1] += num_ids;
+    return OR_OK;
+}
+
 /* ------------------------------------------------------------------ cache write */
 /* k, v: bf16 [num_tokens][num_kv_heads][head_size].  A negative slot means "no write". */
 void oracle_write_kv_bf16(uint16_t* cache, int num_blocks, int block_size, int num_kv_heads,

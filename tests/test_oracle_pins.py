@@ -482,3 +482,101 @@ def test_write_fp8_divides_at_ties(oracle_mod):
     c = cache.reshape(n, 2)
     for j, r in enumerate(rows):
         assert c[j, 0] == int(r[3], 16) and c[j, 1] == int(r[3], 16), r
+
+
+# ------------------------------------------------------------------ block allocation
+# allocate_slots as "Inside vLLM" reading notes, core point 1 describe it: count the new blocks
+# (17 new tokens need ceil(17/16) = 2), check the free pool, take blocks from the head of the
+# free-block queue ("vLLM architecture overview", section 2).  Expected values hand-computed.
+
+def _alloc(om, rows, computed, new, queue, head, count, max_blocks=8, bs=16, capacity=None):
+    q = np.array(queue, np.int32)
+    if capacity is not None:
+        assert q.size == capacity
+    bt = np.full((len(computed), max_blocks), -9, np.int32)
+    for r, row in enumerate(rows):
+        bt[r, :len(row)] = row
+    st = np.array([head, count], np.int32)
+    got = om.allocate_slots(bt, computed, new, bs, q, st)
+    return got, bt, st
+
+
+def test_allocate_worked_example_17_tokens_take_two_blocks_from_head(oracle_mod):
+    got, bt, st = _alloc(oracle_mod, [[]], [0], [17], [7, 3, 9, 1], 0, 4)
+    assert got.tolist() == [2]
+    assert bt[0, :3].tolist() == [7, 3, -9]
+    assert st.tolist() == [2, 2]
+
+
+def test_allocate_continues_a_partly_filled_block(oracle_mod):
+    # (computed, new) -> new blocks: (16, 1) -> 1; (17, 15) -> 0 (positions 17..31 fit block 1);
+    # (17, 16) -> 1; (0, 0) -> 0; (0, 16) -> 1; (0, 32) -> 2
+    cases = [((16, 1), 1), ((17, 15), 0), ((17, 16), 1), ((0, 0), 0), ((0, 16), 1), ((0, 32), 2)]
+    for (c, n), want in cases:
+        have = -(-c // 16)
+        got, bt, st = _alloc(oracle_mod, [[5] * have], [c], [n], [40, 41, 42], 0, 3)
+        assert got.tolist() == [want], (c, n)
+        assert bt[0, :have + want].tolist() == [5] * have + [40, 41, 42][:want]
+        assert bt[0, have + want] == -9
+        assert st.tolist() == [want, 3 - want]
+
+
+def test_allocate_stops_at_first_request_it_cannot_place(oracle_mod):
+    # pool of 3: requests need 2, 2, 1 -> the first is served, the second is not, and neither
+    # is the third (first come, first served stops), leaving one block
+    got, bt, st = _alloc(oracle_mod, [[], [], []], [0, 0, 0], [20, 32, 1], [4, 5, 6, 7], 0, 3)
+    assert got.tolist() == [2, -1, -1]
+    assert bt[0, :2].tolist() == [4, 5] and (bt[1:] == -9).all()
+    assert st.tolist() == [2, 1]
+
+
+def test_allocate_refuses_a_row_past_the_table(oracle_mod):
+    got, bt, st = _alloc(oracle_mod, [[1, 2]], [32], [1], [9, 8], 0, 2, max_blocks=2)
+    assert got.tolist() == [-1] and st.tolist() == [0, 2] and bt[0].tolist() == [1, 2]
+
+
+def test_allocate_wraps_around_the_ring_and_free_appends_at_tail(oracle_mod):
+    queue = np.array([20, 21, 0, 0, 24], np.int32)  # free ids at 4, 0, 1 (head 4, count 3)
+    st = np.array([4, 3], np.int32)
+    bt = np.full((1, 4), -9, np.int32)
+    assert oracle_mod.allocate_slots(bt, [0], [17], 16, queue, st).tolist() == [2]
+    assert bt[0, :2].tolist() == [24, 20] and st.tolist() == [1, 1]
+    oracle_mod.free_blocks([30, 31, 32], queue, st)  # tail at (1 + 1) % 5 = 2: slots 2, 3, 4
+    assert queue.tolist() == [20, 21, 30, 31, 32] and st.tolist() == [1, 4]
+    bt2 = np.full((1, 4), -9, np.int32)
+    assert oracle_mod.allocate_slots(bt2, [0], [64], 16, queue, st).tolist() == [4]
+    assert bt2[0].tolist() == [21, 30, 31, 32] and st.tolist() == [0, 0]
+    with pytest.raises(oracle_mod.OracleError):
+        oracle_mod.free_blocks(list(range(6)), queue, st)  # more than the ring holds
+
+
+def test_allocate_brute_force_invariants(oracle_mod):
+    rng = np.random.default_rng(77)
+    for _ in range(200):
+        B = int(rng.integers(1, 12))
+        cap = int(rng.integers(1, 40))
+        queue = rng.permutation(1000)[:cap].astype(np.int32)
+        head, count = int(rng.integers(0, cap)), int(rng.integers(0, cap + 1))
+        computed = rng.integers(0, 80, B)
+        new = rng.integers(0, 60, B)
+        have = -(-computed // 16)
+        bt = np.full((B, 10), -9, np.int32)
+        for r in range(B):
+            bt[r, :have[r]] = 100 + r
+        before = bt.copy()
+        st = np.array([head, count], np.int32)
+        got = oracle_mod.allocate_slots(bt, computed, new, 16, queue, st)
+        need = -(-(computed + new) // 16) - have
+        taken = []
+        served = True
+        for r in range(B):
+            fits = served and need[r] <= count - len(taken) and have[r] + need[r] <= 10
+            served = fits
+            assert got[r] == (need[r] if fits else -1)
+            if fits:
+                taken += bt[r, have[r]:have[r] + need[r]].tolist()
+            assert (bt[r, :have[r]] == before[r, :have[r]]).all()
+            k = have[r] + (need[r] if fits else 0)
+            assert (bt[r, k:] == -9).all()
+        assert taken == [int(queue[(head + j) % cap]) for j in range(len(taken))]
+        assert st.tolist() == [(head + len(taken)) % cap, count - len(taken)]
