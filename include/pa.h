@@ -100,6 +100,34 @@ int pa_slot_mapping(const int32_t* block_table, int max_blocks_per_seq, const in
                     const int32_t* query_start_loc, int num_seqs, int num_tokens,
                     int block_size, int32_t* slot_mapping, void* stream);
 
+/* Block allocation for a step ([P3] core point 1: allocate_slots counts the new blocks a
+ * request needs -- 17 new tokens take ceil(17/16) = 2 --, checks the free pool and takes the
+ * blocks from the head of the free-block queue; [P2] section 2: the free-block queue).
+ * The queue is a device ring: free_queue int32 [queue_capacity] of block ids and queue_state
+ * int32 [2] = {head index, number of free blocks}; both caller-owned, updated in place.
+ * Request r already holds ceil(num_computed[r] / block_size) blocks (the first entries of its
+ * block_table row) and grows by num_new[r] tokens, so it needs
+ *     ceil((num_computed[r] + num_new[r]) / block_size) - ceil(num_computed[r] / block_size)
+ * new blocks, written in queue order after its existing entries.  Requests are served in
+ * order and service stops at the first request that cannot be placed (too few free blocks,
+ * or a row longer than max_blocks_per_seq): it and every later request get nothing.
+ * num_allocated: device int32 [num_seqs] output, the blocks taken by each request or -1 when
+ * it was not served.  block_table entries other than the new ones are left unchanged.
+ * num_computed, num_new: device int32 [num_seqs], >= 0 (a negative value or a queue state out
+ * of range records a device error and leaves the queue unchanged).  Afterwards the slot
+ * mapping of the step is pa_slot_mapping with seq_lens = num_computed + num_new.
+ * Errors: INVALID_ARG, CUDA. */
+int pa_allocate_slots(int32_t* block_table, int max_blocks_per_seq, const int32_t* num_computed,
+                      const int32_t* num_new, int num_seqs, int block_size,
+                      const int32_t* free_queue, int queue_capacity, int32_t* queue_state,
+                      int32_t* num_allocated, void* stream);
+
+/* Return blocks to the tail of the free-block queue, in the order given ([P2] section 2).
+ * block_ids: device int32 [num_ids].  If the queue would hold more than queue_capacity ids,
+ * nothing is written and a device error is recorded.  Errors: INVALID_ARG, CUDA. */
+int pa_free_blocks(const int32_t* block_ids, int num_ids, int32_t* free_queue,
+                   int queue_capacity, int32_t* queue_state, void* stream);
+
 /* Cache write, reshape_and_cache ([P2] section 3): for every token t with slot s =
  * slot_mapping[t] >= 0 and every kv head h, K and V rows are stored at token s % block_size of
  * block s / block_size.  bf16 pools store the bits unchanged; FP8 pools store

@@ -32,7 +32,7 @@ EXPORTED = [
     "pa_cache_bytes", "pa_alloc_cache", "pa_free_cache", "pa_cache_data", "pa_slot_mapping",
     "pa_write_kv", "pa_attention_workspace_bytes", "pa_attention", "pa_plan_attention",
     "pa_attention_ex", "pa_validate_block_table", "pa_device_error", "pa_status_string",
-    "pa_last_cuda_error", "pa_attention_noalloc",
+    "pa_last_cuda_error", "pa_attention_noalloc", "pa_allocate_slots", "pa_free_blocks",
 ]
 PA_NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -95,6 +95,8 @@ def load() -> ctypes.CDLL:
         "pa_cache_data": (P, [P]),
         "pa_slot_mapping": (I, [P, I, P, P, I, I, I, P, P]),
         "pa_write_kv": (I, [P, P, P, P, I, P]),
+        "pa_allocate_slots": (I, [P, I, P, P, I, I, P, I, P, P, P]),
+        "pa_free_blocks": (I, [P, I, P, I, P, P]),
         "pa_attention_workspace_bytes": (Z, [I, I, I, I]),
         "pa_attention": (I, [P, P, I, P, I, P, P, P, P, I, I, F, P, P, Z, P]),
         "pa_plan_attention": (I, [P, P, I, I, I, I, I, I, I, I, Z,
@@ -174,6 +176,21 @@ def pa_slot_mapping(block_table, max_blocks_per_seq, seq_lens, query_start_loc, 
     _check(load().pa_slot_mapping(_ptr(block_table), max_blocks_per_seq, _ptr(seq_lens),
                                   _ptr(query_start_loc), num_seqs, num_tokens, block_size,
                                   _ptr(slot_mapping), _stream(stream)), "pa_slot_mapping")
+
+
+def pa_allocate_slots(block_table, max_blocks_per_seq, num_computed, num_new, num_seqs,
+                      block_size, free_queue, queue_capacity, queue_state, num_allocated,
+                      stream=None) -> None:
+    _check(load().pa_allocate_slots(_ptr(block_table), max_blocks_per_seq, _ptr(num_computed),
+                                    _ptr(num_new), num_seqs, block_size, _ptr(free_queue),
+                                    queue_capacity, _ptr(queue_state), _ptr(num_allocated),
+                                    _stream(stream)), "pa_allocate_slots")
+
+
+def pa_free_blocks(block_ids, num_ids, free_queue, queue_capacity, queue_state,
+                   stream=None) -> None:
+    _check(load().pa_free_blocks(_ptr(block_ids), num_ids, _ptr(free_queue), queue_capacity,
+                                 _ptr(queue_state), _stream(stream)), "pa_free_blocks")
 
 
 def pa_write_kv(handle, k, v, slot_mapping, num_tokens, stream=None) -> None:

@@ -373,6 +373,34 @@ int pa_slot_mapping(const int32_t* block_table, int max_blocks_per_seq, const in
     return e == cudaSuccess ? PA_OK : fail_cuda(e);
 }
 
+int pa_allocate_slots(int32_t* block_table, int max_blocks_per_seq, const int32_t* num_computed,
+                      const int32_t* num_new, int num_seqs, int block_size,
+                      const int32_t* free_queue, int queue_capacity, int32_t* queue_state,
+                      int32_t* num_allocated, void* stream) {
+    if (num_seqs < 0 || block_size <= 0 || max_blocks_per_seq <= 0 || queue_capacity <= 0 ||
+        !queue_state)
+        return PA_ERR_INVALID_ARG;
+    if (num_seqs == 0) return PA_OK;
+    if (!block_table || !num_computed || !num_new || !free_queue || !num_allocated)
+        return PA_ERR_INVALID_ARG;
+    cudaError_t e = pa::launch_allocate_slots(block_table, max_blocks_per_seq, num_computed,
+                                              num_new, num_seqs, block_size, free_queue,
+                                              queue_capacity, queue_state, num_allocated,
+                                              device_error_ptr(), static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PA_OK : fail_cuda(e);
+}
+
+int pa_free_blocks(const int32_t* block_ids, int num_ids, int32_t* free_queue,
+                   int queue_capacity, int32_t* queue_state, void* stream) {
+    if (num_ids < 0 || queue_capacity <= 0 || !free_queue || !queue_state) return PA_ERR_INVALID_ARG;
+    if (num_ids == 0) return PA_OK;
+    if (!block_ids || num_ids > queue_capacity) return PA_ERR_INVALID_ARG;
+    cudaError_t e = pa::launch_free_blocks(block_ids, num_ids, free_queue, queue_capacity,
+                                           queue_state, device_error_ptr(),
+                                           static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PA_OK : fail_cuda(e);
+}
+
 int pa_write_kv(pa_cache* cache, const void* k, const void* v, const int32_t* slot_mapping,
                 int num_tokens, void* stream) {
     if (!cache || num_tokens < 0) return PA_ERR_INVALID_ARG;

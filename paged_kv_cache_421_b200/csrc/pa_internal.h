@@ -99,6 +99,13 @@ cudaError_t launch_chunk_tc(const CUtensorMap& tmap_blk, const AttnParams& p, co
 cudaError_t launch_reduce(const AttnParams& p, const ChunkList& list, int head_size,
                           cudaStream_t stream);
 cudaError_t launch_zero_counters(int* counters, int n, cudaStream_t stream);
+cudaError_t launch_allocate_slots(int32_t* block_table, int max_blocks_per_seq,
+                                  const int32_t* num_computed, const int32_t* num_new,
+                                  int num_seqs, int block_size, const int32_t* queue, int capacity,
+                                  int32_t* state, int32_t* num_allocated, int* err,
+                                  cudaStream_t stream);
+cudaError_t launch_free_blocks(const int32_t* ids, int num_ids, int32_t* queue, int capacity,
+                               int32_t* state, int* err, cudaStream_t stream);
 cudaError_t launch_slot_mapping(const int32_t* block_table, int max_blocks_per_seq,
                                 const int32_t* seq_lens, const int32_t* qsl, int num_seqs,
                                 int num_tokens, int block_size, int32_t* slot_mapping, int* err,

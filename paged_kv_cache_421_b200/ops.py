@@ -66,6 +66,40 @@ def slot_mapping(block_table: torch.Tensor, seq_lens: torch.Tensor, qsl: torch.T
     return out
 
 
+class BlockQueue:
+    """The free-block queue on the device: a ring of block ids plus (head, count)."""
+
+    def __init__(self, block_ids: torch.Tensor, capacity: Optional[int] = None):
+        n = block_ids.numel()
+        cap = n if capacity is None else capacity
+        assert cap >= n > 0
+        self.queue = torch.zeros(cap, dtype=torch.int32, device=block_ids.device)
+        self.queue[:n] = block_ids.to(torch.int32)
+        self.state = torch.tensor([0, n], dtype=torch.int32, device=block_ids.device)
+
+    @property
+    def capacity(self) -> int:
+        return self.queue.numel()
+
+
+def allocate_slots(block_table: torch.Tensor, num_computed: torch.Tensor, num_new: torch.Tensor,
+                   queue: BlockQueue, block_size: int = 16, out: Optional[torch.Tensor] = None,
+                   stream=None) -> torch.Tensor:
+    """Append each request's new blocks to its block-table row (in place); returns the blocks
+    taken per request, -1 where the request was not served."""
+    if out is None:
+        out = torch.empty(num_computed.numel(), dtype=torch.int32, device=block_table.device)
+    B.pa_allocate_slots(block_table, block_table.shape[1], num_computed, num_new,
+                        num_computed.numel(), block_size, queue.queue, queue.capacity, queue.state,
+                        out, stream)
+    return out
+
+
+def free_blocks(block_ids: torch.Tensor, queue: BlockQueue, stream=None) -> None:
+    B.pa_free_blocks(block_ids, block_ids.numel(), queue.queue, queue.capacity, queue.state,
+                     stream)
+
+
 def write_kv(cache: PagedKVCache, k: torch.Tensor, v: torch.Tensor, slots: torch.Tensor,
              stream=None) -> None:
     assert k.is_contiguous() and v.is_contiguous() and k.dtype == torch.bfloat16

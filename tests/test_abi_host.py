@@ -166,3 +166,20 @@ def test_argument_errors_without_device(lib):
     assert lib.pa_slot_mapping(None, 4, None, None, 1, 1, 16, None, None) == B.PA_ERR_INVALID_ARG
     assert lib.pa_free_cache(None) == B.PA_OK
     assert B.pa_status_string(B.PA_ERR_METADATA) == "PA_ERR_METADATA"
+
+
+def test_allocator_argument_errors_without_device(lib):
+    st = ctypes.c_void_p(0x1000)  # never dereferenced: every call below fails or returns early
+    assert lib.pa_allocate_slots(None, 4, None, None, 0, 16, None, 8, st, None, None) == B.PA_OK
+    assert lib.pa_allocate_slots(None, 4, None, None, 3, 16, None, 8, st, None, None) == \
+        B.PA_ERR_INVALID_ARG
+    assert lib.pa_allocate_slots(None, 4, None, None, -1, 16, None, 8, st, None, None) == \
+        B.PA_ERR_INVALID_ARG
+    assert lib.pa_allocate_slots(None, 4, None, None, 0, 0, None, 8, st, None, None) == \
+        B.PA_ERR_INVALID_ARG
+    assert lib.pa_allocate_slots(None, 4, None, None, 0, 16, None, 0, st, None, None) == \
+        B.PA_ERR_INVALID_ARG
+    assert lib.pa_free_blocks(None, 0, st, 8, st, None) == B.PA_OK
+    assert lib.pa_free_blocks(None, 2, st, 8, st, None) == B.PA_ERR_INVALID_ARG
+    assert lib.pa_free_blocks(st, 9, st, 8, st, None) == B.PA_ERR_INVALID_ARG
+    assert lib.pa_free_blocks(st, 1, None, 8, st, None) == B.PA_ERR_INVALID_ARG
