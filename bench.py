@@ -33,6 +33,7 @@ if ROOT not in sys.path:
 DEFAULT_WORKLOAD = "llama8b_decode"
 METRIC = "paged-attn KV-read GB/s (% of HBM peak) and query tokens/s per batch step"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 L2_FLUSH_BYTES = 256 << 20
 L2_BYTES = 126 << 20
 
@@ -46,6 +47,8 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
+    ap.add_argument("--no-alloc", action="store_true",
+                    help="skip timing the device block allocation")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing")
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
     ap.add_argument("--flush", choices=["auto", "always", "never"], default="auto",
@@ -71,6 +74,18 @@ def decode_kv_bytes(wl) -> int:
         wl.head_size * wl.dtype_bytes
 
 
+def chunk_flops(wl) -> int:
+    """Algorithmic FLOPs of the chunk-kind requests: 4 D per unmasked (query, key) pair per q
+    head (Q K^T and P V); query i of a request with q_len new tokens sees ctx - q_len + i + 1
+    keys."""
+    G = wl.num_q_heads // wl.num_kv_heads
+    total = 0
+    for ctx, ql in zip(wl.seq_lens.astype(np.int64), wl.q_lens.astype(np.int64)):
+        if ql > 0 and ql * G > 8:
+            total += int(ql * (ctx - ql) + ql * (ql + 1) // 2)
+    return total * wl.num_q_heads * 4 * wl.head_size
+
+
 def unique_kv_bytes(wl) -> int:
     used = set()
     for r in range(wl.num_seqs):
@@ -86,6 +101,18 @@ def load_peaks() -> tuple:
         return float(pk["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def load_tensor_peak() -> tuple:
+    """Dense bf16 tensor peak (TFLOP/s): the measured burst figure (the chunk kernel runs tens
+    of microseconds, far from the power-capped sustained regime)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 def source_digest(*names) -> str:
@@ -374,6 +401,28 @@ def run_device_bench(args, rank, world, local):
     if step.plan["chunk_max_splits"] > 1:
         reduce_ms = statistics.mean(e[4].elapsed_time(e[5]) for e in ev)
 
+    # ---- device block allocation for this step's requests (allocate_slots on a queue holding
+    # the whole pool), timed apart from the step: the queue state is restored before each call
+    alloc = None
+    if not args.no_alloc:
+        from paged_kv_cache_421_b200 import ops
+        ql_d = torch.from_numpy(np.ascontiguousarray(wl.q_lens, np.int32)).to(device)
+        comp_d = torch.from_numpy(np.ascontiguousarray(wl.seq_lens - wl.q_lens, np.int32)).to(device)
+        queue = ops.BlockQueue(torch.arange(wl.num_blocks, dtype=torch.int32, device=device))
+        saved = queue.state.clone()
+        abt = torch.full((wl.num_seqs, wl.max_blocks_per_seq), -1, dtype=torch.int32, device=device)
+        taken = ops.allocate_slots(abt, comp_d, ql_d, queue)
+        a_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                for _ in range(args.steps)]
+        for i in range(args.steps):
+            queue.state.copy_(saved)
+            a_ev[i][0].record(stream)
+            ops.allocate_slots(abt, comp_d, ql_d, queue, out=taken)
+            a_ev[i][1].record(stream)
+        torch.cuda.synchronize(device)
+        alloc = {"us_per_call": round(1e3 * statistics.mean(a.elapsed_time(b) for a, b in a_ev), 2),
+                 "requests": wl.num_seqs, "blocks_taken": int(taken.clamp(min=0).sum().item())}
+
     # ---- end-to-end: host inputs (pinned) -> device -> step -> output back to the host
     e2e = None
     if not args.no_e2e:
@@ -443,9 +492,16 @@ def run_device_bench(args, rank, world, local):
                     "traffic": recorded_traffic("decode_kernel", args.workload),
                     "peak_kind": peak_kind, "bytes_per_launch": dec_bytes,
                     "ms_per_launch": round(dec_ms, 4)}
-        elif chunk_ms:
-            roof = {"bound": "tensor", "kernel": "chunk_kernel", "achieved": None, "peak": None,
-                    "unit": "TFLOP/s", "frac": None, "traffic": None}
+        chunk_roof = None
+        if chunk_ms:
+            tflops = chunk_flops(wl) / (chunk_ms * 1e-3) / 1e12
+            tpeak, tkind = load_tensor_peak()
+            chunk_roof = {"bound": "tensor", "kernel": "chunk_tc_kernel", "achieved": round(tflops, 1),
+                          "peak": tpeak, "unit": "TFLOP/s", "frac": round(tflops / tpeak, 4),
+                          "traffic": None, "peak_kind": tkind, "flops_per_launch": chunk_flops(wl),
+                          "ms_per_launch": round(chunk_ms, 4)}
+            if roof is None:
+                roof = chunk_roof
         result = {
             "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
@@ -467,6 +523,8 @@ def run_device_bench(args, rank, world, local):
             "pct_hbm_peak": round(100 * value / world / peak, 2),
             "roofline": roof,
             "kernel_ms": {"decode": dec_ms, "chunk": chunk_ms, "reduce": reduce_ms},
+            "chunk_roofline": chunk_roof,
+            "alloc": alloc,
             "e2e": e2e,
             "gpu_launches": step.launches_per_step() * args.steps,
             "clocks": clk,

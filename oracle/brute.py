@@ -45,8 +45,9 @@ def write_kv_bf16(cache: dict, k, v, slots, num_kv_heads, head_size, block_size)
 
 
 def attention(cache_value, q, num_q_heads, num_kv_heads, head_size, block_table, seq_lens,
-              qsl, block_size, scale):
+              qsl, block_size, scale, window=0):
     """cache_value(block, kv, head, tok, d) -> float.  q: nested [T][Hq][D] bf16 bits.
+    window > 0: the query at position p sees only positions p - window + 1 .. p.
     Returns out as nested lists [T][Hq][D] of floats."""
     group = num_q_heads // num_kv_heads
     T = int(qsl[-1])
@@ -57,11 +58,12 @@ def attention(cache_value, q, num_q_heads, num_kv_heads, head_size, block_table,
         for i in range(q_len):
             t = int(qsl[r]) + i
             visible = ctx - q_len + i + 1
+            start = max(0, visible - window) if window > 0 else 0
             for h in range(num_q_heads):
                 g = h // group
                 qv = [bf16_bits_to_float(q[t][h][d]) for d in range(head_size)]
-                weights = []
-                for p in range(visible):
+                weights = [0.0] * start
+                for p in range(start, visible):
                     b = int(block_table[r][p // block_size])
                     o = p % block_size
                     dot = sum(qv[d] * cache_value(b, 0, g, o, d) for d in range(head_size))
@@ -69,7 +71,7 @@ def attention(cache_value, q, num_q_heads, num_kv_heads, head_size, block_table,
                 total = sum(weights)
                 for d in range(head_size):
                     acc = 0.0
-                    for p in range(visible):
+                    for p in range(start, visible):
                         b = int(block_table[r][p // block_size])
                         o = p % block_size
                         acc += weights[p] * cache_value(b, 1, g, o, d)

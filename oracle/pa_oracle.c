@@ -267,25 +267,34 @@ void oracle_write_kv_fp8(uint8_t* cache, int num_blocks, int block_size, int num
 }
 
 /* ------------------------------------------------------------------ attention core */
-/* One query row against keys 0..limit of contiguous fp64 K, V [*, head_size].
+/* One query row against keys first..limit of contiguous fp64 K, V [*, head_size].
  * Two-pass softmax; writes out[head_size] and returns the natural-log LSE. */
-static double attend_row(const double* qrow, const double* K, const double* V, int limit,
-                         int head_size, double scale, double* s, double* out) {
+static double attend_row(const double* qrow, const double* K, const double* V, int first,
+                         int limit, int head_size, double scale, double* s, double* out) {
     int p, d;
     double mx = -INFINITY, sum = 0.0;
-    for (p = 0; p <= limit; ++p) {
+    for (p = first; p <= limit; ++p) {
         double acc = 0.0;
         for (d = 0; d < head_size; ++d) acc += qrow[d] * K[(int64_t)p * head_size + d];
         s[p] = scale * acc;
         if (s[p] > mx) mx = s[p];
     }
-    for (p = 0; p <= limit; ++p) sum += exp(s[p] - mx);
+    for (p = first; p <= limit; ++p) sum += exp(s[p] - mx);
     for (d = 0; d < head_size; ++d) out[d] = 0.0;
-    for (p = 0; p <= limit; ++p) {
+    for (p = first; p <= limit; ++p) {
         double w = exp(s[p] - mx) / sum;
         for (d = 0; d < head_size; ++d) out[d] += w * V[(int64_t)p * head_size + d];
     }
     return mx + log(sum);
+}
+
+/* First key a query at position `limit` sees: all of them (window 0), else the last `window`
+ * positions up to and including its own -- the sliding window the "vLLM architecture
+ * overview" names (section 2, SlidingWindowManager keeps only the window's blocks; section 6,
+ * SWA), read as a query at position p attending to keys max(0, p - W + 1) .. p. */
+static int first_key(int limit, int window) {
+    if (window <= 0) return 0;
+    return limit - window + 1 > 0 ? limit - window + 1 : 0;
 }
 
 static double cache_value(const void* cache, int kv_dtype, int64_t idx, double scale) {
@@ -302,7 +311,7 @@ int oracle_attention_paged(const void* cache, int kv_dtype, int num_blocks, int 
                            const float* v_scale, const uint16_t* q, int num_q_heads,
                            const int32_t* block_table, int max_blocks_per_seq,
                            const int32_t* seq_lens, const int32_t* qsl, int num_seqs,
-                           double scale, double* out, double* lse) {
+                           double scale, int window, double* out, double* lse) {
     int r, g, i, hh, d, p;
     int group = num_q_heads / num_kv_heads;
     if (group * num_kv_heads != num_q_heads) return OR_BAD_ARG;
@@ -351,8 +360,8 @@ int oracle_attention_paged(const void* cache, int kv_dtype, int num_blocks, int 
                     int64_t row = (int64_t)t * num_q_heads + h;
                     for (d = 0; d < head_size; ++d)
                         qrow[d] = oracle_bf16_to_double(q[row * head_size + d]);
-                    lse[row] = attend_row(qrow, K, V, limit, head_size, scale, s,
-                                          out + row * head_size);
+                    lse[row] = attend_row(qrow, K, V, first_key(limit, window), limit,
+                                          head_size, scale, s, out + row * head_size);
                 }
             }
         }
@@ -370,7 +379,7 @@ int oracle_attention_rows(const uint16_t* k_src, const uint16_t* v_src, int num_
                           int head_size, const int64_t* pos_rows, const int64_t* pos_start,
                           int kv_dtype, const float* k_scale, const float* v_scale,
                           const uint16_t* q, int num_q_heads, const int32_t* seq_lens,
-                          const int32_t* qsl, int num_seqs, double scale,
+                          const int32_t* qsl, int num_seqs, double scale, int window,
                           const int32_t* sel_tokens, const int32_t* sel_heads, int nsel,
                           double* out, double* lse) {
     int j, r, d, p;
@@ -410,7 +419,8 @@ int oracle_attention_rows(const uint16_t* k_src, const uint16_t* v_src, int num_
         }
         for (d = 0; d < head_size; ++d)
             qrow[d] = oracle_bf16_to_double(q[((int64_t)t * num_q_heads + h) * head_size + d]);
-        lse[j] = attend_row(qrow, K, V, limit, head_size, scale, s, out + (int64_t)j * head_size);
+        lse[j] = attend_row(qrow, K, V, first_key(limit, window), limit, head_size, scale, s,
+                            out + (int64_t)j * head_size);
         free(K); free(V); free(s); free(qrow);
     }
     return OR_OK;

@@ -580,3 +580,84 @@ def test_allocate_brute_force_invariants(oracle_mod):
             assert (bt[r, k:] == -9).all()
         assert taken == [int(queue[(head + j) % cap]) for j in range(len(taken))]
         assert st.tolist() == [(head + len(taken)) % cap, count - len(taken)]
+
+
+# ------------------------------------------------------------------ sliding window
+# The pages name the sliding window (architecture overview, section 2: SlidingWindowManager
+# keeps only the window's blocks; section 6: SWA) without defining it; the reading taken: a
+# query at position p sees keys max(0, p - W + 1) .. p.
+
+@pytest.mark.parametrize("case", range(6))
+def test_window_vs_brute(oracle_mod, case):
+    rng = np.random.default_rng(700 + case)
+    bs = int([1, 2, 16, 4, 16, 2][case])
+    B = int(rng.integers(1, 4))
+    ctx = rng.integers(1, 41, size=B)
+    ql = np.array([rng.integers(1, c + 1) for c in ctx])
+    window = int(rng.integers(1, 20))
+    nb = int(sum(-(-c // bs) for c in ctx)) + 3
+    wl = W.make_workload("t", ctx, ql, 2, 1, 4, bs, nb, 300 + case, scale=0.7)
+    cache = _oracle_cache(oracle_mod, wl)
+    out, _ = oracle_mod.attention_paged(cache, W.BF16, nb, bs, 1, 4, W.bits(wl.q), 2,
+                                        wl.block_table, wl.seq_lens, wl.qsl, 0.7, window=window)
+    c5 = cache.reshape(nb, 2, 1, bs, 4)
+
+    def val(b, kv, h, o, d):
+        return brute.bf16_bits_to_float(c5[b, kv, h, o, d])
+
+    want = brute.attention(val, W.bits(wl.q).tolist(), 2, 1, 4, wl.block_table.tolist(),
+                           wl.seq_lens.tolist(), wl.qsl.tolist(), bs, 0.7, window=window)
+    np.testing.assert_allclose(out, np.array(want), rtol=1e-11, atol=1e-12)
+
+
+def test_window_special_cases(oracle_mod):
+    wl = W.make_workload("t", [37, 20], [5, 20], 4, 2, 8, 16, 8, 41)
+    cache = _oracle_cache(oracle_mod, wl)
+    full = _attn_paged(oracle_mod, wl, cache)
+    args = (cache, W.BF16, wl.num_blocks, 16, 2, 8, W.bits(wl.q), 4, wl.block_table,
+            wl.seq_lens, wl.qsl, wl.scale)
+    # a window at least as long as every context is full attention, bit for bit
+    for w in [37, 38, 1000]:
+        o, l = oracle_mod.attention_paged(*args, window=w)
+        assert np.array_equal(o, full[0]) and np.array_equal(l, full[1])
+    # window 1: every query sees only its own position -> its own value row, lse = its score
+    o, l = oracle_mod.attention_paged(*args, window=1)
+    k_src, v_src = wl.kv_src()
+    q = W.bits(wl.q)
+    for r in range(2):
+        ql = int(wl.qsl[r + 1] - wl.qsl[r])
+        for i in range(ql):
+            t = int(wl.qsl[r]) + i
+            p = int(wl.seq_lens[r]) - ql + i
+            row = wl.pos_rows[wl.pos_start[r] + p]
+            for h in range(4):
+                vrow = v_src[row, h // 2].float().numpy()
+                np.testing.assert_array_equal(o[t, h], vrow.astype(np.float64))
+                kk = k_src[row, h // 2].double().numpy()
+                qq = np.array([brute.bf16_bits_to_float(int(x)) for x in q[t, h]])
+                np.testing.assert_allclose(l[t, h], wl.scale * float(kk @ qq), rtol=1e-13)
+    # the unpaged definition agrees under a window too
+    k_bits, v_bits = W.bits(k_src), W.bits(v_src)
+    T, Hq = wl.num_tokens, 4
+    tok = np.repeat(np.arange(T), Hq).astype(np.int32)
+    hed = np.tile(np.arange(Hq), T).astype(np.int32)
+    for w in [1, 5, 16, 17]:
+        o, _ = oracle_mod.attention_paged(*args, window=w)
+        o2, _ = oracle_mod.attention_rows(k_bits, v_bits, wl.pos_rows, wl.pos_start, W.BF16,
+                                          q, wl.seq_lens, wl.qsl, wl.scale, tok, hed, window=w)
+        assert np.array_equal(o.reshape(T * Hq, -1), o2)
+
+
+def test_window_equal_keys_mean_of_window(oracle_mod):
+    # identical keys -> uniform weights over the window -> mean of the window's values
+    wl = W.make_workload("t", [37], [1], 2, 1, 8, 16, 4, 23)
+    wl.k_hist[:] = wl.k_hist[0]
+    wl.k_new[:] = wl.k_hist[0]
+    cache = _oracle_cache(oracle_mod, wl)
+    k_src, v_src = wl.kv_src()
+    for w in [1, 7, 16, 30]:
+        o, _ = oracle_mod.attention_paged(cache, W.BF16, 4, 16, 1, 8, W.bits(wl.q), 2,
+                                          wl.block_table, wl.seq_lens, wl.qsl, wl.scale, window=w)
+        rows = wl.pos_rows[wl.pos_start[0] + np.arange(37 - w, 37)]
+        want = v_src[rows, 0].double().numpy().mean(axis=0)
+        np.testing.assert_allclose(o[0, 0], want, rtol=1e-12, atol=1e-13)
