@@ -223,6 +223,9 @@ typedef struct {
                               [0]/[1] before/after the decode kernel, [2]/[3] around the chunk
                               kernel, [4]/[5] around the split reduce; an entry is recorded
                               only when that kernel is launched; NULL entries are skipped */
+    int sliding_window;    /* > 0: a query at position p sees only keys max(0, p - W + 1) .. p
+                              (the sliding window [P2] section 2 names; its reading here);
+                              0: full causal attention */
 } pa_attention_opts;
 
 /* The planner alone: fills *plan for the given host metadata without touching the GPU.

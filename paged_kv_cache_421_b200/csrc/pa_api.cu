@@ -158,6 +158,8 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
     const int G = Hq / Hkv;
     const int forced = opts ? opts->kv_split_tokens : 0;
     if (forced < 0 || forced % bs) return PA_ERR_INVALID_ARG;
+    const int window = opts ? opts->sliding_window : 0;
+    if (window < 0) return PA_ERR_INVALID_ARG;
     if (B > 0 && qsl[0] != 0) return PA_ERR_METADATA;
     long long dec_units = 0;
     int dec_max_blocks = 0, chunk_max_blocks = 0, chunk_max_qtiles = 0;
@@ -173,9 +175,11 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
         const int blocks = pa::ceil_div(ctx, bs);
         if (blocks > maxb) return PA_ERR_METADATA;
         if (pa::is_decode_kind(ql, G)) {
+            // with a sliding window the decode CTAs walk only the window's blocks
             pl->num_decode_seqs++;
-            dec_units += static_cast<long long>(blocks) * Hkv;
-            if (blocks > dec_max_blocks) dec_max_blocks = blocks;
+            const int eff = blocks - pa::window_first_key(ctx - ql, window) / bs;
+            dec_units += static_cast<long long>(eff) * Hkv;
+            if (eff > dec_max_blocks) dec_max_blocks = eff;
         } else {
             pl->num_chunk_seqs++;
             const int qt = pa::ceil_div(ql * G, chunk_cta_rows);
@@ -183,7 +187,8 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
             if (blocks > chunk_max_blocks) chunk_max_blocks = blocks;
             for (int i = 0; i < qt; ++i) {
                 const int last_row = std::min((i + 1) * chunk_cta_rows, ql * G) - 1;
-                const long long w = pa::ceil_div(ctx - ql + last_row / G + 1, chunk_tile_keys);
+                const int lo = pa::window_first_key(ctx - ql + i * chunk_cta_rows / G, window) / bs * bs;
+                const long long w = pa::ceil_div(ctx - ql + last_row / G + 1 - lo, chunk_tile_keys);
                 chunk_work += w * Hkv;
                 if (w > chunk_work_max) chunk_work_max = w;
             }
@@ -251,7 +256,8 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
         if (ql == 0) continue;
         int ns;
         if (pa::is_decode_kind(ql, G)) {
-            ns = pa::num_splits(sl[r], pl->decode_split_blocks);
+            const int fb = pa::window_first_key(sl[r] - ql, window) / bs;
+            ns = pa::ceil_div(pa::ceil_div(sl[r], bs) - fb, pl->decode_split_blocks);
             pl->decode_ctas += static_cast<int64_t>(ns) * Hkv;
         } else {
             ns = pa::num_splits(sl[r], pl->chunk_split_blocks);
@@ -489,6 +495,7 @@ int pa_attention_ex(const pa_cache* cache, const void* q, int num_q_heads,
     p.chunk_max_qtiles = pl.chunk_max_qtiles > 0 ? pl.chunk_max_qtiles : 1;
     p.reduce_row_tiles = pa::ceil_div(pl.reduce_rows_max > 0 ? pl.reduce_rows_max : 1, 4);
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    p.window = opts ? opts->sliding_window : 0;
     p.err = device_error_ptr();
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -546,8 +553,10 @@ int pa_attention_ex(const pa_cache* cache, const void* q, int num_q_heads,
             for (int qt = 0; qt < nqt; ++qt) {
                 const int last_row = std::min((qt + 1) * cta_rows, ql * p.group) - 1;
                 const int kmax = ctx - ql + last_row / p.group;
+                const int lo = pa::window_first_key(ctx - ql + qt * cta_rows / p.group, p.window) /
+                               cache->block_size * cache->block_size;
                 for (int sp = 0; sp < nsplit; ++sp) {
-                    const int key_lo = sp * csb * cache->block_size;
+                    const int key_lo = std::max(sp * csb * cache->block_size, lo);
                     const int key_hi = std::min(std::min((sp + 1) * csb * cache->block_size, ctx), kmax + 1);
                     const int tiles = key_hi > key_lo ? pa::ceil_div(key_hi - key_lo, tile_keys) : 0;
                     items.emplace_back(tiles, static_cast<uint32_t>(r) | (static_cast<uint32_t>(qt) << 10) |

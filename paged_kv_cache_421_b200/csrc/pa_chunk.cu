@@ -80,7 +80,10 @@ chunk_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
     const int kend = min(je * kBlockSize, ctx);  // keys of this split: [jb*16, kend)
     const int last_row = min(R0 + kChunkRows - 1, rows_total - 1);
     const int kmax = ctx - q_len + last_row / G;   // last key any row of the tile sees
-    const int key_lo = jb * kBlockSize;
+    // the first key any row of the CTA may see: the split's start, or (sliding window) the
+    // window start of the CTA's first row, rounded down to its block
+    const int key_lo = max(jb * kBlockSize,
+                           window_first_key(ctx - q_len + R0 / G, p.window) / kBlockSize * kBlockSize);
     const int key_hi = min(kend, kmax + 1);
     const int ntiles = key_hi > key_lo ? ceil_div(key_hi - key_lo, kTileKeys) : 0;
 
@@ -99,6 +102,7 @@ chunk_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
     const bool vA = rA < rows_total, vB = rB < rows_total;
     const int limA = vA ? ctx - q_len + rA / G : kmax;
     const int limB = vB ? ctx - q_len + rB / G : kmax;
+    const int loA = window_first_key(limA, p.window), loB = window_first_key(limB, p.window);
     const int wlast = min(R0 + 16 * warp + 15, rows_total - 1);
     const int warp_kmax = ctx - q_len + wlast / G;
 
@@ -230,8 +234,8 @@ chunk_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
                 for (int e = 0; e < 2; ++e) {
                     const int pos = key0 + 8 * nt + 2 * tq + e;
                     const bool in = pos < kend;
-                    s[nt][e] = (in && pos <= limA) ? s[nt][e] * sl : -INFINITY;
-                    s[nt][2 + e] = (in && pos <= limB) ? s[nt][2 + e] * sl : -INFINITY;
+                    s[nt][e] = (in && pos <= limA && pos >= loA) ? s[nt][e] * sl : -INFINITY;
+                    s[nt][2 + e] = (in && pos <= limB && pos >= loB) ? s[nt][2 + e] * sl : -INFINITY;
                     mxA = fmaxf(mxA, s[nt][e]);
                     mxB = fmaxf(mxB, s[nt][2 + e]);
                 }

@@ -247,7 +247,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
     const int kend = min(je * kBlockSize, ctx);
     const int last_row = min(R0 + kQTiles * kRows - 1, rows_total - 1);
     const int kmax = ctx - q_len + last_row / G;
-    const int key_lo = jb * kBlockSize;
+    // the first key any row of the CTA may see: the split's start, or (sliding window) the
+    // window start of the CTA's first row, rounded down to its block
+    const int key_lo = max(jb * kBlockSize,
+                           window_first_key(ctx - q_len + R0 / G, p.window) / kBlockSize * kBlockSize);
     const int key_hi = min(kend, kmax + 1);
     const int ntiles = key_hi > key_lo ? ceil_div(key_hi - key_lo, kKeys) : 0;
     const bool two = R0 + kRows < rows_total;  // the second q-tile has rows
@@ -447,6 +450,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
             const bool valid = R < rows_total;
             const int lim = valid ? ctx - q_len + R / G : kmax;
             const int first_lim = ctx - q_len + (R0 + q * kRows) / G;  // smallest limit of the q-tile
+            const int lo = window_first_key(lim, p.window);            // first key this row sees
+            const int last_lo = window_first_key(                      // latest of the q-tile
+                ctx - q_len + min(R0 + q * kRows + kRows - 1, rows_total - 1) / G, p.window);
             const uint32_t tq = tmem + q * 256;
             const uint32_t tmem_lane = tq + (static_cast<uint32_t>((warp & 3) * 32) << 16);
             const float sl = p.scale_log2;
@@ -460,7 +466,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
                 }
                 tc_fence_after();
                 // only tiles crossing a causal limit or the split end need masking
-                const bool masked = !(key0 + kKeys - 1 <= first_lim && key0 + kKeys <= kend);
+                const bool masked =
+                    !(key0 + kKeys - 1 <= first_lim && key0 + kKeys <= kend && key0 >= last_lo);
                 // S of this row: all four loads in flight, one wait (TMEM load latency is long)
                 float sv[kKeys];
 #pragma unroll
@@ -475,7 +482,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
 #pragma unroll
                     for (int c = 0; c < kKeys; ++c) {
                         const int pos = key0 + c;
-                        if (pos > lim || pos >= kend) sv[c] = -INFINITY;
+                        if (pos > lim || pos >= kend || pos < lo) sv[c] = -INFINITY;
                     }
                 }
                 // the row max with independent partial maxima (short dependency chains)

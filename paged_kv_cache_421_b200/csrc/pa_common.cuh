@@ -29,6 +29,12 @@ constexpr int kErrMetadata = 4;   // device metadata disagrees with the planned 
 
 // A request is served by the decode kernel when all its query rows of one kv head fit one
 // 8-wide MMA tile, otherwise by the chunk kernel.  q_len == 0 requests produce nothing.
+// First key a query at position `limit` may see: 0, or with a sliding window of `window`
+// keys the last `window` positions up to its own.
+__host__ __device__ inline int window_first_key(int limit, int window) {
+    return (window > 0 && limit - window + 1 > 0) ? limit - window + 1 : 0;
+}
+
 __host__ __device__ inline bool is_decode_kind(int q_len, int group) {
     return q_len > 0 && q_len * group <= kDecodeRows;
 }

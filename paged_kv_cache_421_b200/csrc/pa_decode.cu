@@ -81,9 +81,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
         ctx = p.max_blocks_per_seq * kBlockSize;
     }
     const int nblocks = ceil_div(ctx, kBlockSize);
-    const int nsplit = ceil_div(nblocks, p.decode_split_blocks);
+    // with a sliding window the splits cover only the blocks from the window of the first row
+    const int fb = window_first_key(ctx - q_len, p.window) / kBlockSize;
+    const int nsplit = ceil_div(nblocks - fb, p.decode_split_blocks);
     if (split >= nsplit) return;
-    const int jb = split * p.decode_split_blocks;
+    const int jb = fb + split * p.decode_split_blocks;
     const int je = min(nblocks, jb + p.decode_split_blocks);
 
     extern __shared__ uint8_t smem_raw[];
@@ -177,6 +179,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
     const int lim0 = row0 < rows ? ctx - q_len + row0 / p.group : ctx - 1;
     const int lim1 = row1 < rows ? ctx - q_len + row1 / p.group : ctx - 1;
     const int lim_min = min(lim0, lim1);
+    // first visible key of the two rows, and of the group's last row (the latest window start)
+    const int lo0 = window_first_key(lim0, p.window), lo1 = window_first_key(lim1, p.window);
+    const int lo_last = window_first_key(ctx - 1, p.window);
 
     float o[C::kKSteps][4];
 #pragma unroll
@@ -298,15 +303,15 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
             // ---- online softmax over the unit's keys (log2 domain).  Units whose keys every
             // row may see skip the mask; a key past the round's blocks (the missing second
             // block of a unit) is masked like a future key.
-            if (kb + BPU * kBlockSize - 1 > min(lim_min, kend - 1)) {
+            if (kb + BPU * kBlockSize - 1 > min(lim_min, kend - 1) || kb < lo_last) {
 #pragma unroll
                 for (int h = 0; h < BPU; ++h) {
                     const int p0 = kb + h * kBlockSize + key_of_row<FP8>(gq);
                     const int p1 = kb + h * kBlockSize + key_of_row<FP8>(gq + 8);
-                    if (p0 > lim0 || p0 >= kend) x[h][0] = -INFINITY;
-                    if (p0 > lim1 || p0 >= kend) x[h][1] = -INFINITY;
-                    if (p1 > lim0 || p1 >= kend) x[h][2] = -INFINITY;
-                    if (p1 > lim1 || p1 >= kend) x[h][3] = -INFINITY;
+                    if (p0 > lim0 || p0 >= kend || p0 < lo0) x[h][0] = -INFINITY;
+                    if (p0 > lim1 || p0 >= kend || p0 < lo1) x[h][1] = -INFINITY;
+                    if (p1 > lim0 || p1 >= kend || p1 < lo0) x[h][2] = -INFINITY;
+                    if (p1 > lim1 || p1 >= kend || p1 < lo1) x[h][3] = -INFINITY;
                 }
             }
             float mx0 = fmaxf(x[0][0], x[0][2]), mx1 = fmaxf(x[0][1], x[0][3]);

@@ -69,6 +69,7 @@ struct AttnParams {
     float scale_log2;           // softmax scale * log2(e)
     int* err;                   // device error word
     int chunk_fused_merge;      // tcgen05 chunk kernel merges its own splits (<= kMaxFusedSplits)
+    int window;                 // sliding window in keys, 0 = full causal attention
 };
 
 // The chunk-kind requests of a launch, longest context first (passed by value, so the chunk
