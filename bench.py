@@ -47,6 +47,8 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
+    ap.add_argument("--sliding-window", type=int, default=0,
+                    help="attend to the last W keys only (0 = full causal attention)")
     ap.add_argument("--no-alloc", action="store_true",
                     help="skip timing the device block allocation")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing")
@@ -59,30 +61,40 @@ def parse_args(argv=None):
     return ap.parse_args(argv)
 
 
-def kv_bytes(wl) -> int:
-    """Algorithmic KV bytes the step's attention reads: every request's full context of K
+def visible_keys(wl, window: int = 0) -> np.ndarray:
+    """Keys each request's rows read: its whole context, or with a sliding window W the keys
+    from the window start of its first new token (ctx - q_len - W + 1) to the end."""
+    ctx = wl.seq_lens.astype(np.int64)
+    if window <= 0:
+        return ctx
+    return ctx - np.maximum(0, ctx - wl.q_lens.astype(np.int64) - window + 1)
+
+
+def kv_bytes(wl, window: int = 0) -> int:
+    """Algorithmic KV bytes the step's attention reads: every request's visible keys of K
     and V once per kv head (the GQA group shares one read)."""
-    return int(np.sum(wl.seq_lens.astype(np.int64))) * 2 * wl.num_kv_heads * wl.head_size * \
+    return int(np.sum(visible_keys(wl, window))) * 2 * wl.num_kv_heads * wl.head_size * \
         wl.dtype_bytes
 
 
-def decode_kv_bytes(wl) -> int:
+def decode_kv_bytes(wl, window: int = 0) -> int:
     G = wl.num_q_heads // wl.num_kv_heads
     ql = wl.q_lens
     dec = (ql > 0) & (ql * G <= 8)
-    return int(np.sum(wl.seq_lens[dec].astype(np.int64))) * 2 * wl.num_kv_heads * \
+    return int(np.sum(visible_keys(wl, window)[dec])) * 2 * wl.num_kv_heads * \
         wl.head_size * wl.dtype_bytes
 
 
-def chunk_flops(wl) -> int:
+def chunk_flops(wl, window: int = 0) -> int:
     """Algorithmic FLOPs of the chunk-kind requests: 4 D per unmasked (query, key) pair per q
     head (Q K^T and P V); query i of a request with q_len new tokens sees ctx - q_len + i + 1
-    keys."""
+    keys (at most W with a sliding window)."""
     G = wl.num_q_heads // wl.num_kv_heads
     total = 0
     for ctx, ql in zip(wl.seq_lens.astype(np.int64), wl.q_lens.astype(np.int64)):
         if ql > 0 and ql * G > 8:
-            total += int(ql * (ctx - ql) + ql * (ql + 1) // 2)
+            vis = ctx - ql + np.arange(1, ql + 1, dtype=np.int64)
+            total += int(np.sum(np.minimum(vis, window) if window > 0 else vis))
     return total * wl.num_q_heads * 4 * wl.head_size
 
 
@@ -230,7 +242,7 @@ def oracle_requests_for_budget(wl, kv_token_heads_budget: int) -> int:
 
 
 # ---------------------------------------------------------------- CPU oracle timing
-def oracle_step_timer(wl):
+def oracle_step_timer(wl, window: int = 0):
     """Build the oracle's cache (untimed) and return a function that times the oracle over
     the first n requests of the step: slot mapping, cache write of their new tokens and
     attention of their queries.  Returns (seconds, kv_bytes_of_those_requests)."""
@@ -257,13 +269,15 @@ def oracle_step_timer(wl):
                         k_bits[:T], v_bits[:T], slots, ks, vs)
         oracle.attention_paged(cache, wl.kv_dtype, wl.num_blocks, 16, wl.num_kv_heads,
                                wl.head_size, q_bits[:T], wl.num_q_heads, bt, sl, qsl, wl.scale,
-                               ks, vs)
-        return time.perf_counter() - t0, int(np.sum(sl.astype(np.int64))) * per_tok
+                               ks, vs, window=window)
+        ctx = sl.astype(np.int64)
+        keys = ctx if window <= 0 else ctx - np.maximum(0, ctx - np.diff(qsl) - window + 1)
+        return time.perf_counter() - t0, int(np.sum(keys)) * per_tok
     return run
 
 
-def cpu_baseline(wl, budget_s: float) -> dict:
-    run = oracle_step_timer(wl)
+def cpu_baseline(wl, budget_s: float, window: int = 0) -> dict:
+    run = oracle_step_timer(wl, window)
     # grow the sample until it takes about budget_s of CPU time
     n = 1
     sec, nbytes = run(n)
@@ -278,9 +292,10 @@ def cpu_baseline(wl, budget_s: float) -> dict:
 
 # ---------------------------------------------------------------- device step
 class DeviceStep:
-    def __init__(self, wl, device, kv_split_tokens: int = 0):
+    def __init__(self, wl, device, kv_split_tokens: int = 0, sliding_window: int = 0):
         import torch
         self.kv_split_tokens = kv_split_tokens
+        self.window = sliding_window
         from paged_kv_cache_421_b200 import ops
         from paged_kv_cache_421_b200 import workloads as W
         self.wl, self.dev, self.ops, self.torch = wl, device, ops, torch
@@ -308,13 +323,15 @@ class DeviceStep:
         self.out = torch.empty(T, wl.num_q_heads, wl.head_size, dtype=torch.float32,
                                device=device)
         nb = ops.workspace_bytes_for(self.cache, wl.seq_lens, wl.qsl, wl.num_q_heads,
-                                     wl.max_blocks_per_seq, kv_split_tokens)
+                                     wl.max_blocks_per_seq, kv_split_tokens,
+                                     sliding_window=sliding_window)
         self.workspace = torch.empty(max(nb, 256), dtype=torch.uint8, device=device)
         self.plan = ops.B.pa_plan_attention(
             wl.seq_lens, wl.qsl, wl.num_q_heads, wl.num_kv_heads, wl.head_size,
             wl.max_blocks_per_seq,
             torch.cuda.get_device_properties(device).multi_processor_count,
-            self.workspace.numel(), kv_split_tokens=kv_split_tokens)
+            self.workspace.numel(), kv_split_tokens=kv_split_tokens,
+            sliding_window=sliding_window)
         torch.cuda.synchronize(device)
 
     def launches_per_step(self) -> int:
@@ -337,7 +354,8 @@ class DeviceStep:
         B.pa_attention_ex(self.cache.handle, self.q if q is None else q, wl.num_q_heads, bt,
                           bt.shape[1], sl, qsl, wl.seq_lens, wl.qsl, wl.num_seqs, T, wl.scale,
                           self.out, self.workspace, self.workspace.numel(),
-                          kv_split_tokens=self.kv_split_tokens, events=events)
+                          kv_split_tokens=self.kv_split_tokens, events=events,
+                          sliding_window=self.window)
 
 
 def run_device_bench(args, rank, world, local):
@@ -348,10 +366,10 @@ def run_device_bench(args, rank, world, local):
     device = torch.device(f"cuda:{local}")
     torch.cuda.set_device(device)
     wl = W.CONFIGS[args.workload](device=device)
-    step = DeviceStep(wl, device, args.kv_split_tokens)
+    step = DeviceStep(wl, device, args.kv_split_tokens, args.sliding_window)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
-    nbytes = kv_bytes(wl)
-    dec_bytes = decode_kv_bytes(wl)
+    nbytes = kv_bytes(wl, args.sliding_window)
+    dec_bytes = decode_kv_bytes(wl, args.sliding_window)
     flush_l2 = args.flush == "always" or (args.flush == "auto" and nbytes < 4 * L2_BYTES)
 
     def barrier():
@@ -497,11 +515,12 @@ def run_device_bench(args, rank, world, local):
                     "ms_per_launch": round(dec_ms, 4)}
         chunk_roof = None
         if chunk_ms:
-            tflops = chunk_flops(wl) / (chunk_ms * 1e-3) / 1e12
+            tflops = chunk_flops(wl, args.sliding_window) / (chunk_ms * 1e-3) / 1e12
             tpeak, tkind = load_tensor_peak()
             chunk_roof = {"bound": "tensor", "kernel": "chunk_tc_kernel", "achieved": round(tflops, 1),
                           "peak": tpeak, "unit": "TFLOP/s", "frac": round(tflops / tpeak, 4),
-                          "traffic": None, "peak_kind": tkind, "flops_per_launch": chunk_flops(wl),
+                          "traffic": None, "peak_kind": tkind,
+                          "flops_per_launch": chunk_flops(wl, args.sliding_window),
                           "ms_per_launch": round(chunk_ms, 4)}
             if roof is None:
                 roof = chunk_roof
@@ -521,6 +540,7 @@ def run_device_bench(args, rank, world, local):
                               f"inputs larger than L2: {nbytes / 1e6:.0f} MB of KV per step vs "
                               f"126 MB L2, no flush"),
                        "kv_split_tokens": args.kv_split_tokens or "planner",
+                       "sliding_window": args.sliding_window or None,
                        "parallelism": f"replicas x{world} (one batch per GPU)"},
             "tokens_per_s": round(world * wl.num_tokens / (ms_per_step * 1e-3), 1),
             "pct_hbm_peak": round(100 * value / world / peak, 2),
@@ -542,7 +562,7 @@ def reference_arm(args, rank, world):
         return None
     from paged_kv_cache_421_b200 import workloads as W
     wl = W.CONFIGS[args.workload]()
-    run = oracle_step_timer(wl)
+    run = oracle_step_timer(wl, args.sliding_window)
     n = oracle_requests_for_budget(wl, 60_000_000)
     for _ in range(max(args.warmup, 0)):
         run(n)
@@ -587,7 +607,7 @@ def main(argv=None):
     result, wl = run_device_bench(args, rank, world, local)
     if rank == 0:
         if not args.no_cpu_baseline:
-            result["cpu_baseline"] = cpu_baseline(wl, args.cpu_budget_s)
+            result["cpu_baseline"] = cpu_baseline(wl, args.cpu_budget_s, args.sliding_window)
         print(json.dumps(result), flush=True)
     if world > 1:
         import torch.distributed as dist
