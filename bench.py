@@ -341,9 +341,10 @@ class DeviceStep:
         return 2 + int(p["decode_max_splits"] > 1) + (p["num_decode_seqs"] > 0) + \
             (p["num_chunk_seqs"] > 0) + int(p["chunk_max_splits"] > 1)
 
-    def run(self, events=None, q=None, k=None, v=None, bt=None, sl=None, qsl=None):
+    def run(self, events=None, q=None, k=None, v=None, bt=None, sl=None, qsl=None, out=None):
         B = self.ops.B
         wl = self.wl
+        out = self.out if out is None else out
         bt = self.bt if bt is None else bt
         sl = self.sl if sl is None else sl
         qsl = self.qsl if qsl is None else qsl
@@ -353,7 +354,7 @@ class DeviceStep:
                       self.slots, T)
         B.pa_attention_ex(self.cache.handle, self.q if q is None else q, wl.num_q_heads, bt,
                           bt.shape[1], sl, qsl, wl.seq_lens, wl.qsl, wl.num_seqs, T, wl.scale,
-                          self.out, self.workspace, self.workspace.numel(),
+                          out, self.workspace, self.workspace.numel(),
                           kv_split_tokens=self.kv_split_tokens, events=events,
                           sliding_window=self.window)
 
@@ -393,9 +394,36 @@ def run_device_bench(args, rank, world, local):
                           else f"/tmp/clocks_{os.getpid()}.csv")
     clocks.start()
     time.sleep(0.3)
+    stream = torch.cuda.current_stream(device)
+    # the headline timing: K steps between one pair of events (consecutive kernels overlap
+    # their prologues through programmatic dependent launch; events recorded between kernels
+    # would serialise them)
+    # (with an L2 flush between steps, each step gets its own event pair so the flush stays
+    # outside the timing)
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    fl_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+             for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize(device)
-    stream = torch.cuda.current_stream(device)
+    t_start.record(stream)
+    for i in range(args.steps):
+        if flush_l2:
+            flush.zero_()
+            fl_ev[i][0].record(stream)
+        step.run()
+        if flush_l2:
+            fl_ev[i][1].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize(device)
+    barrier()
+    clk = clocks.stop()
+    timed = (sum(a.elapsed_time(b) for a, b in fl_ev) if flush_l2
+             else t_start.elapsed_time(t_end))
+    total_ms = max_over_ranks(timed, world, device)
+    ms_per_step = total_ms / args.steps
+    # the same K steps again with events around every kernel, for the per-kernel durations
+    barrier()
+    torch.cuda.synchronize(device)
     for i in range(args.steps):
         if flush_l2:
             flush.zero_()
@@ -404,10 +432,7 @@ def run_device_bench(args, rank, world, local):
         st_ev[i][1].record(stream)
     torch.cuda.synchronize(device)
     barrier()
-    clk = clocks.stop()
-    step_ms = [a.elapsed_time(b) for a, b in st_ev]
-    total_ms = max_over_ranks(sum(step_ms), world, device)
-    ms_per_step = total_ms / args.steps
+    ms_per_step_events = statistics.mean(a.elapsed_time(b) for a, b in st_ev)
     dec_ms = None
     if step.plan["num_decode_seqs"]:
         dec_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
@@ -467,44 +492,78 @@ def run_device_bench(args, rank, world, local):
         hbuf = torch.zeros(total, dtype=torch.uint8).pin_memory()
         for o, t in zip(offs, parts):
             hbuf[o:o + t.numel()] = t
-        dbuf = torch.empty(total, dtype=torch.uint8, device=device)
+        # two device input buffers and two output buffers: step i+1's inputs go up and step
+        # i's output comes back on copy streams while step i computes (every step still copies
+        # its inputs from pinned host memory and reads its output back to the host)
+        dbufs = [torch.empty(total, dtype=torch.uint8, device=device) for _ in range(2)]
+        douts = [torch.empty_like(step.out) for _ in range(2)]
+        houts = [torch.empty(step.out.shape, dtype=torch.float32).pin_memory() for _ in range(2)]
+        up, down = torch.cuda.Stream(device), torch.cuda.Stream(device)
 
-        def dview(i, dtype, shape):
+        def dview(buf, i, dtype, shape):
             n = int(np.prod(shape)) * torch.tensor([], dtype=dtype).element_size()
-            return dbuf[offs[i]:offs[i] + n].view(dtype).view(*shape)
-        dq = dview(0, torch.bfloat16, step.q.shape)
-        dk = dview(1, torch.bfloat16, step.k.shape)
-        dv = dview(2, torch.bfloat16, step.v.shape)
-        dbt = dview(3, torch.int32, step.bt.shape)
-        dsl = dview(4, torch.int32, step.sl.shape)
-        dqsl = dview(5, torch.int32, step.qsl.shape)
-        hout = torch.empty(step.out.shape, dtype=torch.float32).pin_memory()
-        h2d = total  # bytes the one H2D copy moves (inputs plus 256-byte alignment padding)
-        d2h = hout.numel() * hout.element_size()
+            return buf[offs[i]:offs[i] + n].view(dtype).view(*shape)
+        views = [dict(q=dview(bf, 0, torch.bfloat16, step.q.shape),
+                      k=dview(bf, 1, torch.bfloat16, step.k.shape),
+                      v=dview(bf, 2, torch.bfloat16, step.v.shape),
+                      bt=dview(bf, 3, torch.int32, step.bt.shape),
+                      sl=dview(bf, 4, torch.int32, step.sl.shape),
+                      qsl=dview(bf, 5, torch.int32, step.qsl.shape)) for bf in dbufs]
+        h2d = total  # bytes each step's H2D copy moves (inputs plus 256-byte alignment padding)
+        d2h = houts[0].numel() * houts[0].element_size()
 
-        def e2e_step():
-            dbuf.copy_(hbuf, non_blocking=True)
-            step.run(q=dq, k=dk, v=dv, bt=dbt, sl=dsl, qsl=dqsl)
-            hout.copy_(step.out, non_blocking=True)
+        def e2e_steps(n, t0=None, t1=None):
+            ev = lambda: torch.cuda.Event()  # noqa: E731
+            up_done = [ev(), ev()]
+            comp_done = [ev(), ev()]
+            down_done = [ev(), ev()]
+            if t0 is not None:
+                t0.record(up)
+            with torch.cuda.stream(up):
+                dbufs[0].copy_(hbuf, non_blocking=True)
+                up_done[0].record(up)
+            for i in range(n):
+                b = i & 1
+                if i + 1 < n:  # next step's inputs, once step i-1 has finished with that buffer
+                    with torch.cuda.stream(up):
+                        if i >= 1:
+                            up.wait_event(comp_done[1 - b])
+                        dbufs[1 - b].copy_(hbuf, non_blocking=True)
+                        up_done[1 - b].record(up)
+                stream.wait_event(up_done[b])
+                if i >= 2:  # step i-2's output has been read back from this buffer
+                    stream.wait_event(down_done[b])
+                if flush_l2:
+                    flush.zero_()
+                step.run(out=douts[b], **views[b])
+                comp_done[b].record(stream)
+                with torch.cuda.stream(down):
+                    down.wait_event(comp_done[b])
+                    houts[b].copy_(douts[b], non_blocking=True)
+                    down_done[b].record(down)
+            stream.wait_event(down_done[(n - 1) & 1])
+            if n >= 2:
+                stream.wait_event(down_done[n & 1])
+            if t1 is not None:
+                t1.record(stream)
 
-        for _ in range(max(args.warmup, 0)):
-            e2e_step()
+        e2e_steps(max(args.warmup, 1))
         torch.cuda.synchronize(device)
         barrier()
-        e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                for _ in range(args.steps)]
-        for i in range(args.steps):
-            if flush_l2:
-                flush.zero_()
-            e_ev[i][0].record(stream)
-            e2e_step()
-            e_ev[i][1].record(stream)
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e2e_steps(args.steps, t0, t1)
         torch.cuda.synchronize(device)
         barrier()
-        e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e_ev), world, device) / args.steps
+        e2e_ms = max_over_ranks(t0.elapsed_time(t1), world, device) / args.steps
+        # the pipelined path returns what the device-resident step computes, bit for bit
+        step.run()
+        torch.cuda.synchronize(device)
+        if not torch.equal(houts[(args.steps - 1) & 1], step.out.cpu()):
+            raise RuntimeError("end-to-end output differs from the device-resident step")
         e2e = {"value": round(world * nbytes / (e2e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
-               "ms_per_step": round(e2e_ms, 4)}
+               "ms_per_step": round(e2e_ms, 4),
+               "pipelining": "step i+1's H2D and step i's D2H overlap step i's compute"}
 
     result = None
     if rank == 0:
@@ -551,6 +610,7 @@ def run_device_bench(args, rank, world, local):
             "pct_hbm_peak": round(100 * value / world / peak, 2),
             "roofline": roof,
             "kernel_ms": {"decode": dec_ms, "chunk": chunk_ms, "reduce": reduce_ms},
+            "ms_per_step_with_kernel_events": round(ms_per_step_events, 4),
             "chunk_roofline": chunk_roof,
             "alloc": alloc,
             "e2e": e2e,
