@@ -82,3 +82,33 @@ def test_bench_byte_accounting():
     assert bench.unique_kv_bytes(wl) < bench.kv_bytes(wl)
     args = bench.parse_args([])
     assert args.gpus == 1 and args.steps > 0 and args.warmup >= 3
+
+
+def test_bench_flop_and_window_accounting():
+    """The algorithmic FLOPs and windowed bytes bench.py reports, against brute-force counts
+    of the unmasked (query, key) pairs and visible keys."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from paged_kv_cache_421_b200 import workloads as W
+    wl = W.mixed_step()
+    # the mixed step's prefill FLOPs: 4 D per unmasked pair per q head (about 21.5 GFLOP)
+    pairs = 0
+    for ctx, ql in zip(wl.seq_lens, wl.q_lens):
+        if ql * (wl.num_q_heads // wl.num_kv_heads) > 8:
+            pairs += sum(int(ctx) - int(ql) + i + 1 for i in range(int(ql)))
+    assert bench.chunk_flops(wl) == pairs * wl.num_q_heads * 4 * wl.head_size
+    assert abs(bench.chunk_flops(wl) / 1e9 - 21.48) < 0.01
+    for window in [1, 100, 700, 5000]:
+        pairs_w = 0
+        for ctx, ql in zip(wl.seq_lens, wl.q_lens):
+            if ql * 4 > 8:
+                pairs_w += sum(min(int(ctx) - int(ql) + i + 1, window) for i in range(int(ql)))
+        assert bench.chunk_flops(wl, window) == pairs_w * wl.num_q_heads * 4 * wl.head_size
+        keys = 0
+        for ctx, ql in zip(wl.seq_lens, wl.q_lens):
+            first = max(0, int(ctx) - int(ql) - window + 1)  # window start of the first query
+            keys += int(ctx) - first
+        assert bench.kv_bytes(wl, window) == keys * 2 * wl.num_kv_heads * wl.head_size * 2
+    # a window as long as every context changes nothing
+    assert bench.kv_bytes(wl, int(wl.seq_lens.max())) == bench.kv_bytes(wl)
+    assert bench.chunk_flops(wl, int(wl.seq_lens.max())) == bench.chunk_flops(wl)
