@@ -127,11 +127,20 @@ def load_tensor_peak() -> tuple:
         return FALLBACK_BF16_TFLOPS, "fallback"
 
 
+def _code_only(text: str) -> str:
+    """Source text without comments and blank-line or indentation differences, so that a
+    comment edit does not retire a recorded measurement of unchanged code."""
+    import re
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", "", text)
+    return "\n".join(line.strip() for line in text.splitlines() if line.strip())
+
+
 def source_digest(*names) -> str:
     h = hashlib.sha256()
     for n in names:
-        with open(os.path.join(ROOT, "paged_kv_cache_421_b200", "csrc", n), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, "paged_kv_cache_421_b200", "csrc", n)) as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -12,8 +12,11 @@
 // Data movement.  Each (physical block, K|V, kv head) tile is 16 tokens x head_size
 // contiguous in the pool and arrives in shared memory by one or two 2-D TMA loads with
 // 128-byte swizzling, completing on an mbarrier.  Every warp owns a private ring of
-// NS stages and the blocks j = warp, warp + NW, ... of the split, so warps never wait for
-// one another inside the stream; the CTA merges its warps' (m, l, O) at the end.
+// NS stages and the units u = warp, warp + NW, ... of the split (a unit is one block, two
+// for an FP8 cache), so warps never wait for one another inside the stream; the CTA merges
+// its warps' (m, l, O) at the end, and with several splits the last CTA of each (request,
+// kv head) to finish merges the splits.  With a sliding window the splits cover only the
+// blocks from the window start of the request's first query row.
 //
 // Math.  The MMA runs transposed: S^T = K Q^T with the 16 keys of a block on M and the
 // query rows (GQA group x q_len, padded to 8) on N of an m16n8k16 tile, so a group of 8
@@ -21,8 +24,8 @@
 // and O^T += V^T P^T reads V through ldmatrix.trans.  Softmax runs in the log2 domain.
 // FP8 E4M3 caches: S^T = K Q^T runs on FP8 tensor cores from the cache bytes (Q split
 // exactly into two E4M3 terms), and V tiles are stored dim-major so that ldmatrix hands out
-// four consecutive keys per word, decoded to f16 (exact) for O^T += V^T P^T; the K scale
-// folds into the score scale and the V scale into the epilogue.
+// four consecutive keys per word, widened exactly to f16 (as 2^-8 V, by moving bits) for
+// O^T += V^T P^T; the K scale folds into the score scale and the V scale into the epilogue.
 #include <cstdlib>
 
 #include "pa_internal.h"
