@@ -398,9 +398,9 @@ def run_device_bench(args, rank, world, local):
     for e in ev:  # torch creates events lazily: record once so the library gets real handles
         for x in e:
             x.record()
-    clocks = ClockSampler(local, os.path.join(ROOT, "gpurun_out", f".clocks_{rank}.csv")
-                          if os.path.isdir(os.path.join(ROOT, "gpurun_out"))
-                          else f"/tmp/clocks_{os.getpid()}.csv")
+    import tempfile
+    clocks = ClockSampler(local, os.path.join(tempfile.gettempdir(),
+                                              f"pa_clocks_{os.getpid()}_{rank}.csv"))
     clocks.start()
     time.sleep(0.3)
     stream = torch.cuda.current_stream(device)
