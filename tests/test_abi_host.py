@@ -183,3 +183,31 @@ def test_allocator_argument_errors_without_device(lib):
     assert lib.pa_free_blocks(None, 2, st, 8, st, None) == B.PA_ERR_INVALID_ARG
     assert lib.pa_free_blocks(st, 9, st, 8, st, None) == B.PA_ERR_INVALID_ARG
     assert lib.pa_free_blocks(st, 1, None, 8, st, None) == B.PA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("window", [1, 16, 100, 1000, 5000])
+def test_plan_with_sliding_window(lib, window):
+    """Decode CTAs cover only the blocks from the window start of each request's first query
+    row; chunk requests keep their split partition; a window past every context changes
+    nothing."""
+    wl = W.mixed_step()
+    ws = B.pa_attention_workspace_bytes(wl.num_tokens, wl.num_q_heads, wl.head_size, 1 << 16)
+    args = (wl.seq_lens, wl.qsl, wl.num_q_heads, wl.num_kv_heads, wl.head_size,
+            wl.max_blocks_per_seq, 148, ws)
+    p = B.pa_plan_attention(*args, sliding_window=window)
+    full = B.pa_plan_attention(*args)
+    G = wl.num_q_heads // wl.num_kv_heads
+    dec = (wl.q_lens > 0) & (wl.q_lens * G <= 8)
+    ctx, ql = wl.seq_lens.astype(np.int64), wl.q_lens.astype(np.int64)
+    first = np.maximum(0, ctx - ql - window + 1) // 16
+    eff = -(-ctx // 16) - first
+    sb = p["decode_split_blocks"]
+    assert p["decode_max_splits"] == int((-(-eff[dec] // sb)).max())
+    assert p["decode_ctas"] == int((-(-eff[dec] // sb)).sum()) * wl.num_kv_heads
+    assert p["decode_ctas"] <= full["decode_ctas"]
+    assert p["num_chunk_seqs"] == full["num_chunk_seqs"]
+    huge = B.pa_plan_attention(*args, sliding_window=int(ctx.max()) + 1)
+    assert huge == full
+    with pytest.raises(B.PaError) as e:
+        B.pa_plan_attention(*args, sliding_window=-1)
+    assert e.value.status == B.PA_ERR_INVALID_ARG
