@@ -153,7 +153,11 @@ size_t pa_attention_workspace_bytes(int num_tokens, int num_q_heads, int head_si
  * seq_lens_host, query_start_loc_host: host copies of the same arrays, used only to plan the
  *   launch (kernel choice, split count, grid size); they must equal the device contents.
  * Query i of request r attends to positions 0 .. seq_lens[r] - q_len + i (causal within a
- *   chunk; a decode row sees the whole context), with the softmax scale `scale`.
+ *   chunk; a decode row sees the whole context), with the softmax scale `scale`; with
+ *   pa_attention_opts.sliding_window = W > 0 (pa_attention_ex) only to the last W of them.
+ * Requests with q_len * (num_q_heads / num_kv_heads) <= 8 run in the decode kernel, the others
+ *   in the chunked-prefill kernel, which needs a bf16 cache (an FP8 cache with such a request
+ *   -> PA_ERR_UNSUPPORTED).
  * out: device fp32 [num_tokens][num_q_heads][head_size].
  * workspace: device scratch of workspace_bytes for split-KV partials (may be NULL/0: then no
  *   request is split).  Its contents are opaque; it must not be shared by calls that
