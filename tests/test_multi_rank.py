@@ -9,9 +9,6 @@ import socket
 import subprocess
 import sys
 
-import numpy as np
-import pytest
-import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 
