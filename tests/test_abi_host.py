@@ -211,3 +211,31 @@ def test_plan_with_sliding_window(lib, window):
     with pytest.raises(B.PaError) as e:
         B.pa_plan_attention(*args, sliding_window=-1)
     assert e.value.status == B.PA_ERR_INVALID_ARG
+
+
+def test_struct_layouts_match_the_header(tmp_path):
+    """The ctypes mirrors of pa_plan and pa_attention_opts have the header's sizes and field
+    offsets (compiled with the host C compiler against include/pa.h)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no host C compiler")
+    fields = {"pa_plan": [f[0] for f in B.pa_plan._fields_],
+              "pa_attention_opts": [f[0] for f in B.pa_attention_opts._fields_]}
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "pa.h"', 'int main(void) {']
+    for st, names in fields.items():
+        lines.append(f'printf("{st} size %zu\\n", sizeof({st}));')
+        for n in names:
+            lines.append(f'printf("{st} {n} %zu\\n", offsetof({st}, {n}));')
+    lines += ['return 0;', '}']
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")
+    got = {tuple(line.split()[:2]): int(line.split()[2]) for line in out if line.strip()}
+    for st, cls in [("pa_plan", B.pa_plan), ("pa_attention_opts", B.pa_attention_opts)]:
+        assert got[(st, "size")] == ctypes.sizeof(cls), st
+        for n in fields[st]:
+            assert got[(st, n)] == getattr(cls, n).offset, (st, n)
