@@ -87,10 +87,10 @@ def _load():
     lib.oracle_write_kv_fp8.argtypes = [P, i32, i32, i32, i32, P, P, P, P, P, i32]
     lib.oracle_attention_paged.restype = i32
     lib.oracle_attention_paged.argtypes = [P, i32, i32, i32, i32, i32, P, P, P, i32, P, i32,
-                                           P, P, i32, f64, i32, P, P]
+                                           P, P, i32, f64, i32, i32, P, P]
     lib.oracle_attention_rows.restype = i32
     lib.oracle_attention_rows.argtypes = [P, P, i32, i32, P, P, i32, P, P, P, i32, P, P, i32,
-                                          f64, i32, P, P, i32, P, P]
+                                          f64, i32, i32, P, P, i32, P, P]
     _lib = lib
     return lib
 
@@ -205,9 +205,11 @@ def write_kv(cache: np.ndarray, kv_dtype: int, num_blocks: int, block_size: int,
 def attention_paged(cache: np.ndarray, kv_dtype: int, num_blocks: int, block_size: int,
                     num_kv_heads: int, head_size: int, q_bits: np.ndarray, num_q_heads: int,
                     block_table: np.ndarray, seq_lens: np.ndarray, qsl: np.ndarray,
-                    scale: float, k_scale=None, v_scale=None, window: int = 0):
+                    scale: float, k_scale=None, v_scale=None, window: int = 0,
+                    local_chunk: int = 0):
     """Exact attention over the paged cache.  Returns (out [T][Hq][D], lse [T][Hq]) fp64.
-    window > 0: a query at position p sees keys max(0, p - window + 1) .. p."""
+    window > 0: a query at position p sees keys max(0, p - window + 1) .. p;
+    local_chunk > 0: only keys floor(p / local_chunk) * local_chunk .. p."""
     q = _c(q_bits, np.uint16)
     bt = _c(block_table, np.int32)
     sl = _c(seq_lens, np.int32)
@@ -220,7 +222,7 @@ def attention_paged(cache: np.ndarray, kv_dtype: int, num_blocks: int, block_siz
     _check(_load().oracle_attention_paged(
         _p(cache), kv_dtype, num_blocks, block_size, num_kv_heads, head_size, _p(ks), _p(vs),
         _p(q), num_q_heads, _p(bt), bt.shape[1], _p(sl), _p(qs), sl.size, float(scale),
-        int(window), _p(out), _p(lse)), "oracle_attention_paged")
+        int(window), int(local_chunk), _p(out), _p(lse)), "oracle_attention_paged")
     return out, lse
 
 
@@ -228,7 +230,7 @@ def attention_rows(k_src: np.ndarray, v_src: np.ndarray, pos_rows: np.ndarray,
                    pos_start: np.ndarray, kv_dtype: int, q_bits: np.ndarray,
                    seq_lens: np.ndarray, qsl: np.ndarray, scale: float,
                    sel_tokens: np.ndarray, sel_heads: np.ndarray, k_scale=None, v_scale=None,
-                   window: int = 0):
+                   window: int = 0, local_chunk: int = 0):
     """Unpaged exact attention for selected (token, q head) rows.
 
     k_src, v_src: uint16 bf16 bits [rows][Hkv][D]; request r's position p reads source row
@@ -250,6 +252,7 @@ def attention_rows(k_src: np.ndarray, v_src: np.ndarray, pos_rows: np.ndarray,
     vs = None if v_scale is None else _c(v_scale, np.float32)
     _check(_load().oracle_attention_rows(
         _p(k), _p(v), num_kv_heads, head_size, _p(pr), _p(ps), kv_dtype, _p(ks), _p(vs),
-        _p(q), num_q_heads, _p(sl), _p(qs), sl.size, float(scale), int(window), _p(st), _p(sh),
+        _p(q), num_q_heads, _p(sl), _p(qs), sl.size, float(scale), int(window),
+        int(local_chunk), _p(st), _p(sh),
         st.size, _p(out), _p(lse)), "oracle_attention_rows")
     return out, lse

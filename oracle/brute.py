@@ -45,9 +45,10 @@ def write_kv_bf16(cache: dict, k, v, slots, num_kv_heads, head_size, block_size)
 
 
 def attention(cache_value, q, num_q_heads, num_kv_heads, head_size, block_table, seq_lens,
-              qsl, block_size, scale, window=0):
+              qsl, block_size, scale, window=0, local_chunk=0):
     """cache_value(block, kv, head, tok, d) -> float.  q: nested [T][Hq][D] bf16 bits.
-    window > 0: the query at position p sees only positions p - window + 1 .. p.
+    window > 0: the query at position p sees only positions p - window + 1 .. p;
+    local_chunk > 0: only positions from the start of its chunk, floor(p / C) * C .. p.
     Returns out as nested lists [T][Hq][D] of floats."""
     group = num_q_heads // num_kv_heads
     T = int(qsl[-1])
@@ -59,6 +60,8 @@ def attention(cache_value, q, num_q_heads, num_kv_heads, head_size, block_table,
             t = int(qsl[r]) + i
             visible = ctx - q_len + i + 1
             start = max(0, visible - window) if window > 0 else 0
+            if local_chunk > 0:
+                start = max(start, (visible - 1) // local_chunk * local_chunk)
             for h in range(num_q_heads):
                 g = h // group
                 qv = [bf16_bits_to_float(q[t][h][d]) for d in range(head_size)]

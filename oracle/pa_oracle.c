@@ -288,13 +288,19 @@ static double attend_row(const double* qrow, const double* K, const double* V, i
     return mx + log(sum);
 }
 
-/* First key a query at position `limit` sees: all of them (window 0), else the last `window`
- * positions up to and including its own -- the sliding window the "vLLM architecture
- * overview" names (section 2, SlidingWindowManager keeps only the window's blocks; section 6,
- * SWA), read as a query at position p attending to keys max(0, p - W + 1) .. p. */
-static int first_key(int limit, int window) {
-    if (window <= 0) return 0;
-    return limit - window + 1 > 0 ? limit - window + 1 : 0;
+/* First key a query at position `limit` sees: all of them (window 0, local_chunk 0), else
+ * - the last `window` positions up to and including its own -- the sliding window the "vLLM
+ *   architecture overview" names (section 2, SlidingWindowManager keeps only the window's
+ *   blocks; section 6, SWA), read as a query at position p attending to keys
+ *   max(0, p - W + 1) .. p;
+ * - the start of its own chunk of `local_chunk` positions -- the chunked local attention of
+ *   the same section (ChunkedLocalAttentionManager), read as keys floor(p / C) * C .. p;
+ * and the later of the two when both are set. */
+static int first_key(int limit, int window, int local_chunk) {
+    int lo = 0;
+    if (window > 0 && limit - window + 1 > lo) lo = limit - window + 1;
+    if (local_chunk > 0 && limit / local_chunk * local_chunk > lo) lo = limit / local_chunk * local_chunk;
+    return lo;
 }
 
 static double cache_value(const void* cache, int kv_dtype, int64_t idx, double scale) {
@@ -311,7 +317,8 @@ int oracle_attention_paged(const void* cache, int kv_dtype, int num_blocks, int 
                            const float* v_scale, const uint16_t* q, int num_q_heads,
                            const int32_t* block_table, int max_blocks_per_seq,
                            const int32_t* seq_lens, const int32_t* qsl, int num_seqs,
-                           double scale, int window, double* out, double* lse) {
+                           double scale, int window, int local_chunk, double* out,
+                           double* lse) {
     int r, g, i, hh, d, p;
     int group = num_q_heads / num_kv_heads;
     if (group * num_kv_heads != num_q_heads) return OR_BAD_ARG;
@@ -360,7 +367,7 @@ int oracle_attention_paged(const void* cache, int kv_dtype, int num_blocks, int 
                     int64_t row = (int64_t)t * num_q_heads + h;
                     for (d = 0; d < head_size; ++d)
                         qrow[d] = oracle_bf16_to_double(q[row * head_size + d]);
-                    lse[row] = attend_row(qrow, K, V, first_key(limit, window), limit,
+                    lse[row] = attend_row(qrow, K, V, first_key(limit, window, local_chunk), limit,
                                           head_size, scale, s, out + row * head_size);
                 }
             }
@@ -380,6 +387,7 @@ int oracle_attention_rows(const uint16_t* k_src, const uint16_t* v_src, int num_
                           int kv_dtype, const float* k_scale, const float* v_scale,
                           const uint16_t* q, int num_q_heads, const int32_t* seq_lens,
                           const int32_t* qsl, int num_seqs, double scale, int window,
+                          int local_chunk,
                           const int32_t* sel_tokens, const int32_t* sel_heads, int nsel,
                           double* out, double* lse) {
     int j, r, d, p;
@@ -419,7 +427,8 @@ int oracle_attention_rows(const uint16_t* k_src, const uint16_t* v_src, int num_
         }
         for (d = 0; d < head_size; ++d)
             qrow[d] = oracle_bf16_to_double(q[((int64_t)t * num_q_heads + h) * head_size + d]);
-        lse[j] = attend_row(qrow, K, V, first_key(limit, window), limit, head_size, scale, s,
+        lse[j] = attend_row(qrow, K, V, first_key(limit, window, local_chunk), limit, head_size,
+                            scale, s,
                             out + (int64_t)j * head_size);
         free(K); free(V); free(s); free(qrow);
     }

@@ -661,3 +661,69 @@ def test_window_equal_keys_mean_of_window(oracle_mod):
         rows = wl.pos_rows[wl.pos_start[0] + np.arange(37 - w, 37)]
         want = v_src[rows, 0].double().numpy().mean(axis=0)
         np.testing.assert_allclose(o[0, 0], want, rtol=1e-12, atol=1e-13)
+
+
+# ------------------------------------------------------------------ chunked local attention
+# The architecture overview (section 2) also names ChunkedLocalAttentionManager without
+# defining it; the reading taken: a query at position p sees keys floor(p / C) * C .. p.
+
+@pytest.mark.parametrize("case", range(6))
+def test_local_chunk_vs_brute(oracle_mod, case):
+    rng = np.random.default_rng(800 + case)
+    bs = int([1, 2, 16, 4, 16, 2][case])
+    B = int(rng.integers(1, 4))
+    ctx = rng.integers(1, 41, size=B)
+    ql = np.array([rng.integers(1, c + 1) for c in ctx])
+    chunk = int(rng.integers(1, 20))
+    window = int(rng.choice([0, 0, 7]))
+    nb = int(sum(-(-c // bs) for c in ctx)) + 3
+    wl = W.make_workload("t", ctx, ql, 2, 1, 4, bs, nb, 400 + case, scale=0.7)
+    cache = _oracle_cache(oracle_mod, wl)
+    out, _ = oracle_mod.attention_paged(cache, W.BF16, nb, bs, 1, 4, W.bits(wl.q), 2,
+                                        wl.block_table, wl.seq_lens, wl.qsl, 0.7,
+                                        window=window, local_chunk=chunk)
+    c5 = cache.reshape(nb, 2, 1, bs, 4)
+
+    def val(b, kv, h, o, d):
+        return brute.bf16_bits_to_float(c5[b, kv, h, o, d])
+
+    want = brute.attention(val, W.bits(wl.q).tolist(), 2, 1, 4, wl.block_table.tolist(),
+                           wl.seq_lens.tolist(), wl.qsl.tolist(), bs, 0.7, window=window,
+                           local_chunk=chunk)
+    np.testing.assert_allclose(out, np.array(want), rtol=1e-11, atol=1e-12)
+
+
+def test_local_chunk_special_cases(oracle_mod):
+    wl = W.make_workload("t", [37, 20], [5, 20], 4, 2, 8, 16, 8, 43)
+    cache = _oracle_cache(oracle_mod, wl)
+    full = _attn_paged(oracle_mod, wl, cache)
+    args = (cache, W.BF16, wl.num_blocks, 16, 2, 8, W.bits(wl.q), 4, wl.block_table,
+            wl.seq_lens, wl.qsl, wl.scale)
+    # a chunk longer than every context is full attention; chunk 1 equals window 1
+    for c in [37, 1000]:
+        o, l = oracle_mod.attention_paged(*args, local_chunk=c)
+        assert np.array_equal(o, full[0]) and np.array_equal(l, full[1])
+    o1, l1 = oracle_mod.attention_paged(*args, local_chunk=1)
+    ow, lw = oracle_mod.attention_paged(*args, window=1)
+    assert np.array_equal(o1, ow) and np.array_equal(l1, lw)
+    # the first query of a chunk (p % C == 0) sees exactly its own key
+    k_src, v_src = wl.kv_src()
+    o, _ = oracle_mod.attention_paged(*args, local_chunk=16)
+    for r in range(2):
+        ql = int(wl.qsl[r + 1] - wl.qsl[r])
+        for i in range(ql):
+            p = int(wl.seq_lens[r]) - ql + i
+            if p % 16 == 0:
+                t = int(wl.qsl[r]) + i
+                row = wl.pos_rows[wl.pos_start[r] + p]
+                np.testing.assert_array_equal(o[t, 0], v_src[row, 0].float().numpy().astype(np.float64))
+    # paged agrees with unpaged under a local chunk
+    T, Hq = wl.num_tokens, 4
+    tok = np.repeat(np.arange(T), Hq).astype(np.int32)
+    hed = np.tile(np.arange(Hq), T).astype(np.int32)
+    for c in [3, 16, 17]:
+        o, _ = oracle_mod.attention_paged(*args, local_chunk=c)
+        o2, _ = oracle_mod.attention_rows(W.bits(k_src), W.bits(v_src), wl.pos_rows, wl.pos_start,
+                                          W.BF16, W.bits(wl.q), wl.seq_lens, wl.qsl, wl.scale,
+                                          tok, hed, local_chunk=c)
+        assert np.array_equal(o.reshape(T * Hq, -1), o2)
