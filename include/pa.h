@@ -154,7 +154,8 @@ size_t pa_attention_workspace_bytes(int num_tokens, int num_q_heads, int head_si
  *   launch (kernel choice, split count, grid size); they must equal the device contents.
  * Query i of request r attends to positions 0 .. seq_lens[r] - q_len + i (causal within a
  *   chunk; a decode row sees the whole context), with the softmax scale `scale`; with
- *   pa_attention_opts.sliding_window = W > 0 (pa_attention_ex) only to the last W of them.
+ *   pa_attention_opts.sliding_window = W > 0 (pa_attention_ex) only to the last W of them,
+ *   and with pa_attention_opts.local_chunk = C > 0 only to those from floor(p / C) * C.
  * Requests with q_len * (num_q_heads / num_kv_heads) <= 8 run in the decode kernel, the others
  *   in the chunked-prefill kernel, which needs a bf16 cache (an FP8 cache with such a request
  *   -> PA_ERR_UNSUPPORTED).
@@ -230,6 +231,10 @@ typedef struct {
     int sliding_window;    /* > 0: a query at position p sees only keys max(0, p - W + 1) .. p
                               (the sliding window [P2] section 2 names; its reading here);
                               0: full causal attention */
+    int local_chunk;       /* > 0: chunked local attention ([P2] section 2 names it; reading
+                              here): a query at position p sees only keys
+                              floor(p / C) * C .. p; combined with sliding_window the later
+                              start applies; 0: off */
 } pa_attention_opts;
 
 /* The planner alone: fills *plan for the given host metadata without touching the GPU.

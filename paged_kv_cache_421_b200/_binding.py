@@ -63,6 +63,7 @@ class pa_attention_opts(ctypes.Structure):
         ("num_sms", ctypes.c_int),
         ("events", ctypes.c_void_p * 6),
         ("sliding_window", ctypes.c_int),
+        ("local_chunk", ctypes.c_int),
     ]
 
 
@@ -206,12 +207,14 @@ def pa_attention_workspace_bytes(num_tokens, num_q_heads, head_size, max_splits)
 
 def pa_plan_attention(seq_lens_host, query_start_loc_host, num_q_heads, num_kv_heads,
                       head_size, max_blocks_per_seq, num_sms, workspace_bytes,
-                      kv_split_tokens=0, block_size=16, sliding_window=0) -> dict:
+                      kv_split_tokens=0, block_size=16, sliding_window=0,
+                      local_chunk=0) -> dict:
     sl = _host_i32(seq_lens_host)
     qs = _host_i32(query_start_loc_host)
     opts = pa_attention_opts()
     opts.kv_split_tokens = kv_split_tokens
     opts.sliding_window = sliding_window
+    opts.local_chunk = local_chunk
     plan = pa_plan()
     _check(load().pa_plan_attention(sl.ctypes.data, qs.ctypes.data, sl.size, int(qs[-1]),
                                     num_q_heads, num_kv_heads, head_size, block_size,
@@ -235,13 +238,15 @@ def pa_attention(handle, q, num_q_heads, block_table, max_blocks_per_seq, seq_le
 def pa_attention_ex(handle, q, num_q_heads, block_table, max_blocks_per_seq, seq_lens,
                     query_start_loc, seq_lens_host, query_start_loc_host, num_seqs, num_tokens,
                     scale, out, workspace=None, workspace_bytes=0, kv_split_tokens=0,
-                    num_sms=0, events=None, sliding_window=0, stream=None) -> None:
+                    num_sms=0, events=None, sliding_window=0, local_chunk=0,
+                    stream=None) -> None:
     sl = _host_i32(seq_lens_host)
     qs = _host_i32(query_start_loc_host)
     opts = pa_attention_opts()
     opts.kv_split_tokens = kv_split_tokens
     opts.num_sms = num_sms
     opts.sliding_window = sliding_window
+    opts.local_chunk = local_chunk
     for i, ev in enumerate(events or []):
         if ev is not None:
             opts.events[i] = ev.cuda_event if hasattr(ev, "cuda_event") else int(ev)

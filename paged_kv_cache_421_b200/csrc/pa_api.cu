@@ -159,7 +159,8 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
     const int forced = opts ? opts->kv_split_tokens : 0;
     if (forced < 0 || forced % bs) return PA_ERR_INVALID_ARG;
     const int window = opts ? opts->sliding_window : 0;
-    if (window < 0) return PA_ERR_INVALID_ARG;
+    const int local_chunk = opts ? opts->local_chunk : 0;
+    if (window < 0 || local_chunk < 0) return PA_ERR_INVALID_ARG;
     if (B > 0 && qsl[0] != 0) return PA_ERR_METADATA;
     long long dec_units = 0;
     int dec_max_blocks = 0, chunk_max_blocks = 0, chunk_max_qtiles = 0;
@@ -177,7 +178,7 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
         if (pa::is_decode_kind(ql, G)) {
             // with a sliding window the decode CTAs walk only the window's blocks
             pl->num_decode_seqs++;
-            const int eff = blocks - pa::window_first_key(ctx - ql, window) / bs;
+            const int eff = blocks - pa::first_visible_key(ctx - ql, window, local_chunk) / bs;
             dec_units += static_cast<long long>(eff) * Hkv;
             if (eff > dec_max_blocks) dec_max_blocks = eff;
         } else {
@@ -187,7 +188,8 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
             if (blocks > chunk_max_blocks) chunk_max_blocks = blocks;
             for (int i = 0; i < qt; ++i) {
                 const int last_row = std::min((i + 1) * chunk_cta_rows, ql * G) - 1;
-                const int lo = pa::window_first_key(ctx - ql + i * chunk_cta_rows / G, window) / bs * bs;
+                const int lo = pa::first_visible_key(ctx - ql + i * chunk_cta_rows / G, window,
+                                                     local_chunk) / bs * bs;
                 const long long w = pa::ceil_div(ctx - ql + last_row / G + 1 - lo, chunk_tile_keys);
                 chunk_work += w * Hkv;
                 if (w > chunk_work_max) chunk_work_max = w;
@@ -256,7 +258,7 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
         if (ql == 0) continue;
         int ns;
         if (pa::is_decode_kind(ql, G)) {
-            const int fb = pa::window_first_key(sl[r] - ql, window) / bs;
+            const int fb = pa::first_visible_key(sl[r] - ql, window, local_chunk) / bs;
             ns = pa::ceil_div(pa::ceil_div(sl[r], bs) - fb, pl->decode_split_blocks);
             pl->decode_ctas += static_cast<int64_t>(ns) * Hkv;
         } else {
@@ -496,6 +498,7 @@ int pa_attention_ex(const pa_cache* cache, const void* q, int num_q_heads,
     p.reduce_row_tiles = pa::ceil_div(pl.reduce_rows_max > 0 ? pl.reduce_rows_max : 1, 4);
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     p.window = opts ? opts->sliding_window : 0;
+    p.local_chunk = opts ? opts->local_chunk : 0;
     p.err = device_error_ptr();
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -553,7 +556,8 @@ int pa_attention_ex(const pa_cache* cache, const void* q, int num_q_heads,
             for (int qt = 0; qt < nqt; ++qt) {
                 const int last_row = std::min((qt + 1) * cta_rows, ql * p.group) - 1;
                 const int kmax = ctx - ql + last_row / p.group;
-                const int lo = pa::window_first_key(ctx - ql + qt * cta_rows / p.group, p.window) /
+                const int lo = pa::first_visible_key(ctx - ql + qt * cta_rows / p.group, p.window,
+                                                     p.local_chunk) /
                                cache->block_size * cache->block_size;
                 for (int sp = 0; sp < nsplit; ++sp) {
                     const int key_lo = std::max(sp * csb * cache->block_size, lo);

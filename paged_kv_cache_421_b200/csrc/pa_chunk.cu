@@ -83,7 +83,8 @@ chunk_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
     // the first key any row of the CTA may see: the split's start, or (sliding window) the
     // window start of the CTA's first row, rounded down to its block
     const int key_lo = max(jb * kBlockSize,
-                           window_first_key(ctx - q_len + R0 / G, p.window) / kBlockSize * kBlockSize);
+                           first_visible_key(ctx - q_len + R0 / G, p.window, p.local_chunk) /
+                               kBlockSize * kBlockSize);
     const int key_hi = min(kend, kmax + 1);
     const int ntiles = key_hi > key_lo ? ceil_div(key_hi - key_lo, kTileKeys) : 0;
 
@@ -102,7 +103,8 @@ chunk_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
     const bool vA = rA < rows_total, vB = rB < rows_total;
     const int limA = vA ? ctx - q_len + rA / G : kmax;
     const int limB = vB ? ctx - q_len + rB / G : kmax;
-    const int loA = window_first_key(limA, p.window), loB = window_first_key(limB, p.window);
+    const int loA = first_visible_key(limA, p.window, p.local_chunk);
+    const int loB = first_visible_key(limB, p.window, p.local_chunk);
     const int wlast = min(R0 + 16 * warp + 15, rows_total - 1);
     const int warp_kmax = ctx - q_len + wlast / G;
 

@@ -250,7 +250,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
     // the first key any row of the CTA may see: the split's start, or (sliding window) the
     // window start of the CTA's first row, rounded down to its block
     const int key_lo = max(jb * kBlockSize,
-                           window_first_key(ctx - q_len + R0 / G, p.window) / kBlockSize * kBlockSize);
+                           first_visible_key(ctx - q_len + R0 / G, p.window, p.local_chunk) /
+                               kBlockSize * kBlockSize);
     const int key_hi = min(kend, kmax + 1);
     const int ntiles = key_hi > key_lo ? ceil_div(key_hi - key_lo, kKeys) : 0;
     const bool two = R0 + kRows < rows_total;  // the second q-tile has rows
@@ -450,9 +451,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
             const bool valid = R < rows_total;
             const int lim = valid ? ctx - q_len + R / G : kmax;
             const int first_lim = ctx - q_len + (R0 + q * kRows) / G;  // smallest limit of the q-tile
-            const int lo = window_first_key(lim, p.window);            // first key this row sees
-            const int last_lo = window_first_key(                      // latest of the q-tile
-                ctx - q_len + min(R0 + q * kRows + kRows - 1, rows_total - 1) / G, p.window);
+            const int lo = first_visible_key(lim, p.window, p.local_chunk);  // this row's first key
+            const int last_lo = first_visible_key(  // the latest first key of the q-tile
+                ctx - q_len + min(R0 + q * kRows + kRows - 1, rows_total - 1) / G, p.window,
+                p.local_chunk);
             const uint32_t tq = tmem + q * 256;
             const uint32_t tmem_lane = tq + (static_cast<uint32_t>((warp & 3) * 32) << 16);
             const float sl = p.scale_log2;

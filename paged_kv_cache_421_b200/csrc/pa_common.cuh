@@ -29,10 +29,15 @@ constexpr int kErrMetadata = 4;   // device metadata disagrees with the planned 
 
 // A request is served by the decode kernel when all its query rows of one kv head fit one
 // 8-wide MMA tile, otherwise by the chunk kernel.  q_len == 0 requests produce nothing.
-// First key a query at position `limit` may see: 0, or with a sliding window of `window`
-// keys the last `window` positions up to its own.
-__host__ __device__ inline int window_first_key(int limit, int window) {
-    return (window > 0 && limit - window + 1 > 0) ? limit - window + 1 : 0;
+// First key a query at position `limit` may see: 0; with a sliding window of `window` keys,
+// the last `window` positions up to its own; with chunked local attention of `local_chunk`
+// positions, the start of its own chunk; the later of the two when both are set.  It never
+// decreases as `limit` grows.
+__host__ __device__ inline int first_visible_key(int limit, int window, int local_chunk) {
+    int lo = 0;
+    if (window > 0 && limit - window + 1 > lo) lo = limit - window + 1;
+    if (local_chunk > 0 && limit / local_chunk * local_chunk > lo) lo = limit / local_chunk * local_chunk;
+    return lo;
 }
 
 __host__ __device__ inline bool is_decode_kind(int q_len, int group) {

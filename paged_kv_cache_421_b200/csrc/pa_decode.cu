@@ -15,8 +15,8 @@
 // NS stages and the units u = warp, warp + NW, ... of the split (a unit is one block, two
 // for an FP8 cache), so warps never wait for one another inside the stream; the CTA merges
 // its warps' (m, l, O) at the end, and with several splits the last CTA of each (request,
-// kv head) to finish merges the splits.  With a sliding window the splits cover only the
-// blocks from the window start of the request's first query row.
+// kv head) to finish merges the splits.  With a sliding window or chunked local attention
+// the splits cover only the blocks from the first key the request's first query row sees.
 //
 // Math.  The MMA runs transposed: S^T = K Q^T with the 16 keys of a block on M and the
 // query rows (GQA group x q_len, padded to 8) on N of an m16n8k16 tile, so a group of 8
@@ -84,8 +84,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
         ctx = p.max_blocks_per_seq * kBlockSize;
     }
     const int nblocks = ceil_div(ctx, kBlockSize);
-    // with a sliding window the splits cover only the blocks from the window of the first row
-    const int fb = window_first_key(ctx - q_len, p.window) / kBlockSize;
+    // with a window or local chunks the splits cover only the blocks the first row may see
+    const int fb = first_visible_key(ctx - q_len, p.window, p.local_chunk) / kBlockSize;
     const int nsplit = ceil_div(nblocks - fb, p.decode_split_blocks);
     if (split >= nsplit) return;
     const int jb = fb + split * p.decode_split_blocks;
@@ -183,8 +183,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
     const int lim1 = row1 < rows ? ctx - q_len + row1 / p.group : ctx - 1;
     const int lim_min = min(lim0, lim1);
     // first visible key of the two rows, and of the group's last row (the latest window start)
-    const int lo0 = window_first_key(lim0, p.window), lo1 = window_first_key(lim1, p.window);
-    const int lo_last = window_first_key(ctx - 1, p.window);
+    const int lo0 = first_visible_key(lim0, p.window, p.local_chunk);
+    const int lo1 = first_visible_key(lim1, p.window, p.local_chunk);
+    const int lo_last = first_visible_key(ctx - 1, p.window, p.local_chunk);
 
     float o[C::kKSteps][4];
 #pragma unroll

@@ -70,6 +70,7 @@ struct AttnParams {
     int* err;                   // device error word
     int chunk_fused_merge;      // tcgen05 chunk kernel merges its own splits (<= kMaxFusedSplits)
     int window;                 // sliding window in keys, 0 = full causal attention
+    int local_chunk;            // chunked local attention: chunk length in keys, 0 = off
 };
 
 // The chunk-kind requests of a launch, longest context first (passed by value, so the chunk

@@ -59,11 +59,13 @@ class GpuStep:
                                      wl.scale, kv_split_tokens=kv_split_tokens)
         torch.cuda.synchronize()
 
-    def attend(self, kv_split_tokens: int = 0, sliding_window: int = 0) -> torch.Tensor:
+    def attend(self, kv_split_tokens: int = 0, sliding_window: int = 0,
+               local_chunk: int = 0) -> torch.Tensor:
         wl = self.wl
         out = ops.attention(self.cache, wl.q.cuda().contiguous(), self.step["bt"],
                             self.step["sl"], self.step["qsl"], wl.seq_lens, wl.qsl, wl.scale,
-                            kv_split_tokens=kv_split_tokens, sliding_window=sliding_window)
+                            kv_split_tokens=kv_split_tokens, sliding_window=sliding_window,
+                            local_chunk=local_chunk)
         torch.cuda.synchronize()
         return out
 
@@ -89,13 +91,14 @@ def oracle_cache(wl: W.Workload) -> np.ndarray:
     return cache
 
 
-def oracle_attention_all(wl: W.Workload, cache: np.ndarray, window: int = 0):
+def oracle_attention_all(wl: W.Workload, cache: np.ndarray, window: int = 0,
+                         local_chunk: int = 0):
     ks = None if wl.k_scale is None else wl.k_scale.cpu().numpy()
     vs = None if wl.v_scale is None else wl.v_scale.cpu().numpy()
     return oracle.attention_paged(cache, wl.kv_dtype, wl.num_blocks, wl.block_size,
                                   wl.num_kv_heads, wl.head_size, W.bits(wl.q), wl.num_q_heads,
                                   wl.block_table, wl.seq_lens, wl.qsl, wl.scale, ks, vs,
-                                  window=window)
+                                  window=window, local_chunk=local_chunk)
 
 
 def oracle_attention_rows(wl: W.Workload, tokens, heads):

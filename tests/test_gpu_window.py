@@ -55,3 +55,32 @@ def test_window_longer_than_context_is_full_attention():
     full = st.attend().cpu().numpy()
     assert np.array_equal(st.attend(sliding_window=1200).cpu().numpy(), full)
     assert np.array_equal(st.attend(sliding_window=1 << 20).cpu().numpy(), full)
+
+
+# chunked local attention: a query at position p sees keys floor(p / C) * C .. p
+@pytest.mark.parametrize("case", sorted(CASES))
+@pytest.mark.parametrize("chunk", [1, 16, 100, 1000])
+def test_local_chunk_matches_oracle(case, chunk):
+    ctx, ql, hq, hkv, d = CASES[case]
+    wl = _wl(ctx, ql, hq, hkv, d, seed=hash((case, chunk, "c")) % 997)
+    st = GpuStep(wl, run_attention=False)
+    want, _ = oracle_attention_all(wl, oracle_cache(wl), local_chunk=chunk)
+    for split in [0, 64]:
+        got = st.attend(kv_split_tokens=split, local_chunk=chunk).cpu().numpy()
+        assert_close(got, want, wl.kv_dtype, f"{case} C={chunk} split={split}")
+    assert B.pa_device_error(reset=True) == 0
+
+
+def test_local_chunk_with_window_and_fp8():
+    wl = _wl([5000, 37, 900], [1, 1, 1], 32, 8, 128, seed=7, kv_dtype=W.FP8_E4M3)
+    st = GpuStep(wl, run_attention=False)
+    for window, chunk in [(0, 512), (300, 1024), (2000, 256)]:
+        want, _ = oracle_attention_all(wl, oracle_cache(wl), window=window, local_chunk=chunk)
+        got = st.attend(sliding_window=window, local_chunk=chunk).cpu().numpy()
+        assert_close(got, want, wl.kv_dtype, f"fp8 W={window} C={chunk}")
+    wl = _wl([600, 1500], [600, 300], 8, 2, 128, seed=8)
+    st = GpuStep(wl, run_attention=False)
+    want, _ = oracle_attention_all(wl, oracle_cache(wl), window=200, local_chunk=256)
+    for split in [0, 64]:
+        got = st.attend(kv_split_tokens=split, sliding_window=200, local_chunk=256).cpu().numpy()
+        assert_close(got, want, wl.kv_dtype, f"chunks W=200 C=256 split={split}")
