@@ -49,6 +49,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end leg")
     ap.add_argument("--sliding-window", type=int, default=0,
                     help="attend to the last W keys only (0 = full causal attention)")
+    ap.add_argument("--local-chunk", type=int, default=0,
+                    help="chunked local attention: a query at position p sees keys "
+                         "floor(p / C) * C .. p (0 = off)")
     ap.add_argument("--no-alloc", action="store_true",
                     help="skip timing the device block allocation")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing")
@@ -61,40 +64,51 @@ def parse_args(argv=None):
     return ap.parse_args(argv)
 
 
-def visible_keys(wl, window: int = 0) -> np.ndarray:
-    """Keys each request's rows read: its whole context, or with a sliding window W the keys
-    from the window start of its first new token (ctx - q_len - W + 1) to the end."""
+def first_key(pos, window: int = 0, local_chunk: int = 0):
+    """First key a query at position pos sees: 0 for full causal attention, pos - W + 1 with a
+    sliding window W, floor(pos / C) * C with local chunks of C keys; the later of these."""
+    pos = np.asarray(pos, dtype=np.int64)
+    lo = np.zeros_like(pos)
+    if window > 0:
+        lo = np.maximum(lo, pos - window + 1)
+    if local_chunk > 0:
+        lo = np.maximum(lo, pos // local_chunk * local_chunk)
+    return lo
+
+
+def visible_keys(wl, window: int = 0, local_chunk: int = 0) -> np.ndarray:
+    """Keys each request's rows read: from the first key its first new token sees (at
+    position ctx - q_len) to the end of its context.  The first key never decreases with the
+    position, so later rows read a subset."""
     ctx = wl.seq_lens.astype(np.int64)
-    if window <= 0:
-        return ctx
-    return ctx - np.maximum(0, ctx - wl.q_lens.astype(np.int64) - window + 1)
+    return ctx - first_key(ctx - wl.q_lens.astype(np.int64), window, local_chunk)
 
 
-def kv_bytes(wl, window: int = 0) -> int:
+def kv_bytes(wl, window: int = 0, local_chunk: int = 0) -> int:
     """Algorithmic KV bytes the step's attention reads: every request's visible keys of K
     and V once per kv head (the GQA group shares one read)."""
-    return int(np.sum(visible_keys(wl, window))) * 2 * wl.num_kv_heads * wl.head_size * \
-        wl.dtype_bytes
-
-
-def decode_kv_bytes(wl, window: int = 0) -> int:
-    G = wl.num_q_heads // wl.num_kv_heads
-    ql = wl.q_lens
-    dec = (ql > 0) & (ql * G <= 8)
-    return int(np.sum(visible_keys(wl, window)[dec])) * 2 * wl.num_kv_heads * \
+    return int(np.sum(visible_keys(wl, window, local_chunk))) * 2 * wl.num_kv_heads * \
         wl.head_size * wl.dtype_bytes
 
 
-def chunk_flops(wl, window: int = 0) -> int:
+def decode_kv_bytes(wl, window: int = 0, local_chunk: int = 0) -> int:
+    G = wl.num_q_heads // wl.num_kv_heads
+    ql = wl.q_lens
+    dec = (ql > 0) & (ql * G <= 8)
+    return int(np.sum(visible_keys(wl, window, local_chunk)[dec])) * 2 * wl.num_kv_heads * \
+        wl.head_size * wl.dtype_bytes
+
+
+def chunk_flops(wl, window: int = 0, local_chunk: int = 0) -> int:
     """Algorithmic FLOPs of the chunk-kind requests: 4 D per unmasked (query, key) pair per q
-    head (Q K^T and P V); query i of a request with q_len new tokens sees ctx - q_len + i + 1
-    keys (at most W with a sliding window)."""
+    head (Q K^T and P V); query i of a request with q_len new tokens sits at position
+    p = ctx - q_len + i and sees the keys first_key(p) .. p."""
     G = wl.num_q_heads // wl.num_kv_heads
     total = 0
     for ctx, ql in zip(wl.seq_lens.astype(np.int64), wl.q_lens.astype(np.int64)):
         if ql > 0 and ql * G > 8:
-            vis = ctx - ql + np.arange(1, ql + 1, dtype=np.int64)
-            total += int(np.sum(np.minimum(vis, window) if window > 0 else vis))
+            pos = ctx - ql + np.arange(ql, dtype=np.int64)
+            total += int(np.sum(pos + 1 - first_key(pos, window, local_chunk)))
     return total * wl.num_q_heads * 4 * wl.head_size
 
 
@@ -251,7 +265,7 @@ def oracle_requests_for_budget(wl, kv_token_heads_budget: int) -> int:
 
 
 # ---------------------------------------------------------------- CPU oracle timing
-def oracle_step_timer(wl, window: int = 0):
+def oracle_step_timer(wl, window: int = 0, local_chunk: int = 0):
     """Build the oracle's cache (untimed) and return a function that times the oracle over
     the first n requests of the step: slot mapping, cache write of their new tokens and
     attention of their queries.  Returns (seconds, kv_bytes_of_those_requests)."""
@@ -278,15 +292,15 @@ def oracle_step_timer(wl, window: int = 0):
                         k_bits[:T], v_bits[:T], slots, ks, vs)
         oracle.attention_paged(cache, wl.kv_dtype, wl.num_blocks, 16, wl.num_kv_heads,
                                wl.head_size, q_bits[:T], wl.num_q_heads, bt, sl, qsl, wl.scale,
-                               ks, vs, window=window)
+                               ks, vs, window=window, local_chunk=local_chunk)
         ctx = sl.astype(np.int64)
-        keys = ctx if window <= 0 else ctx - np.maximum(0, ctx - np.diff(qsl) - window + 1)
+        keys = ctx - first_key(ctx - np.diff(qsl), window, local_chunk)
         return time.perf_counter() - t0, int(np.sum(keys)) * per_tok
     return run
 
 
-def cpu_baseline(wl, budget_s: float, window: int = 0) -> dict:
-    run = oracle_step_timer(wl, window)
+def cpu_baseline(wl, budget_s: float, window: int = 0, local_chunk: int = 0) -> dict:
+    run = oracle_step_timer(wl, window, local_chunk)
     # grow the sample until it takes about budget_s of CPU time
     n = 1
     sec, nbytes = run(n)
@@ -301,10 +315,12 @@ def cpu_baseline(wl, budget_s: float, window: int = 0) -> dict:
 
 # ---------------------------------------------------------------- device step
 class DeviceStep:
-    def __init__(self, wl, device, kv_split_tokens: int = 0, sliding_window: int = 0):
+    def __init__(self, wl, device, kv_split_tokens: int = 0, sliding_window: int = 0,
+                 local_chunk: int = 0):
         import torch
         self.kv_split_tokens = kv_split_tokens
         self.window = sliding_window
+        self.local_chunk = local_chunk
         from paged_kv_cache_421_b200 import ops
         from paged_kv_cache_421_b200 import workloads as W
         self.wl, self.dev, self.ops, self.torch = wl, device, ops, torch
@@ -333,14 +349,14 @@ class DeviceStep:
                                device=device)
         nb = ops.workspace_bytes_for(self.cache, wl.seq_lens, wl.qsl, wl.num_q_heads,
                                      wl.max_blocks_per_seq, kv_split_tokens,
-                                     sliding_window=sliding_window)
+                                     sliding_window=sliding_window, local_chunk=local_chunk)
         self.workspace = torch.empty(max(nb, 256), dtype=torch.uint8, device=device)
         self.plan = ops.B.pa_plan_attention(
             wl.seq_lens, wl.qsl, wl.num_q_heads, wl.num_kv_heads, wl.head_size,
             wl.max_blocks_per_seq,
             torch.cuda.get_device_properties(device).multi_processor_count,
             self.workspace.numel(), kv_split_tokens=kv_split_tokens,
-            sliding_window=sliding_window)
+            sliding_window=sliding_window, local_chunk=local_chunk)
         torch.cuda.synchronize(device)
 
     def launches_per_step(self) -> int:
@@ -365,7 +381,7 @@ class DeviceStep:
                           bt.shape[1], sl, qsl, wl.seq_lens, wl.qsl, wl.num_seqs, T, wl.scale,
                           out, self.workspace, self.workspace.numel(),
                           kv_split_tokens=self.kv_split_tokens, events=events,
-                          sliding_window=self.window)
+                          sliding_window=self.window, local_chunk=self.local_chunk)
 
 
 def run_device_bench(args, rank, world, local):
@@ -376,10 +392,10 @@ def run_device_bench(args, rank, world, local):
     device = torch.device(f"cuda:{local}")
     torch.cuda.set_device(device)
     wl = W.CONFIGS[args.workload](device=device)
-    step = DeviceStep(wl, device, args.kv_split_tokens, args.sliding_window)
+    step = DeviceStep(wl, device, args.kv_split_tokens, args.sliding_window, args.local_chunk)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
-    nbytes = kv_bytes(wl, args.sliding_window)
-    dec_bytes = decode_kv_bytes(wl, args.sliding_window)
+    nbytes = kv_bytes(wl, args.sliding_window, args.local_chunk)
+    dec_bytes = decode_kv_bytes(wl, args.sliding_window, args.local_chunk)
     flush_l2 = args.flush == "always" or (args.flush == "auto" and nbytes < 4 * L2_BYTES)
 
     def barrier():
@@ -588,12 +604,13 @@ def run_device_bench(args, rank, world, local):
                     "ms_per_launch": round(dec_ms, 4)}
         chunk_roof = None
         if chunk_ms:
-            tflops = chunk_flops(wl, args.sliding_window) / (chunk_ms * 1e-3) / 1e12
+            flops = chunk_flops(wl, args.sliding_window, args.local_chunk)
+            tflops = flops / (chunk_ms * 1e-3) / 1e12
             tpeak, tkind = load_tensor_peak()
             chunk_roof = {"bound": "tensor", "kernel": "chunk_tc_kernel", "achieved": round(tflops, 1),
                           "peak": tpeak, "unit": "TFLOP/s", "frac": round(tflops / tpeak, 4),
                           "traffic": None, "peak_kind": tkind,
-                          "flops_per_launch": chunk_flops(wl, args.sliding_window),
+                          "flops_per_launch": flops,
                           "ms_per_launch": round(chunk_ms, 4)}
             if roof is None:
                 roof = chunk_roof
@@ -614,6 +631,7 @@ def run_device_bench(args, rank, world, local):
                               f"126 MB L2, no flush"),
                        "kv_split_tokens": args.kv_split_tokens or "planner",
                        "sliding_window": args.sliding_window or None,
+                       "local_chunk": args.local_chunk or None,
                        "parallelism": f"replicas x{world} (one batch per GPU)"},
             "tokens_per_s": round(world * wl.num_tokens / (ms_per_step * 1e-3), 1),
             "pct_hbm_peak": round(100 * value / world / peak, 2),
@@ -636,7 +654,7 @@ def reference_arm(args, rank, world):
         return None
     from paged_kv_cache_421_b200 import workloads as W
     wl = W.CONFIGS[args.workload]()
-    run = oracle_step_timer(wl, args.sliding_window)
+    run = oracle_step_timer(wl, args.sliding_window, args.local_chunk)
     n = oracle_requests_for_budget(wl, 60_000_000)
     for _ in range(max(args.warmup, 0)):
         run(n)
@@ -681,7 +699,8 @@ def main(argv=None):
     result, wl = run_device_bench(args, rank, world, local)
     if rank == 0:
         if not args.no_cpu_baseline:
-            result["cpu_baseline"] = cpu_baseline(wl, args.cpu_budget_s, args.sliding_window)
+            result["cpu_baseline"] = cpu_baseline(wl, args.cpu_budget_s, args.sliding_window,
+                                                  args.local_chunk)
         print(json.dumps(result), flush=True)
     if world > 1:
         import torch.distributed as dist

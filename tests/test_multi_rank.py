@@ -109,3 +109,26 @@ def test_bench_flop_and_window_accounting():
     # a window as long as every context changes nothing
     assert bench.kv_bytes(wl, int(wl.seq_lens.max())) == bench.kv_bytes(wl)
     assert bench.chunk_flops(wl, int(wl.seq_lens.max())) == bench.chunk_flops(wl)
+
+
+def test_bench_local_chunk_accounting():
+    """Chunked local attention: a query at position p sees p % C + 1 keys (its own chunk up to
+    itself), and with a window W as well, the smaller of that and W."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from paged_kv_cache_421_b200 import workloads as W
+    wl = W.mixed_step()
+    big = 1 << 40
+    for C, Wn in [(1, 0), (16, 0), (100, 0), (1000, 0), (100, 37), (1000, 5000), (64, 1)]:
+        pairs = keys = 0
+        for ctx, ql in zip(wl.seq_lens.astype(int), wl.q_lens.astype(int)):
+            p0 = ctx - ql
+            keys += ctx - p0 + min(p0, Wn - 1 if Wn else big, p0 % C)
+            if ql * 4 > 8:
+                pairs += sum(min(p % C + 1, Wn if Wn else big) for p in range(p0, ctx))
+        assert bench.chunk_flops(wl, Wn, C) == pairs * wl.num_q_heads * 4 * wl.head_size
+        assert bench.kv_bytes(wl, Wn, C) == keys * 2 * wl.num_kv_heads * wl.head_size * 2
+    # chunks at least as long as every context change nothing
+    assert bench.kv_bytes(wl, 0, int(wl.seq_lens.max()) + 1) == bench.kv_bytes(wl)
+    assert bench.chunk_flops(wl, 0, int(wl.seq_lens.max()) + 1) == bench.chunk_flops(wl)
+    assert bench.parse_args(["--local-chunk", "8192"]).local_chunk == 8192
