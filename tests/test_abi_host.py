@@ -239,3 +239,83 @@ def test_struct_layouts_match_the_header(tmp_path):
         assert got[(st, "size")] == ctypes.sizeof(cls), st
         for n in fields[st]:
             assert got[(st, n)] == getattr(cls, n).offset, (st, n)
+
+
+@pytest.mark.parametrize("chunk", [1, 16, 100, 1000, 8192])
+def test_plan_with_local_chunk(lib, chunk):
+    """Chunked local attention: decode CTAs cover only the blocks from the first key of each
+    request's first query row, floor(p / C) * C; chunks at least as long as every context
+    change nothing."""
+    wl = W.mixed_step()
+    ws = B.pa_attention_workspace_bytes(wl.num_tokens, wl.num_q_heads, wl.head_size, 1 << 16)
+    args = (wl.seq_lens, wl.qsl, wl.num_q_heads, wl.num_kv_heads, wl.head_size,
+            wl.max_blocks_per_seq, 148, ws)
+    p = B.pa_plan_attention(*args, local_chunk=chunk)
+    full = B.pa_plan_attention(*args)
+    G = wl.num_q_heads // wl.num_kv_heads
+    dec = (wl.q_lens > 0) & (wl.q_lens * G <= 8)
+    ctx, ql = wl.seq_lens.astype(np.int64), wl.q_lens.astype(np.int64)
+    p0 = ctx - ql
+    eff = -(-ctx // 16) - (p0 - p0 % chunk) // 16
+    sb = p["decode_split_blocks"]
+    assert p["decode_max_splits"] == int((-(-eff[dec] // sb)).max())
+    assert p["decode_ctas"] == int((-(-eff[dec] // sb)).sum()) * wl.num_kv_heads
+    assert p["decode_ctas"] <= full["decode_ctas"]
+    assert B.pa_plan_attention(*args, local_chunk=int(ctx.max()) + 1) == full
+    with pytest.raises(B.PaError) as e:
+        B.pa_plan_attention(*args, local_chunk=-1)
+    assert e.value.status == B.PA_ERR_INVALID_ARG
+
+
+def test_plan_random_metadata_stays_inside_the_workspace(lib):
+    """Every plan the planner accepts indexes only the splits its workspace holds: for random
+    batches, windows, local chunks, forced splits and workspace sizes, each request's split
+    count (computed the way the kernels compute it) is at most the plan's maximum, and that
+    maximum's workspace fits in the bytes given."""
+    rng = np.random.default_rng(4217)
+    accepted = 0
+    for _ in range(300):
+        n = int(rng.integers(1, 40))
+        Hkv = int(rng.choice([1, 2, 8]))
+        Hq = Hkv * int(rng.choice([1, 4, 8]))
+        D = int(rng.choice([64, 128]))
+        ql = rng.choice([0, 1, 1, 1, 2, 3, 17, 130, 600], size=n).astype(np.int64)
+        ctx = ql + rng.integers(0, 20000, size=n)
+        ctx = np.where(ctx == 0, 0, np.maximum(ctx, 1))
+        qsl = np.concatenate([[0], np.cumsum(ql)])
+        T = int(qsl[-1])
+        maxb = int(max(1, (-(-ctx // 16)).max())) + int(rng.integers(0, 3))
+        window = int(rng.choice([0, 0, 1, 77, 4096]))
+        chunk = int(rng.choice([0, 0, 1, 100, 8192]))
+        forced = int(rng.choice([0, 0, 0, 16, 256, 4096]))
+        smax_ws = int(rng.choice([0, 1, 2, 5, 64, 1 << 12]))
+        ws = B.pa_attention_workspace_bytes(max(T, 1), Hq, D, smax_ws) if smax_ws > 1 else 0
+        try:
+            p = B.pa_plan_attention(ctx, qsl, Hq, Hkv, D, maxb, 148, ws, kv_split_tokens=forced,
+                                    sliding_window=window, local_chunk=chunk)
+        except B.PaError as e:
+            assert forced and e.status == B.PA_ERR_WORKSPACE, e
+            continue
+        accepted += 1
+        G = Hq // Hkv
+        blocks = -(-ctx // 16)
+        smax = max(p["decode_max_splits"], p["chunk_max_splits"])
+        assert p["decode_max_splits"] <= 1024
+        if smax > 1:
+            assert p["workspace_needed"] <= ws
+        for r in range(n):
+            if ql[r] == 0:
+                continue
+            if ql[r] * G <= 8:  # decode kind
+                lim = int(ctx[r] - ql[r])
+                lo = 0
+                if window:
+                    lo = max(lo, lim - window + 1)
+                if chunk:
+                    lo = max(lo, lim // chunk * chunk)
+                ns = -(-(int(blocks[r]) - lo // 16) // p["decode_split_blocks"])
+                assert 1 <= ns <= p["decode_max_splits"]
+            else:
+                ns = -(-int(blocks[r]) // p["chunk_split_blocks"])
+                assert 1 <= ns <= p["chunk_max_splits"]
+    assert accepted > 150
