@@ -88,6 +88,12 @@ def _load():
     lib.oracle_attention_paged.restype = i32
     lib.oracle_attention_paged.argtypes = [P, i32, i32, i32, i32, i32, P, P, P, i32, P, i32,
                                            P, P, i32, f64, i32, i32, P, P]
+    lib.oracle_dcp_local_len.restype = i32
+    lib.oracle_dcp_local_len.argtypes = [i32, i32, i32, i32]
+    lib.oracle_dcp_slot_mapping.restype = i32
+    lib.oracle_dcp_slot_mapping.argtypes = [P, i32, P, P, i32, i32, i32, i32, P]
+    lib.oracle_merge_partials.restype = None
+    lib.oracle_merge_partials.argtypes = [P, P, i32, i64, i32, P, P]
     lib.oracle_attention_rows.restype = i32
     lib.oracle_attention_rows.argtypes = [P, P, i32, i32, P, P, i32, P, P, P, i32, P, P, i32,
                                           f64, i32, i32, P, P, i32, P, P]
@@ -255,4 +261,41 @@ def attention_rows(k_src: np.ndarray, v_src: np.ndarray, pos_rows: np.ndarray,
         _p(q), num_q_heads, _p(sl), _p(qs), sl.size, float(scale), int(window),
         int(local_chunk), _p(st), _p(sh),
         st.size, _p(out), _p(lse)), "oracle_attention_rows")
+    return out, lse
+
+
+# ---------------------------------------------------------------- context parallelism
+def dcp_local_len(seq_lens, block_size: int, rank: int, world: int) -> np.ndarray:
+    """Keys rank `rank` of `world` holds of each request: block j of a request lives on rank
+    j mod world (see oracle_dcp_local_len)."""
+    lib = _load()
+    return np.array([lib.oracle_dcp_local_len(int(c), block_size, rank, world)
+                     for c in np.asarray(seq_lens).ravel()], np.int32)
+
+
+def dcp_slot_mapping(local_table: np.ndarray, seq_lens: np.ndarray, qsl: np.ndarray,
+                     block_size: int, rank: int, world: int) -> np.ndarray:
+    """Slots of the step's new tokens on one rank: -1 where another rank owns the token's
+    block (see oracle_dcp_slot_mapping).  seq_lens are total request lengths."""
+    bt = _c(local_table, np.int32)
+    sl = _c(seq_lens, np.int32)
+    q = _c(qsl, np.int32)
+    out = np.full(int(q[-1]), -2, np.int32)
+    _check(_load().oracle_dcp_slot_mapping(_p(bt), bt.shape[1], _p(sl), _p(q), sl.size,
+                                           block_size, rank, world, _p(out)),
+           "oracle_dcp_slot_mapping")
+    return out
+
+
+def merge_partials(part_o: np.ndarray, part_lse: np.ndarray):
+    """LSE merge of attention over disjoint key sets.  part_o [P][..., D], part_lse [P][...]
+    (natural log); returns (out [..., D], lse [...]) in fp64."""
+    o = _c(part_o, np.float64)
+    l = _c(part_lse, np.float64)
+    P, D = o.shape[0], o.shape[-1]
+    rows = l[0].size
+    assert o.size == P * rows * D and l.size == P * rows
+    out = np.zeros(o.shape[1:], np.float64)
+    lse = np.zeros(l.shape[1:], np.float64)
+    _load().oracle_merge_partials(_p(o), _p(l), P, rows, D, _p(out), _p(lse))
     return out, lse

@@ -434,3 +434,85 @@ int oracle_attention_rows(const uint16_t* k_src, const uint16_t* v_src, int num_
     }
     return OR_OK;
 }
+
+/* ------------------------------------------------------------------ context parallelism */
+/* Decode context parallelism (DCP): the "vLLM architecture overview" (section 8, its index of
+ * the FlashAttention document) names it without describing it.  Reading taken: a group of
+ * `world` ranks shares every request's KV; logical block j of a request lives on rank
+ * j mod world, as that rank's local logical block j / world, so each rank's share is an
+ * ordinary paged cache with its own block table.  Each rank attends the queries to its share
+ * and yields (O_r, lse_r); the shares are disjoint key sets, so their results combine exactly
+ * as the splits of split-KV attention do (oracle_merge_partials). */
+
+/* Keys of a request of total length ctx held by rank `rank` of `world`: the positions
+ * p < ctx whose block p / block_size the rank owns, counted one by one. */
+int oracle_dcp_local_len(int ctx, int block_size, int rank, int world) {
+    int p, n = 0;
+    for (p = 0; p < ctx; ++p)
+        if ((p / block_size) % world == rank) ++n;
+    return n;
+}
+
+/* Slots of a step's new tokens on rank `rank`.  seq_lens are the requests' total lengths
+ * (this step's tokens included); local_table is the rank's own block table.  The token at
+ * position p is stored only by the owner of its block j = p / bs, at local block j / world,
+ * offset p % bs; every other rank gets slot -1 (skip). */
+int oracle_dcp_slot_mapping(const int32_t* local_table, int max_blocks_per_seq,
+                            const int32_t* seq_lens, const int32_t* qsl, int num_seqs,
+                            int block_size, int rank, int world, int32_t* slot_mapping) {
+    int r, i;
+    if (world <= 0 || rank < 0 || rank >= world) return OR_BAD_ARG;
+    for (r = 0; r < num_seqs; ++r) {
+        int q_len = qsl[r + 1] - qsl[r];
+        int ctx = seq_lens[r];
+        if (q_len < 0 || q_len > ctx) return OR_BAD_META;
+        for (i = 0; i < q_len; ++i) {
+            int p = ctx - q_len + i;
+            int j = p / block_size;
+            int t = qsl[r] + i;
+            if (j % world != rank) {
+                slot_mapping[t] = -1;
+                continue;
+            }
+            if (j / world >= max_blocks_per_seq) return OR_BAD_META;
+            slot_mapping[t] =
+                local_table[(int64_t)r * max_blocks_per_seq + j / world] * block_size
+                + p % block_size;
+        }
+    }
+    return OR_OK;
+}
+
+/* Merge of attention results over disjoint key sets (the LSE combination that lets partial
+ * softmax results be merged, FlashAttention, article 7 outline of the first page).  Part k of
+ * row n holds O_k (normalised by its own softmax sum) and lse_k (natural log of that sum).
+ * With L = max_k lse_k:
+ *     out = sum_k e^(lse_k - L) O_k / sum_k e^(lse_k - L),   lse = L + ln sum_k e^(lse_k - L).
+ * A part with lse_k = -inf saw no key and carries no weight; a row whose parts all saw no key
+ * gets out = 0 and lse = -inf.  part_o: [num_parts][rows][head_size]; part_lse:
+ * [num_parts][rows]; out: [rows][head_size]; lse: [rows]. */
+void oracle_merge_partials(const double* part_o, const double* part_lse, int num_parts,
+                           int64_t rows, int head_size, double* out, double* lse) {
+    int64_t n;
+    int k, d;
+    for (n = 0; n < rows; ++n) {
+        double L = -INFINITY, wsum = 0.0;
+        for (k = 0; k < num_parts; ++k)
+            if (part_lse[(int64_t)k * rows + n] > L) L = part_lse[(int64_t)k * rows + n];
+        for (d = 0; d < head_size; ++d) out[n * head_size + d] = 0.0;
+        if (L == -INFINITY) {
+            lse[n] = -INFINITY;
+            continue;
+        }
+        for (k = 0; k < num_parts; ++k) {
+            double lk = part_lse[(int64_t)k * rows + n];
+            double w = lk == -INFINITY ? 0.0 : exp(lk - L);
+            wsum += w;
+            if (w == 0.0) continue;
+            for (d = 0; d < head_size; ++d)
+                out[n * head_size + d] += w * part_o[((int64_t)k * rows + n) * head_size + d];
+        }
+        for (d = 0; d < head_size; ++d) out[n * head_size + d] /= wsum;
+        lse[n] = L + log(wsum);
+    }
+}

@@ -727,3 +727,106 @@ def test_local_chunk_special_cases(oracle_mod):
                                           W.BF16, W.bits(wl.q), wl.seq_lens, wl.qsl, wl.scale,
                                           tok, hed, local_chunk=c)
         assert np.array_equal(o.reshape(T * Hq, -1), o2)
+
+
+# ------------------------------------------------------------------ context parallelism
+# The architecture overview names decode context parallelism (DCP) without describing it.
+# Reading taken: logical block j of a request lives on rank j mod world as that rank's local
+# block j / world; each rank attends to its share and the shares merge by their LSEs.
+
+def _dcp_local_tables(block_table, world):
+    """Each rank's block table over the same physical pool: rank r's local block l is the
+    global table's block l * world + r."""
+    B, M = block_table.shape
+    out = []
+    for r in range(world):
+        t = np.zeros((B, max(1, -(-M // world))), np.int32)
+        own = block_table[:, r::world]
+        t[:, :own.shape[1]] = own
+        out.append(t)
+    return out
+
+
+def test_dcp_local_len_golden_and_partition(oracle_mod):
+    # hand-counted: 40 keys in blocks of 16 over two ranks -> rank 0 holds blocks 0 and 2
+    # (16 + 8 keys), rank 1 block 1 (16 keys); 17 keys over four ranks -> 16, 1, 0, 0
+    assert list(oracle_mod.dcp_local_len([40], 16, 0, 2)) == [24]
+    assert list(oracle_mod.dcp_local_len([40], 16, 1, 2)) == [16]
+    assert [int(oracle_mod.dcp_local_len([17], 16, r, 4)[0]) for r in range(4)] == [16, 1, 0, 0]
+    ctx = np.arange(0, 300)
+    for world in [1, 2, 3, 5]:
+        parts = np.stack([oracle_mod.dcp_local_len(ctx, 16, r, world) for r in range(world)])
+        assert np.array_equal(parts.sum(axis=0), ctx)  # every key on exactly one rank
+        # whole rounds of `world` blocks give every rank the same share
+        full = ctx[ctx % (16 * world) == 0]
+        for r in range(world):
+            assert np.array_equal(oracle_mod.dcp_local_len(full, 16, r, world), full // world)
+    assert np.array_equal(oracle_mod.dcp_local_len(ctx, 16, 0, 1), ctx)
+
+
+@pytest.mark.parametrize("world", [1, 2, 3, 4])
+def test_dcp_slots_match_the_global_slots_on_the_owner(oracle_mod, world):
+    """With every rank's table drawn from one pool, the owner's local slot of a token is its
+    global slot and every other rank skips it: the sharded write stores each token exactly
+    once, where the unsharded write would."""
+    wl = W.make_workload("t", [1, 16, 17, 40, 100, 333], [1, 1, 17, 5, 100, 64], 4, 2, 16, 16,
+                         64, 87)
+    glob = oracle_mod.slot_mapping(wl.block_table, wl.seq_lens, wl.qsl, 16)
+    tables = _dcp_local_tables(wl.block_table, world)
+    per_rank = np.stack([oracle_mod.dcp_slot_mapping(tables[r], wl.seq_lens, wl.qsl, 16, r, world)
+                         for r in range(world)])
+    assert np.all(per_rank >= -1)
+    assert np.array_equal((per_rank >= 0).sum(axis=0), np.ones(wl.num_tokens))
+    assert np.array_equal(per_rank.max(axis=0), glob)
+    if world == 1:
+        assert np.array_equal(per_rank[0], glob)
+
+
+def test_merge_partials_closed_forms(oracle_mod):
+    rng = np.random.default_rng(5)
+    o = rng.standard_normal((1, 3, 8))
+    l = rng.standard_normal((1, 3))
+    out, lse = oracle_mod.merge_partials(o, l)          # one part: itself
+    assert np.array_equal(out, o[0]) and np.allclose(lse, l[0], rtol=0, atol=1e-15)
+    out, lse = oracle_mod.merge_partials(np.stack([o[0], o[0]]), np.stack([l[0], l[0]]))
+    np.testing.assert_allclose(out, o[0], rtol=1e-15)  # two equal halves: same O, sum doubled
+    np.testing.assert_allclose(lse, l[0] + math.log(2), rtol=1e-15)
+    inf = np.full((2, 3), -np.inf)
+    out, lse = oracle_mod.merge_partials(np.stack([o[0], 2 * o[0]]), inf)  # nothing seen
+    assert np.all(out == 0) and np.all(lse == -np.inf)
+    l2 = np.stack([l[0], np.full(3, -np.inf)])           # an empty part carries no weight
+    out, lse = oracle_mod.merge_partials(np.stack([o[0], np.full((3, 8), np.nan)]), l2)
+    assert np.array_equal(out, o[0]) and np.array_equal(lse, l[0])
+    # weights follow e^lse: lse 0 and ln 3 give weights 1/4 and 3/4
+    out, lse = oracle_mod.merge_partials(np.stack([np.ones((1, 2)), np.zeros((1, 2))]),
+                                         np.array([[0.0], [math.log(3)]]))
+    np.testing.assert_allclose(out, [[0.25, 0.25]], rtol=1e-15)
+    np.testing.assert_allclose(lse, [math.log(4)], rtol=1e-15)
+
+
+@pytest.mark.parametrize("world", [2, 3, 4])
+def test_dcp_shards_merge_to_full_attention(oracle_mod, world):
+    """Attention of each rank's share (its local table and local length, on the same pool),
+    merged by the LSEs, is the unsharded attention; ranks that hold no key of a request add
+    nothing (short contexts leave later ranks empty)."""
+    ctx = [1, 5, 16, 17, 33, 64, 65, 200, 517]
+    wl = W.make_workload("t", ctx, [1] * len(ctx), 8, 2, 16, 16, 80, 90 + world, scale=0.3)
+    cache = _oracle_cache(oracle_mod, wl)
+    full, lse_full = _attn_paged(oracle_mod, wl, cache)
+    tables = _dcp_local_tables(wl.block_table, world)
+    T, Hq, D = wl.num_tokens, wl.num_q_heads, wl.head_size
+    parts_o = np.zeros((world, T, Hq, D))
+    parts_l = np.full((world, T, Hq), -np.inf)
+    for r in range(world):
+        ll = oracle_mod.dcp_local_len(wl.seq_lens, 16, r, world)
+        ql = np.where(ll > 0, 1, 0).astype(np.int32)   # requests with no local key: no rows
+        qsl = np.concatenate([[0], np.cumsum(ql)]).astype(np.int32)
+        rows = np.nonzero(ll > 0)[0]
+        o, l = oracle_mod.attention_paged(cache, W.BF16, wl.num_blocks, 16, wl.num_kv_heads, D,
+                                          W.bits(wl.q)[rows], Hq, tables[r], ll, qsl, wl.scale)
+        parts_o[r, rows] = o
+        parts_l[r, rows] = l
+    assert np.any(parts_l == -np.inf)  # some shares are empty
+    out, lse = oracle_mod.merge_partials(parts_o, parts_l)
+    np.testing.assert_allclose(out, full, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(lse, lse_full, rtol=1e-13)
