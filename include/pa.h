@@ -14,7 +14,9 @@
  *        article 7 outline (FlashAttention tiling, online softmax, LSE, split of K vs Q).
  *   [P2] "vLLM architecture overview" (blog.chen3feng.top/vllm-analysis), section 2
  *        (PagedAttention: fixed-size blocks, int32 block table, shared prefix blocks),
- *        section 3 (kernel layer: PagedAttention V1/V2 kernels, reshape_and_cache).
+ *        section 3 (kernel layer: PagedAttention V1/V2 kernels, reshape_and_cache),
+ *        section 8 (index of its FlashAttention document, which names decode context
+ *        parallelism, DCP).
  *   [P3] "Inside vLLM" reading notes (kb.wilsonhandbook.online), core point 1 (16-token
  *        blocks, per-block bytes, allocate_slots' ceil(n/16)), core point 2 (all requests of
  *        a step flattened into one super-sequence, separated by positions and masks).
@@ -164,7 +166,8 @@ size_t pa_attention_workspace_bytes(int num_tokens, int num_q_heads, int head_si
  *   request is split).  Its contents are opaque; it must not be shared by calls that
  *   overlap on the GPU.
  * Host checks (-> PA_ERR_METADATA): query_start_loc_host non-decreasing from 0 to num_tokens,
- *   0 <= q_len <= seq_len, seq_len > 0 when q_len > 0, ceil(seq_len / block_size) <=
+ *   0 <= q_len <= seq_len, seq_len > 0 when q_len > 0 (with pa_attention_opts.lse_out a
+ *   decode-kind request may have seq_len == 0), ceil(seq_len / block_size) <=
  *   max_blocks_per_seq.  Errors: INVALID_ARG, UNSUPPORTED, METADATA, CUDA. */
 int pa_attention(const pa_cache* cache, const void* q, int num_q_heads,
                  const int32_t* block_table, int max_blocks_per_seq, const int32_t* seq_lens,
@@ -235,6 +238,13 @@ typedef struct {
                               here): a query at position p sees only keys
                               floor(p / C) * C .. p; combined with sliding_window the later
                               start applies; 0: off */
+    float* lse_out;        /* optional device fp32 [num_tokens][num_q_heads]: each row's
+                              log-sum-exp, ln of the sum over its visible keys of
+                              exp(scale * q.k) (its softmax denominator), so that results over
+                              disjoint key sets can be merged (pa_merge_partials).  When given,
+                              decode-kind requests with seq_len == 0 are also accepted: their
+                              rows get out = 0 and lse = -inf (an empty share of a context-
+                              parallel group).  NULL: not written */
 } pa_attention_opts;
 
 /* The planner alone: fills *plan for the given host metadata without touching the GPU.
@@ -251,6 +261,50 @@ int pa_attention_ex(const pa_cache* cache, const void* q, int num_q_heads,
                     const int32_t* query_start_loc_host, int num_seqs, int num_tokens,
                     float scale, float* out, void* workspace, size_t workspace_bytes,
                     const pa_attention_opts* opts, void* stream);
+
+/* Decode context parallelism ([P2] section 8 names DCP; the pages do not describe it, so the
+ * reading here): a group of `world` ranks (one per GPU) shares every request's KV.  Logical
+ * block j of a request lives on rank j mod world, as that rank's local logical block
+ * j / world, so each rank's share is an ordinary paged cache with its own block table.  A
+ * step on each rank: pa_dcp_slot_mapping + pa_write_kv store the new tokens the rank owns;
+ * pa_attention_ex with lse_out and the rank's local lengths (pa_dcp_local_seq_lens) attends
+ * every query to the rank's share; the ranks exchange their (out, lse) (an all-gather over
+ * NCCL); pa_merge_partials combines them into the attention over the whole context.  Every
+ * query row must be decode-kind (q_len * group <= 8): chunk rows need causal masks across
+ * shares, which this split does not express. */
+
+/* Keys of each request that rank `rank` of `world` holds: local_seq_lens_host[r] = number of
+ * positions p < seq_lens_host[r] with (p / block_size) mod world == rank.  Host arrays
+ * [num_seqs]; pure host computation.  Errors: INVALID_ARG (world < 1, rank outside
+ * [0, world), block_size < 1, a negative length). */
+int pa_dcp_local_seq_lens(const int32_t* seq_lens_host, int num_seqs, int block_size,
+                          int rank, int world, int32_t* local_seq_lens_host);
+
+/* Slot mapping of a step's new tokens on rank `rank` of a DCP group.  seq_lens: device int32
+ * [num_seqs], the requests' TOTAL lengths (this step's tokens included); block_table: the
+ * rank's local table, device int32 [num_seqs][max_blocks_per_seq]; query_start_loc as in
+ * pa_slot_mapping.  New token i of request r sits at position p = seq_lens[r] - q_len + i in
+ * block j = p / block_size: the rank that owns j (j mod world) gets slot
+ * block_table[r][j / world] * block_size + p % block_size, every other rank -1, which
+ * pa_write_kv skips.  A local block index >= max_blocks_per_seq gets -1 and records a device
+ * error.  Errors: INVALID_ARG, CUDA. */
+int pa_dcp_slot_mapping(const int32_t* block_table, int max_blocks_per_seq,
+                        const int32_t* seq_lens, const int32_t* query_start_loc, int num_seqs,
+                        int num_tokens, int block_size, int rank, int world,
+                        int32_t* slot_mapping, void* stream);
+
+/* Merge of attention results over disjoint key sets ([P1] article 7: the LSE is what lets
+ * partial softmax results be combined).  part_out: device fp32 [num_parts][num_rows]
+ * [head_size], each part normalised by its own softmax sum; part_lse: device fp32
+ * [num_parts][num_rows], natural log of that sum (-inf: the part saw no key).  With
+ * L = max_k lse_k:
+ *     out = sum_k e^(lse_k - L) O_k / sum_k e^(lse_k - L),  lse = L + ln sum_k e^(lse_k - L);
+ * a row with no key in any part gets out = 0 and lse = -inf.  out: device fp32 [num_rows]
+ * [head_size]; lse_out: device fp32 [num_rows] or NULL.  head_size 64 or 128 (else
+ * UNSUPPORTED); num_parts 1 .. 1024.  Errors: INVALID_ARG, UNSUPPORTED, CUDA. */
+int pa_merge_partials(const float* part_out, const float* part_lse, int num_parts,
+                      int64_t num_rows, int head_size, float* out, float* lse_out,
+                      void* stream);
 
 /* Opt-in device check of the metadata a step will read: every block id that
  * attention would read (logical blocks 0 .. ceil(seq_len / block_size) - 1 of each request)

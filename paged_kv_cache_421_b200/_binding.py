@@ -33,6 +33,7 @@ EXPORTED = [
     "pa_write_kv", "pa_attention_workspace_bytes", "pa_attention", "pa_plan_attention",
     "pa_attention_ex", "pa_validate_block_table", "pa_device_error", "pa_status_string",
     "pa_last_cuda_error", "pa_attention_noalloc", "pa_allocate_slots", "pa_free_blocks",
+    "pa_dcp_local_seq_lens", "pa_dcp_slot_mapping", "pa_merge_partials",
 ]
 PA_NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -64,6 +65,7 @@ class pa_attention_opts(ctypes.Structure):
         ("events", ctypes.c_void_p * 6),
         ("sliding_window", ctypes.c_int),
         ("local_chunk", ctypes.c_int),
+        ("lse_out", ctypes.c_void_p),
     ]
 
 
@@ -110,6 +112,9 @@ def load() -> ctypes.CDLL:
         "pa_status_string": (ctypes.c_char_p, [I]),
         "pa_last_cuda_error": (I, []),
         "pa_attention_noalloc": (I, [P, P, I, P, I, P, P, P, P, I, I, F, P, P]),
+        "pa_dcp_local_seq_lens": (I, [P, I, I, I, I, P]),
+        "pa_dcp_slot_mapping": (I, [P, I, P, P, I, I, I, I, I, P, P]),
+        "pa_merge_partials": (I, [P, P, I, ctypes.c_int64, I, P, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -208,13 +213,16 @@ def pa_attention_workspace_bytes(num_tokens, num_q_heads, head_size, max_splits)
 def pa_plan_attention(seq_lens_host, query_start_loc_host, num_q_heads, num_kv_heads,
                       head_size, max_blocks_per_seq, num_sms, workspace_bytes,
                       kv_split_tokens=0, block_size=16, sliding_window=0,
-                      local_chunk=0) -> dict:
+                      local_chunk=0, with_lse=False) -> dict:
+    """with_lse: plan as a call that exports LSEs (which admits empty decode shares); the
+    planner only tests the pointer for NULL, so a dummy non-NULL value stands in."""
     sl = _host_i32(seq_lens_host)
     qs = _host_i32(query_start_loc_host)
     opts = pa_attention_opts()
     opts.kv_split_tokens = kv_split_tokens
     opts.sliding_window = sliding_window
     opts.local_chunk = local_chunk
+    opts.lse_out = 16 if with_lse else None
     plan = pa_plan()
     _check(load().pa_plan_attention(sl.ctypes.data, qs.ctypes.data, sl.size, int(qs[-1]),
                                     num_q_heads, num_kv_heads, head_size, block_size,
@@ -238,7 +246,7 @@ def pa_attention(handle, q, num_q_heads, block_table, max_blocks_per_seq, seq_le
 def pa_attention_ex(handle, q, num_q_heads, block_table, max_blocks_per_seq, seq_lens,
                     query_start_loc, seq_lens_host, query_start_loc_host, num_seqs, num_tokens,
                     scale, out, workspace=None, workspace_bytes=0, kv_split_tokens=0,
-                    num_sms=0, events=None, sliding_window=0, local_chunk=0,
+                    num_sms=0, events=None, sliding_window=0, local_chunk=0, lse_out=None,
                     stream=None) -> None:
     sl = _host_i32(seq_lens_host)
     qs = _host_i32(query_start_loc_host)
@@ -247,6 +255,7 @@ def pa_attention_ex(handle, q, num_q_heads, block_table, max_blocks_per_seq, seq
     opts.num_sms = num_sms
     opts.sliding_window = sliding_window
     opts.local_chunk = local_chunk
+    opts.lse_out = _ptr(lse_out)
     for i, ev in enumerate(events or []):
         if ev is not None:
             opts.events[i] = ev.cuda_event if hasattr(ev, "cuda_event") else int(ev)
@@ -288,3 +297,27 @@ def pa_device_error(reset: bool = True) -> int:
 
 def pa_status_string(status: int) -> str:
     return load().pa_status_string(status).decode()
+
+
+def pa_dcp_local_seq_lens(seq_lens_host, block_size, rank, world) -> np.ndarray:
+    """Keys of each request that rank `rank` of a `world`-rank DCP group holds (host)."""
+    sl = _host_i32(seq_lens_host)
+    out = np.zeros(sl.size, np.int32)
+    _check(load().pa_dcp_local_seq_lens(sl.ctypes.data, sl.size, block_size, rank, world,
+                                        out.ctypes.data), "pa_dcp_local_seq_lens")
+    return out
+
+
+def pa_dcp_slot_mapping(block_table, max_blocks_per_seq, seq_lens, query_start_loc, num_seqs,
+                        num_tokens, block_size, rank, world, slot_mapping, stream=None) -> None:
+    _check(load().pa_dcp_slot_mapping(_ptr(block_table), max_blocks_per_seq, _ptr(seq_lens),
+                                      _ptr(query_start_loc), num_seqs, num_tokens, block_size,
+                                      rank, world, _ptr(slot_mapping), _stream(stream)),
+           "pa_dcp_slot_mapping")
+
+
+def pa_merge_partials(part_out, part_lse, num_parts, num_rows, head_size, out, lse_out=None,
+                      stream=None) -> None:
+    _check(load().pa_merge_partials(_ptr(part_out), _ptr(part_lse), num_parts, num_rows,
+                                    head_size, _ptr(out), _ptr(lse_out), _stream(stream)),
+           "pa_merge_partials")

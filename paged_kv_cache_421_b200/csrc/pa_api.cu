@@ -161,6 +161,9 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
     const int window = opts ? opts->sliding_window : 0;
     const int local_chunk = opts ? opts->local_chunk : 0;
     if (window < 0 || local_chunk < 0) return PA_ERR_INVALID_ARG;
+    // with an LSE output a decode-kind request may hold no key (an empty context-parallel
+    // share): one CTA per kv head writes out = 0 and lse = -inf for its rows
+    const bool empty_ok = opts && opts->lse_out;
     if (B > 0 && qsl[0] != 0) return PA_ERR_METADATA;
     long long dec_units = 0;
     int dec_max_blocks = 0, chunk_max_blocks = 0, chunk_max_qtiles = 0;
@@ -171,8 +174,14 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
     for (int r = 0; r < B; ++r) {
         const int ql = qsl[r + 1] - qsl[r];
         const int ctx = sl[r];
-        if (ql < 0 || ctx < ql || (ql > 0 && ctx <= 0)) return PA_ERR_METADATA;
+        if (ql < 0 || ctx < 0) return PA_ERR_METADATA;
         if (ql == 0) continue;
+        if (ctx == 0) {
+            if (!empty_ok || !pa::is_decode_kind(ql, G)) return PA_ERR_METADATA;
+            pl->num_decode_seqs++;
+            continue;
+        }
+        if (ctx < ql) return PA_ERR_METADATA;
         const int blocks = pa::ceil_div(ctx, bs);
         if (blocks > maxb) return PA_ERR_METADATA;
         if (pa::is_decode_kind(ql, G)) {
@@ -199,9 +208,10 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
     if (B > 0 && qsl[B] != T) return PA_ERR_METADATA;
     const int allowed = max_splits_for(ws, T, Hq, D);
 
-    // decode partition
+    // decode partition (at least one block long, even when every decode request is empty)
     int dsb = 1;
     if (pl->num_decode_seqs) {
+        if (dec_max_blocks < 1) dec_max_blocks = 1;
         if (forced) {
             dsb = forced / bs;
         } else {
@@ -259,7 +269,7 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
         int ns;
         if (pa::is_decode_kind(ql, G)) {
             const int fb = pa::first_visible_key(sl[r] - ql, window, local_chunk) / bs;
-            ns = pa::ceil_div(pa::ceil_div(sl[r], bs) - fb, pl->decode_split_blocks);
+            ns = std::max(1, pa::ceil_div(pa::ceil_div(sl[r], bs) - fb, pl->decode_split_blocks));
             pl->decode_ctas += static_cast<int64_t>(ns) * Hkv;
         } else {
             ns = pa::num_splits(sl[r], pl->chunk_split_blocks);
@@ -453,7 +463,8 @@ int pa_attention_ex(const pa_cache* cache, const void* q, int num_q_heads,
     if (!(scale > 0.f) || scale != scale) return PA_ERR_INVALID_ARG;
     if (workspace_bytes && !workspace) return PA_ERR_INVALID_ARG;
     if ((reinterpret_cast<uintptr_t>(q) & 15) || (reinterpret_cast<uintptr_t>(out) & 15) ||
-        (reinterpret_cast<uintptr_t>(workspace) & 255))
+        (reinterpret_cast<uintptr_t>(workspace) & 255) ||
+        (opts && (reinterpret_cast<uintptr_t>(opts->lse_out) & 3)))
         return PA_ERR_INVALID_ARG;
     const int num_sms = (opts && opts->num_sms > 0) ? opts->num_sms : device_num_sms();
     if (num_sms <= 0) return fail_cuda(cudaErrorNoDevice);
@@ -499,6 +510,7 @@ int pa_attention_ex(const pa_cache* cache, const void* q, int num_q_heads,
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     p.window = opts ? opts->sliding_window : 0;
     p.local_chunk = opts ? opts->local_chunk : 0;
+    p.lse_out = opts ? opts->lse_out : nullptr;
     p.err = device_error_ptr();
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -619,6 +631,57 @@ int pa_validate_block_table(const pa_cache* cache, const int32_t* block_table,
     if (e == cudaSuccess) e = cudaMemcpyAsync(num_bad, counter, sizeof(int), cudaMemcpyDeviceToHost, s);
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     cudaFreeAsync(counter, s);
+    return e == cudaSuccess ? PA_OK : fail_cuda(e);
+}
+
+int pa_dcp_local_seq_lens(const int32_t* seq_lens_host, int num_seqs, int block_size,
+                          int rank, int world, int32_t* local_seq_lens_host) {
+    if (num_seqs < 0 || block_size < 1 || world < 1 || rank < 0 || rank >= world)
+        return PA_ERR_INVALID_ARG;
+    if (num_seqs == 0) return PA_OK;
+    if (!seq_lens_host || !local_seq_lens_host) return PA_ERR_INVALID_ARG;
+    for (int r = 0; r < num_seqs; ++r)
+        if (seq_lens_host[r] < 0) return PA_ERR_INVALID_ARG;
+    for (int r = 0; r < num_seqs; ++r) {
+        // full blocks j < nb with j mod world == rank hold block_size keys each; the partly
+        // filled block nb holds the remainder
+        const int nb = seq_lens_host[r] / block_size, rem = seq_lens_host[r] % block_size;
+        int n = nb > rank ? ((nb - rank - 1) / world + 1) * block_size : 0;
+        if (rem && nb % world == rank) n += rem;
+        local_seq_lens_host[r] = n;
+    }
+    return PA_OK;
+}
+
+int pa_dcp_slot_mapping(const int32_t* block_table, int max_blocks_per_seq,
+                        const int32_t* seq_lens, const int32_t* query_start_loc, int num_seqs,
+                        int num_tokens, int block_size, int rank, int world,
+                        int32_t* slot_mapping, void* stream) {
+    if (num_seqs < 0 || num_tokens < 0 || block_size <= 0 || max_blocks_per_seq <= 0 ||
+        world < 1 || rank < 0 || rank >= world)
+        return PA_ERR_INVALID_ARG;
+    if (num_seqs == 0 || num_tokens == 0) return PA_OK;
+    if (!block_table || !seq_lens || !query_start_loc || !slot_mapping) return PA_ERR_INVALID_ARG;
+    if (num_seqs > (1 << 30)) return PA_ERR_UNSUPPORTED;
+    cudaError_t e = pa::launch_dcp_slot_mapping(block_table, max_blocks_per_seq, seq_lens,
+                                                query_start_loc, num_seqs, num_tokens,
+                                                block_size, rank, world, slot_mapping,
+                                                device_error_ptr(), static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? PA_OK : fail_cuda(e);
+}
+
+int pa_merge_partials(const float* part_out, const float* part_lse, int num_parts,
+                      int64_t num_rows, int head_size, float* out, float* lse_out, void* stream) {
+    if (num_parts < 1 || num_parts > 1024 || num_rows < 0) return PA_ERR_INVALID_ARG;
+    if (head_size != 64 && head_size != 128) return PA_ERR_UNSUPPORTED;
+    if (num_rows == 0) return PA_OK;
+    if (!part_out || !part_lse || !out) return PA_ERR_INVALID_ARG;
+    if ((reinterpret_cast<uintptr_t>(part_out) | reinterpret_cast<uintptr_t>(out)) & 15)
+        return PA_ERR_INVALID_ARG;  // rows are read and written as 16- or 8-byte vectors
+    if ((reinterpret_cast<uintptr_t>(part_lse) | reinterpret_cast<uintptr_t>(lse_out)) & 3)
+        return PA_ERR_INVALID_ARG;
+    cudaError_t e = pa::launch_merge_partials(part_out, part_lse, num_parts, num_rows, head_size,
+                                              out, lse_out, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? PA_OK : fail_cuda(e);
 }
 

@@ -314,6 +314,9 @@ chunk_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
         float* dst;
         if (direct) {
             dst = p.out + (static_cast<int64_t>(t) * p.num_q_heads + h) * D;
+            if (tq == 0 && p.lse_out)
+                p.lse_out[static_cast<int64_t>(t) * p.num_q_heads + h] =
+                    l > 0.f ? (m + __log2f(l)) * kLn2 : -INFINITY;
         } else {
             const int64_t prow = (static_cast<int64_t>(split) * p.num_tokens + t) * p.num_q_heads + h;
             dst = p.part_o + prow * D;

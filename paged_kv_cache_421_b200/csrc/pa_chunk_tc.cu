@@ -566,10 +566,13 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
             const bool all_ok = __all_sync(0xffffffffu, ok);
             const bool have = all_ok && ntiles > 0;
             const float inv = l > 0.f ? 1.f / l : 0.f;
-            if (all_ok && valid && nsplit > 1) {
+            if (all_ok && valid && (nsplit > 1 || p.lse_out)) {
                 const int t = q0 + R / G, h = g * G + R % G;
-                p.part_lse[(static_cast<int64_t>(split) * p.num_tokens + t) * p.num_q_heads + h] =
-                    l > 0.f ? m_used + __log2f(l) : -INFINITY;
+                const float lse2 = l > 0.f ? m_used + __log2f(l) : -INFINITY;
+                if (nsplit > 1)
+                    p.part_lse[(static_cast<int64_t>(split) * p.num_tokens + t) * p.num_q_heads + h] = lse2;
+                else
+                    p.lse_out[static_cast<int64_t>(t) * p.num_q_heads + h] = lse2 * kLn2;
             }
             if (all_ok) {
                 // O / l through shared memory (this q-tile's Q region: its last MMA has
@@ -655,6 +658,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
                     const float inv = W > 0.f ? 1.f / W : 0.f;
 #pragma unroll
                     for (int sp = 0; sp < kMaxFusedSplits; ++sp) wsm[tid * kMaxFusedSplits + sp] = w[sp] * inv;
+                    if (p.lse_out && Rr < rows_total)
+                        p.lse_out[row_of(Rr)] = W > 0.f ? (M + __log2f(W)) * kLn2 : -INFINITY;
                 }
                 named_barrier_sync(1, kQLoaders);
                 // phase 2: warp w merges rows w, w + 8, ..., lane l the 16 bytes at 4l of each

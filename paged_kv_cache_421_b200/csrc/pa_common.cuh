@@ -27,8 +27,9 @@ constexpr int kErrBadSlotMeta = 2;
 constexpr int kErrBadBlockId = 3;
 constexpr int kErrMetadata = 4;   // device metadata disagrees with the planned launch
 
-// A request is served by the decode kernel when all its query rows of one kv head fit one
-// 8-wide MMA tile, otherwise by the chunk kernel.  q_len == 0 requests produce nothing.
+// Kernels keep the softmax in the log2 domain; a row's exported log-sum-exp is natural log.
+constexpr float kLn2 = 0.69314718055994531f;
+
 // First key a query at position `limit` may see: 0; with a sliding window of `window` keys,
 // the last `window` positions up to its own; with chunked local attention of `local_chunk`
 // positions, the start of its own chunk; the later of the two when both are set.  It never
@@ -40,6 +41,8 @@ __host__ __device__ inline int first_visible_key(int limit, int window, int loca
     return lo;
 }
 
+// A request is served by the decode kernel when all its query rows of one kv head fit one
+// 8-wide MMA tile, otherwise by the chunk kernel.  q_len == 0 requests produce nothing.
 __host__ __device__ inline bool is_decode_kind(int q_len, int group) {
     return q_len > 0 && q_len * group <= kDecodeRows;
 }

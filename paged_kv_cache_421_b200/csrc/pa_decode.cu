@@ -84,9 +84,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
         ctx = p.max_blocks_per_seq * kBlockSize;
     }
     const int nblocks = ceil_div(ctx, kBlockSize);
-    // with a window or local chunks the splits cover only the blocks the first row may see
+    // with a window or local chunks the splits cover only the blocks the first row may see;
+    // a request with no key at all (an empty context-parallel share) keeps one CTA, which
+    // writes out = 0 and lse = -inf
     const int fb = first_visible_key(ctx - q_len, p.window, p.local_chunk) / kBlockSize;
-    const int nsplit = ceil_div(nblocks - fb, p.decode_split_blocks);
+    const int nsplit = max(1, ceil_div(nblocks - fb, p.decode_split_blocks));
     if (split >= nsplit) return;
     const int jb = fb + split * p.decode_split_blocks;
     const int je = min(nblocks, jb + p.decode_split_blocks);
@@ -465,6 +467,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
         const int h = g * p.group + n % p.group;
         if (direct) {
             p.out[(static_cast<int64_t>(t) * p.num_q_heads + h) * D + d] = val;
+            if (d == 0 && p.lse_out)
+                p.lse_out[static_cast<int64_t>(t) * p.num_q_heads + h] =
+                    L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
         } else {
             const int64_t prow = split * stride + static_cast<int64_t>(t) * p.num_q_heads + h;
             p.part_o[prow * D + d] = val;
@@ -500,7 +505,10 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) W += __shfl_xor_sync(kFull, W, off);
-        if (lane == 0) s_inv[n] = W > 0.f ? 1.f / W : 0.f;
+        if (lane == 0) {
+            s_inv[n] = W > 0.f ? 1.f / W : 0.f;
+            if (p.lse_out) p.lse_out[row] = W > 0.f ? (M + __log2f(W)) * kLn2 : -INFINITY;
+        }
     }
     __syncthreads();
     constexpr int kV4 = D / 4;

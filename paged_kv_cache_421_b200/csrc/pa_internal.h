@@ -71,6 +71,7 @@ struct AttnParams {
     int chunk_fused_merge;      // tcgen05 chunk kernel merges its own splits (<= kMaxFusedSplits)
     int window;                 // sliding window in keys, 0 = full causal attention
     int local_chunk;            // chunked local attention: chunk length in keys, 0 = off
+    float* lse_out;             // [T][Hq] natural-log LSE of every row, or null
 };
 
 // The chunk-kind requests of a launch, longest context first (passed by value, so the chunk
@@ -115,6 +116,13 @@ cudaError_t launch_slot_mapping(const int32_t* block_table, int max_blocks_per_s
 cudaError_t launch_write_kv(const pa_cache& c, const void* k, const void* v,
                             const int32_t* slot_mapping, int num_tokens, int* err,
                             cudaStream_t stream);
+cudaError_t launch_dcp_slot_mapping(const int32_t* block_table, int max_blocks_per_seq,
+                                    const int32_t* seq_lens, const int32_t* qsl, int num_seqs,
+                                    int num_tokens, int block_size, int rank, int world,
+                                    int32_t* slot_mapping, int* err, cudaStream_t stream);
+cudaError_t launch_merge_partials(const float* part_out, const float* part_lse, int num_parts,
+                                  int64_t num_rows, int head_size, float* out, float* lse_out,
+                                  cudaStream_t stream);
 cudaError_t launch_validate(const int32_t* block_table, int max_blocks_per_seq,
                             const int32_t* seq_lens, int num_seqs, int block_size,
                             int num_blocks, int* counter, cudaStream_t stream);

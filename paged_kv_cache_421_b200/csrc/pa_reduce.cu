@@ -70,6 +70,7 @@ __global__ void __launch_bounds__(128) reduce_kernel(const AttnParams p,
         for (int off = 16; off > 0; off >>= 1) W += __shfl_xor_sync(0xffffffffu, W, off);
     }
     const float inv = W > 0.f ? 1.f / W : 0.f;
+    if (lane == 0 && p.lse_out) p.lse_out[base] = W > 0.f ? (M + __log2f(W)) * kLn2 : -INFINITY;
     float* dst = p.out + base * D + lane * kVec;
     if constexpr (kVec == 4) {
         *reinterpret_cast<float4*>(dst) =

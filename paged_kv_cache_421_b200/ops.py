@@ -109,7 +109,7 @@ def write_kv(cache: PagedKVCache, k: torch.Tensor, v: torch.Tensor, slots: torch
 def workspace_bytes_for(cache: PagedKVCache, seq_lens_host, qsl_host, num_q_heads: int,
                         max_blocks_per_seq: int, kv_split_tokens: int = 0,
                         num_sms: Optional[int] = None, sliding_window: int = 0,
-                        local_chunk: int = 0) -> int:
+                        local_chunk: int = 0, with_lse: bool = False) -> int:
     if num_sms is None:
         num_sms = torch.cuda.get_device_properties(cache.buffer.device).multi_processor_count
     qs = np.asarray(qsl_host)
@@ -118,7 +118,8 @@ def workspace_bytes_for(cache: PagedKVCache, seq_lens_host, qsl_host, num_q_head
     plan = B.pa_plan_attention(seq_lens_host, qsl_host, num_q_heads, cache.num_kv_heads,
                                cache.head_size, max_blocks_per_seq, num_sms, unlimited,
                                kv_split_tokens=kv_split_tokens, block_size=cache.block_size,
-                               sliding_window=sliding_window, local_chunk=local_chunk)
+                               sliding_window=sliding_window, local_chunk=local_chunk,
+                               with_lse=with_lse)
     return int(plan["workspace_needed"])
 
 
@@ -126,17 +127,24 @@ def attention(cache: PagedKVCache, q: torch.Tensor, block_table: torch.Tensor,
               seq_lens: torch.Tensor, qsl: torch.Tensor, seq_lens_host, qsl_host, scale: float,
               out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
               kv_split_tokens: int = 0, events=None, sliding_window: int = 0,
-              local_chunk: int = 0, stream=None) -> torch.Tensor:
+              local_chunk: int = 0, lse_out: Optional[torch.Tensor] = None,
+              stream=None) -> torch.Tensor:
+    """Paged attention of one step; with ``lse_out`` (fp32 [T][Hq]) each row's natural-log
+    log-sum-exp is written too, and decode-kind requests may hold no key (0 and -inf)."""
     T, Hq, D = q.shape
     if out is None:
         out = torch.empty(T, Hq, D, dtype=torch.float32, device=q.device)
+    if lse_out is not None:
+        assert lse_out.dtype == torch.float32 and lse_out.is_contiguous()
+        assert lse_out.numel() == T * Hq
     if workspace is None:
         nb = workspace_bytes_for(cache, seq_lens_host, qsl_host, Hq, block_table.shape[1],
                                  kv_split_tokens, sliding_window=sliding_window,
-                                 local_chunk=local_chunk)
+                                 local_chunk=local_chunk, with_lse=lse_out is not None)
         workspace = torch.empty(max(nb, 1), dtype=torch.uint8, device=q.device)
     B.pa_attention_ex(cache.handle, q, Hq, block_table, block_table.shape[1], seq_lens, qsl,
                       seq_lens_host, qsl_host, seq_lens.numel(), T, scale, out, workspace,
                       workspace.numel(), kv_split_tokens=kv_split_tokens, events=events,
-                      sliding_window=sliding_window, local_chunk=local_chunk, stream=stream)
+                      sliding_window=sliding_window, local_chunk=local_chunk, lse_out=lse_out,
+                      stream=stream)
     return out
