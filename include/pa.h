@@ -214,10 +214,12 @@ typedef struct {
     int decode_max_splits;    /* largest split count among decode-kind requests */
     int chunk_split_blocks;   /* blocks per KV split for chunk-kind requests */
     int chunk_max_splits;
-    int chunk_max_qtiles;     /* largest number of 64-row query tiles of one (request, kv head) */
+    int chunk_max_qtiles;     /* largest number of query tiles of one (request, kv head): 256
+                                 rows per tile for the tcgen05 kernel (bf16, head_size 128),
+                                 64 rows for the head_size-64 kernel */
     int64_t decode_ctas;      /* CTAs that do work in the decode kernel */
     int64_t chunk_ctas;       /* CTAs that do work in the chunk kernel */
-    int any_split;            /* a reduce launch is needed */
+    int any_split;            /* some request is split: partials go through the workspace */
     size_t workspace_needed;  /* bytes of workspace this plan uses */
     int reduce_rows_max;      /* largest q_len * group among split chunk-kind requests */
 } pa_plan;
