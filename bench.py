@@ -112,6 +112,18 @@ def chunk_flops(wl, window: int = 0, local_chunk: int = 0) -> int:
     return total * wl.num_q_heads * 4 * wl.head_size
 
 
+def launches_for_plan(plan: dict, head_size: int) -> int:
+    """Kernels of ours per step, as pa_attention launches them: slot mapping and write, the
+    split-counter clear (split decode requests, or chunk splits the tcgen05 kernel merges
+    itself: head_size 128 and at most 4 splits), the decode and/or chunk kernel, and the split
+    reduce (chunk splits not merged in the chunk kernel)."""
+    fused = head_size == 128 and plan["chunk_max_splits"] <= 4
+    clear = plan["decode_max_splits"] > 1 or (plan["chunk_max_splits"] > 1 and fused)
+    reduce = plan["chunk_max_splits"] > 1 and not fused
+    return 2 + int(clear) + int(plan["num_decode_seqs"] > 0) + int(plan["num_chunk_seqs"] > 0) + \
+        int(reduce)
+
+
 def unique_kv_bytes(wl) -> int:
     used = set()
     for r in range(wl.num_seqs):
@@ -360,11 +372,7 @@ class DeviceStep:
         torch.cuda.synchronize(device)
 
     def launches_per_step(self) -> int:
-        """Kernels of ours per step: slot mapping, write, the split-counter clear (split
-        decode), decode and/or chunk, chunk reduce."""
-        p = self.plan
-        return 2 + int(p["decode_max_splits"] > 1) + (p["num_decode_seqs"] > 0) + \
-            (p["num_chunk_seqs"] > 0) + int(p["chunk_max_splits"] > 1)
+        return launches_for_plan(self.plan, self.wl.head_size)
 
     def run(self, events=None, q=None, k=None, v=None, bt=None, sl=None, qsl=None, out=None):
         B = self.ops.B

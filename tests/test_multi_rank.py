@@ -132,3 +132,21 @@ def test_bench_local_chunk_accounting():
     assert bench.kv_bytes(wl, 0, int(wl.seq_lens.max()) + 1) == bench.kv_bytes(wl)
     assert bench.chunk_flops(wl, 0, int(wl.seq_lens.max()) + 1) == bench.chunk_flops(wl)
     assert bench.parse_args(["--local-chunk", "8192"]).local_chunk == 8192
+
+
+def test_bench_launch_count_follows_the_launch_sequence():
+    """gpu_launches counts what pa_attention launches: the counter clear for split decodes
+    and for chunk splits merged inside the tcgen05 kernel (<= 4), the reduce otherwise."""
+    sys.path.insert(0, ROOT)
+    import bench
+
+    def plan(dec, chunk, ds, cs):
+        return {"num_decode_seqs": dec, "num_chunk_seqs": chunk, "decode_max_splits": ds,
+                "chunk_max_splits": cs}
+    assert bench.launches_for_plan(plan(4, 0, 1, 0), 128) == 3      # slots, write, decode
+    assert bench.launches_for_plan(plan(4, 0, 3, 0), 128) == 4      # + counter clear
+    assert bench.launches_for_plan(plan(4, 2, 1, 1), 128) == 4      # decode + chunk
+    assert bench.launches_for_plan(plan(0, 2, 0, 3), 128) == 4      # fused merge: clear
+    assert bench.launches_for_plan(plan(0, 2, 0, 9), 128) == 4      # reduce, no clear
+    assert bench.launches_for_plan(plan(4, 2, 5, 9), 128) == 6      # everything
+    assert bench.launches_for_plan(plan(0, 2, 0, 3), 64) == 4       # head_size 64: reduce
