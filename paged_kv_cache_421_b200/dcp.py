@@ -102,15 +102,15 @@ def merge(parts_out: torch.Tensor, parts_lse: torch.Tensor, out: Optional[torch.
 
 
 def attention(cache: ops.PagedKVCache, q: torch.Tensor, local_block_table: torch.Tensor,
-              seq_lens_host, qsl: torch.Tensor, qsl_host, scale: float, group=None,
-              stream=None) -> torch.Tensor:
+              seq_lens_host, qsl: torch.Tensor, qsl_host, scale: float,
+              group=None) -> torch.Tensor:
     """One decode step's attention over the whole context, this rank holding its share in
     `cache` (its local table in `local_block_table`); seq_lens_host are the requests' total
-    lengths.  Every rank of `group` calls this with the same queries and gets the result."""
+    lengths.  Every rank of `group` calls this with the same queries and gets the result.
+    Kernels run on torch's current stream, which NCCL orders the all-gather against."""
     rank, world = dist.get_rank(group), dist.get_world_size(group)
     loc = local_seq_lens(seq_lens_host, rank, world, cache.block_size)
-    loc_dev = torch.from_numpy(loc).to(q.device, non_blocking=False)
-    out, lse = partial_attention(cache, q, local_block_table, loc_dev, qsl, loc, qsl_host, scale,
-                                 stream=stream)
+    loc_dev = torch.from_numpy(loc).to(q.device)
+    out, lse = partial_attention(cache, q, local_block_table, loc_dev, qsl, loc, qsl_host, scale)
     parts_out, parts_lse = exchange(out, lse, group)
-    return merge(parts_out, parts_lse, stream=stream)
+    return merge(parts_out, parts_lse)
