@@ -45,7 +45,7 @@ extern "C" {
 typedef enum {
     PA_OK = 0,
     PA_ERR_INVALID_ARG = 1,   /* null pointer, non-positive size, inconsistent shapes */
-    PA_ERR_UNSUPPORTED = 2,   /* a valid configuration this build has no kernel for */
+    PA_ERR_UNSUPPORTED = 2,   /* a valid configuration the library has no kernel for */
     PA_ERR_OOM = 3,           /* device allocation failed */
     PA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed; see pa_last_cuda_error */
     PA_ERR_WORKSPACE = 5,     /* workspace smaller than the plan needs */
