@@ -250,7 +250,9 @@ typedef struct {
 } pa_attention_opts;
 
 /* The planner alone: fills *plan for the given host metadata without touching the GPU.
- * num_sms must be > 0.  Errors: INVALID_ARG, METADATA, UNSUPPORTED. */
+ * num_sms must be > 0.  It reads opts->lse_out only as a flag (non-NULL: plan a call that
+ * exports LSEs, which admits empty decode shares) and never dereferences it.
+ * Errors: INVALID_ARG, METADATA, UNSUPPORTED. */
 int pa_plan_attention(const int32_t* seq_lens_host, const int32_t* query_start_loc_host,
                       int num_seqs, int num_tokens, int num_q_heads, int num_kv_heads,
                       int head_size, int block_size, int max_blocks_per_seq, int num_sms,
