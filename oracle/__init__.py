@@ -32,35 +32,44 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "pa_oracle.c")
 _OUT_DIR = os.path.join(_HERE, "_build")
 _LIB_PATH = os.path.join(_OUT_DIR, "liboracle.so")
+# the same source built with OpenMP: independent (request, kv head) units and selected rows
+# run on several threads, each with the arithmetic of the plain build
+_OMP_LIB_PATH = os.path.join(_OUT_DIR, "liboracle_omp.so")
 
 BF16 = 0
 FP8_E4M3 = 1
 
 _lib = None
+_omp_lib = None
+
+_CFLAGS = ["-O2", "-std=c99", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math",
+           "-Wall", "-Wextra"]
+
+
+def _compile(path: str, extra: list, force: bool) -> str:
+    if (not force and os.path.exists(path)
+            and os.path.getmtime(path) >= os.path.getmtime(_SRC)):
+        return path
+    tmp = path + f".tmp{os.getpid()}"
+    subprocess.check_call(["gcc", *_CFLAGS, *extra, "-o", tmp, _SRC, "-lm"])
+    os.replace(tmp, path)
+    return path
 
 
 def build(force: bool = False) -> str:
     """Compile pa_oracle.c into a shared library (gcc, strict IEEE: no fast-math, no FMA
-    contraction, so the fp32 divide of the FP8 path is a correctly rounded divide)."""
+    contraction, so the fp32 divide of the FP8 path is a correctly rounded divide), and the
+    same source once more with OpenMP (liboracle_omp.so)."""
     os.makedirs(_OUT_DIR, exist_ok=True)
-    if (not force and os.path.exists(_LIB_PATH)
-            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
-        return _LIB_PATH
-    tmp = _LIB_PATH + f".tmp{os.getpid()}"
-    subprocess.check_call([
-        "gcc", "-O2", "-std=c99", "-fPIC", "-shared", "-ffp-contract=off",
-        "-fno-fast-math", "-Wall", "-Wextra", "-o", tmp, _SRC, "-lm"])
-    os.replace(tmp, _LIB_PATH)
-    return _LIB_PATH
+    _compile(_OMP_LIB_PATH, ["-fopenmp"], force)
+    return _compile(_LIB_PATH, ["-Wno-unknown-pragmas"], force)
 
 
-def _load():
-    global _lib
-    if _lib is not None:
-        return _lib
-    lib = ctypes.CDLL(build())
+def _declare(lib):
     P = ctypes.c_void_p
     i32, i64, f64, u8 = ctypes.c_int, ctypes.c_int64, ctypes.c_double, ctypes.c_uint8
+    lib.oracle_set_threads.restype = i32
+    lib.oracle_set_threads.argtypes = [i32]
     lib.oracle_cache_elems.restype = i64
     lib.oracle_cache_elems.argtypes = [i32, i32, i32, i32]
     lib.oracle_block_bytes.restype = i64
@@ -97,8 +106,42 @@ def _load():
     lib.oracle_attention_rows.restype = i32
     lib.oracle_attention_rows.argtypes = [P, P, i32, i32, P, P, i32, P, P, P, i32, P, P, i32,
                                           f64, i32, i32, P, P, i32, P, P]
-    _lib = lib
     return lib
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        _lib = _declare(ctypes.CDLL(build()))
+    return _lib
+
+
+def _load_omp():
+    global _omp_lib
+    if _omp_lib is None:
+        build()
+        _omp_lib = _declare(ctypes.CDLL(_OMP_LIB_PATH))
+    return _omp_lib
+
+
+def host_cores() -> int:
+    """Host cores this process may run on."""
+    return len(os.sched_getaffinity(0))
+
+
+def _attention_lib(threads):
+    """The plain (single-threaded) oracle for threads None or 1, else the OpenMP build set to
+    that many threads (0: every host core this process may use)."""
+    if threads is None or threads == 1:
+        return _load()
+    lib = _load_omp()
+    lib.oracle_set_threads(host_cores() if threads == 0 else int(threads))
+    return lib
+
+
+def threads_in_use(threads) -> int:
+    """Threads an attention call with this `threads` argument runs on."""
+    return int(_attention_lib(threads).oracle_set_threads(0))
 
 
 def _c(a: np.ndarray, dtype) -> np.ndarray:
@@ -212,10 +255,12 @@ def attention_paged(cache: np.ndarray, kv_dtype: int, num_blocks: int, block_siz
                     num_kv_heads: int, head_size: int, q_bits: np.ndarray, num_q_heads: int,
                     block_table: np.ndarray, seq_lens: np.ndarray, qsl: np.ndarray,
                     scale: float, k_scale=None, v_scale=None, window: int = 0,
-                    local_chunk: int = 0):
+                    local_chunk: int = 0, threads=None):
     """Exact attention over the paged cache.  Returns (out [T][Hq][D], lse [T][Hq]) fp64.
     window > 0: a query at position p sees keys max(0, p - window + 1) .. p;
-    local_chunk > 0: only keys floor(p / local_chunk) * local_chunk .. p."""
+    local_chunk > 0: only keys floor(p / local_chunk) * local_chunk .. p.
+    threads: None / 1 single-threaded; n > 1 (0 = all host cores) the OpenMP build, which
+    returns the same bits."""
     q = _c(q_bits, np.uint16)
     bt = _c(block_table, np.int32)
     sl = _c(seq_lens, np.int32)
@@ -225,7 +270,7 @@ def attention_paged(cache: np.ndarray, kv_dtype: int, num_blocks: int, block_siz
     lse = np.zeros((T, num_q_heads), np.float64)
     ks = None if k_scale is None else _c(k_scale, np.float32)
     vs = None if v_scale is None else _c(v_scale, np.float32)
-    _check(_load().oracle_attention_paged(
+    _check(_attention_lib(threads).oracle_attention_paged(
         _p(cache), kv_dtype, num_blocks, block_size, num_kv_heads, head_size, _p(ks), _p(vs),
         _p(q), num_q_heads, _p(bt), bt.shape[1], _p(sl), _p(qs), sl.size, float(scale),
         int(window), int(local_chunk), _p(out), _p(lse)), "oracle_attention_paged")
@@ -236,11 +281,12 @@ def attention_rows(k_src: np.ndarray, v_src: np.ndarray, pos_rows: np.ndarray,
                    pos_start: np.ndarray, kv_dtype: int, q_bits: np.ndarray,
                    seq_lens: np.ndarray, qsl: np.ndarray, scale: float,
                    sel_tokens: np.ndarray, sel_heads: np.ndarray, k_scale=None, v_scale=None,
-                   window: int = 0, local_chunk: int = 0):
+                   window: int = 0, local_chunk: int = 0, threads=None):
     """Unpaged exact attention for selected (token, q head) rows.
 
     k_src, v_src: uint16 bf16 bits [rows][Hkv][D]; request r's position p reads source row
-    pos_rows[pos_start[r] + p].  Returns (out [nsel][D], lse [nsel]) in fp64."""
+    pos_rows[pos_start[r] + p].  Returns (out [nsel][D], lse [nsel]) in fp64.
+    threads: as for attention_paged."""
     k = _c(k_src, np.uint16)
     v = _c(v_src, np.uint16)
     num_kv_heads, head_size = k.shape[1], k.shape[2]
@@ -256,7 +302,7 @@ def attention_rows(k_src: np.ndarray, v_src: np.ndarray, pos_rows: np.ndarray,
     lse = np.zeros(st.size, np.float64)
     ks = None if k_scale is None else _c(k_scale, np.float32)
     vs = None if v_scale is None else _c(v_scale, np.float32)
-    _check(_load().oracle_attention_rows(
+    _check(_attention_lib(threads).oracle_attention_rows(
         _p(k), _p(v), num_kv_heads, head_size, _p(pr), _p(ps), kv_dtype, _p(ks), _p(vs),
         _p(q), num_q_heads, _p(sl), _p(qs), sl.size, float(scale), int(window),
         int(local_chunk), _p(st), _p(sh),

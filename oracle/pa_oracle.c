@@ -32,9 +32,24 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 enum { OR_OK = 0, OR_BAD_META = 6, OR_NOMEM = 3, OR_BAD_ARG = 1 };
 enum { OR_BF16 = 0, OR_FP8_E4M3 = 1 };
+
+/* Threads an OpenMP build of this file runs independent attention units on (n > 0 sets it);
+ * returns the count in force.  A plain build has no threads and returns 1. */
+int oracle_set_threads(int n) {
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+    return omp_get_max_threads();
+#else
+    (void)n;
+    return 1;
+#endif
+}
 
 /* ------------------------------------------------------------------ layout */
 /* Element (token tok, dim d) of the K (kv = 0) or V (kv = 1) tile of (block, head).  Tiles
@@ -308,10 +323,72 @@ static double cache_value(const void* cache, int kv_dtype, int64_t idx, double s
     return oracle_e4m3_decode(((const uint8_t*)cache)[idx]) * scale;
 }
 
+/* One (request r, kv head g) unit of paged attention: gather the request's keys and values of
+ * head g through its block table into contiguous fp64 arrays, then attend every query row of
+ * the group.  Units share nothing but read-only inputs and disjoint output rows. */
+static int attend_unit(const void* cache, int kv_dtype, int num_blocks, int block_size,
+                       int num_kv_heads, int head_size, const float* k_scale,
+                       const float* v_scale, const uint16_t* q, int num_q_heads,
+                       const int32_t* block_table, int max_blocks_per_seq,
+                       const int32_t* seq_lens, const int32_t* qsl, double scale, int window,
+                       int local_chunk, int r, int g, double* out, double* lse) {
+    int i, hh, d, p;
+    int group = num_q_heads / num_kv_heads;
+    int q_len = qsl[r + 1] - qsl[r];
+    int ctx = seq_lens[r];
+    double ks = k_scale ? (double)k_scale[g] : 1.0;
+    double vs = v_scale ? (double)v_scale[g] : 1.0;
+    double *K, *V, *s, *qrow;
+    if (q_len == 0) return OR_OK;
+    if (q_len < 0 || ctx < q_len || ctx <= 0) return OR_BAD_META;
+    if ((ctx - 1) / block_size >= max_blocks_per_seq) return OR_BAD_META;
+    K = (double*)malloc(sizeof(double) * (size_t)ctx * head_size);
+    V = (double*)malloc(sizeof(double) * (size_t)ctx * head_size);
+    s = (double*)malloc(sizeof(double) * (size_t)ctx);
+    qrow = (double*)malloc(sizeof(double) * (size_t)head_size);
+    if (!K || !V || !s || !qrow) {
+        free(K); free(V); free(s); free(qrow);
+        return OR_NOMEM;
+    }
+    /* gather this request's keys and values through its block table */
+    for (p = 0; p < ctx; ++p) {
+        int64_t b = block_table[(int64_t)r * max_blocks_per_seq + p / block_size];
+        int o = p % block_size;
+        if (b < 0 || b >= num_blocks) {
+            free(K); free(V); free(s); free(qrow);
+            return OR_BAD_META;
+        }
+        for (d = 0; d < head_size; ++d) {
+            K[(int64_t)p * head_size + d] = cache_value(
+                cache, kv_dtype,
+                elem_index_dt(b, 0, g, o, d, num_kv_heads, block_size, head_size, kv_dtype), ks);
+            V[(int64_t)p * head_size + d] = cache_value(
+                cache, kv_dtype,
+                elem_index_dt(b, 1, g, o, d, num_kv_heads, block_size, head_size, kv_dtype), vs);
+        }
+    }
+    for (i = 0; i < q_len; ++i) {
+        int t = qsl[r] + i;
+        int limit = ctx - q_len + i; /* last key this query may see */
+        for (hh = 0; hh < group; ++hh) {
+            int h = g * group + hh;
+            int64_t row = (int64_t)t * num_q_heads + h;
+            for (d = 0; d < head_size; ++d)
+                qrow[d] = oracle_bf16_to_double(q[row * head_size + d]);
+            lse[row] = attend_row(qrow, K, V, first_key(limit, window, local_chunk), limit,
+                                  head_size, scale, s, out + row * head_size);
+        }
+    }
+    free(K); free(V); free(s); free(qrow);
+    return OR_OK;
+}
+
 /* Paged attention over the cache.
  * q: bf16 [num_tokens][num_q_heads][head_size]; block_table int32 [num_seqs][max_blocks];
  * seq_lens [num_seqs]; qsl [num_seqs + 1].  Query head h reads kv head h / (Hq / Hkv).
- * out: fp64 [num_tokens][num_q_heads][head_size]; lse: fp64 [num_tokens][num_q_heads]. */
+ * out: fp64 [num_tokens][num_q_heads][head_size]; lse: fp64 [num_tokens][num_q_heads].
+ * The (request, kv head) units are independent; a build with OpenMP runs them on several
+ * threads, each unit's arithmetic unchanged, so every thread count gives the same bits. */
 int oracle_attention_paged(const void* cache, int kv_dtype, int num_blocks, int block_size,
                            int num_kv_heads, int head_size, const float* k_scale,
                            const float* v_scale, const uint16_t* q, int num_q_heads,
@@ -319,61 +396,68 @@ int oracle_attention_paged(const void* cache, int kv_dtype, int num_blocks, int 
                            const int32_t* seq_lens, const int32_t* qsl, int num_seqs,
                            double scale, int window, int local_chunk, double* out,
                            double* lse) {
-    int r, g, i, hh, d, p;
-    int group = num_q_heads / num_kv_heads;
-    if (group * num_kv_heads != num_q_heads) return OR_BAD_ARG;
-    for (r = 0; r < num_seqs; ++r) {
-        int q_len = qsl[r + 1] - qsl[r];
-        int ctx = seq_lens[r];
-        double *K, *V, *s, *qrow;
-        if (q_len == 0) continue;
-        if (q_len < 0 || ctx < q_len || ctx <= 0) return OR_BAD_META;
-        if ((ctx - 1) / block_size >= max_blocks_per_seq) return OR_BAD_META;
-        K = (double*)malloc(sizeof(double) * (size_t)ctx * head_size);
-        V = (double*)malloc(sizeof(double) * (size_t)ctx * head_size);
-        s = (double*)malloc(sizeof(double) * (size_t)ctx);
-        qrow = (double*)malloc(sizeof(double) * (size_t)head_size);
-        if (!K || !V || !s || !qrow) {
-            free(K); free(V); free(s); free(qrow);
-            return OR_NOMEM;
+    int64_t u, units = (int64_t)num_seqs * num_kv_heads;
+    int status = OR_OK;
+    if (num_kv_heads <= 0 || (num_q_heads / num_kv_heads) * num_kv_heads != num_q_heads)
+        return OR_BAD_ARG;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (u = 0; u < units; ++u) {
+        int rc = attend_unit(cache, kv_dtype, num_blocks, block_size, num_kv_heads, head_size,
+                             k_scale, v_scale, q, num_q_heads, block_table, max_blocks_per_seq,
+                             seq_lens, qsl, scale, window, local_chunk,
+                             (int)(u / num_kv_heads), (int)(u % num_kv_heads), out, lse);
+        if (rc != OR_OK) {
+#pragma omp critical
+            if (status == OR_OK) status = rc;
         }
-        for (g = 0; g < num_kv_heads; ++g) {
-            double ks = k_scale ? (double)k_scale[g] : 1.0;
-            double vs = v_scale ? (double)v_scale[g] : 1.0;
-            /* gather this request's keys and values through its block table */
-            for (p = 0; p < ctx; ++p) {
-                int64_t b = block_table[(int64_t)r * max_blocks_per_seq + p / block_size];
-                int o = p % block_size;
-                if (b < 0 || b >= num_blocks) {
-                    free(K); free(V); free(s); free(qrow);
-                    return OR_BAD_META;
-                }
-                for (d = 0; d < head_size; ++d) {
-                    K[(int64_t)p * head_size + d] = cache_value(
-                        cache, kv_dtype,
-                        elem_index_dt(b, 0, g, o, d, num_kv_heads, block_size, head_size,
-                                      kv_dtype), ks);
-                    V[(int64_t)p * head_size + d] = cache_value(
-                        cache, kv_dtype,
-                        elem_index_dt(b, 1, g, o, d, num_kv_heads, block_size, head_size,
-                                      kv_dtype), vs);
-                }
-            }
-            for (i = 0; i < q_len; ++i) {
-                int t = qsl[r] + i;
-                int limit = ctx - q_len + i; /* last key this query may see */
-                for (hh = 0; hh < group; ++hh) {
-                    int h = g * group + hh;
-                    int64_t row = (int64_t)t * num_q_heads + h;
-                    for (d = 0; d < head_size; ++d)
-                        qrow[d] = oracle_bf16_to_double(q[row * head_size + d]);
-                    lse[row] = attend_row(qrow, K, V, first_key(limit, window, local_chunk), limit,
-                                          head_size, scale, s, out + row * head_size);
-                }
-            }
-        }
-        free(K); free(V); free(s); free(qrow);
     }
+    return status;
+}
+
+/* One selected row of oracle_attention_rows (see there). */
+static int attend_selected_row(const uint16_t* k_src, const uint16_t* v_src, int num_kv_heads,
+                               int head_size, const int64_t* pos_rows, const int64_t* pos_start,
+                               int kv_dtype, const float* k_scale, const float* v_scale,
+                               const uint16_t* q, int num_q_heads, const int32_t* seq_lens,
+                               const int32_t* qsl, int num_seqs, double scale, int window,
+                               int local_chunk, int t, int h, double* out, double* lse) {
+    int r, d, p, g, q_len, ctx, limit;
+    int group = num_q_heads / num_kv_heads;
+    double *K, *V, *s, *qrow;
+    for (r = 0; r < num_seqs; ++r)
+        if (qsl[r] <= t && t < qsl[r + 1]) break;
+    if (r == num_seqs || h < 0 || h >= num_q_heads) return OR_BAD_ARG;
+    g = h / group;
+    q_len = qsl[r + 1] - qsl[r];
+    ctx = seq_lens[r];
+    if (ctx < q_len) return OR_BAD_META;
+    limit = ctx - q_len + (t - qsl[r]);
+    K = (double*)malloc(sizeof(double) * (size_t)(limit + 1) * head_size);
+    V = (double*)malloc(sizeof(double) * (size_t)(limit + 1) * head_size);
+    s = (double*)malloc(sizeof(double) * (size_t)(limit + 1));
+    qrow = (double*)malloc(sizeof(double) * (size_t)head_size);
+    if (!K || !V || !s || !qrow) {
+        free(K); free(V); free(s); free(qrow);
+        return OR_NOMEM;
+    }
+    for (p = 0; p <= limit; ++p) {
+        int64_t src_row = pos_rows[pos_start[r] + p];
+        for (d = 0; d < head_size; ++d) {
+            int64_t idx = (src_row * num_kv_heads + g) * head_size + d;
+            if (kv_dtype == OR_BF16) {
+                K[(int64_t)p * head_size + d] = oracle_bf16_to_double(k_src[idx]);
+                V[(int64_t)p * head_size + d] = oracle_bf16_to_double(v_src[idx]);
+            } else {
+                K[(int64_t)p * head_size + d] = fp8_roundtrip(k_src[idx], k_scale[g]);
+                V[(int64_t)p * head_size + d] = fp8_roundtrip(v_src[idx], v_scale[g]);
+            }
+        }
+    }
+    for (d = 0; d < head_size; ++d)
+        qrow[d] = oracle_bf16_to_double(q[((int64_t)t * num_q_heads + h) * head_size + d]);
+    *lse = attend_row(qrow, K, V, first_key(limit, window, local_chunk), limit, head_size, scale,
+                      s, out);
+    free(K); free(V); free(s); free(qrow);
     return OR_OK;
 }
 
@@ -381,7 +465,8 @@ int oracle_attention_paged(const void* cache, int kv_dtype, int num_blocks, int 
  * k_src, v_src: bf16 [rows][num_kv_heads][head_size]; request r's position p reads source
  * row pos_rows[pos_start[r] + p].  With kv_dtype == FP8 every K/V value is taken through the
  * FP8 round trip (fp32 divide, encode, decode, times scale), i.e. what an FP8 cache holds.
- * Selected (token, q head) pairs: sel_tokens[j], sel_heads[j]; out [nsel][head_size]. */
+ * Selected (token, q head) pairs: sel_tokens[j], sel_heads[j]; out [nsel][head_size].
+ * Rows are independent; an OpenMP build runs them on several threads with the same bits. */
 int oracle_attention_rows(const uint16_t* k_src, const uint16_t* v_src, int num_kv_heads,
                           int head_size, const int64_t* pos_rows, const int64_t* pos_start,
                           int kv_dtype, const float* k_scale, const float* v_scale,
@@ -390,49 +475,21 @@ int oracle_attention_rows(const uint16_t* k_src, const uint16_t* v_src, int num_
                           int local_chunk,
                           const int32_t* sel_tokens, const int32_t* sel_heads, int nsel,
                           double* out, double* lse) {
-    int j, r, d, p;
-    int group = num_q_heads / num_kv_heads;
-    if (group * num_kv_heads != num_q_heads) return OR_BAD_ARG;
+    int j, status = OR_OK;
+    if (num_kv_heads <= 0 || (num_q_heads / num_kv_heads) * num_kv_heads != num_q_heads)
+        return OR_BAD_ARG;
+#pragma omp parallel for schedule(dynamic, 1)
     for (j = 0; j < nsel; ++j) {
-        int t = sel_tokens[j], h = sel_heads[j], g, q_len, ctx, limit;
-        double *K, *V, *s, *qrow;
-        for (r = 0; r < num_seqs; ++r)
-            if (qsl[r] <= t && t < qsl[r + 1]) break;
-        if (r == num_seqs || h < 0 || h >= num_q_heads) return OR_BAD_ARG;
-        g = h / group;
-        q_len = qsl[r + 1] - qsl[r];
-        ctx = seq_lens[r];
-        if (ctx < q_len) return OR_BAD_META;
-        limit = ctx - q_len + (t - qsl[r]);
-        K = (double*)malloc(sizeof(double) * (size_t)(limit + 1) * head_size);
-        V = (double*)malloc(sizeof(double) * (size_t)(limit + 1) * head_size);
-        s = (double*)malloc(sizeof(double) * (size_t)(limit + 1));
-        qrow = (double*)malloc(sizeof(double) * (size_t)head_size);
-        if (!K || !V || !s || !qrow) {
-            free(K); free(V); free(s); free(qrow);
-            return OR_NOMEM;
+        int rc = attend_selected_row(k_src, v_src, num_kv_heads, head_size, pos_rows, pos_start,
+                                     kv_dtype, k_scale, v_scale, q, num_q_heads, seq_lens, qsl,
+                                     num_seqs, scale, window, local_chunk, sel_tokens[j],
+                                     sel_heads[j], out + (int64_t)j * head_size, lse + j);
+        if (rc != OR_OK) {
+#pragma omp critical
+            if (status == OR_OK) status = rc;
         }
-        for (p = 0; p <= limit; ++p) {
-            int64_t src_row = pos_rows[pos_start[r] + p];
-            for (d = 0; d < head_size; ++d) {
-                int64_t idx = (src_row * num_kv_heads + g) * head_size + d;
-                if (kv_dtype == OR_BF16) {
-                    K[(int64_t)p * head_size + d] = oracle_bf16_to_double(k_src[idx]);
-                    V[(int64_t)p * head_size + d] = oracle_bf16_to_double(v_src[idx]);
-                } else {
-                    K[(int64_t)p * head_size + d] = fp8_roundtrip(k_src[idx], k_scale[g]);
-                    V[(int64_t)p * head_size + d] = fp8_roundtrip(v_src[idx], v_scale[g]);
-                }
-            }
-        }
-        for (d = 0; d < head_size; ++d)
-            qrow[d] = oracle_bf16_to_double(q[((int64_t)t * num_q_heads + h) * head_size + d]);
-        lse[j] = attend_row(qrow, K, V, first_key(limit, window, local_chunk), limit, head_size,
-                            scale, s,
-                            out + (int64_t)j * head_size);
-        free(K); free(V); free(s); free(qrow);
     }
-    return OR_OK;
+    return status;
 }
 
 /* ------------------------------------------------------------------ context parallelism */
