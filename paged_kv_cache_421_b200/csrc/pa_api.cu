@@ -4,6 +4,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <algorithm>
+#include <atomic>
 #include <vector>
 #include <new>
 
@@ -17,8 +18,9 @@ thread_local int g_last_cuda_error = 0;
 __device__ int g_device_error_word = 0;
 
 constexpr int kMaxDevices = 64;
-int* g_err_ptr[kMaxDevices] = {nullptr};
-int g_num_sms[kMaxDevices] = {0};
+// Per-device values resolved once; host threads racing on the first call store the same value.
+std::atomic<int*> g_err_ptr[kMaxDevices];
+std::atomic<int> g_num_sms[kMaxDevices];
 
 int fail_cuda(cudaError_t e) {
     g_last_cuda_error = static_cast<int>(e);
@@ -35,23 +37,28 @@ int current_device() {
 int* device_error_ptr() {
     const int dev = current_device();
     if (dev < 0 || dev >= kMaxDevices) return nullptr;
-    if (!g_err_ptr[dev]) {
+    int* ptr = g_err_ptr[dev].load(std::memory_order_acquire);
+    if (!ptr) {
         void* p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_device_error_word) != cudaSuccess) return nullptr;
-        g_err_ptr[dev] = static_cast<int*>(p);
+        if (cudaGetSymbolAddress(&p, g_device_error_word) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        ptr = static_cast<int*>(p);
+        g_err_ptr[dev].store(ptr, std::memory_order_release);
     }
-    return g_err_ptr[dev];
+    return ptr;
 }
 
 int device_num_sms() {
     const int dev = current_device();
     if (dev < 0 || dev >= kMaxDevices) return 0;
-    if (!g_num_sms[dev]) {
-        int n = 0;
+    int n = g_num_sms[dev].load(std::memory_order_relaxed);
+    if (!n) {
         if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
-        g_num_sms[dev] = n;
+        g_num_sms[dev].store(n, std::memory_order_relaxed);
     }
-    return g_num_sms[dev];
+    return n;
 }
 
 int dtype_bytes(int kv_dtype) { return kv_dtype == PA_BF16 ? 2 : (kv_dtype == PA_FP8_E4M3 ? 1 : 0); }
@@ -632,6 +639,37 @@ int pa_validate_block_table(const pa_cache* cache, const int32_t* block_table,
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     cudaFreeAsync(counter, s);
     return e == cudaSuccess ? PA_OK : fail_cuda(e);
+}
+
+int pa_validate_slots(const pa_cache* cache, const int32_t* slot_mapping, int num_tokens,
+                      int* num_out_of_pool, int* num_duplicates, void* stream) {
+    if (!cache || !num_out_of_pool || !num_duplicates || num_tokens < 0) return PA_ERR_INVALID_ARG;
+    *num_out_of_pool = 0;
+    *num_duplicates = 0;
+    if (num_tokens == 0) return PA_OK;
+    if (!slot_mapping) return PA_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const int64_t num_slots = static_cast<int64_t>(cache->num_blocks) * cache->block_size;
+    const size_t words = static_cast<size_t>((num_slots + 31) / 32);
+    // one allocation: two counters, then the bitmap of the pool's slots
+    const size_t bytes = 256 + words * sizeof(uint32_t);
+    char* buf = nullptr;
+    cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&buf), bytes, s);
+    if (e != cudaSuccess) return fail_cuda(e);
+    int* counts = reinterpret_cast<int*>(buf);
+    int host_counts[2] = {0, 0};
+    e = cudaMemsetAsync(buf, 0, bytes, s);
+    if (e == cudaSuccess)
+        e = pa::launch_validate_slots(slot_mapping, num_tokens, num_slots,
+                                      reinterpret_cast<uint32_t*>(buf + 256), counts, s);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(host_counts, counts, sizeof(host_counts), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    cudaFreeAsync(buf, s);
+    if (e != cudaSuccess) return fail_cuda(e);
+    *num_out_of_pool = host_counts[0];
+    *num_duplicates = host_counts[1];
+    return PA_OK;
 }
 
 int pa_dcp_local_seq_lens(const int32_t* seq_lens_host, int num_seqs, int block_size,

@@ -13,6 +13,8 @@
 // is resolved with cudaGetSymbolAddress the first time the entry point runs on a device, with
 // that device current, and cached per device.  Nothing here calls cudaMalloc, cudaFree or any
 // allocating routine.
+#include <atomic>
+
 #include "pa_internal.h"
 
 namespace {
@@ -20,13 +22,10 @@ namespace {
 static __device__ __align__(256) unsigned char g_noalloc_scratch[PA_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxNoallocDevices = 64;
-void* g_noalloc_scratch_addr[kMaxNoallocDevices] = {nullptr};
-
-// Bytes of split partials that two splits of every (token, q head) row need; a call whose
-// rows do not fit twice in the scratch is beyond this entry point's maximum.
-size_t two_split_bytes(int num_tokens, int num_q_heads, int head_size) {
-    return pa_attention_workspace_bytes(num_tokens, num_q_heads, head_size, 2);
-}
+// Device address of the scratch per device, resolved once.  Concurrent first calls from
+// several host threads may each resolve it; they store the same value, and the atomic makes
+// that a well-defined race.  A failed resolution is not cached, so the next call retries.
+std::atomic<void*> g_noalloc_scratch_addr[kMaxNoallocDevices];
 
 }  // namespace
 
@@ -36,26 +35,24 @@ extern "C" int pa_attention_noalloc(const pa_cache* cache, const void* q, int nu
                                     const int32_t* seq_lens_host,
                                     const int32_t* query_start_loc_host, int num_seqs,
                                     int num_tokens, float scale, float* out, void* stream) {
-    if (!cache || num_tokens < 0 || num_q_heads <= 0 || cache->head_size <= 0)
-        return PA_ERR_INVALID_ARG;
-    if (num_tokens > 0 &&
-        two_split_bytes(num_tokens, num_q_heads, cache->head_size) > PA_NOALLOC_SCRATCH_BYTES)
-        return PA_ERR_WORKSPACE;  // the fixed scratch cannot hold this call's partials
-
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxNoallocDevices)
         return PA_ERR_CUDA;
-    if (!g_noalloc_scratch_addr[dev]) {
+    void* ptr = g_noalloc_scratch_addr[dev].load(std::memory_order_acquire);
+    if (!ptr) {
         // one-time set-up on this device (the device is current): resolve the device address
-        void* ptr = nullptr;
         const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-        if (e != cudaSuccess || !ptr) return PA_ERR_CUDA;
-        g_noalloc_scratch_addr[dev] = ptr;
+        if (e != cudaSuccess || !ptr) {
+            cudaGetLastError();
+            return PA_ERR_CUDA;
+        }
+        g_noalloc_scratch_addr[dev].store(ptr, std::memory_order_release);
     }
-    // pa_attention clears the split counters on the stream before its kernels and writes every
-    // partial the merge reads; the planner fits the split-KV partition into the scratch.
+    // pa_attention checks every argument first, then plans a split-KV partition that fits the
+    // scratch (fewer splits, down to none, when the call's rows are many); it clears the split
+    // counters on the stream before its kernels and writes every partial the merge reads.  A
+    // plan that still needs more than the scratch is refused with PA_ERR_WORKSPACE.
     return pa_attention(cache, q, num_q_heads, block_table, max_blocks_per_seq, seq_lens,
                         query_start_loc, seq_lens_host, query_start_loc_host, num_seqs,
-                        num_tokens, scale, out, g_noalloc_scratch_addr[dev],
-                        PA_NOALLOC_SCRATCH_BYTES, stream);
+                        num_tokens, scale, out, ptr, PA_NOALLOC_SCRATCH_BYTES, stream);
 }
