@@ -135,8 +135,9 @@ int pa_free_blocks(const int32_t* block_ids, int num_ids, int32_t* free_queue,
  * block s / block_size.  bf16 pools store the bits unchanged; FP8 pools store
  * e4m3_rn_satfinite(x / scale[h]) with an IEEE fp32 divide.  A negative slot skips the token.
  * k, v: device bf16 [num_tokens][num_kv_heads][head_size], dense.  slot_mapping: device int32
- * [num_tokens].  Slots must lie inside the pool and be distinct within one call (duplicates
- * leave an unspecified one of the rows).  Errors: INVALID_ARG, CUDA. */
+ * [num_tokens].  Slots must lie inside the pool and be distinct within one call: a slot at or
+ * beyond the pool is skipped and records a device error; duplicates leave an unspecified one
+ * of the rows (pa_validate_slots counts both before a write).  Errors: INVALID_ARG, CUDA. */
 int pa_write_kv(pa_cache* cache, const void* k, const void* v, const int32_t* slot_mapping,
                 int num_tokens, void* stream);
 
@@ -189,10 +190,14 @@ int pa_attention(const pa_cache* cache, const void* q, int num_q_heads,
  * otherwise behaves exactly like pa_attention (same arguments, results and errors).
  * It allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
  * Set-up: the first call on a device (with that device current) resolves the scratch's
- *   device address with cudaGetSymbolAddress; make that first call before any stream capture.
- * Limit: calls for which pa_attention_workspace_bytes(num_tokens, num_q_heads, head_size, 2)
- *   (two splits of every row) exceeds PA_NOALLOC_SCRATCH_BYTES return PA_ERR_WORKSPACE and
- *   launch nothing; other calls get a split-KV partition fitted to the scratch.
+ *   device address with cudaGetSymbolAddress and caches it for the device; make that first
+ *   call before any stream capture.  After cudaDeviceReset the cached address is stale: a
+ *   process that resets a device must reload the library before calling this again.
+ * Limit: the split-KV partials of a call must fit PA_NOALLOC_SCRATCH_BYTES.  The planner
+ *   fits them, exactly as pa_attention does with a workspace of that size: a call with many
+ *   rows gets fewer KV splits (down to none) rather than a refusal.  A plan that would still
+ *   need more scratch than that returns PA_ERR_WORKSPACE and launches nothing.  Arguments
+ *   are checked first, with pa_attention's errors.
  * Sharing: all calls on a device share the one scratch, which keeps the last call's contents;
  *   each call clears the split counters it uses (the only part that must start at zero) on its
  *   stream before its kernels run, and writes every partial it reads.  Calls that overlap on
@@ -318,9 +323,22 @@ int pa_validate_block_table(const pa_cache* cache, const int32_t* block_table,
                             int max_blocks_per_seq, const int32_t* seq_lens, int num_seqs,
                             int* num_bad, void* stream);
 
+/* Opt-in device check of one call's slot mapping before pa_write_kv: counts the tokens whose
+ * slot lies at or beyond the pool's num_blocks * block_size slots (*num_out_of_pool) and the
+ * tokens whose slot another token of the same call also holds (*num_duplicates = valid
+ * in-pool tokens minus distinct slots among them).  Negative slots are skips and count as
+ * neither.  slot_mapping: device int32 [num_tokens].  Uses a temporary device bitmap of the
+ * pool's slots (stream-ordered allocation), synchronises `stream`, never traps.
+ * Errors: INVALID_ARG, CUDA. */
+int pa_validate_slots(const pa_cache* cache, const int32_t* slot_mapping, int num_tokens,
+                      int* num_out_of_pool, int* num_duplicates, void* stream);
+
 /* Read (and, if reset != 0, clear) the device error word of the current device: 0 = none,
  * 1 = a bounded wait timed out, 2 = a slot position beyond the block table, 3 = a block id
- * outside the pool.  Synchronises the device.  Returns PA_OK or PA_ERR_CUDA. */
+ * outside the pool, 4 = device metadata (query_start_loc, seq_lens) disagreeing with the
+ * host copies the launch was planned from, or with the launch's own sizes.  The first code
+ * recorded wins until the word is cleared.  Synchronises the device.  Returns PA_OK or
+ * PA_ERR_CUDA. */
 int pa_device_error(int* code, int reset);
 
 /* Human-readable name of a pa_status value. */

@@ -33,7 +33,7 @@ EXPORTED = [
     "pa_write_kv", "pa_attention_workspace_bytes", "pa_attention", "pa_plan_attention",
     "pa_attention_ex", "pa_validate_block_table", "pa_device_error", "pa_status_string",
     "pa_last_cuda_error", "pa_attention_noalloc", "pa_allocate_slots", "pa_free_blocks",
-    "pa_dcp_local_seq_lens", "pa_dcp_slot_mapping", "pa_merge_partials",
+    "pa_dcp_local_seq_lens", "pa_dcp_slot_mapping", "pa_merge_partials", "pa_validate_slots",
 ]
 PA_NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -108,6 +108,7 @@ def load() -> ctypes.CDLL:
         "pa_attention_ex": (I, [P, P, I, P, I, P, P, P, P, I, I, F, P, P, Z,
                                 ctypes.POINTER(pa_attention_opts), P]),
         "pa_validate_block_table": (I, [P, P, I, P, I, ctypes.POINTER(I), P]),
+        "pa_validate_slots": (I, [P, P, I, ctypes.POINTER(I), ctypes.POINTER(I), P]),
         "pa_device_error": (I, [ctypes.POINTER(I), I]),
         "pa_status_string": (ctypes.c_char_p, [I]),
         "pa_last_cuda_error": (I, []),
@@ -287,6 +288,16 @@ def pa_validate_block_table(handle, block_table, max_blocks_per_seq, seq_lens, n
                                           _ptr(seq_lens), num_seqs, ctypes.byref(bad),
                                           _stream(stream)), "pa_validate_block_table")
     return bad.value
+
+
+def pa_validate_slots(handle, slot_mapping, num_tokens, stream=None) -> tuple:
+    """(tokens whose slot lies outside the pool, tokens whose slot another token of the call
+    also holds) for one call's slot mapping; negative slots are skips."""
+    out_of_pool, dups = ctypes.c_int(0), ctypes.c_int(0)
+    _check(load().pa_validate_slots(handle, _ptr(slot_mapping), num_tokens,
+                                    ctypes.byref(out_of_pool), ctypes.byref(dups),
+                                    _stream(stream)), "pa_validate_slots")
+    return out_of_pool.value, dups.value
 
 
 def pa_device_error(reset: bool = True) -> int:

@@ -22,8 +22,8 @@
 // query rows (GQA group x q_len, padded to 8) on N of an m16n8k16 tile, so a group of 8
 // fills the tile with no padding.  P^T is brought into B-operand layout with movmatrix,
 // and O^T += V^T P^T reads V through ldmatrix.trans.  Softmax runs in the log2 domain.
-// FP8 E4M3 caches: S^T = K Q^T runs on FP8 tensor cores from the cache bytes (Q split
-// exactly into two E4M3 terms), and V tiles are stored dim-major so that ldmatrix hands out
+// FP8 E4M3 caches: S^T = K Q^T runs on FP8 tensor cores from the cache bytes (Q split into
+// two E4M3 terms that hold its bf16 value), and V tiles are stored dim-major so that ldmatrix hands out
 // four consecutive keys per word, widened exactly to f16 (as 2^-8 V, by moving bits) for
 // O^T += V^T P^T; the K scale folds into the score scale and the V scale into the epilogue.
 #include <cstdlib>
@@ -111,10 +111,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
     // ---- Q^T as B fragments: row n = gq is (token n / group, head g * group + n % group)
     // bf16 cache: bf16 pairs for m16n8k16.  FP8 cache: S^T = K Q^T runs on FP8 tensor cores
     // (m16n8k32 E4M3) straight from the cache bytes; each Q row is scaled by a power of two
-    // 2^e and split exactly into two E4M3 terms q1 + q2 (q1 = e4m3(q 2^e), q2 = e4m3 of the
-    // fp32-exact remainder), so the product keeps bf16-level precision; qb[0..3] hold q1 and
-    // qb[4..7] q2 (k-steps of 32 dims).  The row's 2^-e, the K scale and the softmax scale
-    // multiply its scores.
+    // 2^e (row max between 112 and 224) and split into two E4M3 terms q1 + q2 (q1 =
+    // e4m3(q 2^e), q2 = e4m3 of the fp32-exact remainder).  A bf16 value keeps 8 significant
+    // bits, q1 the top 4 and the remainder at most 4 more, so the split is exact for scaled
+    // elements of magnitude 2^-2 and above; below that the remainder's bits under E4M3's
+    // smallest subnormal step (2^-9) are rounded away, an absolute error of at most 2^-10 in
+    // the scaled element.  qb[0..3] hold q1 and qb[4..7] q2 (k-steps of 32 dims).  The row's
+    // 2^-e, the K scale and the softmax scale multiply its scores.
     uint32_t qb[C::kKSteps][2];
     float sl0 = p.scale_log2, sl1 = p.scale_log2;  // score multipliers of rows 2tq, 2tq+1
     {

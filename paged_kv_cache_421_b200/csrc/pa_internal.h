@@ -126,5 +126,7 @@ cudaError_t launch_merge_partials(const float* part_out, const float* part_lse, 
 cudaError_t launch_validate(const int32_t* block_table, int max_blocks_per_seq,
                             const int32_t* seq_lens, int num_seqs, int block_size,
                             int num_blocks, int* counter, cudaStream_t stream);
+cudaError_t launch_validate_slots(const int32_t* slots, int num_tokens, int64_t num_slots,
+                                  uint32_t* bitmap, int* counts, cudaStream_t stream);
 
 }  // namespace pa

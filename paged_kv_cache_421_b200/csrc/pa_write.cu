@@ -1,4 +1,4 @@
-// Slot mapping, cache write (reshape_and_cache) and the opt-in block-table validator.
+// Slot mapping, cache write (reshape_and_cache) and the opt-in block-table and slot validators.
 //
 // Slot of a new token ("vLLM: from KV Cache to high-throughput serving", article 3 outline;
 // "Inside vLLM" notes, core point 2): token i of request r sits at position
@@ -10,6 +10,8 @@
 // row, so both the reads of k/v and the writes into the pool are coalesced.  An FP8 pool
 // stores e4m3(x / scale[head]) with an IEEE-rounded fp32 divide and saturating conversion;
 // its V tiles are dim-major, so V bytes are scattered with a 16-byte stride.
+#include <algorithm>
+
 #include "pa_internal.h"
 
 namespace pa {
@@ -116,6 +118,34 @@ __global__ void validate_kernel(const int32_t* __restrict__ bt, int maxb,
     if ((threadIdx.x & 31) == 0 && bad) atomicAdd(counter, bad);
 }
 
+// Slot check: a slot at or beyond the pool's num_slots counts as out of the pool; a slot that
+// another token of the same call already holds counts as a duplicate (set bit already set in
+// a bitmap of the pool's slots, cleared by the host first), so the count is the number of
+// tokens minus the distinct slots among them, whatever the order.  Negative slots are skips.
+__global__ void validate_slots_kernel(const int32_t* __restrict__ slots, int num_tokens,
+                                      int64_t num_slots, uint32_t* bitmap, int* counts) {
+    int out = 0, dup = 0;
+    for (int t = blockIdx.x * blockDim.x + threadIdx.x; t < num_tokens;
+         t += gridDim.x * blockDim.x) {
+        const int s = slots[t];
+        if (s < 0) continue;
+        if (s >= num_slots) {
+            ++out;
+            continue;
+        }
+        const uint32_t bit = 1u << (s & 31);
+        dup += (atomicOr(bitmap + (s >> 5), bit) & bit) != 0;
+    }
+    for (int off = 16; off > 0; off >>= 1) {
+        out += __shfl_xor_sync(0xffffffffu, out, off);
+        dup += __shfl_xor_sync(0xffffffffu, dup, off);
+    }
+    if ((threadIdx.x & 31) == 0) {
+        if (out) atomicAdd(counts, out);
+        if (dup) atomicAdd(counts + 1, dup);
+    }
+}
+
 template <int D, bool FP8>
 cudaError_t launch_write_t(const pa_cache& c, const void* k, const void* v, const int32_t* slots,
                            int num_tokens, int* err, cudaStream_t stream) {
@@ -159,6 +189,15 @@ cudaError_t launch_validate(const int32_t* block_table, int max_blocks_per_seq,
                             int num_blocks, int* counter, cudaStream_t stream) {
     validate_kernel<<<num_seqs, 128, 0, stream>>>(block_table, max_blocks_per_seq, seq_lens,
                                                   block_size, num_blocks, counter);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_validate_slots(const int32_t* slots, int num_tokens, int64_t num_slots,
+                                  uint32_t* bitmap, int* counts, cudaStream_t stream) {
+    const int threads = 256;
+    const int blocks = static_cast<int>(std::min<int64_t>((num_tokens + threads - 1) / threads, 148 * 8));
+    validate_slots_kernel<<<blocks, threads, 0, stream>>>(slots, num_tokens, num_slots, bitmap,
+                                                          counts);
     return cudaGetLastError();
 }
 

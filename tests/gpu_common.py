@@ -91,23 +91,29 @@ def oracle_cache(wl: W.Workload) -> np.ndarray:
     return cache
 
 
+# The oracle's attention runs on its OpenMP build over every host core by default: the same
+# bits as the single-threaded build (pinned by tests/test_oracle_openmp.py), in less time.
+ORACLE_THREADS = 0
+
+
 def oracle_attention_all(wl: W.Workload, cache: np.ndarray, window: int = 0,
-                         local_chunk: int = 0):
+                         local_chunk: int = 0, threads=ORACLE_THREADS):
     ks = None if wl.k_scale is None else wl.k_scale.cpu().numpy()
     vs = None if wl.v_scale is None else wl.v_scale.cpu().numpy()
     return oracle.attention_paged(cache, wl.kv_dtype, wl.num_blocks, wl.block_size,
                                   wl.num_kv_heads, wl.head_size, W.bits(wl.q), wl.num_q_heads,
                                   wl.block_table, wl.seq_lens, wl.qsl, wl.scale, ks, vs,
-                                  window=window, local_chunk=local_chunk)
+                                  window=window, local_chunk=local_chunk, threads=threads)
 
 
-def oracle_attention_rows(wl: W.Workload, tokens, heads):
+def oracle_attention_rows(wl: W.Workload, tokens, heads, threads=ORACLE_THREADS):
     k_src, v_src = wl.kv_src()
     ks = None if wl.k_scale is None else wl.k_scale.cpu().numpy()
     vs = None if wl.v_scale is None else wl.v_scale.cpu().numpy()
     return oracle.attention_rows(W.bits(k_src), W.bits(v_src), wl.pos_rows, wl.pos_start,
                                  wl.kv_dtype, W.bits(wl.q), wl.seq_lens, wl.qsl, wl.scale,
-                                 np.asarray(tokens, np.int32), np.asarray(heads, np.int32), ks, vs)
+                                 np.asarray(tokens, np.int32), np.asarray(heads, np.int32), ks, vs,
+                                 threads=threads)
 
 
 def assert_close(got: np.ndarray, want: np.ndarray, kv_dtype: int, what: str = "") -> dict:

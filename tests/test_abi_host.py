@@ -166,6 +166,14 @@ def test_argument_errors_without_device(lib):
     assert lib.pa_slot_mapping(None, 4, None, None, 1, 1, 16, None, None) == B.PA_ERR_INVALID_ARG
     assert lib.pa_free_cache(None) == B.PA_OK
     assert B.pa_status_string(B.PA_ERR_METADATA) == "PA_ERR_METADATA"
+    n_out, n_dup = ctypes.c_int(7), ctypes.c_int(7)
+    assert lib.pa_validate_slots(None, None, 4, ctypes.byref(n_out), ctypes.byref(n_dup),
+                                 None) == B.PA_ERR_INVALID_ARG
+    fake = ctypes.c_void_p(0x1000)  # never dereferenced: the checks below fail first
+    assert lib.pa_validate_slots(fake, None, -1, ctypes.byref(n_out), ctypes.byref(n_dup),
+                                 None) == B.PA_ERR_INVALID_ARG
+    assert lib.pa_validate_slots(fake, None, 4, None, ctypes.byref(n_dup), None) == \
+        B.PA_ERR_INVALID_ARG
 
 
 def test_allocator_argument_errors_without_device(lib):

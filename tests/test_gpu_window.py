@@ -1,6 +1,8 @@
 """Sliding-window attention (a query at position p sees keys max(0, p - W + 1) .. p) against
 the oracle: decode and chunked-prefill rows, bf16 and FP8 pools, head sizes 64 and 128, and
 forced KV splits whose ranges start below, inside and past the window."""
+import zlib
+
 import numpy as np
 import pytest
 
@@ -30,7 +32,7 @@ CASES = {
 @pytest.mark.parametrize("window", [1, 16, 17, 100, 513, 4096])
 def test_window_matches_oracle(case, window):
     ctx, ql, hq, hkv, d = CASES[case]
-    wl = _wl(ctx, ql, hq, hkv, d, seed=hash((case, window)) % 997)
+    wl = _wl(ctx, ql, hq, hkv, d, seed=zlib.crc32(repr((case, window)).encode()) % 997)
     st = GpuStep(wl, run_attention=False)
     want, _ = oracle_attention_all(wl, oracle_cache(wl), window=window)
     for split in [0, 16, 64, 512]:
@@ -62,7 +64,7 @@ def test_window_longer_than_context_is_full_attention():
 @pytest.mark.parametrize("chunk", [1, 16, 100, 1000])
 def test_local_chunk_matches_oracle(case, chunk):
     ctx, ql, hq, hkv, d = CASES[case]
-    wl = _wl(ctx, ql, hq, hkv, d, seed=hash((case, chunk, "c")) % 997)
+    wl = _wl(ctx, ql, hq, hkv, d, seed=zlib.crc32(repr((case, chunk, "c")).encode()) % 997)
     st = GpuStep(wl, run_attention=False)
     want, _ = oracle_attention_all(wl, oracle_cache(wl), local_chunk=chunk)
     for split in [0, 64]:
