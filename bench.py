@@ -68,6 +68,9 @@ def parse_args(argv=None):
                          "are under 4x the 126 MB L2)")
     ap.add_argument("--kv-split-tokens", type=int, default=0,
                     help="force the KV partition (keys per split); 0 = planner's choice")
+    ap.add_argument("--cascade", choices=["auto", "on", "off"], default="auto",
+                    help="cascade attention over the block-table prefix every request shares "
+                         "(auto: when it spans at least 256 tokens and 8 requests)")
     return ap.parse_args(argv)
 
 
@@ -98,12 +101,22 @@ def kv_bytes(wl, window: int = 0, local_chunk: int = 0) -> int:
         wl.head_size * wl.dtype_bytes
 
 
-def decode_kv_bytes(wl, window: int = 0, local_chunk: int = 0) -> int:
+def decode_kv_bytes(wl, window: int = 0, local_chunk: int = 0, prefix: int = 0) -> int:
+    """KV bytes the decode kernel reads: the visible keys of every decode-kind request, less
+    a shared prefix of `prefix` keys that cascade attention reads in its own pass."""
     G = wl.num_q_heads // wl.num_kv_heads
     ql = wl.q_lens
     dec = (ql > 0) & (ql * G <= 8)
-    return int(np.sum(visible_keys(wl, window, local_chunk)[dec])) * 2 * wl.num_kv_heads * \
-        wl.head_size * wl.dtype_bytes
+    keys = visible_keys(wl, window, local_chunk)[dec] - prefix
+    return int(np.sum(keys)) * 2 * wl.num_kv_heads * wl.head_size * wl.dtype_bytes
+
+
+def prefix_pass_work(wl, prefix: int) -> tuple:
+    """(KV bytes, FLOPs) of the cascade prefix pass: the prefix's keys read once per kv head,
+    and every query row of the step against all of them (4 D FLOPs per (row, key))."""
+    nbytes = prefix * 2 * wl.num_kv_heads * wl.head_size * wl.dtype_bytes
+    flops = wl.num_tokens * wl.num_q_heads * prefix * 4 * wl.head_size
+    return nbytes, flops
 
 
 def chunk_flops(wl, window: int = 0, local_chunk: int = 0) -> int:
@@ -122,13 +135,32 @@ def chunk_flops(wl, window: int = 0, local_chunk: int = 0) -> int:
 def launches_for_plan(plan: dict, head_size: int) -> int:
     """Kernels of ours per step, as pa_attention launches them: slot mapping and write, the
     split-counter clear (split decode requests, or chunk splits the tcgen05 kernel merges
-    itself: head_size 128 and at most 4 splits), the decode and/or chunk kernel, and the split
-    reduce (chunk splits not merged in the chunk kernel)."""
+    itself: head_size 128 and at most 4 splits), the cascade prefix pass, the decode and/or
+    chunk kernel, and the split reduce (chunk splits not merged in the chunk kernel)."""
     fused = head_size == 128 and plan["chunk_max_splits"] <= 4
     clear = plan["decode_max_splits"] > 1 or (plan["chunk_max_splits"] > 1 and fused)
     reduce = plan["chunk_max_splits"] > 1 and not fused
-    return 2 + int(clear) + int(plan["num_decode_seqs"] > 0) + int(plan["num_chunk_seqs"] > 0) + \
-        int(reduce)
+    prefix = plan.get("prefix_splits", 0) > 0
+    return 2 + int(clear) + int(prefix) + int(plan["num_decode_seqs"] > 0) + \
+        int(plan["num_chunk_seqs"] > 0) + int(reduce)
+
+
+def cascade_prefix_tokens(wl, mode: str = "auto") -> int:
+    """Tokens of the block-table prefix every request of the step shares, to be read once by
+    cascade attention; 0 when cascade is off (auto: a prefix of at least 256 tokens over at
+    least 8 requests, every one of them a decode)."""
+    if mode == "off":
+        return 0
+    from paged_kv_cache_421_b200 import _binding as B
+    G = wl.num_q_heads // wl.num_kv_heads
+    ql = wl.q_lens
+    live = ql > 0
+    if not np.all(ql[live] * G <= 8):
+        return 0
+    P = 16 * B.pa_common_prefix_blocks(wl.block_table, wl.seq_lens, wl.qsl)
+    if mode == "auto" and (P < 256 or int(np.sum(live)) < 8):
+        return 0
+    return P
 
 
 def unique_kv_bytes(wl) -> int:
@@ -343,11 +375,13 @@ def cpu_baseline(wl, budget_s: float, window: int = 0, local_chunk: int = 0) -> 
 # ---------------------------------------------------------------- device step
 class DeviceStep:
     def __init__(self, wl, device, kv_split_tokens: int = 0, sliding_window: int = 0,
-                 local_chunk: int = 0):
+                 local_chunk: int = 0, cascade: str = "auto"):
         import torch
         self.kv_split_tokens = kv_split_tokens
         self.window = sliding_window
         self.local_chunk = local_chunk
+        self.prefix = (cascade_prefix_tokens(wl, cascade)
+                       if not (sliding_window or local_chunk) else 0)
         from paged_kv_cache_421_b200 import ops
         from paged_kv_cache_421_b200 import workloads as W
         self.wl, self.dev, self.ops, self.torch = wl, device, ops, torch
@@ -376,14 +410,16 @@ class DeviceStep:
                                device=device)
         nb = ops.workspace_bytes_for(self.cache, wl.seq_lens, wl.qsl, wl.num_q_heads,
                                      wl.max_blocks_per_seq, kv_split_tokens,
-                                     sliding_window=sliding_window, local_chunk=local_chunk)
+                                     sliding_window=sliding_window, local_chunk=local_chunk,
+                                     common_prefix_tokens=self.prefix)
         self.workspace = torch.empty(max(nb, 256), dtype=torch.uint8, device=device)
         self.plan = ops.B.pa_plan_attention(
             wl.seq_lens, wl.qsl, wl.num_q_heads, wl.num_kv_heads, wl.head_size,
             wl.max_blocks_per_seq,
             torch.cuda.get_device_properties(device).multi_processor_count,
             self.workspace.numel(), kv_split_tokens=kv_split_tokens,
-            sliding_window=sliding_window, local_chunk=local_chunk)
+            sliding_window=sliding_window, local_chunk=local_chunk,
+            common_prefix_tokens=self.prefix)
         torch.cuda.synchronize(device)
 
     def launches_per_step(self) -> int:
@@ -404,7 +440,8 @@ class DeviceStep:
                           bt.shape[1], sl, qsl, wl.seq_lens, wl.qsl, wl.num_seqs, T, wl.scale,
                           out, self.workspace, self.workspace.numel(),
                           kv_split_tokens=self.kv_split_tokens, events=events,
-                          sliding_window=self.window, local_chunk=self.local_chunk)
+                          sliding_window=self.window, local_chunk=self.local_chunk,
+                          common_prefix_tokens=self.prefix)
 
 
 def time_step(step, args, flush_l2: bool, flush, stream, world: int, local: int, device,
@@ -477,11 +514,12 @@ def time_step(step, args, flush_l2: bool, flush, stream, world: int, local: int,
     return t
 
 
-def decode_roofline(wl, workload: str, dec_ms: float, window: int, local_chunk: int) -> dict:
+def decode_roofline(wl, workload: str, dec_ms: float, window: int, local_chunk: int,
+                    prefix: int = 0) -> dict:
     """HBM roofline of the decode kernel: algorithmic KV bytes of one launch / its mean
     CUDA-event duration, against the measured copy peak."""
     peak, peak_kind = load_peaks()
-    dec_bytes = decode_kv_bytes(wl, window, local_chunk)
+    dec_bytes = decode_kv_bytes(wl, window, local_chunk, prefix)
     achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
     return {"bound": "hbm", "kernel": "decode_kernel", "achieved": round(achieved, 1),
             "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
@@ -503,7 +541,8 @@ def measure_variant(name: str, args, world: int, local: int, device, flush, stre
     import torch
     from paged_kv_cache_421_b200 import workloads as W
     wl = W.CONFIGS[name](device=device)
-    step = DeviceStep(wl, device, args.kv_split_tokens, args.sliding_window, args.local_chunk)
+    step = DeviceStep(wl, device, args.kv_split_tokens, args.sliding_window, args.local_chunk,
+                      args.cascade)
     nbytes = kv_bytes(wl, args.sliding_window, args.local_chunk)
     flush_l2 = args.flush == "always" or (args.flush == "auto" and nbytes < 4 * L2_BYTES)
     t = time_step(step, args, flush_l2, flush, stream, world, local, device,
@@ -532,7 +571,8 @@ def run_device_bench(args, rank, world, local):
     device = torch.device(f"cuda:{local}")
     torch.cuda.set_device(device)
     wl = W.CONFIGS[args.workload](device=device)
-    step = DeviceStep(wl, device, args.kv_split_tokens, args.sliding_window, args.local_chunk)
+    step = DeviceStep(wl, device, args.kv_split_tokens, args.sliding_window, args.local_chunk,
+                      args.cascade)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     nbytes = kv_bytes(wl, args.sliding_window, args.local_chunk)
     flush_l2 = args.flush == "always" or (args.flush == "auto" and nbytes < 4 * L2_BYTES)
@@ -681,9 +721,19 @@ def run_device_bench(args, rank, world, local):
         roof = None
         if dec_ms:
             roof = decode_roofline(wl, args.workload, dec_ms, args.sliding_window,
-                                   args.local_chunk)
+                                   args.local_chunk, step.prefix)
+            if step.prefix:  # the recorded traffic is of the non-cascade decode kernel
+                roof["traffic"] = None
+        cascade = None
+        if step.prefix:
+            pb, pf = prefix_pass_work(wl, step.prefix)
+            cascade = {"prefix_tokens": step.prefix, "prefix_splits": step.plan["prefix_splits"],
+                       "prefix_pass_ms": round(chunk_ms, 4) if chunk_ms else None,
+                       "prefix_pass_flops": pf, "prefix_pass_kv_bytes": pb,
+                       "prefix_pass_tflops": round(pf / (chunk_ms * 1e-3) / 1e12, 1)
+                       if chunk_ms else None}
         chunk_roof = None
-        if chunk_ms:
+        if chunk_ms and not step.prefix:
             flops = chunk_flops(wl, args.sliding_window, args.local_chunk)
             tflops = flops / (chunk_ms * 1e-3) / 1e12
             tpeak, tkind = load_tensor_peak()
@@ -710,11 +760,18 @@ def run_device_bench(args, rank, world, local):
                               f"inputs larger than L2: {nbytes / 1e6:.0f} MB of KV per step vs "
                               f"126 MB L2, no flush"),
                        "kv_split_tokens": args.kv_split_tokens or "planner",
+                       "cascade_prefix_tokens": step.prefix or None,
                        "sliding_window": args.sliding_window or None,
                        "local_chunk": args.local_chunk or None,
                        "parallelism": f"replicas x{world} (one batch per GPU)"},
             "tokens_per_s": round(world * wl.num_tokens / (ms_per_step * 1e-3), 1),
             "pct_hbm_peak": round(100 * value / world / peak, 2),
+            "unique": ({"kv_bytes_per_step": ub,
+                        "value": round(world * ub / (ms_per_step * 1e-3) / 1e9, 2),
+                        "unit": "GB/s",
+                        "pct_hbm_peak": round(100 * ub / (ms_per_step * 1e-3) / 1e9 / peak, 2)}
+                       if (ub := unique_kv_bytes(wl)) < nbytes else None),
+            "cascade": cascade,
             "roofline": roof,
             "kernel_ms": {"decode": dec_ms, "chunk": chunk_ms, "reduce": reduce_ms},
             "ms_per_step_with_kernel_events": round(ms_per_step_events, 4),

@@ -160,8 +160,8 @@ size_t pa_attention_workspace_bytes(int num_tokens, int num_q_heads, int head_si
  *   pa_attention_opts.sliding_window = W > 0 (pa_attention_ex) only to the last W of them,
  *   and with pa_attention_opts.local_chunk = C > 0 only to those from floor(p / C) * C.
  * Requests with q_len * (num_q_heads / num_kv_heads) <= 8 run in the decode kernel, the others
- *   in the chunked-prefill kernel, which needs a bf16 cache (an FP8 cache with such a request
- *   -> PA_ERR_UNSUPPORTED).
+ *   in the chunked-prefill kernel (bf16 or FP8 E4M3 cache; any mix of the two kinds in one
+ *   call).
  * out: device fp32 [num_tokens][num_q_heads][head_size].
  * workspace: device scratch of workspace_bytes for split-KV partials (may be NULL/0: then no
  *   request is split).  Its contents are opaque; it must not be shared by calls that
@@ -227,6 +227,9 @@ typedef struct {
     int any_split;            /* some request is split: partials go through the workspace */
     size_t workspace_needed;  /* bytes of workspace this plan uses */
     int reduce_rows_max;      /* largest q_len * group among split chunk-kind requests */
+    int prefix_splits;        /* cascade: KV splits of the shared-prefix pass (0: no cascade) */
+    int prefix_split_blocks;  /* cascade: blocks per prefix split */
+    int64_t prefix_ctas;      /* cascade: CTAs of the prefix pass */
 } pa_plan;
 
 /* Options for pa_attention_ex (zero-initialise for defaults). */
@@ -236,7 +239,8 @@ typedef struct {
     int num_sms;           /* > 0: plan for this many SMs instead of the device's count */
     void* events[6];       /* optional cudaEvent_t handles recorded on the call's stream:
                               [0]/[1] before/after the decode kernel, [2]/[3] around the chunk
-                              kernel, [4]/[5] around the split reduce; an entry is recorded
+                              kernel (with a common prefix: its prefix pass), [4]/[5] around
+                              the split reduce; an entry is recorded
                               only when that kernel is launched; NULL entries are skipped */
     int sliding_window;    /* > 0: a query at position p sees only keys max(0, p - W + 1) .. p
                               (the sliding window [P2] section 2 names; its reading here);
@@ -252,6 +256,21 @@ typedef struct {
                               decode-kind requests with seq_len == 0 are also accepted: their
                               rows get out = 0 and lse = -inf (an empty share of a context-
                               parallel group).  NULL: not written */
+    int common_prefix_tokens; /* > 0: cascade attention over a shared prefix ([P2] section 2:
+                              requests whose block tables start with the same physical blocks,
+                              e.g. A = [B0, B3, B7], B = [B0, B3, B1, B5, B8] share B0, B3;
+                              section 6 names cascade attention).  The first
+                              common_prefix_tokens / block_size entries of the block-table row
+                              of every request with q_len > 0 are the same physical blocks
+                              (pa_common_prefix_blocks finds them from a host copy of the
+                              table); the call reads those blocks once for all the step's
+                              queries, attends each request's remaining keys separately and
+                              merges the two by their LSEs -- the result is the same attention.
+                              Requires a multiple of block_size, every request with q_len > 0
+                              decode-kind with seq_len - q_len >= common_prefix_tokens
+                              (else METADATA), no sliding window or local chunk (else
+                              UNSUPPORTED), and workspace for the prefix partials
+                              (pa_plan_attention's workspace_needed; else WORKSPACE).  0: off */
 } pa_attention_opts;
 
 /* The planner alone: fills *plan for the given host metadata without touching the GPU.
@@ -262,6 +281,18 @@ int pa_plan_attention(const int32_t* seq_lens_host, const int32_t* query_start_l
                       int num_seqs, int num_tokens, int num_q_heads, int num_kv_heads,
                       int head_size, int block_size, int max_blocks_per_seq, int num_sms,
                       size_t workspace_bytes, const pa_attention_opts* opts, pa_plan* plan);
+
+/* Longest shared prefix of a step's block tables, for cascade attention
+ * (pa_attention_opts.common_prefix_tokens = *num_blocks * block_size): the largest n such that
+ * every request with q_len > 0 has the same n first block ids as the first such request, and
+ * n * block_size <= seq_len - q_len for each of them (every query sees the whole prefix).
+ * Host arrays: block_table_host [num_seqs][max_blocks_per_seq], seq_lens_host [num_seqs],
+ * query_start_loc_host [num_seqs + 1].  *num_blocks = 0 when no request has a query.  Pure
+ * host computation.  Errors: INVALID_ARG (null pointer, non-positive sizes), METADATA
+ * (q_len < 0 or seq_len < q_len). */
+int pa_common_prefix_blocks(const int32_t* block_table_host, int max_blocks_per_seq,
+                            const int32_t* seq_lens_host, const int32_t* query_start_loc_host,
+                            int num_seqs, int block_size, int* num_blocks);
 
 /* pa_attention with options (opts may be NULL). */
 int pa_attention_ex(const pa_cache* cache, const void* q, int num_q_heads,

@@ -34,6 +34,7 @@ EXPORTED = [
     "pa_attention_ex", "pa_validate_block_table", "pa_device_error", "pa_status_string",
     "pa_last_cuda_error", "pa_attention_noalloc", "pa_allocate_slots", "pa_free_blocks",
     "pa_dcp_local_seq_lens", "pa_dcp_slot_mapping", "pa_merge_partials", "pa_validate_slots",
+    "pa_common_prefix_blocks",
 ]
 PA_NOALLOC_SCRATCH_BYTES = 64 << 20
 
@@ -52,6 +53,9 @@ class pa_plan(ctypes.Structure):
         ("any_split", ctypes.c_int),
         ("workspace_needed", ctypes.c_size_t),
         ("reduce_rows_max", ctypes.c_int),
+        ("prefix_splits", ctypes.c_int),
+        ("prefix_split_blocks", ctypes.c_int),
+        ("prefix_ctas", ctypes.c_int64),
     ]
 
     def as_dict(self) -> dict:
@@ -66,6 +70,7 @@ class pa_attention_opts(ctypes.Structure):
         ("sliding_window", ctypes.c_int),
         ("local_chunk", ctypes.c_int),
         ("lse_out", ctypes.c_void_p),
+        ("common_prefix_tokens", ctypes.c_int),
     ]
 
 
@@ -109,6 +114,7 @@ def load() -> ctypes.CDLL:
                                 ctypes.POINTER(pa_attention_opts), P]),
         "pa_validate_block_table": (I, [P, P, I, P, I, ctypes.POINTER(I), P]),
         "pa_validate_slots": (I, [P, P, I, ctypes.POINTER(I), ctypes.POINTER(I), P]),
+        "pa_common_prefix_blocks": (I, [P, I, P, P, I, I, ctypes.POINTER(I)]),
         "pa_device_error": (I, [ctypes.POINTER(I), I]),
         "pa_status_string": (ctypes.c_char_p, [I]),
         "pa_last_cuda_error": (I, []),
@@ -214,7 +220,7 @@ def pa_attention_workspace_bytes(num_tokens, num_q_heads, head_size, max_splits)
 def pa_plan_attention(seq_lens_host, query_start_loc_host, num_q_heads, num_kv_heads,
                       head_size, max_blocks_per_seq, num_sms, workspace_bytes,
                       kv_split_tokens=0, block_size=16, sliding_window=0,
-                      local_chunk=0, with_lse=False) -> dict:
+                      local_chunk=0, with_lse=False, common_prefix_tokens=0) -> dict:
     """with_lse: plan as a call that exports LSEs (which admits empty decode shares); the
     planner only tests the pointer for NULL, so a dummy non-NULL value stands in."""
     sl = _host_i32(seq_lens_host)
@@ -224,6 +230,7 @@ def pa_plan_attention(seq_lens_host, query_start_loc_host, num_q_heads, num_kv_h
     opts.sliding_window = sliding_window
     opts.local_chunk = local_chunk
     opts.lse_out = 16 if with_lse else None
+    opts.common_prefix_tokens = common_prefix_tokens
     plan = pa_plan()
     _check(load().pa_plan_attention(sl.ctypes.data, qs.ctypes.data, sl.size, int(qs[-1]),
                                     num_q_heads, num_kv_heads, head_size, block_size,
@@ -248,7 +255,7 @@ def pa_attention_ex(handle, q, num_q_heads, block_table, max_blocks_per_seq, seq
                     query_start_loc, seq_lens_host, query_start_loc_host, num_seqs, num_tokens,
                     scale, out, workspace=None, workspace_bytes=0, kv_split_tokens=0,
                     num_sms=0, events=None, sliding_window=0, local_chunk=0, lse_out=None,
-                    stream=None) -> None:
+                    common_prefix_tokens=0, stream=None) -> None:
     sl = _host_i32(seq_lens_host)
     qs = _host_i32(query_start_loc_host)
     opts = pa_attention_opts()
@@ -257,6 +264,7 @@ def pa_attention_ex(handle, q, num_q_heads, block_table, max_blocks_per_seq, seq
     opts.sliding_window = sliding_window
     opts.local_chunk = local_chunk
     opts.lse_out = _ptr(lse_out)
+    opts.common_prefix_tokens = common_prefix_tokens
     for i, ev in enumerate(events or []):
         if ev is not None:
             opts.events[i] = ev.cuda_event if hasattr(ev, "cuda_event") else int(ev)
@@ -288,6 +296,20 @@ def pa_validate_block_table(handle, block_table, max_blocks_per_seq, seq_lens, n
                                           _ptr(seq_lens), num_seqs, ctypes.byref(bad),
                                           _stream(stream)), "pa_validate_block_table")
     return bad.value
+
+
+def pa_common_prefix_blocks(block_table_host, seq_lens_host, query_start_loc_host,
+                            block_size=16) -> int:
+    """Leading block-table entries that every request with queries shares, each request's
+    queries seeing all of them (host arrays)."""
+    bt = np.ascontiguousarray(block_table_host, dtype=np.int32)
+    sl = _host_i32(seq_lens_host)
+    qs = _host_i32(query_start_loc_host)
+    n = ctypes.c_int(0)
+    _check(load().pa_common_prefix_blocks(bt.ctypes.data, bt.shape[1], sl.ctypes.data,
+                                          qs.ctypes.data, sl.size, block_size, ctypes.byref(n)),
+           "pa_common_prefix_blocks")
+    return n.value
 
 
 def pa_validate_slots(handle, slot_mapping, num_tokens, stream=None) -> tuple:

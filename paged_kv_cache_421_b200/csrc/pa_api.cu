@@ -144,6 +144,12 @@ int max_splits_for(size_t ws, int num_tokens, int num_q_heads, int head_size) {
 
 int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
+// Cascade prefix partials: [S][T][Hq][D] normalised outputs, then [S][T][Hq] log2 LSEs.
+size_t prefix_part_bytes(int num_tokens, int num_q_heads, int head_size, int splits) {
+    const size_t rows = static_cast<size_t>(splits) * num_tokens * num_q_heads;
+    return align256(rows * head_size * sizeof(float)) + align256(rows * sizeof(float));
+}
+
 // Planner constants.
 constexpr int kDecodeCtasPerSm = 3;    // decode kernel residency (64 KB of stages per CTA)
 constexpr int kMaxDecodeSplits = 1024;  // merge weights of one row fit the CTA's shared memory
@@ -152,6 +158,7 @@ constexpr int kMinDecodeSplitBlocks = 64;   // >= 1024 keys per split
 constexpr int kMinChunkSplitBlocks = 16;
 constexpr int kMinChunkSplitTiles = 4;      // a chunk split walks at least four key tiles
 constexpr int kMaxChunkSplitBlocks = 1024;  // chunk kernels stage up to 1024 block ids
+constexpr int kMaxPrefixSplits = 8;         // prefix partials each decode row merges
 
 int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int Hkv, int D,
               int bs, int maxb, int num_sms, size_t ws, const pa_attention_opts* opts,
@@ -168,6 +175,11 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
     const int window = opts ? opts->sliding_window : 0;
     const int local_chunk = opts ? opts->local_chunk : 0;
     if (window < 0 || local_chunk < 0) return PA_ERR_INVALID_ARG;
+    // cascade attention over a shared prefix of P keys: decode-kind requests only, full
+    // attention only; each request's own work is its keys after the prefix
+    const int P = opts ? opts->common_prefix_tokens : 0;
+    if (P < 0 || P % bs) return PA_ERR_INVALID_ARG;
+    if (P > 0 && (window > 0 || local_chunk > 0)) return PA_ERR_UNSUPPORTED;
     // with an LSE output a decode-kind request may hold no key (an empty context-parallel
     // share): one CTA per kv head writes out = 0 and lse = -inf for its rows
     const bool empty_ok = opts && opts->lse_out;
@@ -184,17 +196,23 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
         if (ql < 0 || ctx < 0) return PA_ERR_METADATA;
         if (ql == 0) continue;
         if (ctx == 0) {
-            if (!empty_ok || !pa::is_decode_kind(ql, G)) return PA_ERR_METADATA;
+            if (!empty_ok || !pa::is_decode_kind(ql, G) || P > 0) return PA_ERR_METADATA;
             pl->num_decode_seqs++;
             continue;
         }
         if (ctx < ql) return PA_ERR_METADATA;
         const int blocks = pa::ceil_div(ctx, bs);
         if (blocks > maxb) return PA_ERR_METADATA;
+        if (P > 0) {
+            if (!pa::is_decode_kind(ql, G)) return PA_ERR_UNSUPPORTED;
+            if (ctx - ql < P) return PA_ERR_METADATA;
+        }
         if (pa::is_decode_kind(ql, G)) {
-            // with a sliding window the decode CTAs walk only the window's blocks
+            // with a sliding window the decode CTAs walk only the window's blocks; after a
+            // shared prefix, only the blocks past it
             pl->num_decode_seqs++;
-            const int eff = blocks - pa::first_visible_key(ctx - ql, window, local_chunk) / bs;
+            const int eff = blocks - P / bs -
+                            pa::first_visible_key(ctx - ql, window, local_chunk) / bs;
             dec_units += static_cast<long long>(eff) * Hkv;
             if (eff > dec_max_blocks) dec_max_blocks = eff;
         } else {
@@ -276,7 +294,7 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
         int ns;
         if (pa::is_decode_kind(ql, G)) {
             const int fb = pa::first_visible_key(sl[r] - ql, window, local_chunk) / bs;
-            ns = std::max(1, pa::ceil_div(pa::ceil_div(sl[r], bs) - fb, pl->decode_split_blocks));
+            ns = std::max(1, pa::ceil_div(pa::ceil_div(sl[r] - P, bs) - fb, pl->decode_split_blocks));
             pl->decode_ctas += static_cast<int64_t>(ns) * Hkv;
         } else {
             ns = pa::num_splits(sl[r], pl->chunk_split_blocks);
@@ -289,6 +307,31 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
                                                                    : pl->chunk_max_splits;
     pl->any_split = smax > 1;
     pl->workspace_needed = workspace_for(T, Hq, D, smax);
+    if (P > 0 && pl->num_decode_seqs > 0) {
+        // the prefix pass: all T * G query rows of each kv head against the P prefix keys,
+        // split so that the chunk kernel fills the SMs (each split at least two key tiles)
+        const int rows_per_cta = pa::chunk_rows(D, 1);
+        const int tile_blocks = (D == 128 ? 128 : 64) / bs;
+        const long long qtiles = pa::ceil_div(T * G, rows_per_cta);
+        const int pblocks = P / bs;
+        const int ptiles = pa::ceil_div(pblocks, tile_blocks);
+        if (qtiles > pa::kMaxChunkWork) return PA_ERR_UNSUPPORTED;  // the work list holds them
+        long long sp = (num_sms + qtiles * Hkv - 1) / (qtiles * Hkv);
+        sp = std::min<long long>(sp, std::max(1, ptiles / 2));
+        sp = std::min<long long>(sp, pa::kMaxChunkWork / qtiles);
+        sp = std::min<long long>(std::max<long long>(sp, 1), kMaxPrefixSplits);
+        // the prefix partials follow the split partials in the workspace
+        const size_t base = pl->workspace_needed;
+        const size_t per = prefix_part_bytes(T, Hq, D, 1);
+        if (base + per > ws) return PA_ERR_WORKSPACE;
+        sp = std::min<long long>(sp, static_cast<long long>((ws - base) / per));
+        while (sp > 1 && base + prefix_part_bytes(T, Hq, D, static_cast<int>(sp)) > ws) --sp;
+        int psb = round_up(pa::ceil_div(pblocks, static_cast<int>(sp)), tile_blocks);
+        pl->prefix_split_blocks = psb;
+        pl->prefix_splits = pa::ceil_div(pblocks, psb);
+        pl->prefix_ctas = qtiles * Hkv * pl->prefix_splits;
+        pl->workspace_needed = base + prefix_part_bytes(T, Hq, D, pl->prefix_splits);
+    }
     return PA_OK;
 }
 
@@ -480,7 +523,11 @@ int pa_attention_ex(const pa_cache* cache, const void* q, int num_q_heads,
                        cache->num_kv_heads, cache->head_size, cache->block_size,
                        max_blocks_per_seq, num_sms, workspace_bytes, opts, &pl);
     if (st != PA_OK) return st;
-    if (pl.num_chunk_seqs && cache->kv_dtype != PA_BF16) return PA_ERR_UNSUPPORTED;
+    // chunk kernels: tcgen05 for head_size 128 (bf16 or FP8 cache), mma.sync for bf16 head_size 64
+    const bool chunk_ok = cache->head_size == 128 || cache->kv_dtype == PA_BF16;
+    if (pl.num_chunk_seqs && !chunk_ok) return PA_ERR_UNSUPPORTED;
+    const bool cascade = pl.prefix_splits > 0;
+    if (cascade && !chunk_ok) return PA_ERR_UNSUPPORTED;
     if (pl.workspace_needed > workspace_bytes) return PA_ERR_WORKSPACE;
 
     pa::AttnParams p;
@@ -501,6 +548,7 @@ int pa_attention_ex(const pa_cache* cache, const void* q, int num_q_heads,
         p.split_counters = reinterpret_cast<int*>(reinterpret_cast<char*>(p.part_lse) +
                                                   align256(rows * sizeof(float)));
     }
+    p.cache = static_cast<const uint8_t*>(cache->data);
     p.k_scale = cache->k_scale;
     p.v_scale = cache->v_scale;
     p.max_blocks_per_seq = max_blocks_per_seq;
@@ -519,6 +567,23 @@ int pa_attention_ex(const pa_cache* cache, const void* q, int num_q_heads,
     p.local_chunk = opts ? opts->local_chunk : 0;
     p.lse_out = opts ? opts->lse_out : nullptr;
     p.err = device_error_ptr();
+    int prefix_row = 0;
+    if (cascade) {
+        // the shared prefix's blocks are read from the first request with queries; its split
+        // partials sit in the workspace after the split-KV partials
+        while (prefix_row < num_seqs &&
+               query_start_loc_host[prefix_row + 1] == query_start_loc_host[prefix_row])
+            ++prefix_row;
+        const int smax = pl.decode_max_splits > pl.chunk_max_splits ? pl.decode_max_splits
+                                                                     : pl.chunk_max_splits;
+        const size_t base = workspace_for(num_tokens, num_q_heads, cache->head_size, smax);
+        const size_t rows = static_cast<size_t>(pl.prefix_splits) * num_tokens * num_q_heads;
+        p.prefix_keys = opts->common_prefix_tokens;
+        p.prefix_parts = pl.prefix_splits;
+        p.prefix_o = reinterpret_cast<const float*>(static_cast<char*>(workspace) + base);
+        p.prefix_lse = reinterpret_cast<const float*>(
+            static_cast<char*>(workspace) + base + align256(rows * cache->head_size * sizeof(float)));
+    }
 
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     void* const* ev = opts ? opts->events : nullptr;
@@ -529,6 +594,48 @@ int pa_attention_ex(const pa_cache* cache, const void* q, int num_q_heads,
     if (pl.decode_max_splits > 1 || (pl.chunk_max_splits > 1 && chunk_merge_fused)) {
         e = pa::launch_zero_counters(p.split_counters, num_tokens * cache->num_kv_heads, s);
         if (e != cudaSuccess) return fail_cuda(e);
+    }
+    if (cascade) {
+        // the prefix pass: every query row of the step against the shared prefix's keys, read
+        // once per (kv head, split) instead of once per request; each split's partials go to
+        // the workspace, where the decode kernel below merges them into its rows
+        pa::AttnParams pp = p;
+        pp.prefix_launch = 1;
+        pp.prefix_row = prefix_row;
+        pp.prefix_parts = 0;
+        pp.prefix_o = nullptr;
+        pp.prefix_lse = nullptr;
+        pp.part_o = const_cast<float*>(p.prefix_o);
+        pp.part_lse = const_cast<float*>(p.prefix_lse);
+        pp.max_splits = pl.prefix_splits;
+        pp.chunk_split_blocks = pl.prefix_split_blocks;
+        pp.chunk_fused_merge = 0;
+        pp.lse_out = nullptr;
+        const int rows_per_cta = pa::chunk_rows(cache->head_size, 1);
+        const int tile_keys = cache->head_size == 128 ? 128 : 64;
+        const int qtiles = pa::ceil_div(num_tokens * pp.group, rows_per_cta);
+        pp.chunk_max_qtiles = qtiles;
+        static thread_local pa::ChunkWork pwork;
+        static thread_local std::vector<std::pair<int, uint32_t>> pitems;
+        pitems.clear();
+        for (int qt = 0; qt < qtiles; ++qt)
+            for (int sp = 0; sp < pl.prefix_splits; ++sp) {
+                const int k0 = sp * pl.prefix_split_blocks * cache->block_size;
+                const int k1 = std::min(p.prefix_keys, k0 + pl.prefix_split_blocks * cache->block_size);
+                pitems.emplace_back(pa::ceil_div(k1 - k0, tile_keys),
+                                    (static_cast<uint32_t>(qt) << 10) | (static_cast<uint32_t>(sp) << 22));
+            }
+        std::stable_sort(pitems.begin(), pitems.end(),
+                         [](const std::pair<int, uint32_t>& a, const std::pair<int, uint32_t>& b) {
+                             return a.first > b.first;
+                         });
+        pwork.count = 0;
+        for (const auto& it : pitems) pwork.item[pwork.count++] = it.second;
+        if (ev) record(ev[2], s);
+        e = pa::launch_chunk(cache->tmap, cache->tmap_blk, pp, pwork, cache->head_size,
+                             cache->kv_dtype, pl.prefix_splits, s);
+        if (e != cudaSuccess) return fail_cuda(e);
+        if (ev) record(ev[3], s);
     }
     if (pl.num_decode_seqs) {
         if (ev) record(ev[0], s);
@@ -639,6 +746,35 @@ int pa_validate_block_table(const pa_cache* cache, const int32_t* block_table,
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     cudaFreeAsync(counter, s);
     return e == cudaSuccess ? PA_OK : fail_cuda(e);
+}
+
+int pa_common_prefix_blocks(const int32_t* block_table_host, int max_blocks_per_seq,
+                            const int32_t* seq_lens_host, const int32_t* query_start_loc_host,
+                            int num_seqs, int block_size, int* num_blocks) {
+    if (!num_blocks) return PA_ERR_INVALID_ARG;
+    *num_blocks = 0;
+    if (num_seqs < 0 || max_blocks_per_seq <= 0 || block_size <= 0) return PA_ERR_INVALID_ARG;
+    if (num_seqs == 0) return PA_OK;
+    if (!block_table_host || !seq_lens_host || !query_start_loc_host) return PA_ERR_INVALID_ARG;
+    int first = -1, n = max_blocks_per_seq;
+    for (int r = 0; r < num_seqs; ++r) {
+        const int ql = query_start_loc_host[r + 1] - query_start_loc_host[r];
+        if (ql < 0 || seq_lens_host[r] < ql) return PA_ERR_METADATA;
+        if (ql == 0) continue;
+        // every query of the request must see the whole prefix
+        n = std::min(n, (seq_lens_host[r] - ql) / block_size);
+        if (first < 0) {
+            first = r;
+            continue;
+        }
+        const int32_t* a = block_table_host + static_cast<int64_t>(first) * max_blocks_per_seq;
+        const int32_t* b = block_table_host + static_cast<int64_t>(r) * max_blocks_per_seq;
+        int j = 0;
+        while (j < n && a[j] == b[j]) ++j;
+        n = j;
+    }
+    *num_blocks = first < 0 ? 0 : n;
+    return PA_OK;
 }
 
 int pa_validate_slots(const pa_cache* cache, const int32_t* slot_mapping, int num_tokens,

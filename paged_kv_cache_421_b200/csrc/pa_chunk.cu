@@ -55,35 +55,53 @@ chunk_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
         g = blockIdx.y;
     }
     if (r >= p.num_seqs || g >= p.num_kv_heads) return;
-    const int q0 = p.qsl[r];
-    const int q_len = p.qsl[r + 1] - q0;
-    if (q_len <= 0 || is_decode_kind(q_len, p.group)) return;
-    if (q0 < 0 || q0 + q_len > p.num_tokens) {  // never index q/out past num_tokens
-        if (blockIdx.x == 0 && threadIdx.x == 0) raise_error(p.err, kErrMetadata);
-        return;
+    // The request this CTA serves: one of the step's chunk-kind requests, or, in the prefix
+    // launch of a cascade call, every query row of the step over the shared prefix's keys
+    // (block-table row prefix_row), which all of them see: no causal mask.
+    const bool prefix = p.prefix_launch != 0;
+    int q0, q_len, ctx, trow;
+    if (prefix) {
+        q0 = 0;
+        q_len = p.num_tokens;
+        ctx = p.prefix_keys;
+        trow = p.prefix_row;
+        if (ctx <= 0 || trow < 0 || trow >= p.num_seqs) return;
+    } else {
+        q0 = p.qsl[r];
+        q_len = p.qsl[r + 1] - q0;
+        ctx = p.seq_lens[r];
+        trow = r;
+        if (q_len <= 0 || is_decode_kind(q_len, p.group)) return;
+        if (q0 < 0 || q0 + q_len > p.num_tokens) {  // never index q/out past num_tokens
+            if (blockIdx.x == 0 && threadIdx.x == 0) raise_error(p.err, kErrMetadata);
+            return;
+        }
     }
     const int G = p.group;
     const int rows_total = q_len * G;
     const int R0 = qt * kChunkRows;
     if (R0 >= rows_total) return;
-    const int ctx = p.seq_lens[r];
-    if (ctx > p.max_blocks_per_seq * kBlockSize || ctx < q_len) {  // never read past the table
+    if (ctx > p.max_blocks_per_seq * kBlockSize || (!prefix && ctx < q_len)) {
         if (blockIdx.x == 0 && threadIdx.x == 0) raise_error(p.err, kErrMetadata);
         return;
     }
+    // last key row R sees: bottom-right causal inside a chunk, every prefix key in a prefix launch
+    auto row_lim = [&](int R) { return prefix ? ctx - 1 : ctx - q_len + R / G; };
     const int nblocks = ceil_div(ctx, kBlockSize);
     const int nsplit = ceil_div(nblocks, p.chunk_split_blocks);
     if (split >= nsplit) return;
-    if (nsplit > 1 && split >= p.max_splits) return;
+    // results go to the split partials (several splits, or any prefix launch) or to out
+    const bool to_parts = nsplit > 1 || prefix;
+    if (to_parts && split >= p.max_splits) return;
     const int jb = split * p.chunk_split_blocks;
     const int je = min(nblocks, jb + p.chunk_split_blocks);
     const int kend = min(je * kBlockSize, ctx);  // keys of this split: [jb*16, kend)
     const int last_row = min(R0 + kChunkRows - 1, rows_total - 1);
-    const int kmax = ctx - q_len + last_row / G;   // last key any row of the tile sees
+    const int kmax = row_lim(last_row);   // last key any row of the tile sees
     // the first key any row of the CTA may see: the split's start, or (sliding window) the
     // window start of the CTA's first row, rounded down to its block
     const int key_lo = max(jb * kBlockSize,
-                           first_visible_key(ctx - q_len + R0 / G, p.window, p.local_chunk) /
+                           first_visible_key(row_lim(R0), p.window, p.local_chunk) /
                                kBlockSize * kBlockSize);
     const int key_hi = min(kend, kmax + 1);
     const int ntiles = key_hi > key_lo ? ceil_div(key_hi - key_lo, kTileKeys) : 0;
@@ -101,12 +119,12 @@ chunk_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
     // rows A = R0 + 16 warp + gq and B = A + 8; invalid rows get a harmless visibility range
     const int rA = R0 + 16 * warp + gq, rB = rA + 8;
     const bool vA = rA < rows_total, vB = rB < rows_total;
-    const int limA = vA ? ctx - q_len + rA / G : kmax;
-    const int limB = vB ? ctx - q_len + rB / G : kmax;
+    const int limA = vA ? row_lim(rA) : kmax;
+    const int limB = vB ? row_lim(rB) : kmax;
     const int loA = first_visible_key(limA, p.window, p.local_chunk);
     const int loB = first_visible_key(limB, p.window, p.local_chunk);
     const int wlast = min(R0 + 16 * warp + 15, rows_total - 1);
-    const int warp_kmax = ctx - q_len + wlast / G;
+    const int warp_kmax = row_lim(wlast);
 
     uint32_t qa[C::kKSteps][4];
     {
@@ -132,7 +150,7 @@ chunk_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
         mbar_init(smem_u32(&bars[1]), 1);
     }
     for (int k = tid; k < min(je - jb, kMaxIds); k += 128) {
-        int blk = p.block_table[static_cast<int64_t>(r) * p.max_blocks_per_seq + jb + k];
+        int blk = p.block_table[static_cast<int64_t>(trow) * p.max_blocks_per_seq + jb + k];
         if (blk < 0 || blk >= p.num_blocks) {
             raise_error(err, kErrBadBlockId);
             blk = 0;
@@ -155,7 +173,7 @@ chunk_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
             if (j0 + b - jb < kMaxIds) {
                 blk = ids[j0 + b - jb];
             } else {
-                blk = p.block_table[static_cast<int64_t>(r) * p.max_blocks_per_seq + j0 + b];
+                blk = p.block_table[static_cast<int64_t>(trow) * p.max_blocks_per_seq + j0 + b];
                 if (blk < 0 || blk >= p.num_blocks) {
                     raise_error(err, kErrBadBlockId);
                     blk = 0;
@@ -302,7 +320,7 @@ chunk_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
     lA += __shfl_xor_sync(kFull, lA, 2);
     lB += __shfl_xor_sync(kFull, lB, 1);
     lB += __shfl_xor_sync(kFull, lB, 2);
-    const bool direct = nsplit == 1;
+    const bool direct = !to_parts;
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
         const int row = half ? rB : rA;
@@ -351,8 +369,8 @@ cudaError_t launch_chunk_t(const CUtensorMap& tmap, const AttnParams& p, const C
 cudaError_t launch_chunk(const CUtensorMap& tmap, const CUtensorMap& tmap_blk, const AttnParams& p,
                          const ChunkWork& work, int head_size, int kv_dtype, int max_splits,
                          cudaStream_t stream) {
+    if (head_size == 128) return launch_chunk_tc(tmap, tmap_blk, p, work, kv_dtype, max_splits, stream);
     if (kv_dtype != PA_BF16) return cudaErrorInvalidValue;
-    if (head_size == 128) return launch_chunk_tc(tmap_blk, p, work, max_splits, stream);
     if (head_size == 64) return launch_chunk_t<64>(tmap, p, work, max_splits, stream);
     return cudaErrorInvalidValue;
 }

@@ -1,5 +1,5 @@
 // Chunked-prefill paged attention on the 5th-generation tensor cores (tcgen05, sm_100a),
-// head_size 128, bf16 cache.
+// head_size 128, bf16 or FP8 E4M3 cache.
 //
 // What it computes is the chunk kernel's: exact softmax attention of a request's query
 // rows -- (token, head of the GQA group) pairs, token-major -- over its paged keys, with the
@@ -25,6 +25,16 @@
 // denominator share it, so results are exact).  Full/empty mbarriers and tcgen05.commit
 // replace CTA barriers inside the loop.  Every wait is bounded: on a timeout each role
 // records the error and stops, and the CTA frees its TMEM and returns.
+//
+// FP8 E4M3 cache ("vLLM: from KV Cache to high-throughput serving", article 6 outline names
+// the format).  The same schedule runs on kind::f8f6f4 MMAs with both operands E4M3, straight
+// from the cache bytes: a K tile is eight 2 KB block tiles [16 keys][128 B] (2-D TMA, 128-byte
+// swizzle: the K-major B operand of S = Q K^T), a V tile eight dim-major block tiles [128 dims]
+// [16 keys] (bulk copies of the stored bytes: K-major B operand of O += P V without swizzle,
+// 16-key core matrices 2 KB apart).  Q and P keep bf16-level precision as two E4M3 terms each
+// (x ~ e4m3(x) + e4m3(x - e4m3(x)), Q after scaling each row by a power of two), and every
+// product is issued once per term.  The K scale and the row's power of two multiply the
+// scores, the V scale the output.
 #include "pa_internal.h"
 
 namespace pa {
@@ -47,6 +57,12 @@ constexpr int kBlockTile = kBlockSize * 2 * kHalfRows;  // 4 KB: one block's 16 
 constexpr int kKBytes = kTileBlocks * kBlockTile;       // 32 KB per K or V tile
 constexpr int kKSlots = 2, kVSlots = 2;
 constexpr int kSmemBytes = kQTiles * kQBytes + (kKSlots + kVSlots) * kKBytes + 1024;  // 193 KB
+// FP8 cache: 2 KB block tiles, 16 KB K or V tiles; each q-tile holds two E4M3 terms of Q,
+// [128 rows][128 B] each (one 128-byte swizzle atom per row), in the same 32 KB as bf16 Q.
+constexpr int kBlockTile8 = kBlockSize * kD;              // 2 KB
+constexpr int kKBytes8 = kTileBlocks * kBlockTile8;       // 16 KB per K or V tile
+constexpr int kQTerm8 = kRows * 128;                      // 16 KB per E4M3 term of a q-tile
+constexpr int kSmemBytes8 = kQTiles * kQBytes + (kKSlots + kVSlots) * kKBytes8 + 1024;  // 129 KB
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColO = 128;                  // q-tile q: S/P [256q, 256q+128), O after it
 constexpr int kMaxIds = 1024;                    // block ids staged in shared memory
@@ -59,6 +75,10 @@ constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) |
 constexpr uint32_t kIdescPV = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
                               (static_cast<uint32_t>(kD >> 3) << 17) |
                               (static_cast<uint32_t>(kRows >> 4) << 24);
+// kind::f8f6f4: fp32 accumulate, E4M3 A and B (format 0), both K-major, M = 128, N = 128 (keys
+// for S = Q K^T, dims for O = P V).
+constexpr uint32_t kIdesc8 = (1u << 4) | (static_cast<uint32_t>(128 >> 3) << 17) |
+                             (static_cast<uint32_t>(kRows >> 4) << 24);
 
 // Shared-memory matrix descriptor: start address, leading / stride byte offsets (16-byte
 // units), descriptor version 1, 128-byte swizzle.
@@ -82,6 +102,40 @@ __device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, 
         "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
         "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc));
+}
+
+// Shared-memory matrix descriptor without swizzle (canonical K-major core matrices of 8 rows
+// x 16 bytes): lbo = bytes between core matrices adjacent along K, sbo = along M/N.
+__device__ __forceinline__ uint64_t smem_desc_noswizzle(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    return static_cast<uint64_t>((addr >> 4) & 0x3FFFu) |
+           (static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16) |
+           (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+
+__device__ __forceinline__ void mma_ss8(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                        uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+        "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+
+__device__ __forceinline__ void mma_ts8(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                        uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+        "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc));
+}
+
+// Bulk copy of `bytes` contiguous bytes global -> shared (no tensor map), completion counted
+// on an mbarrier.  Both addresses 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
+        : "memory");
 }
 
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
@@ -167,6 +221,25 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
         : "memory");
 }
 
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+        : "memory");
+}
+
+// Two probabilities -> their two-term E4M3 split: hi = e4m3(a) and lo = e4m3(a - hi) (the
+// remainder is exact in fp32), two 8-bit codes each with a.x in the low byte.
+__device__ __forceinline__ void split_e4m3x2(float2 a, uint32_t& hi, uint32_t& lo) {
+    const __nv_fp8x2_storage_t c1 = __nv_cvt_float2_to_fp8x2(a, __NV_SATFINITE, __NV_E4M3);
+    const __half2 h = __half2(__nv_cvt_fp8x2_to_halfraw2(c1, __NV_E4M3));
+    const float2 back = __half22float2(h);
+    const __nv_fp8x2_storage_t c2 = __nv_cvt_float2_to_fp8x2(
+        make_float2(a.x - back.x, a.y - back.y), __NV_SATFINITE, __NV_E4M3);
+    hi = c1;
+    lo = c2;
+}
+
 // One (block, K|V, kv head) tile through the 4-D view: box (64, 8, 2, 2) at 8-row group `grp`.
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                             int grp) {
@@ -200,9 +273,14 @@ constexpr int kMergeRows = 8;            // rows a warp merges with all loads in
 static_assert(8 * 32 * kRegsSoftmax + 4 * 32 * kRegsProducer <= kThreads * 168,
               "register split exceeds the launch's registers");
 
+// tmap: bf16 cache -- the 4-D whole-tile view of the pool; FP8 cache -- the 2-D view (rows of
+// 128 bytes, 16-row boxes, 128-byte swizzle).
+template <bool FP8>
 __global__ void __launch_bounds__(kThreads, 1)
-chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p,
+chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
                 const __grid_constant__ ChunkWork work) {
+    constexpr int kSlotBytes = FP8 ? kKBytes8 : kKBytes;   // one K or V tile in shared memory
+    constexpr int kTileLoadBytes = FP8 ? kBlockTile8 : kBlockTile;  // one block's tile
     pdl_trigger();
     pdl_wait();
     int* err = p.err;
@@ -222,35 +300,53 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
         g = blockIdx.y;
     }
     if (r >= p.num_seqs || g >= p.num_kv_heads) return;
-    const int q0 = p.qsl[r];
-    const int q_len = p.qsl[r + 1] - q0;
-    if (q_len <= 0 || is_decode_kind(q_len, p.group)) return;
-    if (q0 < 0 || q0 + q_len > p.num_tokens) {
-        if (blockIdx.x == 0 && threadIdx.x == 0) raise_error(err, kErrMetadata);
-        return;
+    // The request this CTA serves: one of the step's chunk-kind requests, or, in the prefix
+    // launch of a cascade call, every query row of the step over the shared prefix's keys
+    // (block-table row prefix_row), which all of them see: no causal mask.
+    const bool prefix = p.prefix_launch != 0;
+    int q0, q_len, ctx, trow;
+    if (prefix) {
+        q0 = 0;
+        q_len = p.num_tokens;
+        ctx = p.prefix_keys;
+        trow = p.prefix_row;
+        if (ctx <= 0 || trow < 0 || trow >= p.num_seqs) return;
+    } else {
+        q0 = p.qsl[r];
+        q_len = p.qsl[r + 1] - q0;
+        ctx = p.seq_lens[r];
+        trow = r;
+        if (q_len <= 0 || is_decode_kind(q_len, p.group)) return;
+        if (q0 < 0 || q0 + q_len > p.num_tokens) {
+            if (blockIdx.x == 0 && threadIdx.x == 0) raise_error(err, kErrMetadata);
+            return;
+        }
     }
     const int G = p.group;
     const int rows_total = q_len * G;
     const int R0 = qt * kRows * kQTiles;
     if (R0 >= rows_total) return;
-    const int ctx = p.seq_lens[r];
-    if (ctx > p.max_blocks_per_seq * kBlockSize || ctx < q_len) {
+    if (ctx > p.max_blocks_per_seq * kBlockSize || (!prefix && ctx < q_len)) {
         if (blockIdx.x == 0 && threadIdx.x == 0) raise_error(err, kErrMetadata);
         return;
     }
+    // last key row R sees: bottom-right causal inside a chunk, every prefix key in a prefix launch
+    auto row_lim = [&](int R) { return prefix ? ctx - 1 : ctx - q_len + R / G; };
     const int nblocks = ceil_div(ctx, kBlockSize);
     const int nsplit = ceil_div(nblocks, p.chunk_split_blocks);
     if (split >= nsplit) return;
-    if (nsplit > 1 && split >= p.max_splits) return;
+    // results go to the split partials (several splits, or any prefix launch) or to out
+    const bool to_parts = nsplit > 1 || prefix;
+    if (to_parts && split >= p.max_splits) return;
     const int jb = split * p.chunk_split_blocks;
     const int je = min(nblocks, jb + p.chunk_split_blocks);
     const int kend = min(je * kBlockSize, ctx);
     const int last_row = min(R0 + kQTiles * kRows - 1, rows_total - 1);
-    const int kmax = ctx - q_len + last_row / G;
+    const int kmax = row_lim(last_row);
     // the first key any row of the CTA may see: the split's start, or (sliding window) the
     // window start of the CTA's first row, rounded down to its block
     const int key_lo = max(jb * kBlockSize,
-                           first_visible_key(ctx - q_len + R0 / G, p.window, p.local_chunk) /
+                           first_visible_key(row_lim(R0), p.window, p.local_chunk) /
                                kBlockSize * kBlockSize);
     const int key_hi = min(kend, kmax + 1);
     const int ntiles = key_hi > key_lo ? ceil_div(key_hi - key_lo, kKeys) : 0;
@@ -264,11 +360,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
     __shared__ uint64_t bar_q;                             // Q staged by the softmax warps
     __shared__ uint32_t tmem_holder;
     __shared__ int ids[kMaxIds];  // physical ids of the split's first kMaxIds logical blocks
+    __shared__ float qfac[FP8 ? kQTiles * kRows : 1];  // FP8: each row's 2^-e (Q was scaled by 2^e)
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const uint32_t q_s = smem_u32(smem);                      // [q-tile][32 KB]
-    const uint32_t k_s = q_s + kQTiles * kQBytes;             // [K slot][32 KB]
-    const uint32_t v_s = k_s + kKSlots * kKBytes;             // [V slot][32 KB]
+    const uint32_t k_s = q_s + kQTiles * kQBytes;             // [K slot][kSlotBytes]
+    const uint32_t v_s = k_s + kKSlots * kSlotBytes;          // [V slot][kSlotBytes]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -280,7 +377,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     if (tid == 0) {
-        prefetch_tensor_map(&tmap_blk);
+        prefetch_tensor_map(&tmap);
         for (int i = 0; i < kKSlots; ++i) {
             mbar_init(smem_u32(&bar_kf[i]), 1);
             mbar_init(smem_u32(&bar_ke[i]), 1);
@@ -298,7 +395,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
         fence_barrier_init();
     }
     for (int k = tid; k < min(je - jb, kMaxIds); k += kThreads) {
-        int blk = p.block_table[static_cast<int64_t>(r) * p.max_blocks_per_seq + jb + k];
+        int blk = p.block_table[static_cast<int64_t>(trow) * p.max_blocks_per_seq + jb + k];
         if (blk < 0 || blk >= p.num_blocks) {
             raise_error(err, kErrBadBlockId);
             blk = 0;
@@ -321,10 +418,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
             auto load = [&](int t, int which) {
                 const int st = t & 1;
                 const uint32_t bar = smem_u32(which ? &bar_vf[st] : &bar_kf[st]);
-                const uint32_t dst = (which ? v_s : k_s) + st * kKBytes;
+                const uint32_t dst = (which ? v_s : k_s) + st * kSlotBytes;
                 const int j0 = key_lo / kBlockSize + t * kTileBlocks;
                 const int nload = min(kTileBlocks, je - j0);
-                if (lane == 0) mbar_arrive_expect_tx(bar, nload * kBlockTile);
+                if (lane == 0) mbar_arrive_expect_tx(bar, nload * kTileLoadBytes);
                 __syncwarp();
                 if (lane < nload) {
                     const int b2 = lane;
@@ -332,14 +429,23 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
                     if (j0 + b2 - jb < kMaxIds) {
                         blk = ids[j0 + b2 - jb];
                     } else {
-                        blk = p.block_table[static_cast<int64_t>(r) * p.max_blocks_per_seq + j0 + b2];
+                        blk = p.block_table[static_cast<int64_t>(trow) * p.max_blocks_per_seq + j0 + b2];
                         if (blk < 0 || blk >= p.num_blocks) {
                             raise_error(err, kErrBadBlockId);
                             blk = 0;
                         }
                     }
                     const int row = blk * kv_rows_per_block + (which * p.num_kv_heads + g) * kBlockSize;
-                    tma_load_4d(dst + b2 * kBlockTile, &tmap_blk, bar, row / 8);
+                    if constexpr (!FP8) {
+                        tma_load_4d(dst + b2 * kBlockTile, &tmap, bar, row / 8);
+                    } else if (which == 0) {
+                        // K: 16 rows of 128 bytes, swizzled into the operand layout
+                        tma_load_2d(dst + b2 * kBlockTile8, &tmap, bar, 0, row);
+                    } else {
+                        // V: the stored dim-major bytes as they are
+                        bulk_load(dst + b2 * kBlockTile8,
+                                  p.cache + static_cast<int64_t>(row) * kD, kBlockTile8, bar);
+                    }
                 }
                 __syncwarp();
             };
@@ -366,23 +472,46 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
             // ================= MMA issuer
             if (lane == 0 && ntiles > 0) {
                 auto qk = [&](int q, int t) {  // S_q = Q_q K_t^T
-                    const uint32_t ks = k_s + (t & 1) * kKBytes;
+                    const uint32_t ks = k_s + (t & 1) * kSlotBytes;
+                    if constexpr (!FP8) {
 #pragma unroll
-                    for (int k = 0; k < kD / 16; ++k) {
-                        const uint32_t off = q * kQBytes + (k >> 2) * kQHalf + (k & 3) * 32;
-                        const uint32_t koff = (k >> 2) * kAtom + (k & 3) * 32;
-                        mma_ss(tmem + q * 256, smem_desc(q_s + off, 16, 1024),
-                               smem_desc(ks + koff, 16, kGroupStride), kIdescQK, k > 0);
+                        for (int k = 0; k < kD / 16; ++k) {
+                            const uint32_t off = q * kQBytes + (k >> 2) * kQHalf + (k & 3) * 32;
+                            const uint32_t koff = (k >> 2) * kAtom + (k & 3) * 32;
+                            mma_ss(tmem + q * 256, smem_desc(q_s + off, 16, 1024),
+                                   smem_desc(ks + koff, 16, kGroupStride), kIdescQK, k > 0);
+                        }
+                    } else {
+                        // 32 dims per MMA (32 bytes of each 128-byte row); both Q terms
+#pragma unroll
+                        for (int k = 0; k < kD / 32; ++k)
+#pragma unroll
+                            for (int term = 0; term < 2; ++term)
+                                mma_ss8(tmem + q * 256,
+                                        smem_desc(q_s + q * kQBytes + term * kQTerm8 + k * 32, 16, 1024),
+                                        smem_desc(ks + k * 32, 16, 1024), kIdesc8, (k | term) > 0);
                     }
                     mma_commit(smem_u32(&bar_sf[q]));
                 };
                 auto pv = [&](int q, int t) {  // O_q += P_q V_t (P from TMEM)
-                    const uint32_t vs = v_s + (t & 1) * kKBytes;
+                    const uint32_t vs = v_s + (t & 1) * kSlotBytes;
+                    if constexpr (!FP8) {
 #pragma unroll
-                    for (int j = 0; j < kKeys / 16; ++j)
-                        mma_ts(tmem + q * 256 + kColO, tmem + q * 256 + 8 * j,
-                               smem_desc(vs + j * kBlockTile, kAtom, kGroupStride), kIdescPV,
-                               (t > 0 || j > 0) ? 1u : 0u);
+                        for (int j = 0; j < kKeys / 16; ++j)
+                            mma_ts(tmem + q * 256 + kColO, tmem + q * 256 + 8 * j,
+                                   smem_desc(vs + j * kBlockTile, kAtom, kGroupStride), kIdescPV,
+                                   (t > 0 || j > 0) ? 1u : 0u);
+                    } else {
+                        // 32 keys per MMA: P's two terms (columns [0, 32) and [32, 64), four
+                        // E4M3 codes per column) against block tiles 2j and 2j + 1
+#pragma unroll
+                        for (int j = 0; j < kKeys / 32; ++j)
+#pragma unroll
+                            for (int term = 0; term < 2; ++term)
+                                mma_ts8(tmem + q * 256 + kColO, tmem + q * 256 + 32 * term + 8 * j,
+                                        smem_desc_noswizzle(vs + 2 * j * kBlockTile8, kBlockTile8, 128),
+                                        kIdesc8, (t > 0 || j > 0 || term > 0) ? 1u : 0u);
+                    }
                     mma_commit(smem_u32(&bar_o[q]));
                 };
                 if (mbar_wait(smem_u32(&bar_q), 0, kWaitLimitNs, err) &&
@@ -419,7 +548,63 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
         // Q tiles -> shared memory in the swizzled K-major layout [q-tile][half][row][128 B],
         // by the softmax warps while the producer already fetches the first K / V tiles; every
         // load of a thread is issued before its first store, so their latencies overlap
-        {
+        if constexpr (FP8) {
+            // FP8 cache: each row is scaled by 2^e (its max |q| to between 112 and 224) and
+            // split into two E4M3 terms, stored [q-tile][term][row][128 B] (swizzled).  Eight
+            // threads share a row, 16 dims each; 32 rows per pass, eight passes.
+            constexpr int kPasses = kQTiles * kRows / 32;
+            const int sub = tid & 7;
+            uint4 v[kPasses][2];
+#pragma unroll
+            for (int i = 0; i < kPasses; ++i) {
+                const int rr = (tid >> 3) + 32 * i, Rr = R0 + rr;
+                v[i][0] = v[i][1] = make_uint4(0, 0, 0, 0);
+                if (Rr < rows_total) {
+                    const uint4* src = reinterpret_cast<const uint4*>(
+                        p.q + (static_cast<int64_t>(q0 + Rr / G) * p.num_q_heads + g * G + Rr % G) * kD +
+                        sub * 16);
+                    v[i][0] = __ldg(src);
+                    v[i][1] = __ldg(src + 1);
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < kPasses; ++i) {
+                const int rr = (tid >> 3) + 32 * i;
+                const uint32_t w[8] = {v[i][0].x, v[i][0].y, v[i][0].z, v[i][0].w,
+                                       v[i][1].x, v[i][1].y, v[i][1].z, v[i][1].w};
+                float x[16];
+                float mx = 0.f;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    x[2 * j] = __uint_as_float(w[j] << 16);
+                    x[2 * j + 1] = __uint_as_float(w[j] & 0xffff0000u);
+                    mx = fmax3(mx, fabsf(x[2 * j]), fabsf(x[2 * j + 1]));
+                }
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                int e = 0;
+                if (mx > 0.f) e = min(max(static_cast<int>(floorf(log2f(448.f / mx))) - 1, -120), 120);
+                const float up = ldexpf(1.f, e);
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    uint32_t h0, l0, h1, l1;
+                    split_e4m3x2(make_float2(x[4 * j] * up, x[4 * j + 1] * up), h0, l0);
+                    split_e4m3x2(make_float2(x[4 * j + 2] * up, x[4 * j + 3] * up), h1, l1);
+                    hi[j] = h0 | (h1 << 16);
+                    lo[j] = l0 | (l1 << 16);
+                }
+                uint8_t* base = smem + (rr >> 7) * kQBytes;
+                const uint32_t off = sw128(rr & (kRows - 1), sub);
+                *reinterpret_cast<uint4*>(base + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4*>(base + kQTerm8 + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                if (sub == 0) qfac[rr] = ldexpf(1.f, -e);
+            }
+            fence_proxy_async();  // generic-proxy stores, before the tensor core reads them
+            mbar_arrive(smem_u32(&bar_q));
+            named_barrier_sync(1, kQLoaders);  // every row's factor is in qfac
+        } else {
             constexpr int kVecs = kQTiles * kRows * (kD / 8), kPer = kVecs / kQLoaders;
             uint4 v[kPer];
 #pragma unroll
@@ -449,15 +634,18 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
             const int row = tid & (kRows - 1);
             const int R = R0 + q * kRows + row;
             const bool valid = R < rows_total;
-            const int lim = valid ? ctx - q_len + R / G : kmax;
-            const int first_lim = ctx - q_len + (R0 + q * kRows) / G;  // smallest limit of the q-tile
+            const int lim = valid ? row_lim(R) : kmax;
+            const int first_lim = row_lim(R0 + q * kRows);  // smallest limit of the q-tile
             const int lo = first_visible_key(lim, p.window, p.local_chunk);  // this row's first key
             const int last_lo = first_visible_key(  // the latest first key of the q-tile
-                ctx - q_len + min(R0 + q * kRows + kRows - 1, rows_total - 1) / G, p.window,
+                row_lim(min(R0 + q * kRows + kRows - 1, rows_total - 1)), p.window,
                 p.local_chunk);
             const uint32_t tq = tmem + q * 256;
             const uint32_t tmem_lane = tq + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-            const float sl = p.scale_log2;
+            // score multiplier: softmax scale in log2 units; FP8: times the K scale and this row's
+            // 2^-e (the scores come from Q 2^e and the K codes)
+            const float sl = FP8 ? p.scale_log2 * p.k_scale[g] * qfac[q * kRows + row]
+                                 : p.scale_log2;
             float m_used = -INFINITY, l = 0.f;
             for (int kt = 0; kt < ntiles; ++kt) {
                 const int key0 = key_lo + kt * kKeys;
@@ -524,15 +712,38 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
                 float2 sp[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
                 for (int c = 0; c < kKeys / 32; ++c) {
-                    uint32_t packed[16];
+                    if constexpr (!FP8) {
+                        uint32_t packed[16];
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float2 x = ffma2(make_float2(sv[32 * c + 2 * i], sv[32 * c + 2 * i + 1]), sl2, nr2);
-                        const float2 a = make_float2(ex2(x.x), ex2(x.y));
-                        sp[i & 1] = fadd2(sp[i & 1], a);
-                        packed[i] = pack_bf16(a.x, a.y);
+                        for (int i = 0; i < 16; ++i) {
+                            const float2 x = ffma2(make_float2(sv[32 * c + 2 * i], sv[32 * c + 2 * i + 1]), sl2, nr2);
+                            const float2 a = make_float2(ex2(x.x), ex2(x.y));
+                            sp[i & 1] = fadd2(sp[i & 1], a);
+                            packed[i] = pack_bf16(a.x, a.y);
+                        }
+                        tmem_st16(tmem_lane + 16 * c, packed);
+                    } else {
+                        // two E4M3 terms of P, four keys per 32-bit column: the first term in
+                        // columns [0, 32), the second in [32, 64)
+                        uint32_t hi[8], lo[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const int k0 = 32 * c + 4 * i;
+                            const float2 x0 = ffma2(make_float2(sv[k0], sv[k0 + 1]), sl2, nr2);
+                            const float2 x1 = ffma2(make_float2(sv[k0 + 2], sv[k0 + 3]), sl2, nr2);
+                            const float2 a0 = make_float2(ex2(x0.x), ex2(x0.y));
+                            const float2 a1 = make_float2(ex2(x1.x), ex2(x1.y));
+                            sp[0] = fadd2(sp[0], a0);
+                            sp[1] = fadd2(sp[1], a1);
+                            uint32_t h0, l0, h1, l1;
+                            split_e4m3x2(a0, h0, l0);
+                            split_e4m3x2(a1, h1, l1);
+                            hi[i] = h0 | (h1 << 16);
+                            lo[i] = l0 | (l1 << 16);
+                        }
+                        tmem_st8(tmem_lane + 8 * c, hi);
+                        tmem_st8(tmem_lane + 32 + 8 * c, lo);
                     }
-                    tmem_st16(tmem_lane + 16 * c, packed);
                 }
                 l += (sp[0].x + sp[0].y) + (sp[1].x + sp[1].y);
                 tmem_wait_st();
@@ -545,13 +756,36 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
                         ok = false;
                         break;
                     }
-                    uint8_t* vg = smem + kQTiles * kQBytes + (kKSlots + vslot) * kKBytes;
+                    uint8_t* vg = smem + kQTiles * kQBytes + (kKSlots + vslot) * kSlotBytes;
                     const int nvalid = kend - key0;
-                    for (int idx = row; idx < (kKeys - nvalid) * 2 * 8; idx += kRows) {
-                        const int kk = nvalid + idx / 16, c = idx % 16;
-                        *reinterpret_cast<uint4*>(vg + (kk >> 3) * kGroupStride + (c >> 3) * kAtom +
-                                              (kk & 7) * kHalfRows + (c & 7) * 16) =
-                            make_uint4(0, 0, 0, 0);
+                    if constexpr (!FP8) {
+                        for (int idx = row; idx < (kKeys - nvalid) * 2 * 8; idx += kRows) {
+                            const int kk = nvalid + idx / 16, c = idx % 16;
+                            *reinterpret_cast<uint4*>(vg + (kk >> 3) * kGroupStride + (c >> 3) * kAtom +
+                                                  (kk & 7) * kHalfRows + (c & 7) * 16) =
+                                make_uint4(0, 0, 0, 0);
+                        }
+                    } else {
+                        // dim-major block tiles: in the partly valid block, thread d clears bytes
+                        // o0..15 of dim row d; the block tiles after it (never loaded: stale
+                        // bytes, maybe E4M3 NaN codes) are zeroed whole
+                        const int bv = nvalid / kBlockSize, o0 = nvalid % kBlockSize;
+                        if (o0) {
+                            uint4* rp = reinterpret_cast<uint4*>(vg + bv * kBlockTile8 + row * 16);
+                            uint4 x = *rp;
+                            uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const int keep = min(max(o0 - 4 * j, 0), 4);  // valid bytes of word j
+                                w[j] = keep == 4 ? w[j] : (w[j] & ((1u << (8 * keep)) - 1u));
+                            }
+                            *rp = make_uint4(w[0], w[1], w[2], w[3]);
+                        }
+                        const int first_zero = bv + (o0 ? 1 : 0);
+                        for (int idx = row; idx < (kTileBlocks - first_zero) * (kBlockTile8 / 16);
+                             idx += kRows)
+                            *reinterpret_cast<uint4*>(vg + first_zero * kBlockTile8 + idx * 16) =
+                                make_uint4(0, 0, 0, 0);
                     }
                     fence_proxy_async();
                 }
@@ -565,11 +799,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
             // tcgen05.ld is warp-collective: the whole warp loads (or none of it)
             const bool all_ok = __all_sync(0xffffffffu, ok);
             const bool have = all_ok && ntiles > 0;
-            const float inv = l > 0.f ? 1.f / l : 0.f;
-            if (all_ok && valid && (nsplit > 1 || p.lse_out)) {
+            // FP8: the V codes were multiplied in unscaled; the V scale returns here
+            const float inv = l > 0.f ? (FP8 ? p.v_scale[g] : 1.f) / l : 0.f;
+            if (all_ok && valid && (to_parts || p.lse_out)) {
                 const int t = q0 + R / G, h = g * G + R % G;
                 const float lse2 = l > 0.f ? m_used + __log2f(l) : -INFINITY;
-                if (nsplit > 1)
+                if (to_parts)
                     p.part_lse[(static_cast<int64_t>(split) * p.num_tokens + t) * p.num_q_heads + h] = lse2;
                 else
                     p.lse_out[static_cast<int64_t>(t) * p.num_q_heads + h] = lse2 * kLn2;
@@ -605,7 +840,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
                         const int Rr = row_base + rl;
                         if (Rr < rows_total) {
                             const int t = q0 + Rr / G, h = g * G + Rr % G;
-                            float* dst = nsplit == 1
+                            float* dst = !to_parts
                                              ? p.out + (static_cast<int64_t>(t) * p.num_q_heads + h) * kD
                                              : p.part_o + ((static_cast<int64_t>(split) * p.num_tokens + t) *
                                                                p.num_q_heads + h) * kD;
@@ -617,7 +852,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
                 }
             }
         }
-        if (nsplit > 1 && p.chunk_fused_merge) {
+        if (nsplit > 1 && p.chunk_fused_merge && !prefix) {
             // ---- split merge: the last CTA of this (q-tile pair, kv head) to finish merges
             // every split's (O_s, lse_s): out = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M),
             // M = max_s lse_s (at most kMaxFusedSplits splits; the host launches the reduce
@@ -704,20 +939,30 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap_blk, const AttnParams p
                      : "memory");
 }
 
-}  // namespace
-
-cudaError_t launch_chunk_tc(const CUtensorMap& tmap_blk, const AttnParams& p, const ChunkWork& work,
-                            int max_splits, cudaStream_t stream) {
+template <bool FP8>
+cudaError_t launch_chunk_tc_t(const CUtensorMap& tmap, const AttnParams& p, const ChunkWork& work,
+                              int max_splits, cudaStream_t stream) {
+    constexpr int smem = FP8 ? kSmemBytes8 : kSmemBytes;
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        cudaError_t e = cudaFuncSetAttribute(chunk_tc_kernel<FP8>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
     const dim3 grid = work.count > 0 ? dim3(p.num_kv_heads, work.count, 1)
                                      : dim3(p.chunk_max_qtiles * max_splits, p.num_kv_heads, p.num_seqs);
-    return launch_pdl(chunk_tc_kernel, grid, dim3(kThreads), kSmemBytes, stream, tmap_blk, p, work);
+    return launch_pdl(chunk_tc_kernel<FP8>, grid, dim3(kThreads), smem, stream, tmap, p, work);
+}
+
+}  // namespace
+
+// bf16 cache: the 4-D whole-tile view; FP8: the 2-D view of the pool.
+cudaError_t launch_chunk_tc(const CUtensorMap& tmap, const CUtensorMap& tmap_blk,
+                            const AttnParams& p, const ChunkWork& work, int kv_dtype,
+                            int max_splits, cudaStream_t stream) {
+    if (kv_dtype == PA_FP8_E4M3) return launch_chunk_tc_t<true>(tmap, p, work, max_splits, stream);
+    return launch_chunk_tc_t<false>(tmap_blk, p, work, max_splits, stream);
 }
 
 }  // namespace pa

@@ -78,10 +78,18 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
         if (split == 0 && threadIdx.x == 0) raise_error(p.err, kErrMetadata);
         return;
     }
-    int ctx = p.seq_lens[r];
-    if (ctx > p.max_blocks_per_seq * kBlockSize) {  // never read past the table row
+    // With a shared prefix (cascade attention) this launch sees only the keys after it: the
+    // request's remaining blocks, from table entry `skip` on, as a context of its own; the
+    // prefix's partials are merged in at the end.
+    const int skip = p.prefix_keys / kBlockSize;
+    int ctx = p.seq_lens[r] - p.prefix_keys;
+    if (ctx < (p.prefix_keys ? q_len : 0)) {  // the host checked seq_len - q_len >= prefix
         if (split == 0 && threadIdx.x == 0) raise_error(p.err, kErrMetadata);
-        ctx = p.max_blocks_per_seq * kBlockSize;
+        return;
+    }
+    if (ctx > (p.max_blocks_per_seq - skip) * kBlockSize) {  // never read past the table row
+        if (split == 0 && threadIdx.x == 0) raise_error(p.err, kErrMetadata);
+        ctx = (p.max_blocks_per_seq - skip) * kBlockSize;
     }
     const int nblocks = ceil_div(ctx, kBlockSize);
     // with a window or local chunks the splits cover only the blocks the first row may see;
@@ -206,7 +214,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
         const int rn = min(kIdsPerRound, je - rb);
         __syncthreads();  // every warp reaches this once per round, even after an error
         for (int k = tid; k < rn; k += NW * 32) {
-            int b = p.block_table[static_cast<int64_t>(r) * p.max_blocks_per_seq + rb + k];
+            int b = p.block_table[static_cast<int64_t>(r) * p.max_blocks_per_seq + skip + rb + k];
             if (b < 0 || b >= p.num_blocks) {
                 raise_error(p.err, kErrBadBlockId);
                 b = 0;
@@ -465,14 +473,32 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
                 acc += red_o[(w * D + d) * 8 + n] * e;
             }
         }
-        const float val = L > 0.f ? acc / L * vscale : 0.f;
+        float val = L > 0.f ? acc / L * vscale : 0.f;
         const int t = q0 + n / p.group;
         const int h = g * p.group + n % p.group;
         if (direct) {
-            p.out[(static_cast<int64_t>(t) * p.num_q_heads + h) * D + d] = val;
-            if (d == 0 && p.lse_out)
-                p.lse_out[static_cast<int64_t>(t) * p.num_q_heads + h] =
-                    L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
+            const int64_t row = static_cast<int64_t>(t) * p.num_q_heads + h;
+            float lse2 = L > 0.f ? M + __log2f(L) : -INFINITY;
+            if (p.prefix_parts > 0) {
+                // cascade: merge the shared prefix's partials (normalised, log2 LSEs) with this
+                // row's suffix result: out = sum_k 2^(lse_k - X) O_k / sum_k 2^(lse_k - X)
+                float X = lse2;
+                for (int k = 0; k < p.prefix_parts; ++k) X = fmaxf(X, __ldcg(p.prefix_lse + k * stride + row));
+                float W = 0.f, a = 0.f;
+                if (X != -INFINITY) {
+                    W = fast_exp2(lse2 - X);
+                    a = W * val;
+                    for (int k = 0; k < p.prefix_parts; ++k) {
+                        const float w = fast_exp2(__ldcg(p.prefix_lse + k * stride + row) - X);
+                        W += w;
+                        a += w * __ldcg(p.prefix_o + (k * stride + row) * D + d);
+                    }
+                }
+                val = W > 0.f ? a / W : 0.f;
+                lse2 = W > 0.f ? X + __log2f(W) : -INFINITY;
+            }
+            p.out[row * D + d] = val;
+            if (d == 0 && p.lse_out) p.lse_out[row] = lse2 * kLn2;
         } else {
             const int64_t prow = split * stride + static_cast<int64_t>(t) * p.num_q_heads + h;
             p.part_o[prow * D + d] = val;
@@ -491,19 +517,25 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    float* s_w = reinterpret_cast<float*>(smem);  // [rows][nsplit] merge weights
-    float* s_inv = s_w + rows * nsplit;           // [rows] 1 / sum of weights
+    // parts: the nsplit splits of this launch, then (cascade) the shared prefix's partials
+    const int nparts = nsplit + p.prefix_parts;
+    auto part_lse = [&](int sp, int64_t row) {
+        return sp < nsplit ? __ldcg(p.part_lse + sp * stride + row)
+                           : __ldcg(p.prefix_lse + (sp - nsplit) * stride + row);
+    };
+    float* s_w = reinterpret_cast<float*>(smem);  // [rows][nparts] merge weights
+    float* s_inv = s_w + rows * nparts;           // [rows] 1 / sum of weights
     for (int n = warp; n < rows; n += NW) {
         const int64_t row = static_cast<int64_t>(q0 + n / p.group) * p.num_q_heads +
                             g * p.group + n % p.group;
         float M = -INFINITY;
-        for (int sp = lane; sp < nsplit; sp += 32) M = fmaxf(M, __ldcg(p.part_lse + sp * stride + row));
+        for (int sp = lane; sp < nparts; sp += 32) M = fmaxf(M, part_lse(sp, row));
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, off));
         float W = 0.f;
-        for (int sp = lane; sp < nsplit; sp += 32) {
-            const float w = M == -INFINITY ? 0.f : fast_exp2(__ldcg(p.part_lse + sp * stride + row) - M);
-            s_w[n * nsplit + sp] = w;
+        for (int sp = lane; sp < nparts; sp += 32) {
+            const float w = M == -INFINITY ? 0.f : fast_exp2(part_lse(sp, row) - M);
+            s_w[n * nparts + sp] = w;
             W += w;
         }
 #pragma unroll
@@ -521,12 +553,21 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
                             g * p.group + n % p.group;
         const float4* src = reinterpret_cast<const float4*>(p.part_o + row * D) + c;
         const int64_t s4 = stride * D / 4;
-        const float* w = s_w + n * nsplit;
+        const float* w = s_w + n * nparts;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 8
         for (int sp = 0; sp < nsplit; ++sp) {
             const float4 v = __ldcg(src + sp * s4);
             const float ws = w[sp];
+            acc.x += ws * v.x;
+            acc.y += ws * v.y;
+            acc.z += ws * v.z;
+            acc.w += ws * v.w;
+        }
+        const float4* psrc = reinterpret_cast<const float4*>(p.prefix_o + row * D) + c;
+        for (int k = 0; k < p.prefix_parts; ++k) {
+            const float4 v = __ldcg(psrc + k * s4);
+            const float ws = w[nsplit + k];
             acc.x += ws * v.x;
             acc.y += ws * v.y;
             acc.z += ws * v.z;

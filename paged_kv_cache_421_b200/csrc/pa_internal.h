@@ -52,6 +52,7 @@ struct AttnParams {
     float* part_o;              // [S][T][Hq][D] split partials (normalised)
     float* part_lse;            // [S][T][Hq]   split log2-sum-exp2 of scaled scores
     int* split_counters;        // [T][Hkv] finished-split counts (zeroed before each launch)
+    const uint8_t* cache;       // the pool (bulk copies of FP8 V tiles)
     const float* k_scale;       // FP8 per-kv-head scales, else null
     const float* v_scale;
     int max_blocks_per_seq;
@@ -72,6 +73,21 @@ struct AttnParams {
     int window;                 // sliding window in keys, 0 = full causal attention
     int local_chunk;            // chunked local attention: chunk length in keys, 0 = off
     float* lse_out;             // [T][Hq] natural-log LSE of every row, or null
+    // Cascade attention over a prefix of prefix_keys positions that every request shares
+    // (the same physical blocks at the start of every block-table row):
+    //  - prefix launch (prefix_launch = 1, chunk kernels): all num_tokens query rows of the
+    //    step form one request that sees every key in [0, prefix_keys) of block-table row
+    //    prefix_row, with no causal mask; each split writes its normalised partial and its
+    //    log2-sum-exp2 to part_o / part_lse at its split index (never to out);
+    //  - suffix launch (prefix_launch = 0, decode kernel): each request walks only its keys
+    //    from prefix_keys on, then merges the prefix_parts partials at prefix_o / prefix_lse
+    //    ([prefix_parts][T][Hq][D] and [prefix_parts][T][Hq], log2 domain) into its result.
+    int prefix_keys;            // 0: no shared prefix
+    int prefix_row;
+    int prefix_launch;
+    int prefix_parts;
+    const float* prefix_o;
+    const float* prefix_lse;
 };
 
 // The chunk-kind requests of a launch, longest context first (passed by value, so the chunk
@@ -97,7 +113,8 @@ cudaError_t launch_decode(const CUtensorMap& tmap, const AttnParams& p, int head
 cudaError_t launch_chunk(const CUtensorMap& tmap, const CUtensorMap& tmap_blk, const AttnParams& p,
                          const ChunkWork& work, int head_size, int kv_dtype, int max_splits,
                          cudaStream_t stream);
-cudaError_t launch_chunk_tc(const CUtensorMap& tmap_blk, const AttnParams& p, const ChunkWork& work,
+cudaError_t launch_chunk_tc(const CUtensorMap& tmap, const CUtensorMap& tmap_blk,
+                            const AttnParams& p, const ChunkWork& work, int kv_dtype,
                             int max_splits, cudaStream_t stream);
 cudaError_t launch_reduce(const AttnParams& p, const ChunkList& list, int head_size,
                           cudaStream_t stream);

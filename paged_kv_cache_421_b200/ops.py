@@ -109,7 +109,8 @@ def write_kv(cache: PagedKVCache, k: torch.Tensor, v: torch.Tensor, slots: torch
 def workspace_bytes_for(cache: PagedKVCache, seq_lens_host, qsl_host, num_q_heads: int,
                         max_blocks_per_seq: int, kv_split_tokens: int = 0,
                         num_sms: Optional[int] = None, sliding_window: int = 0,
-                        local_chunk: int = 0, with_lse: bool = False) -> int:
+                        local_chunk: int = 0, with_lse: bool = False,
+                        common_prefix_tokens: int = 0) -> int:
     if num_sms is None:
         num_sms = torch.cuda.get_device_properties(cache.buffer.device).multi_processor_count
     qs = np.asarray(qsl_host)
@@ -119,7 +120,7 @@ def workspace_bytes_for(cache: PagedKVCache, seq_lens_host, qsl_host, num_q_head
                                cache.head_size, max_blocks_per_seq, num_sms, unlimited,
                                kv_split_tokens=kv_split_tokens, block_size=cache.block_size,
                                sliding_window=sliding_window, local_chunk=local_chunk,
-                               with_lse=with_lse)
+                               with_lse=with_lse, common_prefix_tokens=common_prefix_tokens)
     return int(plan["workspace_needed"])
 
 
@@ -128,9 +129,11 @@ def attention(cache: PagedKVCache, q: torch.Tensor, block_table: torch.Tensor,
               out: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None,
               kv_split_tokens: int = 0, events=None, sliding_window: int = 0,
               local_chunk: int = 0, lse_out: Optional[torch.Tensor] = None,
-              stream=None) -> torch.Tensor:
+              common_prefix_tokens: int = 0, stream=None) -> torch.Tensor:
     """Paged attention of one step; with ``lse_out`` (fp32 [T][Hq]) each row's natural-log
-    log-sum-exp is written too, and decode-kind requests may hold no key (0 and -inf)."""
+    log-sum-exp is written too, and decode-kind requests may hold no key (0 and -inf).
+    ``common_prefix_tokens`` > 0: the requests' block tables share that many leading tokens'
+    blocks (see pa_common_prefix_blocks), read once for all of them (cascade attention)."""
     T, Hq, D = q.shape
     if out is None:
         out = torch.empty(T, Hq, D, dtype=torch.float32, device=q.device)
@@ -140,11 +143,12 @@ def attention(cache: PagedKVCache, q: torch.Tensor, block_table: torch.Tensor,
     if workspace is None:
         nb = workspace_bytes_for(cache, seq_lens_host, qsl_host, Hq, block_table.shape[1],
                                  kv_split_tokens, sliding_window=sliding_window,
-                                 local_chunk=local_chunk, with_lse=lse_out is not None)
+                                 local_chunk=local_chunk, with_lse=lse_out is not None,
+                                 common_prefix_tokens=common_prefix_tokens)
         workspace = torch.empty(max(nb, 1), dtype=torch.uint8, device=q.device)
     B.pa_attention_ex(cache.handle, q, Hq, block_table, block_table.shape[1], seq_lens, qsl,
                       seq_lens_host, qsl_host, seq_lens.numel(), T, scale, out, workspace,
                       workspace.numel(), kv_split_tokens=kv_split_tokens, events=events,
                       sliding_window=sliding_window, local_chunk=local_chunk, lse_out=lse_out,
-                      stream=stream)
+                      common_prefix_tokens=common_prefix_tokens, stream=stream)
     return out

@@ -224,17 +224,18 @@ def llama8b_decode(device="cpu") -> Workload:
                          SEED_BASE + 2, device=device)
 
 
-def mixed_step(device="cpu") -> Workload:
+def mixed_step(kv_dtype: int = BF16, device="cpu") -> Workload:
     """48 decodes (context uniform in [1024, 8192]) then two 512-token prefill chunks with 0
     and 2048 tokens already computed; 1072 tokens of a 2048-token budget; 32/8 heads,
-    head_dim 128, block 16, a 65536-block pool."""
+    head_dim 128, block 16, a 65536-block pool; bf16 or FP8 E4M3 cache."""
     rng = np.random.default_rng(SEED_BASE + 3)
     dec = rng.integers(1024, 8192, size=48, endpoint=True)
     ctx = np.concatenate([dec, [512, 2048 + 512]])
     ql = np.concatenate([np.ones(48, np.int64), [512, 512]])
     assert ql.sum() <= 2048
-    return make_workload("mixed_step", ctx, ql, 32, 8, 128, 16, 65536, SEED_BASE + 3,
-                         device=device)
+    name = "mixed_step" + ("_fp8" if kv_dtype == FP8_E4M3 else "")
+    return make_workload(name, ctx, ql, 32, 8, 128, 16, 65536, SEED_BASE + 3,
+                         kv_dtype=kv_dtype, device=device)
 
 
 def prefix_share_decode(device="cpu") -> Workload:
@@ -264,6 +265,7 @@ CONFIGS = {
     "prefix_share_decode": prefix_share_decode,
     "long70b_decode": long70b_decode,
     "long70b_decode_fp8": lambda device="cpu": long70b_decode(FP8_E4M3, device=device),
+    "mixed_step_fp8": lambda device="cpu": mixed_step(FP8_E4M3, device=device),
 }
 
 

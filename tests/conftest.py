@@ -18,7 +18,7 @@ def pytest_configure(config):
 # Config-level parity tests build a full-size step and its oracle once per config and keep only
 # the current one; running every test of one config before the next avoids rebuilding them.
 CONFIG_ORDER = ["tiny_decode", "llama8b_decode", "mixed_step", "prefix_share_decode",
-                "long70b_decode", "long70b_decode_fp8"]
+                "long70b_decode", "long70b_decode_fp8", "mixed_step_fp8"]
 
 
 def pytest_collection_modifyitems(session, config, items):

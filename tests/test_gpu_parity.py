@@ -18,7 +18,7 @@ from paged_kv_cache_421_b200 import workloads as W
 pytestmark = pytest.mark.gpu
 
 ALL_CONFIGS = ["tiny_decode", "llama8b_decode", "mixed_step", "prefix_share_decode",
-               "long70b_decode", "long70b_decode_fp8"]
+               "long70b_decode", "long70b_decode_fp8", "mixed_step_fp8"]
 
 
 @pytest.fixture(autouse=True)
@@ -117,7 +117,7 @@ def test_attention_sampled_rows(name):
     print(name, stats, len(tokens), "rows")
 
 
-@pytest.mark.parametrize("name", ["mixed_step"])
+@pytest.mark.parametrize("name", ["mixed_step", "mixed_step_fp8"])
 def test_mixed_step_chunks_all_rows(name):
     # every row of both prefill chunks (the chunk kernel's causal diagonal tiles included),
     # against the unpaged oracle
@@ -194,7 +194,9 @@ def test_edge_case(case):
 
 
 @pytest.mark.parametrize("kv_dtype,q_lens", [(W.BF16, [1, 1, 1, 1]), (W.FP8_E4M3, [1, 1, 1, 1]),
-                                             (W.BF16, [17, 9, 5, 60])])
+                                             (W.BF16, [17, 9, 5, 60]),
+                                             (W.FP8_E4M3, [17, 9, 5, 60])],
+                         ids=["bf16-decode", "fp8-decode", "bf16-chunks", "fp8-chunks"])
 def test_nan_garbage_in_unwritten_slots(kv_dtype, q_lens):
     # stale NaN patterns in the unused tail of partly filled blocks must not reach the output
     # (decode rows, and prefill chunks whose last key tile ends inside a block)
@@ -223,6 +225,50 @@ def test_random_small_steps(seed):
     assert np.array_equal(st.cache_host(), oracle_cache(wl).view(np.uint8))
     want, _ = oracle_attention_all(wl, oracle_cache(wl))
     assert_close(st.out.cpu().numpy(), want, wl.kv_dtype, f"seed {seed}")
+
+
+FP8_CHUNK_CASES = {
+    # FP8 E4M3 cache with chunk-kind requests (q_len * group > 8): the tcgen05 chunk kernel's
+    # kind::f8f6f4 path, alone and mixed with decodes
+    "first_chunk": ([70], [70], 8, 2),
+    "chunk_after_history": ([1000], [333], 16, 2),
+    "spec_decode_g8_qlen2": ([300, 517], [2, 2], 64, 8),
+    "qlen3_g4": ([50, 300], [3, 3], 8, 2),
+    "mixed_decodes_and_chunk": ([2000, 3001, 600, 700], [1, 1, 200, 1], 32, 8),
+    "ragged_chunk_tails": ([129, 255, 17], [129, 100, 17], 8, 1),
+}
+
+
+@pytest.mark.parametrize("case", sorted(FP8_CHUNK_CASES))
+def test_fp8_chunk_case(case):
+    ctx, ql, hq, hkv = FP8_CHUNK_CASES[case]
+    wl = _small(ctx, ql, hq, hkv, 128, seed=zlib.crc32(case.encode()) % 1000,
+                kv_dtype=W.FP8_E4M3)
+    st = GpuStep(wl)
+    ocache = oracle_cache(wl)
+    assert np.array_equal(st.cache_host(), ocache)
+    want, want_lse = oracle_attention_all(wl, ocache)
+    assert_close(st.out.cpu().numpy(), want, W.FP8_E4M3, case)
+    # forced partitions: fused split merges (<= 4 splits) and the reduce kernel (more)
+    for split in [64, 256]:
+        assert_close(st.attend(kv_split_tokens=split).cpu().numpy(), want, W.FP8_E4M3,
+                     f"{case} split {split}")
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_random_small_steps_fp8_with_chunks(seed):
+    rng = np.random.default_rng(3000 + seed)
+    B_ = int(rng.integers(1, 8))
+    hkv = int(rng.choice([1, 2, 4]))
+    G = int(rng.choice([1, 2, 4, 8]))
+    ctx = rng.integers(1, 900, size=B_)
+    ql = np.array([int(rng.choice([1, 2, int(rng.integers(1, c + 1))])) for c in ctx])
+    ql = np.minimum(ql, ctx)
+    wl = _small(ctx, ql, hkv * G, hkv, 128, seed=seed, kv_dtype=W.FP8_E4M3)
+    st = GpuStep(wl)
+    assert np.array_equal(st.cache_host(), oracle_cache(wl))
+    want, _ = oracle_attention_all(wl, oracle_cache(wl))
+    assert_close(st.out.cpu().numpy(), want, W.FP8_E4M3, f"fp8 chunks seed {seed}")
 
 
 def test_random_small_steps_fp8():
