@@ -271,6 +271,15 @@ typedef struct {
                               (else METADATA), no sliding window or local chunk (else
                               UNSUPPORTED), and workspace for the prefix partials
                               (pa_plan_attention's workspace_needed; else WORKSPACE).  0: off */
+    int test_skip_decode_load; /* test hook of the bounded waits, 0 in normal use.  k > 0: in
+                              the decode kernel's CTA (split 0, kv head 0, request 0), warp 0
+                              leaves the load of its k-th unit (a block, two for FP8) of its
+                              first round unissued, so its wait for it runs out: the CTA
+                              records code 1 in the device error word and returns without
+                              writing its rows (the call's output is then incomplete).  Nothing
+                              is in flight when the wait gives up. */
+    int test_wait_limit_us;   /* with test_skip_decode_load: that CTA's wait limit in
+                              microseconds (> 0); otherwise ignored (waits give up after 2 s) */
 } pa_attention_opts;
 
 /* The planner alone: fills *plan for the given host metadata without touching the GPU.

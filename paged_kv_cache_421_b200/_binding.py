@@ -71,6 +71,8 @@ class pa_attention_opts(ctypes.Structure):
         ("local_chunk", ctypes.c_int),
         ("lse_out", ctypes.c_void_p),
         ("common_prefix_tokens", ctypes.c_int),
+        ("test_skip_decode_load", ctypes.c_int),
+        ("test_wait_limit_us", ctypes.c_int),
     ]
 
 
@@ -255,7 +257,8 @@ def pa_attention_ex(handle, q, num_q_heads, block_table, max_blocks_per_seq, seq
                     query_start_loc, seq_lens_host, query_start_loc_host, num_seqs, num_tokens,
                     scale, out, workspace=None, workspace_bytes=0, kv_split_tokens=0,
                     num_sms=0, events=None, sliding_window=0, local_chunk=0, lse_out=None,
-                    common_prefix_tokens=0, stream=None) -> None:
+                    common_prefix_tokens=0, test_skip_decode_load=0, test_wait_limit_us=0,
+                    stream=None) -> None:
     sl = _host_i32(seq_lens_host)
     qs = _host_i32(query_start_loc_host)
     opts = pa_attention_opts()
@@ -265,6 +268,8 @@ def pa_attention_ex(handle, q, num_q_heads, block_table, max_blocks_per_seq, seq
     opts.local_chunk = local_chunk
     opts.lse_out = _ptr(lse_out)
     opts.common_prefix_tokens = common_prefix_tokens
+    opts.test_skip_decode_load = test_skip_decode_load
+    opts.test_wait_limit_us = test_wait_limit_us
     for i, ev in enumerate(events or []):
         if ev is not None:
             opts.events[i] = ev.cuda_event if hasattr(ev, "cuda_event") else int(ev)

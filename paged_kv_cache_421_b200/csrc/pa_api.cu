@@ -5,6 +5,7 @@
 #include <cstring>
 #include <algorithm>
 #include <atomic>
+#include <mutex>
 #include <vector>
 #include <new>
 
@@ -59,6 +60,42 @@ int device_num_sms() {
         g_num_sms[dev].store(n, std::memory_order_relaxed);
     }
     return n;
+}
+
+// Mixed steps: the chunk kernel runs on a second stream of the device while the decode kernel
+// runs on the caller's, so that the chunk CTAs (tensor-bound, one per SM) take a subset of the
+// SMs while the decode CTAs keep HBM busy on the others.  The stream has the device's highest
+// priority, so its CTAs are dispatched first; events fork it from and join it back into the
+// caller's stream, which keeps every call stream-ordered (and capturable in a graph).
+constexpr bool kOverlapChunksWithDecode = true;
+
+struct SideStream {
+    std::mutex mu;  // one fork/join at a time per device: the events are shared
+    cudaStream_t stream = nullptr;
+    cudaEvent_t fork = nullptr, join = nullptr;
+    bool ready = false;
+};
+SideStream g_side[kMaxDevices];
+std::mutex g_side_init;
+
+// The side stream of the current device, created on first use; nullptr if that fails.
+SideStream* side_stream() {
+    const int dev = current_device();
+    if (dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lk(g_side_init);
+    SideStream& ss = g_side[dev];
+    if (!ss.ready) {
+        int least = 0, greatest = 0;
+        if (cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess ||
+            cudaStreamCreateWithPriority(&ss.stream, cudaStreamNonBlocking, greatest) != cudaSuccess ||
+            cudaEventCreateWithFlags(&ss.fork, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&ss.join, cudaEventDisableTiming) != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
+        ss.ready = true;
+    }
+    return &ss;
 }
 
 int dtype_bytes(int kv_dtype) { return kv_dtype == PA_BF16 ? 2 : (kv_dtype == PA_FP8_E4M3 ? 1 : 0); }
@@ -177,6 +214,9 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
     if (window < 0 || local_chunk < 0) return PA_ERR_INVALID_ARG;
     // cascade attention over a shared prefix of P keys: decode-kind requests only, full
     // attention only; each request's own work is its keys after the prefix
+    if (opts && (opts->test_skip_decode_load < 0 || opts->test_wait_limit_us < 0 ||
+                 (opts->test_skip_decode_load > 0 && opts->test_wait_limit_us <= 0)))
+        return PA_ERR_INVALID_ARG;  // the bounded-wait test hook needs its own wait limit
     const int P = opts ? opts->common_prefix_tokens : 0;
     if (P < 0 || P % bs) return PA_ERR_INVALID_ARG;
     if (P > 0 && (window > 0 || local_chunk > 0)) return PA_ERR_UNSUPPORTED;
@@ -504,6 +544,20 @@ int pa_attention_ex(const pa_cache* cache, const void* q, int num_q_heads,
                     const int32_t* query_start_loc_host, int num_seqs, int num_tokens,
                     float scale, float* out, void* workspace, size_t workspace_bytes,
                     const pa_attention_opts* opts, void* stream) {
+    return pa::attention_call(cache, q, num_q_heads, block_table, max_blocks_per_seq, seq_lens,
+                              query_start_loc, seq_lens_host, query_start_loc_host, num_seqs,
+                              num_tokens, scale, out, workspace, workspace_bytes, opts, stream,
+                              true);
+}
+
+}  // extern "C"
+
+int pa::attention_call(const pa_cache* cache, const void* q, int num_q_heads,
+                       const int32_t* block_table, int max_blocks_per_seq, const int32_t* seq_lens,
+                       const int32_t* query_start_loc, const int32_t* seq_lens_host,
+                       const int32_t* query_start_loc_host, int num_seqs, int num_tokens,
+                       float scale, float* out, void* workspace, size_t workspace_bytes,
+                       const pa_attention_opts* opts, void* stream, bool allow_side_stream) {
     if (!cache || num_seqs < 0 || num_tokens < 0 || num_q_heads <= 0) return PA_ERR_INVALID_ARG;
     if (num_q_heads % cache->num_kv_heads) return PA_ERR_INVALID_ARG;
     if (num_tokens == 0) return PA_OK;
@@ -512,6 +566,7 @@ int pa_attention_ex(const pa_cache* cache, const void* q, int num_q_heads,
         return PA_ERR_INVALID_ARG;
     if (!(scale > 0.f) || scale != scale) return PA_ERR_INVALID_ARG;
     if (workspace_bytes && !workspace) return PA_ERR_INVALID_ARG;
+
     if ((reinterpret_cast<uintptr_t>(q) & 15) || (reinterpret_cast<uintptr_t>(out) & 15) ||
         (reinterpret_cast<uintptr_t>(workspace) & 255) ||
         (opts && (reinterpret_cast<uintptr_t>(opts->lse_out) & 3)))
@@ -567,6 +622,10 @@ int pa_attention_ex(const pa_cache* cache, const void* q, int num_q_heads,
     p.local_chunk = opts ? opts->local_chunk : 0;
     p.lse_out = opts ? opts->lse_out : nullptr;
     p.err = device_error_ptr();
+    if (opts && opts->test_skip_decode_load > 0) {
+        p.test_skip_unit = opts->test_skip_decode_load;
+        p.test_wait_ns = static_cast<uint64_t>(opts->test_wait_limit_us) * 1000u;
+    }
     int prefix_row = 0;
     if (cascade) {
         // the shared prefix's blocks are read from the first request with queries; its split
@@ -637,17 +696,13 @@ int pa_attention_ex(const pa_cache* cache, const void* q, int num_q_heads,
         if (e != cudaSuccess) return fail_cuda(e);
         if (ev) record(ev[3], s);
     }
-    if (pl.num_decode_seqs) {
-        if (ev) record(ev[0], s);
-        e = pa::launch_decode(cache->tmap, p, cache->head_size, cache->kv_dtype,
-                              pl.decode_max_splits, s);
-        if (e != cudaSuccess) return fail_cuda(e);
-        if (ev) record(ev[1], s);
-    }
     // the chunk-kind requests, longest context first; a longer list falls back to a grid over
     // every request
     static thread_local pa::ChunkList list;
+    static thread_local pa::ChunkWork work;
+    static thread_local std::vector<std::pair<int, uint32_t>> items;
     list.count = 0;
+    work.count = 0;
     if (pl.num_chunk_seqs) {
         if (pl.num_chunk_seqs <= pa::kMaxChunkList) {
             for (int r = 0; r < num_seqs; ++r) {
@@ -659,9 +714,6 @@ int pa_attention_ex(const pa_cache* cache, const void* q, int num_q_heads,
             });
         }
         // the chunk CTAs, most key tiles first; a list that does not fit falls back to the grid
-        static thread_local pa::ChunkWork work;
-        static thread_local std::vector<std::pair<int, uint32_t>> items;
-        work.count = 0;
         items.clear();
         const int cta_rows = pa::chunk_rows(cache->head_size, 1);
         const int tile_keys = cache->head_size == 128 ? 128 : 64;
@@ -701,11 +753,48 @@ int pa_attention_ex(const pa_cache* cache, const void* q, int num_q_heads,
                              });
             for (const auto& it : items) work.item[work.count++] = it.second;
         }
+    }
+    // a step with both kinds: the chunk kernel on the side stream, forked from this stream after
+    // the counter clear and joined back before the split reduce
+    SideStream* side = nullptr;
+    std::unique_lock<std::mutex> side_lock;
+    if (kOverlapChunksWithDecode && allow_side_stream && pl.num_decode_seqs && pl.num_chunk_seqs &&
+        !cascade) {
+        side = side_stream();
+        if (side) {
+            side_lock = std::unique_lock<std::mutex>(side->mu);
+            e = cudaEventRecord(side->fork, s);
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(side->stream, side->fork, 0);
+            if (e != cudaSuccess) return fail_cuda(e);
+        }
+    }
+    const cudaStream_t cs = side ? side->stream : s;  // the chunk kernel's stream
+    if (pl.num_chunk_seqs && side) {
+        if (ev) record(ev[2], cs);
+        e = pa::launch_chunk(cache->tmap, cache->tmap_blk, p, work, cache->head_size,
+                             cache->kv_dtype, pl.chunk_max_splits, cs);
+        if (e != cudaSuccess) return fail_cuda(e);
+        if (ev) record(ev[3], cs);
+    }
+    if (pl.num_decode_seqs) {
+        if (ev) record(ev[0], s);
+        e = pa::launch_decode(cache->tmap, p, cache->head_size, cache->kv_dtype,
+                              pl.decode_max_splits, s);
+        if (e != cudaSuccess) return fail_cuda(e);
+        if (ev) record(ev[1], s);
+    }
+    if (pl.num_chunk_seqs && !side) {
         if (ev) record(ev[2], s);
         e = pa::launch_chunk(cache->tmap, cache->tmap_blk, p, work, cache->head_size,
                              cache->kv_dtype, pl.chunk_max_splits, s);
         if (e != cudaSuccess) return fail_cuda(e);
         if (ev) record(ev[3], s);
+    }
+    if (side) {
+        e = cudaEventRecord(side->join, cs);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(s, side->join, 0);
+        if (e != cudaSuccess) return fail_cuda(e);
+        side_lock.unlock();
     }
     if (pl.chunk_max_splits > 1 && !chunk_merge_fused) {
         if (ev) record(ev[4], s);
@@ -715,6 +804,8 @@ int pa_attention_ex(const pa_cache* cache, const void* q, int num_q_heads,
     }
     return PA_OK;
 }
+
+extern "C" {
 
 int pa_attention(const pa_cache* cache, const void* q, int num_q_heads,
                  const int32_t* block_table, int max_blocks_per_seq, const int32_t* seq_lens,

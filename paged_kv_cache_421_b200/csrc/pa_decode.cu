@@ -100,6 +100,11 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
     if (split >= nsplit) return;
     const int jb = fb + split * p.decode_split_blocks;
     const int je = min(nblocks, jb + p.decode_split_blocks);
+    // test hook of the bounded waits: one CTA leaves one of warp 0's loads unissued, so that
+    // warp's wait for it runs out (after test_wait_ns) with no copy in flight
+    const bool inject = p.test_skip_unit > 0 && split == 0 && g == 0 && r == 0;
+    const uint64_t wait_ns = inject ? p.test_wait_ns : kWaitLimitNs;
+    const uint64_t wind_ns = inject ? p.test_wait_ns : kWindDownLimitNs;
 
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t bars[NW * NS];
@@ -229,6 +234,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
         const int kend = (rb + rn) * kBlockSize;  // first position past this round's blocks
 
         auto issue = [&](int i, uint32_t n) {
+            if (inject && warp == 0 && rb == jb && i == p.test_skip_unit - 1) return;
             const int u0 = (warp + i * NW) * BPU;  // round index of the unit's first block
             const int nb = min(BPU, rn - u0);
             const uint32_t st = n % NS;
@@ -255,7 +261,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
         for (int i = 0; i < mine; ++i) {
             const uint32_t n = loads + i;
             const uint32_t st = n % NS;
-            if (!mbar_wait(smem_u32(&bars[warp * NS + st]), (n / NS) & 1u, kWaitLimitNs, p.err)) {
+            if (!mbar_wait(smem_u32(&bars[warp * NS + st]), (n / NS) & 1u, wait_ns, p.err)) {
                 ok = false;
                 fail_i = i;
                 break;
@@ -417,7 +423,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
             // wind down: wait (bounded, 0.1 s each) for this warp's loads still in flight
             for (int i = fail_i; i < min(fail_i + NS, mine); ++i) {
                 const uint32_t n = loads + i;
-                mbar_wait(smem_u32(&bars[warp * NS + n % NS]), (n / NS) & 1u, kWindDownLimitNs,
+                mbar_wait(smem_u32(&bars[warp * NS + n % NS]), (n / NS) & 1u, wind_ns,
                           p.err);
             }
         }

@@ -88,6 +88,11 @@ struct AttnParams {
     int prefix_parts;
     const float* prefix_o;
     const float* prefix_lse;
+    // Test hook of the bounded waits (decode kernel): > 0 makes CTA (split 0, kv head 0,
+    // request 0) skip the load of warp 0's unit test_skip_unit - 1 of its first round, and that
+    // CTA's waits give up after test_wait_ns; 0 = off.
+    int test_skip_unit;
+    uint64_t test_wait_ns;
 };
 
 // The chunk-kind requests of a launch, longest context first (passed by value, so the chunk
@@ -107,6 +112,15 @@ struct ChunkWork {
     int count;
     uint32_t item[kMaxChunkWork];
 };
+
+// The body of pa_attention_ex.  allow_side_stream = false keeps every launch on `stream` and
+// creates no stream or event (pa_attention_noalloc allocates nothing, not even those).
+int attention_call(const pa_cache* cache, const void* q, int num_q_heads,
+                   const int32_t* block_table, int max_blocks_per_seq, const int32_t* seq_lens,
+                   const int32_t* query_start_loc, const int32_t* seq_lens_host,
+                   const int32_t* query_start_loc_host, int num_seqs, int num_tokens, float scale,
+                   float* out, void* workspace, size_t workspace_bytes,
+                   const pa_attention_opts* opts, void* stream, bool allow_side_stream);
 
 cudaError_t launch_decode(const CUtensorMap& tmap, const AttnParams& p, int head_size,
                           int kv_dtype, int max_splits, cudaStream_t stream);

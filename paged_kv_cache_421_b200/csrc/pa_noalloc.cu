@@ -48,11 +48,13 @@ extern "C" int pa_attention_noalloc(const pa_cache* cache, const void* q, int nu
         }
         g_noalloc_scratch_addr[dev].store(ptr, std::memory_order_release);
     }
-    // pa_attention checks every argument first, then plans a split-KV partition that fits the
-    // scratch (fewer splits, down to none, when the call's rows are many); it clears the split
-    // counters on the stream before its kernels and writes every partial the merge reads.  A
-    // plan that still needs more than the scratch is refused with PA_ERR_WORKSPACE.
-    return pa_attention(cache, q, num_q_heads, block_table, max_blocks_per_seq, seq_lens,
-                        query_start_loc, seq_lens_host, query_start_loc_host, num_seqs,
-                        num_tokens, scale, out, ptr, PA_NOALLOC_SCRATCH_BYTES, stream);
+    // The call checks every argument first (as pa_attention), then plans a split-KV partition
+    // that fits the scratch (fewer splits, down to none, when the call's rows are many); it
+    // clears the split counters on the stream before its kernels and writes every partial the
+    // merge reads.  A plan that still needs more than the scratch is refused with
+    // PA_ERR_WORKSPACE.  Every launch stays on `stream`: no second stream or event is created.
+    return pa::attention_call(cache, q, num_q_heads, block_table, max_blocks_per_seq, seq_lens,
+                              query_start_loc, seq_lens_host, query_start_loc_host, num_seqs,
+                              num_tokens, scale, out, ptr, PA_NOALLOC_SCRATCH_BYTES, nullptr,
+                              stream, false);
 }

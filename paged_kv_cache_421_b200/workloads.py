@@ -238,6 +238,13 @@ def mixed_step(kv_dtype: int = BF16, device="cpu") -> Workload:
                          kv_dtype=kv_dtype, device=device)
 
 
+def prefill_chunks(device="cpu") -> Workload:
+    """The mixed step's two prefill chunks alone, the chunk kernel's share of that step: 512
+    new tokens over 0 and over 2048 computed ones; 32/8 heads, head_dim 128, block 16."""
+    return make_workload("prefill_chunks", [512, 2048 + 512], [512, 512], 32, 8, 128, 16,
+                         65536, SEED_BASE + 6, device=device)
+
+
 def prefix_share_decode(device="cpu") -> Workload:
     """128 decode requests sharing a 1024-token prefix (the same 64 physical blocks in every
     table) plus private suffixes of uniform [64, 512] tokens; 32/8 heads, head_dim 128."""
@@ -266,6 +273,7 @@ CONFIGS = {
     "long70b_decode": long70b_decode,
     "long70b_decode_fp8": lambda device="cpu": long70b_decode(FP8_E4M3, device=device),
     "mixed_step_fp8": lambda device="cpu": mixed_step(FP8_E4M3, device=device),
+    "prefill_chunks": prefill_chunks,
 }
 
 

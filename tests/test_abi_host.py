@@ -174,6 +174,17 @@ def test_argument_errors_without_device(lib):
                                  None) == B.PA_ERR_INVALID_ARG
     assert lib.pa_validate_slots(fake, None, 4, None, ctypes.byref(n_dup), None) == \
         B.PA_ERR_INVALID_ARG
+    # the bounded-wait test hook needs a wait limit of its own
+    opts = B.pa_attention_opts()
+    plan = B.pa_plan()
+    sl = (ctypes.c_int * 1)(40)
+    qs = (ctypes.c_int * 2)(0, 1)
+    for skip, limit, status in [(1, 0, B.PA_ERR_INVALID_ARG), (-1, 10, B.PA_ERR_INVALID_ARG),
+                                (1, -5, B.PA_ERR_INVALID_ARG), (1, 1000, B.PA_OK),
+                                (0, 0, B.PA_OK)]:
+        opts.test_skip_decode_load, opts.test_wait_limit_us = skip, limit
+        assert lib.pa_plan_attention(sl, qs, 1, 1, 8, 2, 128, 16, 4, 148, 0, ctypes.byref(opts),
+                                     ctypes.byref(plan)) == status, (skip, limit)
 
 
 def test_allocator_argument_errors_without_device(lib):

@@ -346,6 +346,28 @@ def test_slot_validator_counts_out_of_pool_and_duplicate_slots(seed):
     assert got == want and want[1] > 0 and want[0] == 100
 
 
+@pytest.mark.parametrize("kv_dtype", [W.BF16, W.FP8_E4M3])
+def test_decode_wait_runs_out_and_is_reported(kv_dtype):
+    # one decode CTA leaves one of its TMA loads unissued (test hook): its bounded wait gives up
+    # after 1 ms, the kernel records code 1 and returns, and the context stays usable
+    wl = _small([2000, 700], [1, 1], 8, 2, 128, seed=13, kv_dtype=kv_dtype)
+    st = GpuStep(wl)
+    want, _ = oracle_attention_all(wl, oracle_cache(wl))
+    assert_close(st.out.cpu().numpy(), want, kv_dtype, "before")
+    nb = ops.workspace_bytes_for(st.cache, wl.seq_lens, wl.qsl, wl.num_q_heads,
+                                 wl.max_blocks_per_seq)
+    ws = torch.empty(max(nb, 256), dtype=torch.uint8, device="cuda")
+    out = torch.zeros(wl.num_tokens, wl.num_q_heads, 128, device="cuda")
+    B.pa_attention_ex(st.cache.handle, wl.q.cuda(), wl.num_q_heads, st.step["bt"],
+                      wl.max_blocks_per_seq, st.step["sl"], st.step["qsl"], wl.seq_lens, wl.qsl,
+                      wl.num_seqs, wl.num_tokens, wl.scale, out, ws, ws.numel(),
+                      test_skip_decode_load=4, test_wait_limit_us=1000)
+    torch.cuda.synchronize()
+    assert B.pa_device_error(reset=True) == 1
+    # the next call runs normally
+    assert_close(st.attend().cpu().numpy(), want, kv_dtype, "after")
+
+
 def test_slot_beyond_table_is_reported():
     bt = torch.zeros(1, 2, dtype=torch.int32, device="cuda")
     sl = torch.tensor([40], dtype=torch.int32, device="cuda")
