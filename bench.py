@@ -507,9 +507,13 @@ def time_step(step, args, flush_l2: bool, flush, stream, world: int, local: int,
     if step.plan["num_decode_seqs"]:
         t["decode"] = max_over_ranks(statistics.mean(e[0].elapsed_time(e[1]) for e in ev),
                                      world, device)
-    if step.plan["num_chunk_seqs"]:
+    # the chunk slot times the chunk kernel, or the prefix pass of a cascade step
+    if step.plan["num_chunk_seqs"] or step.plan.get("prefix_splits", 0):
         t["chunk"] = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
-    if step.plan["chunk_max_splits"] > 1:  # decode splits merge inside the decode kernel
+    # the split reduce runs only for chunk splits the chunk kernel does not merge itself
+    # (decode splits merge inside the decode kernel)
+    if step.plan["chunk_max_splits"] > 1 and not (step.wl.head_size == 128 and
+                                                  step.plan["chunk_max_splits"] <= 4):
         t["reduce"] = statistics.mean(e[4].elapsed_time(e[5]) for e in ev)
     return t
 

@@ -195,7 +195,7 @@ constexpr int kMinDecodeSplitBlocks = 64;   // >= 1024 keys per split
 constexpr int kMinChunkSplitBlocks = 16;
 constexpr int kMinChunkSplitTiles = 4;      // a chunk split walks at least four key tiles
 constexpr int kMaxChunkSplitBlocks = 1024;  // chunk kernels stage up to 1024 block ids
-constexpr int kMaxPrefixSplits = 8;         // prefix partials each decode row merges
+constexpr int kMaxPrefixSplits = pa::kMaxPrefixParts;  // prefix partials a decode row merges
 
 int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int Hkv, int D,
               int bs, int maxb, int num_sms, size_t ws, const pa_attention_opts* opts,

@@ -20,6 +20,7 @@ constexpr int kDecodeRows = 8;      // decode tile: q_len * group <= 8 rows shar
 constexpr int kChunkRows = 64;      // mma.sync chunk tile: 64 (token, q head) rows per CTA
 constexpr int kMaxFusedSplits = 4;    // tcgen05 chunk kernel: splits it merges itself
 constexpr int kChunkRowsTc = 256;   // tcgen05 chunk CTA: two 128-row q-tiles (TMEM lanes)
+constexpr int kMaxPrefixParts = 4;  // cascade: prefix partials a decode row merges (planner cap)
 
 // Error codes written to the device error word.
 constexpr int kErrWaitTimeout = 1;
@@ -239,6 +240,17 @@ __device__ __forceinline__ void e4m3x4_to_f16x2_scaled(uint32_t r, uint32_t& eve
                                                        uint32_t& odd) {
     even = ((r << 7) & 0x3f803f80u) | ((r << 8) & 0x80008000u);
     odd = ((r >> 1) & 0x3f803f80u) | (r & 0x80008000u);
+}
+
+// Four E4M3 codes (bytes b0..b3 of r) -> two f16x2 words holding their values, by the
+// hardware conversion (exact: every E4M3 value is an f16): even = (b0, b2), odd = (b1, b3).
+// The NaN codes (0x7f / 0xff) give NaN, so stale bytes must not reach an MMA.
+__device__ __forceinline__ void e4m3x4_to_f16x2_cvt(uint32_t r, uint32_t& even, uint32_t& odd) {
+    const uint32_t q = __byte_perm(r, 0u, 0x3120);  // bytes (b0, b2, b1, b3)
+    asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, lo;\n\tcvt.rn.f16x2.e4m3x2 %1, hi;\n\t}"
+        : "=r"(even), "=r"(odd)
+        : "r"(q));
 }
 
 __device__ __forceinline__ float fast_exp2(float x) { return exp2f(x); }

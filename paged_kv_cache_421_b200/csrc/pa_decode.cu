@@ -24,8 +24,8 @@
 // and O^T += V^T P^T reads V through ldmatrix.trans.  Softmax runs in the log2 domain.
 // FP8 E4M3 caches: S^T = K Q^T runs on FP8 tensor cores from the cache bytes (Q split into
 // two E4M3 terms that hold its bf16 value), and V tiles are stored dim-major so that ldmatrix hands out
-// four consecutive keys per word, widened exactly to f16 (as 2^-8 V, by moving bits) for
-// O^T += V^T P^T; the K scale folds into the score scale and the V scale into the epilogue.
+// four consecutive keys per word, widened exactly to f16 for O^T += V^T P^T; the K scale
+// folds into the score scale and the V scale into the epilogue.
 #include <cstdlib>
 
 #include "pa_internal.h"
@@ -35,6 +35,10 @@ namespace {
 
 constexpr uint32_t kFull = 0xffffffffu;
 constexpr int kIdsPerRound = 1024;  // block ids staged in shared memory per round
+// FP8 V widening: true -- the hardware E4M3 -> f16x2 conversion (3 instructions per four codes,
+// exact values; stale bytes past the context are cleared first, as NaN codes would convert to
+// NaN); false -- the bit move to 2^-8 V (7 instructions, finite for every byte).
+constexpr bool kFp8WidenCvt = true;
 
 // Key of the block held by row m (0..15) of the S^T = K Q^T tile.  With a bf16 cache rows are
 // keys in order.  With an FP8 cache the rows are permuted so that, after movmatrix, thread
@@ -102,9 +106,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
     const int je = min(nblocks, jb + p.decode_split_blocks);
     // test hook of the bounded waits: one CTA leaves one of warp 0's loads unissued, so that
     // warp's wait for it runs out (after test_wait_ns) with no copy in flight
-    const bool inject = p.test_skip_unit > 0 && split == 0 && g == 0 && r == 0;
-    const uint64_t wait_ns = inject ? p.test_wait_ns : kWaitLimitNs;
-    const uint64_t wind_ns = inject ? p.test_wait_ns : kWindDownLimitNs;
+    auto inject = [&]() {
+        return p.test_skip_unit > 0 && blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0;
+    };
 
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t bars[NW * NS];
@@ -229,12 +233,14 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
         __syncthreads();
         // a unit is kBpu consecutive blocks of the round; warp w takes units w, w + NW, ...
         constexpr int BPU = C::kBpu;
+        // the unit whose load the test hook leaves unissued (first round, warp 0), else -1
+        const int skip_i = (rb == jb && warp == 0 && inject()) ? p.test_skip_unit - 1 : -1;
         const int units = (rn + BPU - 1) / BPU;
         const int mine = (ok && units > warp) ? (units - warp + NW - 1) / NW : 0;
         const int kend = (rb + rn) * kBlockSize;  // first position past this round's blocks
 
         auto issue = [&](int i, uint32_t n) {
-            if (inject && warp == 0 && rb == jb && i == p.test_skip_unit - 1) return;
+            if (i == skip_i) return;
             const int u0 = (warp + i * NW) * BPU;  // round index of the unit's first block
             const int nb = min(BPU, rn - u0);
             const uint32_t st = n % NS;
@@ -261,7 +267,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
         for (int i = 0; i < mine; ++i) {
             const uint32_t n = loads + i;
             const uint32_t st = n % NS;
-            if (!mbar_wait(smem_u32(&bars[warp * NS + st]), (n / NS) & 1u, wait_ns, p.err)) {
+            if (!mbar_wait(smem_u32(&bars[warp * NS + st]), (n / NS) & 1u,
+                           inject() ? p.test_wait_ns : kWaitLimitNs, p.err)) {
                 ok = false;
                 fail_i = i;
                 break;
@@ -272,8 +279,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
             if constexpr (!FP8) {
                 if (kb + kBlockSize > ctx) {
                     // last, partly filled block: clear V past the context so that stale cache
-                    // bytes (possibly NaN patterns) cannot reach P.V.  FP8 V needs no clearing:
-                    // its f16 widening is finite for every byte, and masked keys get P = 0.
+                    // bytes (possibly NaN patterns) cannot reach P.V (FP8: see above).
                     const int nz = ctx - kb;
                     uint8_t* vg = smem + (stage + C::kTileBytes - smem_u32(smem));
                     for (int idx = lane; idx < (kBlockSize - nz) * C::kBoxes * 8; idx += 32) {
@@ -281,6 +287,34 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
                         const int c = idx % (C::kBoxes * 8);
                         *reinterpret_cast<uint4*>(vg + (c >> 3) * 2048 + row * 128 + (c & 7) * 16) =
                             make_uint4(0, 0, 0, 0);
+                    }
+                    fence_proxy_async();  // order these writes before the stage's next TMA fill
+                    __syncwarp();
+                }
+            }
+
+            if constexpr (FP8 && kFp8WidenCvt) {
+                if (kb + BPU * kBlockSize > min(ctx, kend)) {
+                    // the unit's last keys lie past the context or past this round's blocks
+                    // (a never-loaded second block): zero their V bytes, dim row by dim row,
+                    // so that no stale NaN code reaches P.V (masked keys get P = 0)
+#pragma unroll
+                    for (int h = 0; h < BPU; ++h) {
+                        const int k0 = kb + h * kBlockSize;
+                        const int nz = k0 >= kend ? 0 : min(max(ctx - k0, 0), kBlockSize);
+                        if (nz == kBlockSize) continue;
+                        uint8_t* vg = smem + (stage + (2 * h + 1) * C::kTileBytes - smem_u32(smem));
+                        for (int d = lane; d < D; d += 32) {
+                            uint4* cp = reinterpret_cast<uint4*>(vg + sw128(d >> 3, d & 7));
+                            uint4 x = *cp;
+                            uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const int keep = min(max(nz - 4 * j, 0), 4);  // valid codes of word j
+                                w[j] = keep == 4 ? w[j] : (w[j] & ((1u << (8 * keep)) - 1u));
+                            }
+                            *cp = make_uint4(w[0], w[1], w[2], w[3]);
+                        }
                     }
                     fence_proxy_async();  // order these writes before the stage's next TMA fill
                     __syncwarp();
@@ -393,7 +427,7 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
             } else {
                 // P^T for keys (4t, 4t+2 | 4t+1, 4t+3) (the row permutation of S^T) against the
                 // dim-major V tile: one ldmatrix word per dim row holds keys 4t..4t+3, widened
-                // exactly to f16 (as 2^-8 V) in an even and an odd half
+                // exactly to f16 in an even and an odd half
 #pragma unroll
                 for (int h = 0; h < BPU; ++h) {
                     const uint32_t vt = stage + (2 * h + 1) * C::kTileBytes;
@@ -406,10 +440,17 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
                         uint32_t r0, r1, r2, r3;
                         ldsm_x4(vt + sw128(d >> 3, d & 7), r0, r1, r2, r3);
                         uint32_t e0, d0, e1, d1, e2, d2, e3, d3;
-                        e4m3x4_to_f16x2_scaled(r0, e0, d0);
-                        e4m3x4_to_f16x2_scaled(r1, e1, d1);
-                        e4m3x4_to_f16x2_scaled(r2, e2, d2);
-                        e4m3x4_to_f16x2_scaled(r3, e3, d3);
+                        if constexpr (kFp8WidenCvt) {
+                            e4m3x4_to_f16x2_cvt(r0, e0, d0);
+                            e4m3x4_to_f16x2_cvt(r1, e1, d1);
+                            e4m3x4_to_f16x2_cvt(r2, e2, d2);
+                            e4m3x4_to_f16x2_cvt(r3, e3, d3);
+                        } else {
+                            e4m3x4_to_f16x2_scaled(r0, e0, d0);
+                            e4m3x4_to_f16x2_scaled(r1, e1, d1);
+                            e4m3x4_to_f16x2_scaled(r2, e2, d2);
+                            e4m3x4_to_f16x2_scaled(r3, e3, d3);
+                        }
                         mma_f16(o[2 * mp], e0, e1, d0, d1, pb0, pb1);
                         mma_f16(o[2 * mp + 1], e2, e3, d2, d3, pb0, pb1);
                     }
@@ -423,7 +464,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
             // wind down: wait (bounded, 0.1 s each) for this warp's loads still in flight
             for (int i = fail_i; i < min(fail_i + NS, mine); ++i) {
                 const uint32_t n = loads + i;
-                mbar_wait(smem_u32(&bars[warp * NS + n % NS]), (n / NS) & 1u, wind_ns,
+                mbar_wait(smem_u32(&bars[warp * NS + n % NS]), (n / NS) & 1u,
+                          inject() ? p.test_wait_ns : kWindDownLimitNs,
                           p.err);
             }
         }
@@ -458,13 +500,82 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
     }
     if (!__syncthreads_and(ok)) return;
 
-    const float vscale = FP8 ? 256.f * p.v_scale[g] : 1.f;  // FP8 V was widened as 2^-8 V
+    // FP8: the V scale, times 2^8 when V was widened as 2^-8 V
+    const float vscale = FP8 ? (kFp8WidenCvt ? 1.f : 256.f) * p.v_scale[g] : 1.f;
     const bool direct = nsplit == 1;
     if (!direct && split >= p.max_splits) {  // workspace bound (a planned launch never hits it)
         if (tid == 0) raise_error(p.err, kErrMetadata);
         return;
     }
     const int64_t stride = static_cast<int64_t>(p.num_tokens) * p.num_q_heads;  // one split
+    if (direct && p.prefix_parts > 0) {
+        // cascade, one split: merge the shared prefix's partials (normalised, log2 LSEs) into
+        // each row, out = sum_k 2^(lse_k - X) O_k / sum_k 2^(lse_k - X).  One warp per row, lane
+        // l owning dims l, l + 32, ...; every partial of the row is loaded before any is used,
+        // so their latencies overlap.
+        constexpr int DL = D / 32;
+        const int parts = min(p.prefix_parts, kMaxPrefixParts);
+        for (int n = warp; n < rows; n += NW) {
+            const int64_t row = static_cast<int64_t>(q0 + n / p.group) * p.num_q_heads +
+                                g * p.group + n % p.group;
+            float plse[kMaxPrefixParts], po[kMaxPrefixParts][DL];
+#pragma unroll
+            for (int k = 0; k < kMaxPrefixParts; ++k) {
+                plse[k] = -INFINITY;
+#pragma unroll
+                for (int i = 0; i < DL; ++i) po[k][i] = 0.f;
+                if (k < parts) {
+                    plse[k] = __ldcg(p.prefix_lse + k * stride + row);
+#pragma unroll
+                    for (int i = 0; i < DL; ++i)
+                        po[k][i] = __ldcg(p.prefix_o + (k * stride + row) * D + lane + 32 * i);
+                }
+            }
+            // this row's result over its own keys, from the warps' states
+            float M = -INFINITY;
+#pragma unroll
+            for (int w = 0; w < NW; ++w) M = fmaxf(M, red_m[w * 8 + n]);
+            float L = 0.f, acc[DL];
+#pragma unroll
+            for (int i = 0; i < DL; ++i) acc[i] = 0.f;
+            if (M != -INFINITY) {
+#pragma unroll
+                for (int w = 0; w < NW; ++w) {
+                    const float e = fast_exp2(red_m[w * 8 + n] - M);
+                    L += red_l[w * 8 + n] * e;
+#pragma unroll
+                    for (int i = 0; i < DL; ++i) acc[i] += red_o[(w * D + lane + 32 * i) * 8 + n] * e;
+                }
+            }
+            const float lse2 = L > 0.f ? M + __log2f(L) : -INFINITY;
+            float X = lse2;
+#pragma unroll
+            for (int k = 0; k < kMaxPrefixParts; ++k) X = fmaxf(X, plse[k]);
+            float W = 0.f, o[DL];
+#pragma unroll
+            for (int i = 0; i < DL; ++i) o[i] = 0.f;
+            if (X != -INFINITY) {
+                if (L > 0.f) {
+                    const float ws = fast_exp2(lse2 - X);
+                    W = ws;
+#pragma unroll
+                    for (int i = 0; i < DL; ++i) o[i] = ws * (acc[i] / L * vscale);
+                }
+#pragma unroll
+                for (int k = 0; k < kMaxPrefixParts; ++k) {
+                    const float wk = fast_exp2(plse[k] - X);  // 0 for parts past `parts`
+                    W += wk;
+#pragma unroll
+                    for (int i = 0; i < DL; ++i) o[i] += wk * po[k][i];
+                }
+            }
+            const float inv = W > 0.f ? 1.f / W : 0.f;
+#pragma unroll
+            for (int i = 0; i < DL; ++i) p.out[row * D + lane + 32 * i] = o[i] * inv;
+            if (lane == 0 && p.lse_out) p.lse_out[row] = W > 0.f ? (X + __log2f(W)) * kLn2 : -INFINITY;
+        }
+        return;
+    }
     for (int idx = tid; idx < rows * D; idx += NW * 32) {
         const int n = idx / D, d = idx % D;
         float M = -INFINITY;
@@ -479,32 +590,13 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
                 acc += red_o[(w * D + d) * 8 + n] * e;
             }
         }
-        float val = L > 0.f ? acc / L * vscale : 0.f;
+        const float val = L > 0.f ? acc / L * vscale : 0.f;
         const int t = q0 + n / p.group;
         const int h = g * p.group + n % p.group;
         if (direct) {
             const int64_t row = static_cast<int64_t>(t) * p.num_q_heads + h;
-            float lse2 = L > 0.f ? M + __log2f(L) : -INFINITY;
-            if (p.prefix_parts > 0) {
-                // cascade: merge the shared prefix's partials (normalised, log2 LSEs) with this
-                // row's suffix result: out = sum_k 2^(lse_k - X) O_k / sum_k 2^(lse_k - X)
-                float X = lse2;
-                for (int k = 0; k < p.prefix_parts; ++k) X = fmaxf(X, __ldcg(p.prefix_lse + k * stride + row));
-                float W = 0.f, a = 0.f;
-                if (X != -INFINITY) {
-                    W = fast_exp2(lse2 - X);
-                    a = W * val;
-                    for (int k = 0; k < p.prefix_parts; ++k) {
-                        const float w = fast_exp2(__ldcg(p.prefix_lse + k * stride + row) - X);
-                        W += w;
-                        a += w * __ldcg(p.prefix_o + (k * stride + row) * D + d);
-                    }
-                }
-                val = W > 0.f ? a / W : 0.f;
-                lse2 = W > 0.f ? X + __log2f(W) : -INFINITY;
-            }
             p.out[row * D + d] = val;
-            if (d == 0 && p.lse_out) p.lse_out[row] = lse2 * kLn2;
+            if (d == 0 && p.lse_out) p.lse_out[row] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
         } else {
             const int64_t prow = split * stride + static_cast<int64_t>(t) * p.num_q_heads + h;
             p.part_o[prow * D + d] = val;

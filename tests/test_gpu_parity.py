@@ -328,7 +328,8 @@ def test_slot_validator_counts_out_of_pool_and_duplicate_slots(seed):
     # seeded bad slot maps: some slots pushed past the pool, some copied onto other tokens'
     # slots, some skips; the expected counts are taken from the map itself
     rng = np.random.default_rng(500 + seed)
-    wl = _small([int(x) for x in rng.integers(20, 300, 6)], [1] * 6, 8, 2, 128, seed=seed)
+    wl = _small([int(x) for x in rng.integers(20, 300, 6)], [1] * 6, 8, 2, 128, seed=seed,
+                nb=512)
     st = GpuStep(wl, run_attention=False)
     num_slots = wl.num_blocks * 16
     n = 4000
