@@ -360,12 +360,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
 
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t bar_kf[kKSlots], bar_ke[kKSlots], bar_vf[kVSlots], bar_ve[kVSlots];
-    // per q-tile and S buffer: S computed / P stored.  The softmax may store P of tile j + 1
-    // before the MMA warp has taken P of tile j, so one P barrier per buffer keeps every
-    // parity wait within one phase of its barrier.
-    __shared__ uint64_t bar_sf[kQTiles][2], bar_pf[kQTiles][2];
+    __shared__ uint64_t bar_sf[kQTiles][2], bar_pf[kQTiles];  // S buffer computed / P stored
     __shared__ uint64_t bar_o[kQTiles];                    // a P V of the q-tile done
-    __shared__ uint64_t bar_done[kQTiles];                 // every MMA of the q-tile done
     __shared__ uint64_t bar_q;                             // Q staged by the softmax warps
     __shared__ uint32_t tmem_holder;
     __shared__ int ids[kMaxIds];  // physical ids of the split's first kMaxIds logical blocks
@@ -398,10 +394,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
         for (int q = 0; q < kQTiles; ++q) {
             mbar_init(smem_u32(&bar_sf[q][0]), 1);
             mbar_init(smem_u32(&bar_sf[q][1]), 1);
-            mbar_init(smem_u32(&bar_pf[q][0]), kRows);
-            mbar_init(smem_u32(&bar_pf[q][1]), kRows);
+            mbar_init(smem_u32(&bar_pf[q]), kRows);
             mbar_init(smem_u32(&bar_o[q]), 1);
-            mbar_init(smem_u32(&bar_done[q]), 1);
         }
         mbar_init(smem_u32(&bar_q), kQLoaders);
         fence_barrier_init();
@@ -556,7 +550,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
                         break;
                     bool w = true;
                     for (int q = 0; q < nq; ++q) {
-                        if (!mbar_wait(smem_u32(&bar_pf[q][kt & 1]), (kt >> 1) & 1, kWaitLimitNs, err)) {
+                        if (!mbar_wait(smem_u32(&bar_pf[q]), kt & 1, kWaitLimitNs, err)) {
                             w = false;
                             break;
                         }
@@ -567,10 +561,6 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
                     if (!w) break;
                     mma_commit(smem_u32(&bar_ve[kt % kVSlots]));
                     if (more) mma_commit(smem_u32(&bar_ke[tk % kKSlots]));
-                    // after the last tile: one more commit per q-tile, which completes once
-                    // every MMA issued so far has (the epilogue's single wait)
-                    if (kt + 1 == ntiles)
-                        for (int q = 0; q < nq; ++q) mma_commit(smem_u32(&bar_done[q]));
                 }
             }
         }
@@ -828,13 +818,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
                     fence_proxy_async();
                 }
                 tc_fence_before();
-                mbar_arrive(smem_u32(&bar_pf[q][kt & 1]));
+                mbar_arrive(smem_u32(&bar_pf[q]));
             }
-            // ---- epilogue: O / l for this row, once every MMA of the q-tile has completed.  (The
-            // last two P V may both be outstanding or both done here; a parity wait on bar_o
-            // cannot tell "two phases ahead" from "none", so the MMA warp commits once more to
-            // bar_done, a barrier of a single phase.)
-            if (ok && ntiles > 0 && !mbar_wait(smem_u32(&bar_done[q]), 0, kWaitLimitNs, err))
+            // ---- epilogue: O / l for this row.  The S of tile ntiles - 1 was committed after
+            // P V (ntiles - 3), so the last two P V of the q-tile may be outstanding: wait for
+            // them in order (a parity wait tells one pending phase from none, not two).
+            if (ok && ntiles > 1 &&
+                !mbar_wait(smem_u32(&bar_o[q]), (ntiles - 2) & 1, kWaitLimitNs, err))
+                ok = false;
+            if (ok && ntiles > 0 && !mbar_wait(smem_u32(&bar_o[q]), (ntiles - 1) & 1, kWaitLimitNs, err))
                 ok = false;
             // tcgen05.ld is warp-collective: the whole warp loads (or none of it)
             const bool all_ok = __all_sync(0xffffffffu, ok);
