@@ -228,7 +228,7 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
     int dec_max_blocks = 0, chunk_max_blocks = 0, chunk_max_qtiles = 0;
     // chunk work in key tiles: the CTA of each q-tile walks the keys its last row may see
     const int chunk_cta_rows = pa::chunk_rows(D, 1);
-    const int chunk_tile_keys = pa::kChunkTileKeys;
+    const int chunk_tile_keys = D == 128 ? 128 : 64;
     long long chunk_work = 0, chunk_work_max = 0;
     for (int r = 0; r < B; ++r) {
         const int ql = qsl[r + 1] - qsl[r];
@@ -351,7 +351,7 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
         // the prefix pass: all T * G query rows of each kv head against the P prefix keys,
         // split so that the chunk kernel fills the SMs (each split at least two key tiles)
         const int rows_per_cta = pa::chunk_rows(D, 1);
-        const int tile_blocks = pa::kChunkTileKeys / bs;
+        const int tile_blocks = (D == 128 ? 128 : 64) / bs;
         const long long qtiles = pa::ceil_div(T * G, rows_per_cta);
         const int pblocks = P / bs;
         const int ptiles = pa::ceil_div(pblocks, tile_blocks);
@@ -671,7 +671,7 @@ int pa::attention_call(const pa_cache* cache, const void* q, int num_q_heads,
         pp.chunk_fused_merge = 0;
         pp.lse_out = nullptr;
         const int rows_per_cta = pa::chunk_rows(cache->head_size, 1);
-        const int tile_keys = pa::kChunkTileKeys;
+        const int tile_keys = cache->head_size == 128 ? 128 : 64;
         const int qtiles = pa::ceil_div(num_tokens * pp.group, rows_per_cta);
         pp.chunk_max_qtiles = qtiles;
         static thread_local pa::ChunkWork pwork;
@@ -716,7 +716,7 @@ int pa::attention_call(const pa_cache* cache, const void* q, int num_q_heads,
         // the chunk CTAs, most key tiles first; a list that does not fit falls back to the grid
         items.clear();
         const int cta_rows = pa::chunk_rows(cache->head_size, 1);
-        const int tile_keys = pa::kChunkTileKeys;
+        const int tile_keys = cache->head_size == 128 ? 128 : 64;
         const int csb = p.chunk_split_blocks;
         bool fits = list.count > 0;
         for (int i = 0; i < list.count && fits; ++i) {

@@ -16,7 +16,7 @@ namespace pa {
 namespace {
 
 constexpr uint32_t kFull = 0xffffffffu;
-constexpr int kTileKeys = kChunkTileKeys;
+constexpr int kTileKeys = 64;
 constexpr int kBlocksPerTile = kTileKeys / kBlockSize;
 constexpr int kMaxIds = 1024;  // block ids staged in shared memory
 

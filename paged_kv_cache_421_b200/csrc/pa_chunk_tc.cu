@@ -9,28 +9,27 @@
 // How.  One CTA owns two 128-row query tiles (256 rows of one (request, kv head)) and
 // optionally one KV split; one CTA per SM.  Its warps specialise: warps 0-7 run the softmax
 // (warps 4q..4q+3 serve q-tile q; thread i of the q-tile owns row i, which is TMEM lane i),
-// warp 8 issues the tensor-core MMAs, warp 9 the TMA loads.  Keys are walked in tiles of 64
-// (four physical blocks from the block table); each block's K and V tiles arrive by TMA (4-D
-// loads, 128-byte swizzle) into four-slot K and V rings laid out [8-key group][64-dim half]
-// [8 keys][128 B], so one layout is the K-major B operand of S = Q K^T and the MN-major B
-// operand of O += P V.  TMEM (512 columns): per q-tile two S buffers of 64 columns, in whose
-// first 32 columns the softmax stores its tile's P (bf16 pairs), and O (128 columns).
-// S of tiles 0 and 1 are computed first; then for tile j the MMA warp issues
-//     O_0 += P_0 V_j,  S_0(j+2) = Q_0 K_{j+2}^T,  O_1 += P_1 V_j,  S_1(j+2) = Q_1 K_{j+2}^T
-// (tcgen05.mma with M 128 and K 16, N 128 dims or 64 keys, fp32 accumulate), the S of tile
-// j + 2 into the buffer that P V of tile j has just read: tcgen05.mma instructions of one
-// thread execute in issue order.  So each softmax warpgroup finds the S of its next tile
-// already computed when it finishes one, and the tensor core works on one q-tile while the
-// other's softmax runs.  O is rescaled lazily, only when a row's max grows by more than 2^8 (a
-// stale max keeps every probability <= 256; numerator and denominator share it, so results
-// are exact), after waiting for the q-tile's previous P V.  Full/empty mbarriers and
-// tcgen05.commit replace CTA barriers inside the loop.  Every wait is bounded: on a timeout
-// each role records the error and stops, and the CTA frees its TMEM and returns.
+// warp 8 issues the tensor-core MMAs, warp 9 the TMA loads.  Keys are walked in tiles of 128
+// (eight physical blocks from the block table); each block's K and V tiles arrive by TMA (2-D
+// loads, 128-byte swizzle) into two-slot K and V rings laid out [64-dim half][key][128 B], so
+// one layout is the K-major B operand of S = Q K^T and the MN-major B operand of O += P V.
+// TMEM (512 columns): per q-tile an S buffer of 128 columns, in whose first 64 columns the
+// softmax stores P (bf16 pairs), and O (128 columns).  Per tile j the MMA warp issues
+//     O_0 += P_0 V_j,  S_0 = Q_0 K_{j+1}^T,  O_1 += P_1 V_j,  S_1 = Q_1 K_{j+1}^T
+// (8 tcgen05.mma each: M 128, N 128, K 16, fp32 accumulate), so the tensor core computes one
+// q-tile's products while the other q-tile's softmax runs.  S_q of tile j+1 overwrites P_q of
+// tile j only after the P V that reads it: tcgen05.mma instructions of one thread execute in
+// issue order.  For the same reason the commit that signals S_q(j+1) also covers O_q += P_q
+// V_j, so the softmax may rescale O as soon as it sees S.  O is rescaled lazily, only when a
+// row's max grows by more than 2^8 (a stale max keeps every probability <= 256; numerator and
+// denominator share it, so results are exact).  Full/empty mbarriers and tcgen05.commit
+// replace CTA barriers inside the loop.  Every wait is bounded: on a timeout each role
+// records the error and stops, and the CTA frees its TMEM and returns.
 //
 // FP8 E4M3 cache ("vLLM: from KV Cache to high-throughput serving", article 6 outline names
 // the format).  The same schedule runs on kind::f8f6f4 MMAs with both operands E4M3, straight
-// from the cache bytes: a K tile is four 2 KB block tiles [16 keys][128 B] (2-D TMA, 128-byte
-// swizzle: the K-major B operand of S = Q K^T), a V tile four dim-major block tiles [128 dims]
+// from the cache bytes: a K tile is eight 2 KB block tiles [16 keys][128 B] (2-D TMA, 128-byte
+// swizzle: the K-major B operand of S = Q K^T), a V tile eight dim-major block tiles [128 dims]
 // [16 keys] (bulk copies of the stored bytes: K-major B operand of O += P V without swizzle,
 // 16-key core matrices 2 KB apart).  Q and P keep bf16-level precision as two E4M3 terms each
 // (x ~ e4m3(x) + e4m3(x - e4m3(x)), Q after scaling each row by a power of two), and every
@@ -44,46 +43,42 @@ namespace {
 constexpr int kD = 128;
 constexpr int kRows = 128;                       // query rows per q-tile = TMEM lanes
 constexpr int kQTiles = 2;                       // q-tiles per CTA, sharing every K/V tile
-constexpr int kKeys = kChunkTileKeys;            // keys per tile (64)
-constexpr int kTileBlocks = kKeys / kBlockSize;  // 4 physical blocks
+constexpr int kKeys = 128;                       // keys per tile
+constexpr int kTileBlocks = kKeys / kBlockSize;  // 8 physical blocks
 constexpr int kHalfRows = 128;                   // bytes per swizzled row (64 bf16)
 constexpr int kQHalf = kRows * kHalfRows;        // 16 KB: one 64-dim half of a q-tile
 constexpr int kQBytes = 2 * kQHalf;              // 32 KB per q-tile
-// A K or V tile (64 keys x 128 dims, 16 KB) is four 4 KB block tiles, each laid out as
+// A K or V tile (128 keys x 128 dims, 32 KB) is eight 4 KB block tiles, each laid out as
 // [8-row group][64-dim half][8 rows][128 B]: 8-key groups are kGroupStride apart for every key
 // of the tile, the two halves of a group kAtom apart (one 128-byte swizzle atom each).
 constexpr int kAtom = 8 * kHalfRows;             // 1 KB: 8 rows x 128 B
 constexpr int kGroupStride = 2 * kAtom;          // 2 KB between consecutive 8-key groups
 constexpr int kBlockTile = kBlockSize * 2 * kHalfRows;  // 4 KB: one block's 16 x 128 tile
-constexpr int kKBytes = kTileBlocks * kBlockTile;       // 16 KB per K or V tile
-constexpr int kKSlots = 4, kVSlots = 4;                 // ring depths (K runs two tiles ahead)
+constexpr int kKBytes = kTileBlocks * kBlockTile;       // 32 KB per K or V tile
+constexpr int kKSlots = 2, kVSlots = 2;
 constexpr int kSmemBytes = kQTiles * kQBytes + (kKSlots + kVSlots) * kKBytes + 1024;  // 193 KB
 // FP8 cache: 2 KB block tiles, 16 KB K or V tiles; each q-tile holds two E4M3 terms of Q,
 // [128 rows][128 B] each (one 128-byte swizzle atom per row), in the same 32 KB as bf16 Q.
 constexpr int kBlockTile8 = kBlockSize * kD;              // 2 KB
-constexpr int kKBytes8 = kTileBlocks * kBlockTile8;       // 8 KB per K or V tile
+constexpr int kKBytes8 = kTileBlocks * kBlockTile8;       // 16 KB per K or V tile
 constexpr int kQTerm8 = kRows * 128;                      // 16 KB per E4M3 term of a q-tile
 constexpr int kSmemBytes8 = kQTiles * kQBytes + (kKSlots + kVSlots) * kKBytes8 + 1024;  // 129 KB
 constexpr uint32_t kTmemCols = 512;
-// TMEM of q-tile q: two S buffers of kKeys columns at 256q and 256q + kKeys (P is written over
-// the first columns of its tile's S), then O at 256q + 128
-constexpr uint32_t kColO = 128;
+constexpr uint32_t kColO = 128;                  // q-tile q: S/P [256q, 256q+128), O after it
 constexpr int kMaxIds = 1024;                    // block ids staged in shared memory
 
 // Instruction descriptors (kind::f16): fp32 accumulate, bf16 A and B, M = 128.
-// S = Q K^T: A and B K-major, N = kKeys.  O = P V: B (V) MN-major, N = 128 dims.
+// S = Q K^T: A and B K-major, N = 128 keys.  O = P V: B (V) MN-major, N = 128 dims.
 constexpr uint32_t kIdescQK = (1u << 4) | (1u << 7) | (1u << 10) |
                               (static_cast<uint32_t>(kKeys >> 3) << 17) |
                               (static_cast<uint32_t>(kRows >> 4) << 24);
 constexpr uint32_t kIdescPV = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
                               (static_cast<uint32_t>(kD >> 3) << 17) |
                               (static_cast<uint32_t>(kRows >> 4) << 24);
-// kind::f8f6f4: fp32 accumulate, E4M3 A and B (format 0), both K-major, M = 128; N = kKeys for
-// S = Q K^T, N = 128 dims for O = P V.
-constexpr uint32_t kIdesc8QK = (1u << 4) | (static_cast<uint32_t>(kKeys >> 3) << 17) |
-                               (static_cast<uint32_t>(kRows >> 4) << 24);
-constexpr uint32_t kIdesc8PV = (1u << 4) | (static_cast<uint32_t>(kD >> 3) << 17) |
-                               (static_cast<uint32_t>(kRows >> 4) << 24);
+// kind::f8f6f4: fp32 accumulate, E4M3 A and B (format 0), both K-major, M = 128, N = 128 (keys
+// for S = Q K^T, dims for O = P V).
+constexpr uint32_t kIdesc8 = (1u << 4) | (static_cast<uint32_t>(128 >> 3) << 17) |
+                             (static_cast<uint32_t>(kRows >> 4) << 24);
 
 // Shared-memory matrix descriptor: start address, leading / stride byte offsets (16-byte
 // units), descriptor version 1, 128-byte swizzle.
@@ -360,7 +355,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
 
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t bar_kf[kKSlots], bar_ke[kKSlots], bar_vf[kVSlots], bar_ve[kVSlots];
-    __shared__ uint64_t bar_sf[kQTiles][2], bar_pf[kQTiles];  // S buffer computed / P stored
+    __shared__ uint64_t bar_sf[kQTiles], bar_pf[kQTiles];  // S computed / P stored
     __shared__ uint64_t bar_o[kQTiles];                    // a P V of the q-tile done
     __shared__ uint64_t bar_q;                             // Q staged by the softmax warps
     __shared__ uint32_t tmem_holder;
@@ -392,8 +387,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
             mbar_init(smem_u32(&bar_ve[i]), 1);
         }
         for (int q = 0; q < kQTiles; ++q) {
-            mbar_init(smem_u32(&bar_sf[q][0]), 1);
-            mbar_init(smem_u32(&bar_sf[q][1]), 1);
+            mbar_init(smem_u32(&bar_sf[q]), 1);
             mbar_init(smem_u32(&bar_pf[q]), kRows);
             mbar_init(smem_u32(&bar_o[q]), 1);
         }
@@ -417,12 +411,12 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
     if (warp >= 8) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsProducer));
         if (warp == 9) {
-            // ================= TMA producer: K two tiles ahead of V (S of tile j + 2 is computed
-            // right after P V of tile j).  The expected bytes are posted first, then lane i
-            // issues block i's whole tile, so the per-copy issue latency overlaps across the warp.
+            // ================= TMA producer: K one tile ahead of V.  The expected bytes are
+            // posted first, then lane i issues block i's whole 4 KB tile, so the per-copy
+            // issue latency overlaps across the warp.
             const int kv_rows_per_block = 2 * p.num_kv_heads * kBlockSize;
             auto load = [&](int t, int which) {
-                const int st = t % (which ? kVSlots : kKSlots);
+                const int st = t & 1;
                 const uint32_t bar = smem_u32(which ? &bar_vf[st] : &bar_kf[st]);
                 const uint32_t dst = (which ? v_s : k_s) + st * kSlotBytes;
                 const int j0 = key_lo / kBlockSize + t * kTileBlocks;
@@ -455,23 +449,21 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
                 }
                 __syncwarp();
             };
-            // step t issues K(t) and V(t - 2); a slot is free once the MMAs that read its
+            // step t issues K(t) and V(t - 1); a slot is free once the MMAs that read its
             // previous tile have completed (their commit arrives on the slot's empty barrier)
-            for (int t = 0; t < ntiles + 2 && ok; ++t) {
+            for (int t = 0; t < ntiles + 1 && ok; ++t) {
                 if (t < ntiles) {
                     if (t >= kKSlots &&
-                        !__all_sync(0xffffffffu,
-                                    mbar_wait(smem_u32(&bar_ke[t % kKSlots]), ((t / kKSlots) + 1) & 1,
-                                              kWaitLimitNs, err)))
+                        !__all_sync(0xffffffffu, mbar_wait(smem_u32(&bar_ke[t & 1]), ((t >> 1) + 1) & 1,
+                                                           kWaitLimitNs, err)))
                         ok = false;
                     if (ok) load(t, 0);
                 }
-                const int tv = t - 2;
-                if (ok && tv >= 0 && tv < ntiles) {
+                const int tv = t - 1;
+                if (ok && tv >= 0) {
                     if (tv >= kVSlots &&
-                        !__all_sync(0xffffffffu,
-                                    mbar_wait(smem_u32(&bar_ve[tv % kVSlots]), ((tv / kVSlots) + 1) & 1,
-                                              kWaitLimitNs, err)))
+                        !__all_sync(0xffffffffu, mbar_wait(smem_u32(&bar_ve[tv & 1]), ((tv >> 1) + 1) & 1,
+                                                           kWaitLimitNs, err)))
                         ok = false;
                     if (ok) load(tv, 1);
                 }
@@ -479,15 +471,14 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
         } else if (warp == 8) {
             // ================= MMA issuer
             if (lane == 0 && ntiles > 0) {
-                auto qk = [&](int q, int t) {  // S_q(t) = Q_q K_t^T into S buffer t % 2
-                    const uint32_t ks = k_s + (t % kKSlots) * kSlotBytes;
-                    const uint32_t sd = tmem + q * 256 + (t & 1) * kKeys;
+                auto qk = [&](int q, int t) {  // S_q = Q_q K_t^T
+                    const uint32_t ks = k_s + (t & 1) * kSlotBytes;
                     if constexpr (!FP8) {
 #pragma unroll
                         for (int k = 0; k < kD / 16; ++k) {
                             const uint32_t off = q * kQBytes + (k >> 2) * kQHalf + (k & 3) * 32;
                             const uint32_t koff = (k >> 2) * kAtom + (k & 3) * 32;
-                            mma_ss(sd, smem_desc(q_s + off, 16, 1024),
+                            mma_ss(tmem + q * 256, smem_desc(q_s + off, 16, 1024),
                                    smem_desc(ks + koff, 16, kGroupStride), kIdescQK, k > 0);
                         }
                     } else {
@@ -496,56 +487,45 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
                         for (int k = 0; k < kD / 32; ++k)
 #pragma unroll
                             for (int term = 0; term < 2; ++term)
-                                mma_ss8(sd,
+                                mma_ss8(tmem + q * 256,
                                         smem_desc(q_s + q * kQBytes + term * kQTerm8 + k * 32, 16, 1024),
-                                        smem_desc(ks + k * 32, 16, 1024), kIdesc8QK, (k | term) > 0);
+                                        smem_desc(ks + k * 32, 16, 1024), kIdesc8, (k | term) > 0);
                     }
-                    mma_commit(smem_u32(&bar_sf[q][t & 1]));
+                    mma_commit(smem_u32(&bar_sf[q]));
                 };
-                auto pv = [&](int q, int t) {  // O_q += P_q(t) V_t (P from TMEM, S buffer t % 2)
-                    const uint32_t vs = v_s + (t % kVSlots) * kSlotBytes;
-                    const uint32_t pa = tmem + q * 256 + (t & 1) * kKeys;
+                auto pv = [&](int q, int t) {  // O_q += P_q V_t (P from TMEM)
+                    const uint32_t vs = v_s + (t & 1) * kSlotBytes;
                     if constexpr (!FP8) {
 #pragma unroll
                         for (int j = 0; j < kKeys / 16; ++j)
-                            mma_ts(tmem + q * 256 + kColO, pa + 8 * j,
+                            mma_ts(tmem + q * 256 + kColO, tmem + q * 256 + 8 * j,
                                    smem_desc(vs + j * kBlockTile, kAtom, kGroupStride), kIdescPV,
                                    (t > 0 || j > 0) ? 1u : 0u);
                     } else {
-                        // 32 keys per MMA: P's two terms (kKeys / 4 columns each, four E4M3 codes
-                        // per column) against block tiles 2j and 2j + 1
+                        // 32 keys per MMA: P's two terms (columns [0, 32) and [32, 64), four
+                        // E4M3 codes per column) against block tiles 2j and 2j + 1
 #pragma unroll
                         for (int j = 0; j < kKeys / 32; ++j)
 #pragma unroll
                             for (int term = 0; term < 2; ++term)
-                                mma_ts8(tmem + q * 256 + kColO, pa + term * (kKeys / 4) + 8 * j,
+                                mma_ts8(tmem + q * 256 + kColO, tmem + q * 256 + 32 * term + 8 * j,
                                         smem_desc_noswizzle(vs + 2 * j * kBlockTile8, kBlockTile8, 128),
-                                        kIdesc8PV, (t > 0 || j > 0 || term > 0) ? 1u : 0u);
+                                        kIdesc8, (t > 0 || j > 0 || term > 0) ? 1u : 0u);
                     }
                     mma_commit(smem_u32(&bar_o[q]));
                 };
-                // S of tiles 0 and 1 up front; then, per tile j and q-tile: P V (j), and S of tile
-                // j + 2 into the buffer that P V (j) has just read (tcgen05 MMAs of one thread run
-                // in issue order)
-                if (mbar_wait(smem_u32(&bar_q), 0, kWaitLimitNs, err)) {
-                    for (int t = 0; t < min(2, ntiles) && ok; ++t) {
-                        if (!mbar_wait(smem_u32(&bar_kf[t]), 0, kWaitLimitNs, err)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        for (int q = 0; q < nq; ++q) qk(q, t);
-                        mma_commit(smem_u32(&bar_ke[t]));
-                    }
+                if (mbar_wait(smem_u32(&bar_q), 0, kWaitLimitNs, err) &&
+                    mbar_wait(smem_u32(&bar_kf[0]), 0, kWaitLimitNs, err)) {
+                    tc_fence_after();
+                    for (int q = 0; q < nq; ++q) qk(q, 0);
+                    mma_commit(smem_u32(&bar_ke[0]));
                 } else {
                     ok = false;
                 }
                 for (int kt = 0; kt < ntiles && ok; ++kt) {
-                    const bool more = kt + 2 < ntiles;
-                    const int tk = kt + 2;
-                    if (!mbar_wait(smem_u32(&bar_vf[kt % kVSlots]), (kt / kVSlots) & 1, kWaitLimitNs, err))
-                        break;
-                    if (more && !mbar_wait(smem_u32(&bar_kf[tk % kKSlots]), (tk / kKSlots) & 1,
+                    const bool more = kt + 1 < ntiles;
+                    if (!mbar_wait(smem_u32(&bar_vf[kt & 1]), (kt >> 1) & 1, kWaitLimitNs, err)) break;
+                    if (more && !mbar_wait(smem_u32(&bar_kf[(kt + 1) & 1]), ((kt + 1) >> 1) & 1,
                                            kWaitLimitNs, err))
                         break;
                     bool w = true;
@@ -556,11 +536,11 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
                         }
                         tc_fence_after();
                         pv(q, kt);
-                        if (more) qk(q, tk);  // overwrites P_q(kt) after the P V above
+                        if (more) qk(q, kt + 1);  // overwrites P_q(kt) after the P V above
                     }
                     if (!w) break;
-                    mma_commit(smem_u32(&bar_ve[kt % kVSlots]));
-                    if (more) mma_commit(smem_u32(&bar_ke[tk % kKSlots]));
+                    mma_commit(smem_u32(&bar_ve[kt & 1]));
+                    if (more) mma_commit(smem_u32(&bar_ke[(kt + 1) & 1]));
                 }
             }
         }
@@ -670,22 +650,20 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
             for (int kt = 0; kt < ntiles; ++kt) {
                 const int key0 = key_lo + kt * kKeys;
                 // waits end warp-uniformly: the tcgen05 loads below are warp-collective
-                if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&bar_sf[q][kt & 1]), (kt >> 1) & 1,
-                                                       kWaitLimitNs, err))) {
+                if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&bar_sf[q]), kt & 1, kWaitLimitNs, err))) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t tbuf = tmem_lane + (kt & 1) * kKeys;  // this tile's S, then P
                 // only tiles crossing a causal limit or the split end need masking
                 const bool masked =
                     !(key0 + kKeys - 1 <= first_lim && key0 + kKeys <= kend && key0 >= last_lo);
-                // S of this row: all loads in flight, one wait (TMEM load latency is long)
+                // S of this row: all four loads in flight, one wait (TMEM load latency is long)
                 float sv[kKeys];
 #pragma unroll
                 for (int c = 0; c < kKeys / 32; ++c) {
                     uint32_t raw[32];
-                    tmem_ld32(tbuf + c * 32, raw);
+                    tmem_ld32(tmem_lane + c * 32, raw);
 #pragma unroll
                     for (int i = 0; i < 32; ++i) sv[c * 32 + i] = __uint_as_float(raw[i]);
                 }
@@ -714,14 +692,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
                     m_used = m_new;
                 }
                 if (__any_sync(0xffffffffu, alpha != 1.f) && kt > 0) {
-                    // rescale O (this warp's 32 rows) once the q-tile's previous P V has
-                    // completed; the next one is issued only after this tile's P is stored
-                    if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&bar_o[q]), (kt - 1) & 1,
-                                                           kWaitLimitNs, err))) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after();
+                    // rescale O (this warp's 32 rows): the commit that signalled S of this tile
+                    // also covers the q-tile's previous P V
                     l *= alpha;
 #pragma unroll
                     for (int c = 0; c < kD / 32; ++c) {
@@ -734,7 +706,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
                         tmem_st32(tmem_lane + kColO + c * 32, raw);
                     }
                 }
-                // P = 2^(s sl - m) as bf16 pairs over the first S columns, 32 keys at a time
+                // P = 2^(s sl - m) as bf16 pairs over the first 64 S columns, 32 keys at a time
                 const float neg_ref = m_used == -INFINITY ? 0.f : -m_used;
                 const float2 sl2 = make_float2(sl, sl), nr2 = make_float2(neg_ref, neg_ref);
                 float2 sp[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
@@ -749,10 +721,10 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
                             sp[i & 1] = fadd2(sp[i & 1], a);
                             packed[i] = pack_bf16(a.x, a.y);
                         }
-                        tmem_st16(tbuf + 16 * c, packed);
+                        tmem_st16(tmem_lane + 16 * c, packed);
                     } else {
                         // two E4M3 terms of P, four keys per 32-bit column: the first term in
-                        // the buffer's first kKeys / 4 columns, the second in the next ones
+                        // columns [0, 32), the second in [32, 64)
                         uint32_t hi[8], lo[8];
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
@@ -769,8 +741,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
                             hi[i] = h0 | (h1 << 16);
                             lo[i] = l0 | (l1 << 16);
                         }
-                        tmem_st8(tbuf + 8 * c, hi);
-                        tmem_st8(tbuf + kKeys / 4 + 8 * c, lo);
+                        tmem_st8(tmem_lane + 8 * c, hi);
+                        tmem_st8(tmem_lane + 32 + 8 * c, lo);
                     }
                 }
                 l += (sp[0].x + sp[0].y) + (sp[1].x + sp[1].y);
@@ -778,9 +750,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
                 if (q == 0 && key0 + kKeys > kend) {
                     // keys past the split / context: clear their V rows once V has landed (q-tile 0
                     // does it; its P V is issued before q-tile 1's)
-                    const int vslot = kt % kVSlots;
-                    if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&bar_vf[vslot]), (kt / kVSlots) & 1,
-                                                           kWaitLimitNs, err))) {
+                    const int vslot = kt & 1;
+                    if (!__all_sync(0xffffffffu,
+                                    mbar_wait(smem_u32(&bar_vf[vslot]), (kt >> 1) & 1, kWaitLimitNs, err))) {
                         ok = false;
                         break;
                     }
@@ -820,12 +792,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
                 tc_fence_before();
                 mbar_arrive(smem_u32(&bar_pf[q]));
             }
-            // ---- epilogue: O / l for this row.  The S of tile ntiles - 1 was committed after
-            // P V (ntiles - 3), so the last two P V of the q-tile may be outstanding: wait for
-            // them in order (a parity wait tells one pending phase from none, not two).
-            if (ok && ntiles > 1 &&
-                !mbar_wait(smem_u32(&bar_o[q]), (ntiles - 2) & 1, kWaitLimitNs, err))
-                ok = false;
+            // ---- epilogue: O / l for this row.  S of the last tile covers every P V before the
+            // last one, so one phase of the q-tile's P V barrier is outstanding here.
             if (ok && ntiles > 0 && !mbar_wait(smem_u32(&bar_o[q]), (ntiles - 1) & 1, kWaitLimitNs, err))
                 ok = false;
             // tcgen05.ld is warp-collective: the whole warp loads (or none of it)

@@ -21,7 +21,6 @@ constexpr int kChunkRows = 64;      // mma.sync chunk tile: 64 (token, q head) r
 constexpr int kMaxFusedSplits = 4;    // tcgen05 chunk kernel: splits it merges itself
 constexpr int kChunkRowsTc = 256;   // tcgen05 chunk CTA: two 128-row q-tiles (TMEM lanes)
 constexpr int kMaxPrefixParts = 4;  // cascade: prefix partials a decode row merges (planner cap)
-constexpr int kChunkTileKeys = 64;  // keys per tile of both chunk kernels (planner's work unit)
 
 // Error codes written to the device error word.
 constexpr int kErrWaitTimeout = 1;
