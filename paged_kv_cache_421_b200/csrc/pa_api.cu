@@ -160,6 +160,46 @@ int make_tensor_map(pa_cache* c) {
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// Tensor maps of a call's Q, output and (cascade) prefix partials for the tcgen05 chunk kernel
+// (head_size 128): Q as {128, Hq, T} bf16 with 128-byte boxes of G heads x 128 / G tokens (one
+// 128-row q-tile half per box, bf16 cache only: FP8 Q is split on the way in), O as
+// {128, Hq, T} fp32 and the partials as {128, Hq, T, S} fp32 with boxes of 32 floats x G heads x
+// 32 / G tokens (one warp's rows of one 32-column chunk).  A map whose shape does not fit (G
+// not dividing 128 or 32) is left unused.
+void make_chunk_io(pa::ChunkIo& io, const void* q, float* out, const float* part, int T, int Hq,
+                   int G, int S, bool q_ok) {
+    std::memset(&io, 0, sizeof(io));
+    EncodeTiledFn enc = encode_fn();
+    if (!enc || T <= 0) return;
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    if (q_ok && 128 % G == 0) {
+        cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(Hq), static_cast<cuuint64_t>(T)};
+        cuuint64_t strides[2] = {128 * 2, static_cast<cuuint64_t>(Hq) * 128 * 2};
+        cuuint32_t box[3] = {64, static_cast<cuuint32_t>(G), static_cast<cuuint32_t>(128 / G)};
+        if (enc(&io.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(q), dims, strides, box,
+                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
+            io.mode |= 1;
+    }
+    if (32 % G == 0) {
+        cuuint64_t dims[4] = {128, static_cast<cuuint64_t>(Hq), static_cast<cuuint64_t>(T),
+                              static_cast<cuuint64_t>(S > 0 ? S : 1)};
+        cuuint64_t strides[3] = {128 * 4, static_cast<cuuint64_t>(Hq) * 128 * 4,
+                                 static_cast<cuuint64_t>(T) * Hq * 128 * 4};
+        cuuint32_t box[4] = {32, static_cast<cuuint32_t>(G), static_cast<cuuint32_t>(32 / G), 1};
+        if (out && enc(&io.o, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, out, dims, strides, box, estr,
+                       CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                       CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                       CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
+            io.mode |= 2;
+        if (part && S > 0 &&
+            enc(&io.part, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<float*>(part), dims, strides,
+                box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS)
+            io.mode |= 4;
+    }
+}
+
 // Workspace of a plan with up to max_splits splits: partial outputs [S][T][Hq][D], partial
 // LSEs [S][T][Hq], then per-(request, kv head) finished-split counters indexed by the
 // request's first token (at most T x Hkv <= T x Hq of them).
@@ -690,8 +730,14 @@ int pa::attention_call(const pa_cache* cache, const void* q, int num_q_heads,
                          });
         pwork.count = 0;
         for (const auto& it : pitems) pwork.item[pwork.count++] = it.second;
+        static thread_local pa::ChunkIo pio;
+        if (cache->head_size == 128)
+            make_chunk_io(pio, q, nullptr, pp.part_o, num_tokens, num_q_heads, pp.group,
+                          pl.prefix_splits, cache->kv_dtype == PA_BF16);
+        else
+            std::memset(&pio, 0, sizeof(pio));
         if (ev) record(ev[2], s);
-        e = pa::launch_chunk(cache->tmap, cache->tmap_blk, pp, pwork, cache->head_size,
+        e = pa::launch_chunk(cache->tmap, cache->tmap_blk, pp, pwork, pio, cache->head_size,
                              cache->kv_dtype, pl.prefix_splits, s);
         if (e != cudaSuccess) return fail_cuda(e);
         if (ev) record(ev[3], s);
@@ -769,9 +815,15 @@ int pa::attention_call(const pa_cache* cache, const void* q, int num_q_heads,
         }
     }
     const cudaStream_t cs = side ? side->stream : s;  // the chunk kernel's stream
+    static thread_local pa::ChunkIo io;
+    if (pl.num_chunk_seqs && cache->head_size == 128)
+        make_chunk_io(io, q, out, nullptr, num_tokens, num_q_heads, p.group, 0,
+                      cache->kv_dtype == PA_BF16);
+    else
+        std::memset(&io, 0, sizeof(io));
     if (pl.num_chunk_seqs && side) {
         if (ev) record(ev[2], cs);
-        e = pa::launch_chunk(cache->tmap, cache->tmap_blk, p, work, cache->head_size,
+        e = pa::launch_chunk(cache->tmap, cache->tmap_blk, p, work, io, cache->head_size,
                              cache->kv_dtype, pl.chunk_max_splits, cs);
         if (e != cudaSuccess) return fail_cuda(e);
         if (ev) record(ev[3], cs);
@@ -785,7 +837,7 @@ int pa::attention_call(const pa_cache* cache, const void* q, int num_q_heads,
     }
     if (pl.num_chunk_seqs && !side) {
         if (ev) record(ev[2], s);
-        e = pa::launch_chunk(cache->tmap, cache->tmap_blk, p, work, cache->head_size,
+        e = pa::launch_chunk(cache->tmap, cache->tmap_blk, p, work, io, cache->head_size,
                              cache->kv_dtype, pl.chunk_max_splits, s);
         if (e != cudaSuccess) return fail_cuda(e);
         if (ev) record(ev[3], s);

@@ -240,6 +240,40 @@ __device__ __forceinline__ void split_e4m3x2(float2 a, uint32_t& hi, uint32_t& l
     lo = c2;
 }
 
+// 3-D tiled load (the Q map: {dim, head, token}).
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int x, int y, int z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+
+// Tiled stores shared -> global (the O maps), tracked as a bulk async-group of this thread.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int x, int y,
+                                             int z) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(src), "r"(x), "r"(y), "r"(z)
+                 : "memory");
+}
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, uint32_t src, int x, int y,
+                                             int z, int w) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(src), "r"(x), "r"(y), "r"(z), "r"(w)
+        : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until at most one of this thread's bulk groups still reads shared memory
+__device__ __forceinline__ void bulk_wait_read1() {
+    asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+}
+// wait until every bulk group of this thread has completed (its writes are done)
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // One (block, K|V, kv head) tile through the 4-D view: box (64, 8, 2, 2) at 8-row group `grp`.
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
                                             int grp) {
@@ -278,7 +312,7 @@ static_assert(8 * 32 * kRegsSoftmax + 4 * 32 * kRegsProducer <= kThreads * 168,
 template <bool FP8>
 __global__ void __launch_bounds__(kThreads, 1)
 chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
-                const __grid_constant__ ChunkWork work) {
+                const __grid_constant__ ChunkWork work, const __grid_constant__ ChunkIo io) {
     constexpr int kSlotBytes = FP8 ? kKBytes8 : kKBytes;   // one K or V tile in shared memory
     constexpr int kTileLoadBytes = FP8 ? kBlockTile8 : kBlockTile;  // one block's tile
     pdl_trigger();
@@ -352,6 +386,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
     const int ntiles = key_hi > key_lo ? ceil_div(key_hi - key_lo, kKeys) : 0;
     const bool two = R0 + kRows < rows_total;  // the second q-tile has rows
     const int nq = two ? 2 : 1;
+    // Q arrives by TMA (bf16 cache, a map whose boxes hold 128 rows of whole tokens): one box per
+    // q-tile and 64-dim half, issued by the MMA warp; else the softmax warps stage it
+    const bool q_by_tma = !FP8 && (io.mode & 1);
 
     extern __shared__ uint8_t smem_raw[];
     __shared__ uint64_t bar_kf[kKSlots], bar_ke[kKSlots], bar_vf[kVSlots], bar_ve[kVSlots];
@@ -391,7 +428,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
             mbar_init(smem_u32(&bar_pf[q]), kRows);
             mbar_init(smem_u32(&bar_o[q]), 1);
         }
-        mbar_init(smem_u32(&bar_q), kQLoaders);
+        mbar_init(smem_u32(&bar_q), q_by_tma ? 1 : kQLoaders);
         fence_barrier_init();
     }
     for (int k = tid; k < min(je - jb, kMaxIds); k += kThreads) {
@@ -514,6 +551,16 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
                     }
                     mma_commit(smem_u32(&bar_o[q]));
                 };
+                if (q_by_tma) {
+                    // rows R0 + 128 qq .. : tokens q0 + (R0 + 128 qq) / G, heads g G .. g G + G - 1;
+                    // rows past the request (another request's tokens, or zeros past the last
+                    // token) only feed rows whose results are never written
+                    mbar_arrive_expect_tx(smem_u32(&bar_q), nq * kQBytes);
+                    for (int qq = 0; qq < nq; ++qq)
+                        for (int h = 0; h < 2; ++h)
+                            tma_load_3d(q_s + qq * kQBytes + h * kQHalf, &io.q, smem_u32(&bar_q), 64 * h,
+                                        g * G, q0 + (R0 + qq * kRows) / G);
+                }
                 if (mbar_wait(smem_u32(&bar_q), 0, kWaitLimitNs, err) &&
                     mbar_wait(smem_u32(&bar_kf[0]), 0, kWaitLimitNs, err)) {
                     tc_fence_after();
@@ -604,7 +651,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
             fence_proxy_async();  // generic-proxy stores, before the tensor core reads them
             mbar_arrive(smem_u32(&bar_q));
             named_barrier_sync(1, kQLoaders);  // every row's factor is in qfac
-        } else {
+        } else if (!q_by_tma) {
             constexpr int kVecs = kQTiles * kRows * (kD / 8), kPer = kVecs / kQLoaders;
             uint4 v[kPer];
 #pragma unroll
@@ -809,12 +856,55 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
                 else
                     p.lse_out[static_cast<int64_t>(t) * p.num_q_heads + h] = lse2 * kLn2;
             }
-            if (all_ok) {
+            const int row_base = R0 + q * kRows + (warp & 3) * 32;  // this warp's 32 rows
+            // TMA stores: the warp's 32 rows are whole tokens of this request (G divides 32,
+            // rows past the request would land on another request's rows), to out, or to the
+            // cascade prefix partials
+            const bool store_tma = have && row_base + 31 < rows_total &&
+                                   (to_parts ? (prefix && (io.mode & 4)) : (io.mode & 2));
+            if (store_tma) {
+                // O / l of 32 rows x 32 columns at a time into a 4 KB buffer of this q-tile's Q
+                // region (its last MMA has completed), rows of 128 B with the 128-byte swizzle
+                // of the map (so the 16-byte stores of a quarter-warp hit distinct banks); one
+                // lane stores the box; two buffers alternate
+                const uint32_t buf0 = q_s + q * kQBytes + (warp & 3) * 8192;
+                const int t0 = q0 + row_base / G;
+                tc_fence_after();
+#pragma unroll
+                for (int c = 0; c < kD / 32; ++c) {
+                    const uint32_t buf = buf0 + (c & 1) * 4096;
+                    if (c >= 2) {
+                        if (lane == 0) bulk_wait_read1();  // the box of chunk c - 2 has left buf
+                        __syncwarp();
+                    }
+                    uint32_t raw[32];
+                    tmem_ld32(tmem_lane + kColO + c * 32, raw);
+                    tmem_wait_ld();
+                    uint8_t* row = smem + (buf - q_s) + lane * 128;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        *reinterpret_cast<float4*>(row + ((i ^ (lane & 7)) << 4)) =
+                            make_float4(__uint_as_float(raw[4 * i]) * inv,
+                                        __uint_as_float(raw[4 * i + 1]) * inv,
+                                        __uint_as_float(raw[4 * i + 2]) * inv,
+                                        __uint_as_float(raw[4 * i + 3]) * inv);
+                    fence_proxy_async();  // generic-proxy writes, before the TMA unit reads them
+                    __syncwarp();
+                    if (lane == 0) {
+                        if (to_parts)
+                            tma_store_4d(&io.part, buf, 32 * c, g * G, t0, split);
+                        else
+                            tma_store_3d(&io.o, buf, 32 * c, g * G, t0);
+                        bulk_commit();
+                    }
+                }
+                if (lane == 0) bulk_wait_all();  // the rows are written before the CTA ends
+                __syncwarp();
+            } else if (all_ok) {
                 // O / l through shared memory (this q-tile's Q region: its last MMA has
                 // completed), 32 columns at a time, so that each store instruction of the warp
                 // writes four whole 128-byte row segments instead of 32 scattered pieces
                 uint8_t* stage = smem + q * kQBytes + (warp & 3) * kEpiWarpBytes;
-                const int row_base = R0 + q * kRows + (warp & 3) * 32;
                 if (have) tc_fence_after();
 #pragma unroll
                 for (int c = 0; c < kD / 32; ++c) {
@@ -941,7 +1031,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
 
 template <bool FP8>
 cudaError_t launch_chunk_tc_t(const CUtensorMap& tmap, const AttnParams& p, const ChunkWork& work,
-                              int max_splits, cudaStream_t stream) {
+                              const ChunkIo& io, int max_splits, cudaStream_t stream) {
     constexpr int smem = FP8 ? kSmemBytes8 : kSmemBytes;
     static bool attr_set = false;
     if (!attr_set) {
@@ -952,17 +1042,17 @@ cudaError_t launch_chunk_tc_t(const CUtensorMap& tmap, const AttnParams& p, cons
     }
     const dim3 grid = work.count > 0 ? dim3(p.num_kv_heads, work.count, 1)
                                      : dim3(p.chunk_max_qtiles * max_splits, p.num_kv_heads, p.num_seqs);
-    return launch_pdl(chunk_tc_kernel<FP8>, grid, dim3(kThreads), smem, stream, tmap, p, work);
+    return launch_pdl(chunk_tc_kernel<FP8>, grid, dim3(kThreads), smem, stream, tmap, p, work, io);
 }
 
 }  // namespace
 
 // bf16 cache: the 4-D whole-tile view; FP8: the 2-D view of the pool.
 cudaError_t launch_chunk_tc(const CUtensorMap& tmap, const CUtensorMap& tmap_blk,
-                            const AttnParams& p, const ChunkWork& work, int kv_dtype,
-                            int max_splits, cudaStream_t stream) {
-    if (kv_dtype == PA_FP8_E4M3) return launch_chunk_tc_t<true>(tmap, p, work, max_splits, stream);
-    return launch_chunk_tc_t<false>(tmap_blk, p, work, max_splits, stream);
+                            const AttnParams& p, const ChunkWork& work, const ChunkIo& io,
+                            int kv_dtype, int max_splits, cudaStream_t stream) {
+    if (kv_dtype == PA_FP8_E4M3) return launch_chunk_tc_t<true>(tmap, p, work, io, max_splits, stream);
+    return launch_chunk_tc_t<false>(tmap_blk, p, work, io, max_splits, stream);
 }
 
 }  // namespace pa

@@ -113,6 +113,18 @@ struct ChunkWork {
     uint32_t item[kMaxChunkWork];
 };
 
+// Tensor maps of one call's queries and outputs for the tcgen05 chunk kernel, so that a CTA
+// loads its Q tile and stores its O rows with TMA instead of per-thread loads and stores (the
+// per-SM throughput of which bounded a CTA's prologue and epilogue).  A map is used only when
+// its bit is set in `mode`.
+struct ChunkIo {
+    CUtensorMap q;       // bf16 [T][Hq][128] as {128, Hq, T}; box {64, G, 128 / G}  (mode & 1)
+    CUtensorMap o;       // fp32 out [T][Hq][128] as {128, Hq, T}; box {32, G, 32 / G} (mode & 2)
+    CUtensorMap part;    // fp32 partials [S][T][Hq][128] as {128, Hq, T, S}; box {32, G, 32 / G, 1}
+                         // (mode & 4: the prefix launch of a cascade call)
+    int mode;
+};
+
 // The body of pa_attention_ex.  allow_side_stream = false keeps every launch on `stream` and
 // creates no stream or event (pa_attention_noalloc allocates nothing, not even those).
 int attention_call(const pa_cache* cache, const void* q, int num_q_heads,
@@ -125,11 +137,11 @@ int attention_call(const pa_cache* cache, const void* q, int num_q_heads,
 cudaError_t launch_decode(const CUtensorMap& tmap, const AttnParams& p, int head_size,
                           int kv_dtype, int max_splits, cudaStream_t stream);
 cudaError_t launch_chunk(const CUtensorMap& tmap, const CUtensorMap& tmap_blk, const AttnParams& p,
-                         const ChunkWork& work, int head_size, int kv_dtype, int max_splits,
-                         cudaStream_t stream);
+                         const ChunkWork& work, const ChunkIo& io, int head_size, int kv_dtype,
+                         int max_splits, cudaStream_t stream);
 cudaError_t launch_chunk_tc(const CUtensorMap& tmap, const CUtensorMap& tmap_blk,
-                            const AttnParams& p, const ChunkWork& work, int kv_dtype,
-                            int max_splits, cudaStream_t stream);
+                            const AttnParams& p, const ChunkWork& work, const ChunkIo& io,
+                            int kv_dtype, int max_splits, cudaStream_t stream);
 cudaError_t launch_reduce(const AttnParams& p, const ChunkList& list, int head_size,
                           cudaStream_t stream);
 cudaError_t launch_zero_counters(int* counters, int n, cudaStream_t stream);
