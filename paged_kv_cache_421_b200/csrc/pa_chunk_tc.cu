@@ -303,6 +303,11 @@ constexpr uint32_t kRegsSoftmax = 232, kRegsProducer = 40;
 constexpr int kQLoaders = 256;           // the softmax warps stage Q
 constexpr int kEpiRowBytes = 32 * 4 + 16;  // epilogue staging row: 32 floats + 16 B (no conflicts)
 constexpr int kEpiWarpBytes = 32 * kEpiRowBytes;
+// each warp's epilogue region in its q-tile's Q region: two 4 KB TMA-store buffers, or the
+// padded staging rows of the plain path
+constexpr int kEpiWarpRegion = 8192;
+static_assert(kEpiWarpBytes <= kEpiWarpRegion && 4 * kEpiWarpRegion <= kQBytes,
+              "epilogue staging exceeds the q-tile's Q region");
 constexpr int kMergeRows = 8;            // rows a warp merges with all loads in flight
 static_assert(8 * 32 * kRegsSoftmax + 4 * 32 * kRegsProducer <= kThreads * 168,
               "register split exceeds the launch's registers");
@@ -867,7 +872,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
                 // region (its last MMA has completed), rows of 128 B with the 128-byte swizzle
                 // of the map (so the 16-byte stores of a quarter-warp hit distinct banks); one
                 // lane stores the box; two buffers alternate
-                const uint32_t buf0 = q_s + q * kQBytes + (warp & 3) * 8192;
+                const uint32_t buf0 = q_s + q * kQBytes + (warp & 3) * kEpiWarpRegion;
                 const int t0 = q0 + row_base / G;
                 tc_fence_after();
 #pragma unroll
@@ -904,7 +909,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
                 // O / l through shared memory (this q-tile's Q region: its last MMA has
                 // completed), 32 columns at a time, so that each store instruction of the warp
                 // writes four whole 128-byte row segments instead of 32 scattered pieces
-                uint8_t* stage = smem + q * kQBytes + (warp & 3) * kEpiWarpBytes;
+                // (the same 8 KB of the q-tile's Q region per warp as the TMA path above, which
+                // the q-tile's other warps may be using at the same time)
+                uint8_t* stage = smem + q * kQBytes + (warp & 3) * kEpiWarpRegion;
                 if (have) tc_fence_after();
 #pragma unroll
                 for (int c = 0; c < kD / 32; ++c) {

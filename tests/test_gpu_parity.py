@@ -177,6 +177,11 @@ EDGE_CASES = {
     "many_requests": ([int(x) for x in np.random.default_rng(3).integers(1, 200, 300)],
                       [1] * 300, 8, 2, 128),
     "g16_chunk": ([90, 40], [1, 1], 32, 2, 128),
+    # chunk rows whose last q-tile has whole 32-row warps (stored as TMA boxes) next to a
+    # partial warp (plain stores): 48, 704 and 488 rows at G 8
+    "chunk_warp_store_paths": ([300, 90, 400], [6, 88, 61], 16, 2, 128),
+    # G 3 divides neither 128 nor 32: Q staged and O stored by the warps
+    "g3_chunk": ([200, 90], [50, 37], 6, 2, 128),
 }
 
 
