@@ -527,7 +527,10 @@ def decode_roofline(wl, workload: str, dec_ms: float, window: int, local_chunk: 
     achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
     return {"bound": "hbm", "kernel": "decode_kernel", "achieved": round(achieved, 1),
             "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
-            "traffic": recorded_traffic("decode_kernel", workload),
+            # the record holds full-context launches: a window, local chunks or a cascade
+            # prefix change what the kernel reads
+            "traffic": (recorded_traffic("decode_kernel", workload)
+                        if not (window or local_chunk or prefix) else None),
             "peak_kind": peak_kind, "bytes_per_launch": dec_bytes,
             "ms_per_launch": round(dec_ms, 4)}
 
