@@ -419,7 +419,7 @@ class DeviceStep:
             torch.cuda.get_device_properties(device).multi_processor_count,
             self.workspace.numel(), kv_split_tokens=kv_split_tokens,
             sliding_window=sliding_window, local_chunk=local_chunk,
-            common_prefix_tokens=self.prefix)
+            common_prefix_tokens=self.prefix, kv_dtype=self.cache.kv_dtype)
         torch.cuda.synchronize(device)
 
     def launches_per_step(self) -> int:

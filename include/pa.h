@@ -280,12 +280,17 @@ typedef struct {
                               is in flight when the wait gives up. */
     int test_wait_limit_us;   /* with test_skip_decode_load: that CTA's wait limit in
                               microseconds (> 0); otherwise ignored (waits give up after 2 s) */
+    int kv_dtype;             /* pa_plan_attention only: the element type (pa_kv_dtype) of the
+                              cache the plan is for -- an FP8 cache at head_size 128 decodes on
+                              another kernel, with its own split sizes.  pa_attention and its
+                              variants take the type from the cache and ignore this field */
 } pa_attention_opts;
 
 /* The planner alone: fills *plan for the given host metadata without touching the GPU.
  * num_sms must be > 0.  It reads opts->lse_out only as a flag (non-NULL: plan a call that
- * exports LSEs, which admits empty decode shares) and never dereferences it.
- * Errors: INVALID_ARG, METADATA, UNSUPPORTED. */
+ * exports LSEs, which admits empty decode shares) and never dereferences it; opts->kv_dtype
+ * names the cache's element type (PA_BF16 when opts is NULL).
+ * Errors: INVALID_ARG (also an unknown kv_dtype), METADATA, UNSUPPORTED. */
 int pa_plan_attention(const int32_t* seq_lens_host, const int32_t* query_start_loc_host,
                       int num_seqs, int num_tokens, int num_q_heads, int num_kv_heads,
                       int head_size, int block_size, int max_blocks_per_seq, int num_sms,

@@ -73,6 +73,7 @@ class pa_attention_opts(ctypes.Structure):
         ("common_prefix_tokens", ctypes.c_int),
         ("test_skip_decode_load", ctypes.c_int),
         ("test_wait_limit_us", ctypes.c_int),
+        ("kv_dtype", ctypes.c_int),
     ]
 
 
@@ -222,9 +223,11 @@ def pa_attention_workspace_bytes(num_tokens, num_q_heads, head_size, max_splits)
 def pa_plan_attention(seq_lens_host, query_start_loc_host, num_q_heads, num_kv_heads,
                       head_size, max_blocks_per_seq, num_sms, workspace_bytes,
                       kv_split_tokens=0, block_size=16, sliding_window=0,
-                      local_chunk=0, with_lse=False, common_prefix_tokens=0) -> dict:
+                      local_chunk=0, with_lse=False, common_prefix_tokens=0,
+                      kv_dtype=0) -> dict:
     """with_lse: plan as a call that exports LSEs (which admits empty decode shares); the
-    planner only tests the pointer for NULL, so a dummy non-NULL value stands in."""
+    planner only tests the pointer for NULL, so a dummy non-NULL value stands in.  kv_dtype:
+    the cache's element type (PA_BF16 / PA_FP8_E4M3)."""
     sl = _host_i32(seq_lens_host)
     qs = _host_i32(query_start_loc_host)
     opts = pa_attention_opts()
@@ -233,6 +236,7 @@ def pa_plan_attention(seq_lens_host, query_start_loc_host, num_q_heads, num_kv_h
     opts.local_chunk = local_chunk
     opts.lse_out = 16 if with_lse else None
     opts.common_prefix_tokens = common_prefix_tokens
+    opts.kv_dtype = kv_dtype
     plan = pa_plan()
     _check(load().pa_plan_attention(sl.ctypes.data, qs.ctypes.data, sl.size, int(qs[-1]),
                                     num_q_heads, num_kv_heads, head_size, block_size,

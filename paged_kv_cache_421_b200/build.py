@@ -21,7 +21,7 @@ SRC = os.path.join(HERE, "csrc")
 OBJ = os.path.join(SRC, "_build")
 LIB = os.path.join(HERE, "libpa.so")
 INCLUDE = os.path.join(os.path.dirname(HERE), "include")
-SOURCES = ["pa_api.cu", "pa_write.cu", "pa_decode.cu", "pa_chunk.cu", "pa_chunk_tc.cu",
+SOURCES = ["pa_api.cu", "pa_write.cu", "pa_decode.cu", "pa_decode_tc.cu", "pa_chunk.cu", "pa_chunk_tc.cu",
            "pa_reduce.cu", "pa_noalloc.cu", "pa_alloc.cu", "pa_dcp.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC,-O2", "--expt-relaxed-constexpr",

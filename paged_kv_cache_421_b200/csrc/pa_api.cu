@@ -229,6 +229,7 @@ size_t prefix_part_bytes(int num_tokens, int num_q_heads, int head_size, int spl
 
 // Planner constants.
 constexpr int kDecodeCtasPerSm = 3;    // decode kernel residency (64 KB of stages per CTA)
+constexpr int kDecodeTc8CtasPerSm = 2;  // tcgen05 FP8 decode kernel residency (107 KB per CTA)
 constexpr int kMaxDecodeSplits = 1024;  // merge weights of one row fit the CTA's shared memory
 constexpr int kDecodeWaves = 2;             // target waves of decode CTAs (2 measured best)
 constexpr int kMinDecodeSplitBlocks = 64;   // >= 1024 keys per split
@@ -239,7 +240,7 @@ constexpr int kMaxPrefixSplits = pa::kMaxPrefixParts;  // prefix partials a deco
 
 int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int Hkv, int D,
               int bs, int maxb, int num_sms, size_t ws, const pa_attention_opts* opts,
-              pa_plan* pl) {
+              int kv_dtype, pa_plan* pl) {
     std::memset(pl, 0, sizeof(*pl));
     if (B < 0 || T < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || num_sms <= 0 || maxb <= 0)
         return PA_ERR_INVALID_ARG;
@@ -266,6 +267,10 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
     if (B > 0 && qsl[0] != 0) return PA_ERR_METADATA;
     long long dec_units = 0;
     int dec_max_blocks = 0, chunk_max_blocks = 0, chunk_max_qtiles = 0;
+    // the decode kernel that will run: tcgen05 for an FP8 cache at head_size 128 (except under
+    // the bounded-wait test hook), else mma.sync
+    const bool tc8 = kv_dtype == PA_FP8_E4M3 && D == 128 &&
+                     !(opts && opts->test_skip_decode_load > 0);
     // chunk work in key tiles: the CTA of each q-tile walks the keys its last row may see
     const int chunk_cta_rows = pa::chunk_rows(D, 1);
     const int chunk_tile_keys = D == 128 ? 128 : 64;
@@ -320,7 +325,9 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
         if (forced) {
             dsb = forced / bs;
         } else {
-            const long long target = static_cast<long long>(num_sms) * kDecodeCtasPerSm * kDecodeWaves;
+            // two waves of the decode kernel's resident CTAs
+            const long long target = static_cast<long long>(num_sms) *
+                                     (tc8 ? kDecodeTc8CtasPerSm : kDecodeCtasPerSm) * kDecodeWaves;
             long long sb = (dec_units + target - 1) / target;
             if (sb < kMinDecodeSplitBlocks) sb = kMinDecodeSplitBlocks;
             dsb = round_up(static_cast<int>(sb < dec_max_blocks ? sb : dec_max_blocks), 4);
@@ -573,9 +580,11 @@ int pa_plan_attention(const int32_t* seq_lens_host, const int32_t* query_start_l
                       size_t workspace_bytes, const pa_attention_opts* opts, pa_plan* plan) {
     if (!plan) return PA_ERR_INVALID_ARG;
     if (head_size != 64 && head_size != 128) return PA_ERR_UNSUPPORTED;
+    const int kv_dtype = opts ? opts->kv_dtype : PA_BF16;
+    if (kv_dtype != PA_BF16 && kv_dtype != PA_FP8_E4M3) return PA_ERR_INVALID_ARG;
     return plan_impl(seq_lens_host, query_start_loc_host, num_seqs, num_tokens, num_q_heads,
                      num_kv_heads, head_size, block_size, max_blocks_per_seq, num_sms,
-                     workspace_bytes, opts, plan);
+                     workspace_bytes, opts, kv_dtype, plan);
 }
 
 int pa_attention_ex(const pa_cache* cache, const void* q, int num_q_heads,
@@ -616,7 +625,7 @@ int pa::attention_call(const pa_cache* cache, const void* q, int num_q_heads,
     pa_plan pl;
     int st = plan_impl(seq_lens_host, query_start_loc_host, num_seqs, num_tokens, num_q_heads,
                        cache->num_kv_heads, cache->head_size, cache->block_size,
-                       max_blocks_per_seq, num_sms, workspace_bytes, opts, &pl);
+                       max_blocks_per_seq, num_sms, workspace_bytes, opts, cache->kv_dtype, &pl);
     if (st != PA_OK) return st;
     // chunk kernels: tcgen05 for head_size 128 (bf16 or FP8 cache), mma.sync for bf16 head_size 64
     const bool chunk_ok = cache->head_size == 128 || cache->kv_dtype == PA_BF16;

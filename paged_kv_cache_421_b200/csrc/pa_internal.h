@@ -136,6 +136,9 @@ int attention_call(const pa_cache* cache, const void* q, int num_q_heads,
 
 cudaError_t launch_decode(const CUtensorMap& tmap, const AttnParams& p, int head_size,
                           int kv_dtype, int max_splits, cudaStream_t stream);
+// FP8 E4M3 cache, head_size 128: the tcgen05 decode kernel (pa_decode_tc.cu)
+cudaError_t launch_decode_tc8(const CUtensorMap& tmap, const AttnParams& p, int max_splits,
+                              cudaStream_t stream);
 cudaError_t launch_chunk(const CUtensorMap& tmap, const CUtensorMap& tmap_blk, const AttnParams& p,
                          const ChunkWork& work, const ChunkIo& io, int head_size, int kv_dtype,
                          int max_splits, cudaStream_t stream);

@@ -120,7 +120,8 @@ def workspace_bytes_for(cache: PagedKVCache, seq_lens_host, qsl_host, num_q_head
                                cache.head_size, max_blocks_per_seq, num_sms, unlimited,
                                kv_split_tokens=kv_split_tokens, block_size=cache.block_size,
                                sliding_window=sliding_window, local_chunk=local_chunk,
-                               with_lse=with_lse, common_prefix_tokens=common_prefix_tokens)
+                               with_lse=with_lse, common_prefix_tokens=common_prefix_tokens,
+                               kv_dtype=cache.kv_dtype)
     return int(plan["workspace_needed"])
 
 
