@@ -209,13 +209,25 @@ def source_digest(*names) -> str:
     return h.hexdigest()[:16]
 
 
+# the sources each recorded kernel's code comes from (a change to any voids its record)
+KERNEL_SOURCES = {
+    "decode_kernel": ("pa_decode.cu", "pa_decode_epi.cuh", "pa_common.cuh"),
+    "decode_tc8_kernel": ("pa_decode_tc.cu", "pa_decode_epi.cuh", "pa_tc.cuh", "pa_common.cuh"),
+}
+
+
+def decode_kernel_name(wl) -> str:
+    """The decode kernel a workload runs on: tcgen05 for an FP8 cache at head_size 128."""
+    return "decode_tc8_kernel" if (wl.kv_dtype != 0 and wl.head_size == 128) else "decode_kernel"
+
+
 def recorded_traffic(kernel: str, workload: str):
     """DRAM bytes per launch of `kernel` on `workload` from the committed ncu summary, if it
     was taken on the current kernel source; else None."""
     path = os.path.join(ROOT, "profiles", "traffic.txt")
-    if not os.path.exists(path):
+    if not os.path.exists(path) or kernel not in KERNEL_SOURCES:
         return None
-    digest = source_digest("pa_decode.cu", "pa_common.cuh")
+    digest = source_digest(*KERNEL_SOURCES[kernel])
     for line in open(path):
         parts = line.split()
         if len(parts) == 4 and parts[0] == kernel and parts[1] == workload and parts[2] == digest:
@@ -525,11 +537,12 @@ def decode_roofline(wl, workload: str, dec_ms: float, window: int, local_chunk: 
     peak, peak_kind = load_peaks()
     dec_bytes = decode_kv_bytes(wl, window, local_chunk, prefix)
     achieved = dec_bytes / (dec_ms * 1e-3) / 1e9
-    return {"bound": "hbm", "kernel": "decode_kernel", "achieved": round(achieved, 1),
+    kernel = decode_kernel_name(wl)
+    return {"bound": "hbm", "kernel": kernel, "achieved": round(achieved, 1),
             "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
             # the record holds full-context launches: a window, local chunks or a cascade
             # prefix change what the kernel reads
-            "traffic": (recorded_traffic("decode_kernel", workload)
+            "traffic": (recorded_traffic(kernel, workload)
                         if not (window or local_chunk or prefix) else None),
             "peak_kind": peak_kind, "bytes_per_launch": dec_bytes,
             "ms_per_launch": round(dec_ms, 4)}
