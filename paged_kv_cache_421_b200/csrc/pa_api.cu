@@ -6,6 +6,7 @@
 #include <algorithm>
 #include <atomic>
 #include <mutex>
+#include <queue>
 #include <vector>
 #include <new>
 
@@ -238,6 +239,38 @@ constexpr int kMinChunkSplitTiles = 4;      // a chunk split walks at least four
 constexpr int kMaxChunkSplitBlocks = 1024;  // chunk kernels stage up to 1024 block ids
 constexpr int kMaxPrefixSplits = pa::kMaxPrefixParts;  // prefix partials a decode row merges
 
+// Estimated time of the tcgen05 chunk kernel, in key tiles, under KV splits of split_keys keys:
+// its CTAs (one per (q-tile pair, kv head, split), each walking the key tiles of its visible
+// range inside its split) scheduled longest first over num_sms SMs, one CTA per SM.  A CTA also
+// pays about a tile of fixed cost (set-up, epilogue), a split one more (its partial and the
+// merge).  ranges: [lo, hi) per q-tile pair, once per kv head (weight Hkv).
+double chunk_makespan(const std::vector<std::pair<int, int>>& ranges, int Hkv, int split_keys,
+                      int tile_keys, int num_sms) {
+    static thread_local std::vector<double> cost;
+    cost.clear();
+    for (const auto& rg : ranges) {
+        const int nsp = pa::ceil_div(rg.second, split_keys);
+        for (int sp = 0; sp < nsp; ++sp) {
+            const int lo = std::max(sp * split_keys, rg.first);
+            const int hi = std::min((sp + 1) * split_keys, rg.second);
+            if (hi <= lo) continue;
+            const double c = pa::ceil_div(hi - lo, tile_keys) + 1.0 + (nsp > 1 ? 1.0 : 0.0);
+            for (int h = 0; h < Hkv; ++h) cost.push_back(c);
+        }
+    }
+    std::sort(cost.begin(), cost.end(), std::greater<double>());
+    std::priority_queue<double, std::vector<double>, std::greater<double>> sm;
+    for (int i = 0; i < num_sms; ++i) sm.push(0.0);
+    double makespan = 0.0;
+    for (double c : cost) {
+        const double t = sm.top() + c;
+        sm.pop();
+        sm.push(t);
+        makespan = std::max(makespan, t);
+    }
+    return makespan;
+}
+
 int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int Hkv, int D,
               int bs, int maxb, int num_sms, size_t ws, const pa_attention_opts* opts,
               int kv_dtype, pa_plan* pl) {
@@ -275,6 +308,9 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
     const int chunk_cta_rows = pa::chunk_rows(D, 1);
     const int chunk_tile_keys = D == 128 ? 128 : 64;
     long long chunk_work = 0, chunk_work_max = 0;
+    // visible key range [lo, hi) of each chunk CTA's q-tile rows (one entry per kv head's CTA)
+    static thread_local std::vector<std::pair<int, int>> chunk_ranges;
+    chunk_ranges.clear();
     for (int r = 0; r < B; ++r) {
         const int ql = qsl[r + 1] - qsl[r];
         const int ctx = sl[r];
@@ -312,6 +348,7 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
                 const long long w = pa::ceil_div(ctx - ql + last_row / G + 1 - lo, chunk_tile_keys);
                 chunk_work += w * Hkv;
                 if (w > chunk_work_max) chunk_work_max = w;
+                chunk_ranges.emplace_back(lo, ctx - ql + last_row / G + 1);
             }
         }
     }
@@ -352,15 +389,34 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
             if (csb > kMaxChunkSplitBlocks && allowed > 1)  // keep block ids in shared memory
                 csb = round_up(pa::ceil_div(chunk_max_blocks,
                                             pa::ceil_div(chunk_max_blocks, kMaxChunkSplitBlocks)), 4);
-            // one CTA per SM: split the KV walk only when the longest CTA would walk more than
-            // three times the average work per SM.  A split writes fp32 partials of every row
-            // and merges them, which costs more than a 2x imbalance (measured on the mixed step).
-            const long long per_sm = (chunk_work + num_sms - 1) / num_sms;
-            const long long target = std::max<long long>(per_sm, kMinChunkSplitTiles);
-            if (chunk_work_max > 3 * target) {
+            if (D == 128 && allowed > 1 && pl->num_decode_seqs == 0) {
+                // tcgen05 kernel, one CTA per SM, merging up to kMaxFusedSplits splits itself,
+                // with the SMs to itself (in a mixed step the decode kernel runs beside it, and
+                // more chunk CTAs take SMs from it: 0.192 -> 0.219 ms on the mixed step): the
+                // split count whose longest-first schedule of CTAs over the SMs ends first
                 const int tile_blocks = chunk_tile_keys / bs;
-                const int sb = static_cast<int>(target) * tile_blocks;
-                if (sb < csb) csb = round_up(std::max(sb, kMinChunkSplitBlocks), 4);
+                const int ns_max = std::min(pa::kMaxFusedSplits, allowed);
+                double best = chunk_makespan(chunk_ranges, Hkv, csb * bs, chunk_tile_keys, num_sms);
+                for (int n = 2; n <= ns_max; ++n) {
+                    const int sb = round_up(pa::ceil_div(chunk_max_blocks, n), tile_blocks);
+                    if (sb >= csb || sb < kMinChunkSplitTiles * tile_blocks) continue;
+                    const double m = chunk_makespan(chunk_ranges, Hkv, sb * bs, chunk_tile_keys, num_sms);
+                    if (m < 0.95 * best) {
+                        best = m;
+                        csb = sb;
+                    }
+                }
+            } else {
+                // split the KV walk only when the longest CTA would walk more than three times
+                // the average work per SM (a mixed step; the head_size-64 kernel, whose splits
+                // go through the reduce kernel)
+                const long long per_sm = (chunk_work + num_sms - 1) / num_sms;
+                const long long target = std::max<long long>(per_sm, kMinChunkSplitTiles);
+                if (chunk_work_max > 3 * target) {
+                    const int tile_blocks = chunk_tile_keys / bs;
+                    const int sb = static_cast<int>(target) * tile_blocks;
+                    if (sb < csb) csb = round_up(std::max(sb, kMinChunkSplitBlocks), 4);
+                }
             }
         }
         int ns = pa::ceil_div(chunk_max_blocks, csb);
@@ -826,7 +882,8 @@ int pa::attention_call(const pa_cache* cache, const void* q, int num_q_heads,
     const cudaStream_t cs = side ? side->stream : s;  // the chunk kernel's stream
     static thread_local pa::ChunkIo io;
     if (pl.num_chunk_seqs && cache->head_size == 128)
-        make_chunk_io(io, q, out, nullptr, num_tokens, num_q_heads, p.group, 0,
+        make_chunk_io(io, q, out, pl.chunk_max_splits > 1 ? p.part_o : nullptr, num_tokens,
+                      num_q_heads, p.group, p.max_splits,
                       cache->kv_dtype == PA_BF16);
     else
         std::memset(&io, 0, sizeof(io));

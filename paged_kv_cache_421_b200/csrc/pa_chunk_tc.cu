@@ -97,6 +97,11 @@ constexpr int kEpiWarpRegion = 8192;
 static_assert(kEpiWarpBytes <= kEpiWarpRegion && 4 * kEpiWarpRegion <= kQBytes,
               "epilogue staging exceeds the q-tile's Q region");
 constexpr int kMergeRows = 8;            // rows a warp merges with all loads in flight
+// split merge through TMA: each softmax warp's share of the CTA's shared memory (the Q tiles and
+// K/V rings, idle once the last MMA completed), one 4 KB box per split of a 32-column chunk
+constexpr int kMergeWarpBytes = 16384;
+static_assert(kMaxFusedSplits * 4096 <= kMergeWarpBytes, "merge boxes exceed a warp's region");
+static_assert(8 * kMergeWarpBytes <= kSmemBytes8 - 1024, "merge regions exceed shared memory");
 static_assert(8 * 32 * kRegsSoftmax + 4 * 32 * kRegsProducer <= kThreads * 168,
               "register split exceeds the launch's registers");
 
@@ -188,6 +193,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
     __shared__ uint64_t bar_sf[kQTiles], bar_pf[kQTiles];  // S computed / P stored
     __shared__ uint64_t bar_o[kQTiles];                    // a P V of the q-tile done
     __shared__ uint64_t bar_q;                             // Q staged by the softmax warps
+    __shared__ uint64_t bar_merge[8][2];                   // split merge: a warp's boxes loaded
+    __shared__ float s_wts[kQTiles * kRows * kMaxFusedSplits];  // split merge weights per row
     __shared__ uint32_t tmem_holder;
     __shared__ int ids[kMaxIds];  // physical ids of the split's first kMaxIds logical blocks
     __shared__ float qfac[FP8 ? kQTiles * kRows : 1];  // FP8: each row's 2^-e (Q was scaled by 2^e)
@@ -222,6 +229,8 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
             mbar_init(smem_u32(&bar_o[q]), 1);
         }
         mbar_init(smem_u32(&bar_q), q_by_tma ? 1 : kQLoaders);
+        for (int w = 0; w < 8; ++w)
+            for (int b2 = 0; b2 < 2; ++b2) mbar_init(smem_u32(&bar_merge[w][b2]), 1);
         fence_barrier_init();
     }
     for (int k = tid; k < min(je - jb, kMaxIds); k += kThreads) {
@@ -652,9 +661,9 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
             const int row_base = R0 + q * kRows + (warp & 3) * 32;  // this warp's 32 rows
             // TMA stores: the warp's 32 rows are whole tokens of this request (G divides 32,
             // rows past the request would land on another request's rows), to out, or to the
-            // cascade prefix partials
+            // split partials (a split's, or the cascade prefix pass's)
             const bool store_tma = have && row_base + 31 < rows_total &&
-                                   (to_parts ? (prefix && (io.mode & 4)) : (io.mode & 2));
+                                   (to_parts ? (io.mode & 4) : (io.mode & 2));
             if (store_tma) {
                 // O / l of 32 rows x 32 columns at a time into a 4 KB buffer of this q-tile's Q
                 // region (its last MMA has completed), rows of 128 B with the 128-byte swizzle
@@ -744,6 +753,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
             // kernel otherwise).  Counters start at zero on every call (cleared on the stream
             // before the launch); decode requests use other tokens' counters.
             __shared__ int s_last;
+            fence_proxy_async_all();  // this CTA's bulk stores of partials, before the counter
             __threadfence();
             named_barrier_sync(1, kQLoaders);  // every partial of this CTA is written
             if (tid == 0) {
@@ -753,15 +763,41 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
             named_barrier_sync(1, kQLoaders);
             if (s_last) {
                 __threadfence();
+                fence_proxy_async_all();  // the other CTAs' partials, before bulk loads of them
                 const int64_t stride = static_cast<int64_t>(p.num_tokens) * p.num_q_heads;
                 auto row_of = [&](int Rr) {
                     return static_cast<int64_t>(q0 + Rr / G) * p.num_q_heads + g * G + Rr % G;
                 };
-                // phase 1: thread t turns row R0 + t's LSEs into normalised split weights
-                float* wsm = reinterpret_cast<float*>(smem);  // [256 rows][kMaxFusedSplits]
+                // phase 2 runs per warp w over its 32 rows R0 + 32 w .. (a q-tile quarter,
+                // whole tokens).  TMA path: per 32-column chunk, one box of each split into the
+                // warp's 16 KB of the CTA's shared memory (the Q tiles and K/V rings, idle
+                // now), two chunks in flight, combined row by row (lane = row), and the result
+                // stored from the chunk's first box by one bulk tensor store.  Other warps merge
+                // with coalesced 16-byte loads.  The first loads go out before the weights are
+                // computed, so their latency overlaps phase 1.
+                const int row_base = R0 + 32 * warp;
+                const bool merge_tma = (io.mode & 6) == 6 && row_base + 31 < rows_total;
+                const uint32_t region = smem_u32(smem) + warp * kMergeWarpBytes;
+                const int gbytes = nsplit * 4096;                  // one chunk's boxes
+                const int ngrp = kMergeWarpBytes / gbytes >= 2 ? 2 : 1;  // chunks in flight
+                const int t0 = q0 + row_base / G;
+                auto issue = [&](int c) {
+                    if (lane == 0) {
+                        const int grp = c % ngrp;
+                        const uint32_t bar = smem_u32(&bar_merge[warp][grp]);
+                        mbar_arrive_expect_tx(bar, gbytes);
+                        for (int sp = 0; sp < nsplit; ++sp)
+                            tma_load_4d_at(region + grp * gbytes + sp * 4096, &io.part, bar, 32 * c,
+                                           g * G, t0, sp);
+                    }
+                };
+                if (merge_tma)
+                    for (int c = 0; c < ngrp; ++c) issue(c);
+                // phase 1: thread t turns row R0 + t's LSEs into normalised split weights (the
+                // same thread merges that row below when the warp takes the TMA path)
+                const int Rr = R0 + tid;
+                float w[kMaxFusedSplits];
                 {
-                    const int Rr = R0 + tid;
-                    float w[kMaxFusedSplits];
                     float M = -INFINITY;
 #pragma unroll
                     for (int sp = 0; sp < kMaxFusedSplits; ++sp) {
@@ -777,39 +813,88 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
                     }
                     const float inv = W > 0.f ? 1.f / W : 0.f;
 #pragma unroll
-                    for (int sp = 0; sp < kMaxFusedSplits; ++sp) wsm[tid * kMaxFusedSplits + sp] = w[sp] * inv;
+                    for (int sp = 0; sp < kMaxFusedSplits; ++sp) {
+                        w[sp] *= inv;
+                        s_wts[tid * kMaxFusedSplits + sp] = w[sp];
+                    }
                     if (p.lse_out && Rr < rows_total)
                         p.lse_out[row_of(Rr)] = W > 0.f ? (M + __log2f(W)) * kLn2 : -INFINITY;
                 }
                 named_barrier_sync(1, kQLoaders);
-                // phase 2: warp w merges rows w, w + 8, ..., lane l the 16 bytes at 4l of each
-                // row (coalesced), kMergeRows rows with all their loads in flight at once
-                for (int i0 = 0; i0 < 32; i0 += kMergeRows) {
-                    float4 v[kMergeRows][kMaxFusedSplits];
-#pragma unroll
-                    for (int b2 = 0; b2 < kMergeRows; ++b2) {
-                        const int Rr = R0 + warp + 8 * (i0 + b2);
-#pragma unroll
-                        for (int sp = 0; sp < kMaxFusedSplits; ++sp)
-                            v[b2][sp] = (Rr < rows_total && sp < nsplit)
-                                            ? __ldcg(reinterpret_cast<const float4*>(
-                                                         p.part_o + (sp * stride + row_of(Rr)) * kD) + lane)
-                                            : make_float4(0.f, 0.f, 0.f, 0.f);
-                    }
-#pragma unroll
-                    for (int b2 = 0; b2 < kMergeRows; ++b2) {
-                        const int rl = warp + 8 * (i0 + b2), Rr = R0 + rl;
-                        if (Rr >= rows_total) continue;
-                        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-                        for (int sp = 0; sp < kMaxFusedSplits; ++sp) {
-                            const float w = wsm[rl * kMaxFusedSplits + sp];
-                            acc.x += w * v[b2][sp].x;
-                            acc.y += w * v[b2][sp].y;
-                            acc.z += w * v[b2][sp].z;
-                            acc.w += w * v[b2][sp].w;
+                if (merge_tma) {
+                    for (int c = 0; c < kD / 32; ++c) {
+                        const int grp = c % ngrp;
+                        const uint32_t bar = smem_u32(&bar_merge[warp][grp]);
+                        const uint32_t par = (c / ngrp) & 1;
+                        const bool got = mbar_wait(bar, par, kWaitLimitNs, err);
+                        if (!__all_sync(0xffffffffu, got)) {
+                            // boxes may still be in flight: a last bounded wait before leaving
+                            for (int cc = c; cc < min(c + ngrp, kD / 32); ++cc)
+                                mbar_wait(smem_u32(&bar_merge[warp][cc % ngrp]), (cc / ngrp) & 1,
+                                          kWindDownLimitNs, err);
+                            break;
                         }
-                        reinterpret_cast<float4*>(p.out + row_of(Rr) * kD)[lane] = acc;
+                        const uint32_t gb = region + grp * gbytes;
+                        float acc[32];
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+                        for (int sp = 0; sp < nsplit; ++sp) {
+                            const uint8_t* row = smem + (gb - smem_u32(smem)) + sp * 4096 + lane * 128;
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                const float4 v = *reinterpret_cast<const float4*>(row + ((i ^ (lane & 7)) << 4));
+                                acc[4 * i] += w[sp] * v.x;
+                                acc[4 * i + 1] += w[sp] * v.y;
+                                acc[4 * i + 2] += w[sp] * v.z;
+                                acc[4 * i + 3] += w[sp] * v.w;
+                            }
+                        }
+                        uint8_t* orow = smem + (gb - smem_u32(smem)) + lane * 128;
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            *reinterpret_cast<float4*>(orow + ((i ^ (lane & 7)) << 4)) =
+                                make_float4(acc[4 * i], acc[4 * i + 1], acc[4 * i + 2], acc[4 * i + 3]);
+                        fence_proxy_async();  // generic-proxy writes, before the TMA unit reads them
+                        __syncwarp();
+                        if (lane == 0) {
+                            tma_store_3d(&io.o, gb, 32 * c, g * G, t0);
+                            bulk_commit();
+                            // the group is reloaded for chunk c + ngrp once the store has read it
+                            if (c + ngrp < kD / 32) bulk_wait_read0();
+                        }
+                        __syncwarp();
+                        if (c + ngrp < kD / 32) issue(c + ngrp);
+                    }
+                    if (lane == 0) bulk_wait_all();  // the rows are written before the CTA ends
+                    __syncwarp();
+                } else {
+                    for (int i0 = 0; i0 < 32; i0 += kMergeRows) {
+                        float4 v[kMergeRows][kMaxFusedSplits];
+#pragma unroll
+                        for (int b2 = 0; b2 < kMergeRows; ++b2) {
+                            const int Rb = row_base + i0 + b2;
+#pragma unroll
+                            for (int sp = 0; sp < kMaxFusedSplits; ++sp)
+                                v[b2][sp] = (Rb < rows_total && sp < nsplit)
+                                                ? __ldcg(reinterpret_cast<const float4*>(
+                                                             p.part_o + (sp * stride + row_of(Rb)) * kD) + lane)
+                                                : make_float4(0.f, 0.f, 0.f, 0.f);
+                        }
+#pragma unroll
+                        for (int b2 = 0; b2 < kMergeRows; ++b2) {
+                            const int rl = 32 * warp + i0 + b2, Rb = R0 + rl;
+                            if (Rb >= rows_total) continue;
+                            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                            for (int sp = 0; sp < kMaxFusedSplits; ++sp) {
+                                const float ws = s_wts[rl * kMaxFusedSplits + sp];
+                                acc.x += ws * v[b2][sp].x;
+                                acc.y += ws * v[b2][sp].y;
+                                acc.z += ws * v[b2][sp].z;
+                                acc.w += ws * v[b2][sp].w;
+                            }
+                            reinterpret_cast<float4*>(p.out + row_of(Rb) * kD)[lane] = acc;
+                        }
                     }
                 }
             }

@@ -198,6 +198,10 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read1() {
     asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
+// wait until none of this thread's bulk groups still reads shared memory
+__device__ __forceinline__ void bulk_wait_read0() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
 // wait until every bulk group of this thread has completed (its writes are done)
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
@@ -209,6 +213,23 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* map
         " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(0), "r"(0), "r"(0), "r"(grp)
         : "memory");
+}
+
+// 4-D tiled load at coordinates (x, y, z, w) (the split-partial map: {dim, head, token, split}).
+__device__ __forceinline__ void tma_load_4d_at(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                               int x, int y, int z, int w) {
+    asm volatile(
+        "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y), "r"(z), "r"(w)
+        : "memory");
+}
+
+// Orders this thread's earlier accesses in any proxy with its later ones in any other proxy,
+// for global as well as shared memory (here: data that other CTAs wrote with bulk tensor
+// stores, read afterwards with bulk tensor loads).
+__device__ __forceinline__ void fence_proxy_async_all() {
+    asm volatile("fence.proxy.async;" ::: "memory");
 }
 
 // Barrier `id` among the first `count` threads of the CTA (whole warps).
