@@ -490,8 +490,18 @@ decode_tc8_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) 
                 const int nvalid = kend - key0;
                 const int b_lo = nvalid >> 4, b_hi = 2 * ceil_div(nvalid, 32);
                 if (nvalid < kKeys && b_lo < b_hi) {
-                    if (!__all_sync(0xffffffffu, mbar_wait(smem_u32(&bar_vf[t % kVSlots]), (t / kVSlots) & 1u,
-                                                           kWaitLimitNs, p.err))) {
+                    // The softmax runs ahead of the V copies (K has its own ring), so the slot's
+                    // previous tile, t - kVSlots, may still be landing: first wait for the P V
+                    // that read it (which leaves the slot's barrier one phase short of tile t,
+                    // so the parity wait below cannot pass on the older phase), then for V(t).
+                    bool v_ok = true;
+                    if (t >= kVSlots)
+                        v_ok = mbar_wait(smem_u32(&bar_pv[(t - kVSlots) % kPBufs]),
+                                         ((t - kVSlots) / kPBufs) & 1u, kWaitLimitNs, p.err);
+                    if (v_ok)
+                        v_ok = mbar_wait(smem_u32(&bar_vf[t % kVSlots]), (t / kVSlots) & 1u,
+                                         kWaitLimitNs, p.err);
+                    if (!__all_sync(0xffffffffu, v_ok)) {
                         fail = true;
                         continue;
                     }

@@ -276,6 +276,25 @@ def test_random_small_steps_fp8_with_chunks(seed):
     assert_close(st.out.cpu().numpy(), want, W.FP8_E4M3, f"fp8 chunks seed {seed}")
 
 
+@pytest.mark.parametrize("kv_split_tokens", [0, 1024])
+def test_fp8_decode_repeats_bit_identical(kv_split_tokens):
+    # The FP8 decode kernel runs its scores and probabilities ahead of the V copies; any wait
+    # that can pass on an older phase shows up as results that change from call to call.  Many
+    # short requests with partial last tiles (and, at 1024-key splits, many split merges), each
+    # called five times: every call bit-identical, and equal to the oracle within tolerance.
+    rng = np.random.default_rng(4243 + kv_split_tokens)
+    ctx = [int(x) for x in rng.integers(300, 3000, 48)]
+    wl = W.make_workload("fp8-repeat", ctx, [1] * 48, 32, 8, 128, 16, 16 * 1024, 4243,
+                         kv_dtype=W.FP8_E4M3)
+    st = GpuStep(wl, kv_split_tokens=kv_split_tokens)
+    first = st.out.cpu()
+    for i in range(4):
+        again = st.attend(kv_split_tokens=kv_split_tokens).cpu()
+        assert torch.equal(again, first), f"call {i + 1} differs from the first"
+    want, _ = oracle_attention_all(wl, oracle_cache(wl))
+    assert_close(first.numpy(), want, W.FP8_E4M3, "fp8 repeat")
+
+
 def test_random_small_steps_fp8():
     for seed in range(4):
         rng = np.random.default_rng(2000 + seed)
