@@ -135,14 +135,13 @@ def chunk_flops(wl, window: int = 0, local_chunk: int = 0) -> int:
 def launches_for_plan(plan: dict, head_size: int) -> int:
     """Kernels of ours per step, as pa_attention launches them: slot mapping and write, the
     split-counter clear (split decode requests, or chunk splits the tcgen05 kernel merges
-    itself: head_size 128 and at most 4 splits), the cascade prefix pass and final merge, the
-    decode and/or chunk kernel, and the split reduce (chunk splits not merged in the chunk
-    kernel)."""
+    itself: head_size 128 and at most 4 splits), the cascade prefix pass, the decode and/or
+    chunk kernel, and the split reduce (chunk splits not merged in the chunk kernel)."""
     fused = head_size == 128 and plan["chunk_max_splits"] <= 4
     clear = plan["decode_max_splits"] > 1 or (plan["chunk_max_splits"] > 1 and fused)
     reduce = plan["chunk_max_splits"] > 1 and not fused
     prefix = plan.get("prefix_splits", 0) > 0
-    return 2 + int(clear) + 2 * int(prefix) + int(plan["num_decode_seqs"] > 0) + \
+    return 2 + int(clear) + int(prefix) + int(plan["num_decode_seqs"] > 0) + \
         int(plan["num_chunk_seqs"] > 0) + int(reduce)
 
 

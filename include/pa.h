@@ -237,14 +237,11 @@ typedef struct {
     int kv_split_tokens;   /* > 0: force this many keys (multiple of block_size) per split
                               for every request; 0: planner's choice */
     int num_sms;           /* > 0: plan for this many SMs instead of the device's count */
-    void* events[6];       /* optional cudaEvent_t handles: [0]/[1] before/after the decode
-                              kernel, [2]/[3] around the chunk kernel (with a common prefix:
-                              its prefix pass), [4]/[5] around the split reduce (with a common
-                              prefix: the final merge); recorded on the stream the kernel runs
-                              on (the call's, or for the chunk kernel of a step with both kinds
-                              and for the prefix pass, a side stream of the library joined back
-                              before the call returns); an entry is recorded only when that
-                              kernel is launched; NULL entries are skipped */
+    void* events[6];       /* optional cudaEvent_t handles recorded on the call's stream:
+                              [0]/[1] before/after the decode kernel, [2]/[3] around the chunk
+                              kernel (with a common prefix: its prefix pass), [4]/[5] around
+                              the split reduce; an entry is recorded
+                              only when that kernel is launched; NULL entries are skipped */
     int sliding_window;    /* > 0: a query at position p sees only keys max(0, p - W + 1) .. p
                               (the sliding window [P2] section 2 names; its reading here);
                               0: full causal attention */
@@ -267,15 +264,13 @@ typedef struct {
                               of every request with q_len > 0 are the same physical blocks
                               (pa_common_prefix_blocks finds them from a host copy of the
                               table); the call reads those blocks once for all the step's
-                              queries (the prefix pass, on a side stream), attends each
-                              request's remaining keys separately at the same time, and merges
-                              the two by their LSEs -- the result is the same attention.
+                              queries, attends each request's remaining keys separately and
+                              merges the two by their LSEs -- the result is the same attention.
                               Requires a multiple of block_size, every request with q_len > 0
                               decode-kind with seq_len - q_len >= common_prefix_tokens
                               (else METADATA), no sliding window or local chunk (else
-                              UNSUPPORTED), and workspace for the prefix partials and the
-                              suffix result (pa_plan_attention's workspace_needed; else
-                              WORKSPACE).  0: off */
+                              UNSUPPORTED), and workspace for the prefix partials
+                              (pa_plan_attention's workspace_needed; else WORKSPACE).  0: off */
     int test_skip_decode_load; /* test hook of the bounded waits, 0 in normal use.  k > 0: in
                               the decode kernel's CTA (split 0, kv head 0, request 0), warp 0
                               leaves the load of its k-th unit (a block, two for FP8) of its

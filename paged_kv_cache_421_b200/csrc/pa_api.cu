@@ -463,16 +463,17 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
         sp = std::min<long long>(sp, std::max(1, ptiles / 2));
         sp = std::min<long long>(sp, pa::kMaxChunkWork / qtiles);
         sp = std::min<long long>(std::max<long long>(sp, 1), kMaxPrefixSplits);
-        // the prefix partials follow the split partials in the workspace, and the suffix
-        // attention's result follows them as one more part (the two are merged at the end)
+        // the prefix partials follow the split partials in the workspace
         const size_t base = pl->workspace_needed;
-        if (base + prefix_part_bytes(T, Hq, D, 2) > ws) return PA_ERR_WORKSPACE;
-        while (sp > 1 && base + prefix_part_bytes(T, Hq, D, static_cast<int>(sp) + 1) > ws) --sp;
+        const size_t per = prefix_part_bytes(T, Hq, D, 1);
+        if (base + per > ws) return PA_ERR_WORKSPACE;
+        sp = std::min<long long>(sp, static_cast<long long>((ws - base) / per));
+        while (sp > 1 && base + prefix_part_bytes(T, Hq, D, static_cast<int>(sp)) > ws) --sp;
         int psb = round_up(pa::ceil_div(pblocks, static_cast<int>(sp)), tile_blocks);
         pl->prefix_split_blocks = psb;
         pl->prefix_splits = pa::ceil_div(pblocks, psb);
         pl->prefix_ctas = qtiles * Hkv * pl->prefix_splits;
-        pl->workspace_needed = base + prefix_part_bytes(T, Hq, D, pl->prefix_splits + 1);
+        pl->workspace_needed = base + prefix_part_bytes(T, Hq, D, pl->prefix_splits);
     }
     return PA_OK;
 }
@@ -740,7 +741,7 @@ int pa::attention_call(const pa_cache* cache, const void* q, int num_q_heads,
         const int smax = pl.decode_max_splits > pl.chunk_max_splits ? pl.decode_max_splits
                                                                      : pl.chunk_max_splits;
         const size_t base = workspace_for(num_tokens, num_q_heads, cache->head_size, smax);
-        const size_t rows = static_cast<size_t>(pl.prefix_splits + 1) * num_tokens * num_q_heads;
+        const size_t rows = static_cast<size_t>(pl.prefix_splits) * num_tokens * num_q_heads;
         p.prefix_keys = opts->common_prefix_tokens;
         p.prefix_parts = pl.prefix_splits;
         p.prefix_o = reinterpret_cast<const float*>(static_cast<char*>(workspace) + base);
@@ -758,26 +759,10 @@ int pa::attention_call(const pa_cache* cache, const void* q, int num_q_heads,
         e = pa::launch_zero_counters(p.split_counters, num_tokens * cache->num_kv_heads, s);
         if (e != cudaSuccess) return fail_cuda(e);
     }
-    // A cascade call runs its prefix pass, and a step with both kinds its chunk kernel, on the
-    // side stream, forked from this stream after the counter clear and joined back before the
-    // kernels that need both results (the cascade merge, the split reduce).
-    SideStream* side = nullptr;
-    std::unique_lock<std::mutex> side_lock;
-    if (allow_side_stream && pl.num_decode_seqs &&
-        (cascade || (kOverlapChunksWithDecode && pl.num_chunk_seqs))) {
-        side = side_stream();
-        if (side) {
-            side_lock = std::unique_lock<std::mutex>(side->mu);
-            e = cudaEventRecord(side->fork, s);
-            if (e == cudaSuccess) e = cudaStreamWaitEvent(side->stream, side->fork, 0);
-            if (e != cudaSuccess) return fail_cuda(e);
-        }
-    }
-    const cudaStream_t cs = side ? side->stream : s;  // the prefix pass's or chunk kernel's stream
     if (cascade) {
         // the prefix pass: every query row of the step against the shared prefix's keys, read
         // once per (kv head, split) instead of once per request; each split's partials go to
-        // the workspace, where the merge at the end combines them with the suffix attention
+        // the workspace, where the decode kernel below merges them into its rows
         pa::AttnParams pp = p;
         pp.prefix_launch = 1;
         pp.prefix_row = prefix_row;
@@ -816,11 +801,11 @@ int pa::attention_call(const pa_cache* cache, const void* q, int num_q_heads,
                           pl.prefix_splits, cache->kv_dtype == PA_BF16);
         else
             std::memset(&pio, 0, sizeof(pio));
-        if (ev) record(ev[2], cs);
+        if (ev) record(ev[2], s);
         e = pa::launch_chunk(cache->tmap, cache->tmap_blk, pp, pwork, pio, cache->head_size,
-                             cache->kv_dtype, pl.prefix_splits, cs);
+                             cache->kv_dtype, pl.prefix_splits, s);
         if (e != cudaSuccess) return fail_cuda(e);
-        if (ev) record(ev[3], cs);
+        if (ev) record(ev[3], s);
     }
     // the chunk-kind requests, longest context first; a longer list falls back to a grid over
     // every request
@@ -880,6 +865,21 @@ int pa::attention_call(const pa_cache* cache, const void* q, int num_q_heads,
             for (const auto& it : items) work.item[work.count++] = it.second;
         }
     }
+    // a step with both kinds: the chunk kernel on the side stream, forked from this stream after
+    // the counter clear and joined back before the split reduce
+    SideStream* side = nullptr;
+    std::unique_lock<std::mutex> side_lock;
+    if (kOverlapChunksWithDecode && allow_side_stream && pl.num_decode_seqs && pl.num_chunk_seqs &&
+        !cascade) {
+        side = side_stream();
+        if (side) {
+            side_lock = std::unique_lock<std::mutex>(side->mu);
+            e = cudaEventRecord(side->fork, s);
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(side->stream, side->fork, 0);
+            if (e != cudaSuccess) return fail_cuda(e);
+        }
+    }
+    const cudaStream_t cs = side ? side->stream : s;  // the chunk kernel's stream
     static thread_local pa::ChunkIo io;
     if (pl.num_chunk_seqs && cache->head_size == 128)
         make_chunk_io(io, q, out, pl.chunk_max_splits > 1 ? p.part_o : nullptr, num_tokens,
@@ -894,21 +894,9 @@ int pa::attention_call(const pa_cache* cache, const void* q, int num_q_heads,
         if (e != cudaSuccess) return fail_cuda(e);
         if (ev) record(ev[3], cs);
     }
-    // the cascade suffix attention: each request's own keys after the prefix, written as the
-    // last part after the prefix partials (normalised rows, log2 LSEs) instead of to out
-    const int64_t all_rows = static_cast<int64_t>(num_tokens) * num_q_heads;
-    pa::AttnParams pd = p;
-    if (cascade) {
-        pd.prefix_parts = 0;
-        pd.prefix_o = nullptr;
-        pd.prefix_lse = nullptr;
-        pd.out = const_cast<float*>(p.prefix_o) + pl.prefix_splits * all_rows * cache->head_size;
-        pd.lse_out = const_cast<float*>(p.prefix_lse) + pl.prefix_splits * all_rows;
-        pd.lse_log2 = 1;
-    }
     if (pl.num_decode_seqs) {
         if (ev) record(ev[0], s);
-        e = pa::launch_decode(cache->tmap, pd, cache->head_size, cache->kv_dtype,
+        e = pa::launch_decode(cache->tmap, p, cache->head_size, cache->kv_dtype,
                               pl.decode_max_splits, s);
         if (e != cudaSuccess) return fail_cuda(e);
         if (ev) record(ev[1], s);
@@ -929,15 +917,6 @@ int pa::attention_call(const pa_cache* cache, const void* q, int num_q_heads,
     if (pl.chunk_max_splits > 1 && !chunk_merge_fused) {
         if (ev) record(ev[4], s);
         e = pa::launch_reduce(p, list, cache->head_size, s);
-        if (e != cudaSuccess) return fail_cuda(e);
-        if (ev) record(ev[5], s);
-    }
-    if (cascade) {
-        // every row: the prefix splits' and the suffix's (O, lse) merged by their LSEs
-        if (ev) record(ev[4], s);
-        e = pa::launch_merge_partials(p.prefix_o, p.prefix_lse, pl.prefix_splits + 1, all_rows,
-                                      cache->head_size, out, opts ? opts->lse_out : nullptr, s,
-                                      true);
         if (e != cudaSuccess) return fail_cuda(e);
         if (ev) record(ev[5], s);
     }

@@ -59,10 +59,10 @@ template <int D>
 __global__ void __launch_bounds__(128)
 merge_partials_kernel(const float* __restrict__ part_out, const float* __restrict__ part_lse,
                       int num_parts, int64_t num_rows, float* __restrict__ out,
-                      float* __restrict__ lse_out, float to_log2) {
+                      float* __restrict__ lse_out) {
     pdl_trigger();
     pdl_wait();
-    const float kLog2e = to_log2;  // the parts' LSE unit -> log2 (log2 e, or 1 for log2 LSEs)
+    constexpr float kLog2e = 1.44269504088896341f;
     constexpr int kVec = D / 32;  // floats per lane: 4 for D = 128, 2 for D = 64
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int64_t n = static_cast<int64_t>(blockIdx.x) * 4 + warp; n < num_rows;
@@ -126,16 +126,15 @@ cudaError_t launch_dcp_slot_mapping(const int32_t* block_table, int max_blocks_p
 
 cudaError_t launch_merge_partials(const float* part_out, const float* part_lse, int num_parts,
                                   int64_t num_rows, int head_size, float* out, float* lse_out,
-                                  cudaStream_t stream, bool lse_in_log2) {
+                                  cudaStream_t stream) {
     const int64_t want = (num_rows + 3) / 4;
     const int blocks = static_cast<int>(want < 148 * 64 ? want : 148 * 64);
-    const float to_log2 = lse_in_log2 ? 1.f : 1.44269504088896341f;
     if (head_size == 128)
         return launch_pdl(merge_partials_kernel<128>, dim3(blocks), dim3(128), 0, stream,
-                          part_out, part_lse, num_parts, num_rows, out, lse_out, to_log2);
+                          part_out, part_lse, num_parts, num_rows, out, lse_out);
     if (head_size == 64)
         return launch_pdl(merge_partials_kernel<64>, dim3(blocks), dim3(128), 0, stream,
-                          part_out, part_lse, num_parts, num_rows, out, lse_out, to_log2);
+                          part_out, part_lse, num_parts, num_rows, out, lse_out);
     return cudaErrorInvalidValue;
 }
 

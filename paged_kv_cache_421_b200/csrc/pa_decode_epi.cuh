@@ -21,7 +21,6 @@ __device__ __forceinline__ void decode_finish(const AttnParams& p, uint8_t* smem
     const float* red_o = reinterpret_cast<const float*>(smem);  // [NSTATE][D][8]
     const float* red_m = red_o + NSTATE * D * kDecodeRows;      // [NSTATE][8]
     const float* red_l = red_m + NSTATE * kDecodeRows;          // [NSTATE][8]
-    const float lse_unit = p.lse_log2 ? 1.f : kLn2;  // exported LSEs: natural log, or log2
     const bool direct = nsplit == 1;
     if (!direct && split >= p.max_splits) {  // workspace bound (a planned launch never hits it)
         if (tid == 0) raise_error(p.err, kErrMetadata);
@@ -92,7 +91,7 @@ __device__ __forceinline__ void decode_finish(const AttnParams& p, uint8_t* smem
             const float inv = W > 0.f ? 1.f / W : 0.f;
 #pragma unroll
             for (int i = 0; i < DL; ++i) p.out[row * D + lane + 32 * i] = o[i] * inv;
-            if (lane == 0 && p.lse_out) p.lse_out[row] = W > 0.f ? (X + __log2f(W)) * lse_unit : -INFINITY;
+            if (lane == 0 && p.lse_out) p.lse_out[row] = W > 0.f ? (X + __log2f(W)) * kLn2 : -INFINITY;
         }
         return;
     }
@@ -116,7 +115,7 @@ __device__ __forceinline__ void decode_finish(const AttnParams& p, uint8_t* smem
         if (direct) {
             const int64_t row = static_cast<int64_t>(t) * p.num_q_heads + h;
             p.out[row * D + d] = val;
-            if (d == 0 && p.lse_out) p.lse_out[row] = L > 0.f ? (M + __log2f(L)) * lse_unit : -INFINITY;
+            if (d == 0 && p.lse_out) p.lse_out[row] = L > 0.f ? (M + __log2f(L)) * kLn2 : -INFINITY;
         } else {
             const int64_t prow = split * stride + static_cast<int64_t>(t) * p.num_q_heads + h;
             p.part_o[prow * D + d] = val;
@@ -160,7 +159,7 @@ __device__ __forceinline__ void decode_finish(const AttnParams& p, uint8_t* smem
         for (int off = 16; off > 0; off >>= 1) W += __shfl_xor_sync(0xffffffffu, W, off);
         if (lane == 0) {
             s_inv[n] = W > 0.f ? 1.f / W : 0.f;
-            if (p.lse_out) p.lse_out[row] = W > 0.f ? (M + __log2f(W)) * lse_unit : -INFINITY;
+            if (p.lse_out) p.lse_out[row] = W > 0.f ? (M + __log2f(W)) * kLn2 : -INFINITY;
         }
     }
     __syncthreads();

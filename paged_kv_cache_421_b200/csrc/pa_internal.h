@@ -88,7 +88,6 @@ struct AttnParams {
     int prefix_parts;
     const float* prefix_o;
     const float* prefix_lse;
-    int lse_log2;               // decode kernels: lse_out in log2 units (a cascade suffix part)
     // Test hook of the bounded waits (decode kernel): > 0 makes CTA (split 0, kv head 0,
     // request 0) skip the load of warp 0's unit test_skip_unit - 1 of its first round, and that
     // CTA's waits give up after test_wait_ns; 0 = off.
@@ -167,11 +166,9 @@ cudaError_t launch_dcp_slot_mapping(const int32_t* block_table, int max_blocks_p
                                     const int32_t* seq_lens, const int32_t* qsl, int num_seqs,
                                     int num_tokens, int block_size, int rank, int world,
                                     int32_t* slot_mapping, int* err, cudaStream_t stream);
-// lse_in_log2: the parts' LSEs are in log2 units (the kernels' partials) instead of natural log
-// (the exported LSEs); lse_out is natural log either way
 cudaError_t launch_merge_partials(const float* part_out, const float* part_lse, int num_parts,
                                   int64_t num_rows, int head_size, float* out, float* lse_out,
-                                  cudaStream_t stream, bool lse_in_log2 = false);
+                                  cudaStream_t stream);
 cudaError_t launch_validate(const int32_t* block_table, int max_blocks_per_seq,
                             const int32_t* seq_lens, int num_seqs, int block_size,
                             int num_blocks, int* counter, cudaStream_t stream);

@@ -102,8 +102,7 @@ def test_plan_cascade_on_prefix_share_decode(lib):
     # the decode kernel now walks only the suffixes
     assert p["decode_ctas"] <= base["decode_ctas"]
     per = lambda rows: -(-rows // 256) * 256  # noqa: E731  (256-byte aligned regions)
-    # the prefix splits' partials, then the suffix attention's result as one more part
-    rows = (p["prefix_splits"] + 1) * T * Hq
+    rows = p["prefix_splits"] * T * Hq
     assert p["workspace_needed"] == (B.pa_attention_workspace_bytes(
         T, Hq, D, max(p["decode_max_splits"], p["chunk_max_splits"]))
         + per(rows * D * 4) + per(rows * 4))
@@ -132,14 +131,10 @@ def test_plan_cascade_refusals(lib):
 
 
 def test_plan_cascade_fits_a_small_workspace(lib):
-    # fewer prefix splits when the workspace holds fewer partials, down to one (two parts: the
-    # prefix split's and the suffix attention's); one part is too little
+    # fewer prefix splits when the workspace holds fewer partials, down to one
     wl = W.prefix_share_decode()
     T, Hq, D = wl.num_tokens, wl.num_q_heads, wl.head_size
-    two = -(-2 * T * Hq * D * 4 // 256) * 256 + -(-2 * T * Hq * 4 // 256) * 256
-    p = _plan(wl, 1024, ws=two)
-    assert p["prefix_splits"] == 1 and p["workspace_needed"] <= two
-    with pytest.raises(B.PaError) as e:
-        _plan(wl, 1024, ws=two // 2)
-    assert e.value.status == B.PA_ERR_WORKSPACE
+    one = -(-T * Hq * D * 4 // 256) * 256 + -(-T * Hq * 4 // 256) * 256
+    p = _plan(wl, 1024, ws=one)
+    assert p["prefix_splits"] == 1 and p["workspace_needed"] <= one
     assert p["decode_max_splits"] == 1

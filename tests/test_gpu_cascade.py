@@ -109,16 +109,15 @@ def test_cascade_fp8_cache():
 
 
 def test_cascade_with_a_workspace_for_one_prefix_split():
-    # room for two parts: one prefix split's partials and the suffix attention's result
     wl = W.prefix_share_decode()
     st = GpuStep(wl, run_attention=False)
     T, Hq, D = wl.num_tokens, wl.num_q_heads, wl.head_size
-    two = -(-2 * T * Hq * D * 4 // 256) * 256 + -(-2 * T * Hq * 4 // 256) * 256
+    one = -(-T * Hq * D * 4 // 256) * 256 + -(-T * Hq * 4 // 256) * 256
     plan = B.pa_plan_attention(wl.seq_lens, wl.qsl, Hq, wl.num_kv_heads, D,
-                               wl.max_blocks_per_seq, 148, two, common_prefix_tokens=1024)
+                               wl.max_blocks_per_seq, 148, one, common_prefix_tokens=1024)
     assert plan["prefix_splits"] == 1
     want, _ = oracle_attention_all(wl, oracle_cache(wl))
-    got, _ = _cascade(st, 1024, workspace_bytes=two)
+    got, _ = _cascade(st, 1024, workspace_bytes=one)
     assert_close(got, want, W.BF16, "one prefix split")
 
 
