@@ -362,12 +362,16 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
         if (forced) {
             dsb = forced / bs;
         } else {
-            // two waves of the decode kernel's resident CTAs
-            const long long target = static_cast<long long>(num_sms) *
-                                     (tc8 ? kDecodeTc8CtasPerSm : kDecodeCtasPerSm) * kDecodeWaves;
+            // mma.sync kernel: two waves of its resident CTAs.  tcgen05 FP8 kernel (two CTAs
+            // per SM, each long): 1.75 waves, so that the second wave is mostly full rather than
+            // a thin tail, in whole 128-key tiles (long70b_decode_fp8: 0.184 ms at 2.08 waves,
+            // 0.166-0.168 ms at 1.76-1.86, 0.185-0.210 ms at 1.16-1.43)
+            const long long target =
+                tc8 ? static_cast<long long>(num_sms) * kDecodeTc8CtasPerSm * 7 / 4
+                    : static_cast<long long>(num_sms) * kDecodeCtasPerSm * kDecodeWaves;
             long long sb = (dec_units + target - 1) / target;
             if (sb < kMinDecodeSplitBlocks) sb = kMinDecodeSplitBlocks;
-            dsb = round_up(static_cast<int>(sb < dec_max_blocks ? sb : dec_max_blocks), 4);
+            dsb = round_up(static_cast<int>(sb < dec_max_blocks ? sb : dec_max_blocks), tc8 ? 8 : 4);
         }
         int ns = pa::ceil_div(dec_max_blocks, dsb);
         const int cap = allowed < kMaxDecodeSplits ? allowed : kMaxDecodeSplits;
