@@ -232,7 +232,6 @@ size_t prefix_part_bytes(int num_tokens, int num_q_heads, int head_size, int spl
 constexpr int kDecodeCtasPerSm = 3;    // decode kernel residency (64 KB of stages per CTA)
 constexpr int kDecodeTc8CtasPerSm = 2;  // tcgen05 FP8 decode kernel residency (107 KB per CTA)
 constexpr int kMaxDecodeSplits = 1024;  // merge weights of one row fit the CTA's shared memory
-constexpr int kDecodeWaves = 2;             // target waves of decode CTAs (2 measured best)
 constexpr int kMinDecodeSplitBlocks = 64;   // >= 1024 keys per split
 constexpr int kMinChunkSplitBlocks = 16;
 constexpr int kMinChunkSplitTiles = 4;      // a chunk split walks at least four key tiles
@@ -362,13 +361,13 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
         if (forced) {
             dsb = forced / bs;
         } else {
-            // mma.sync kernel: two waves of its resident CTAs.  tcgen05 FP8 kernel (two CTAs
-            // per SM, each long): 1.75 waves, so that the second wave is mostly full rather than
-            // a thin tail, in whole 128-key tiles (long70b_decode_fp8: 0.184 ms at 2.08 waves,
-            // 0.166-0.168 ms at 1.76-1.86, 0.185-0.210 ms at 1.16-1.43)
-            const long long target =
-                tc8 ? static_cast<long long>(num_sms) * kDecodeTc8CtasPerSm * 7 / 4
-                    : static_cast<long long>(num_sms) * kDecodeCtasPerSm * kDecodeWaves;
+            // 1.75 waves of the decode kernel's resident CTAs, so that the second wave is mostly
+            // full rather than a thin tail (measured on the long-context step: bf16 0.322 ms at
+            // 2.09 waves, 0.305 ms at 1.51-1.86, 0.327-0.352 ms at 1.17-1.32; FP8 0.184 ms at
+            // 2.08, 0.166-0.168 ms at 1.76-1.86, 0.185-0.210 ms at 1.16-1.43; short contexts,
+            // llama8b_decode, within 1 % from 1.8 to 3.1 waves); tcgen05 splits in whole tiles
+            const long long target = static_cast<long long>(num_sms) *
+                                     (tc8 ? kDecodeTc8CtasPerSm : kDecodeCtasPerSm) * 7 / 4;
             long long sb = (dec_units + target - 1) / target;
             if (sb < kMinDecodeSplitBlocks) sb = kMinDecodeSplitBlocks;
             dsb = round_up(static_cast<int>(sb < dec_max_blocks ? sb : dec_max_blocks), tc8 ? 8 : 4);
