@@ -456,6 +456,21 @@ class DeviceStep:
                           common_prefix_tokens=self.prefix)
 
 
+def queue_ahead_ms(steps: int) -> float:
+    """Length of the device-side wait in front of K timed steps: about 1 ms of host time per
+    step to enqueue, at least 20 ms."""
+    return min(200.0, max(20.0, 1.0 * steps))
+
+
+def queue_ahead(stream, steps: int):
+    """A device-side wait on `stream`, so that the host enqueues the timed steps while the
+    device waits and the timed region holds device time only (a host slower than a step would
+    otherwise leave the device idle between launches)."""
+    import torch
+    with torch.cuda.stream(stream):
+        torch.cuda._sleep(int(queue_ahead_ms(steps) * 2.0e6))  # cycles at about 2 GHz
+
+
 def time_step(step, args, flush_l2: bool, flush, stream, world: int, local: int, device,
               clock_path: str):
     """Warm up, then time K steps of `step`: once between one pair of CUDA events on the
@@ -488,6 +503,7 @@ def time_step(step, args, flush_l2: bool, flush, stream, world: int, local: int,
              for _ in range(args.steps)]
     barrier()
     torch.cuda.synchronize(device)
+    queue_ahead(stream, args.steps)
     t_start.record(stream)
     for i in range(args.steps):
         if flush_l2:
@@ -505,6 +521,7 @@ def time_step(step, args, flush_l2: bool, flush, stream, world: int, local: int,
     ms_per_step = max_over_ranks(timed, world, device) / args.steps
     barrier()
     torch.cuda.synchronize(device)
+    queue_ahead(stream, args.steps)
     for i in range(args.steps):
         if flush_l2:
             flush.zero_()
@@ -779,6 +796,8 @@ def run_device_bench(args, rank, world, local):
                               if flush_l2 else
                               f"inputs larger than L2: {nbytes / 1e6:.0f} MB of KV per step vs "
                               f"126 MB L2, no flush"),
+                       "launch": (f"the timed steps are enqueued behind a ~{queue_ahead_ms(args.steps):.0f} ms "
+                                  "device-side wait (device time only, no host gaps)"),
                        "kv_split_tokens": args.kv_split_tokens or "planner",
                        "cascade_prefix_tokens": step.prefix or None,
                        "sliding_window": args.sliding_window or None,

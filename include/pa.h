@@ -230,6 +230,11 @@ typedef struct {
     int prefix_splits;        /* cascade: KV splits of the shared-prefix pass (0: no cascade) */
     int prefix_split_blocks;  /* cascade: blocks per prefix split */
     int64_t prefix_ctas;      /* cascade: CTAs of the prefix pass */
+    int chunk_ctas_per_kv_head; /* a step with both kinds (head_size 128, no cascade): the
+                              chunk kernel's CTAs per kv head while it runs beside the decode
+                              kernel, each walking several of its (q-tile pair, split) items
+                              -- the fewest whose longest-first schedule is estimated to end
+                              within the decode kernel's time; 0: one CTA per item */
 } pa_plan;
 
 /* Options for pa_attention_ex (zero-initialise for defaults). */

@@ -56,6 +56,7 @@ class pa_plan(ctypes.Structure):
         ("prefix_splits", ctypes.c_int),
         ("prefix_split_blocks", ctypes.c_int),
         ("prefix_ctas", ctypes.c_int64),
+        ("chunk_ctas_per_kv_head", ctypes.c_int),
     ]
 
     def as_dict(self) -> dict:

@@ -63,10 +63,13 @@ int device_num_sms() {
     return n;
 }
 
-// Mixed steps: the chunk kernel runs on a second stream of the device while the decode kernel
+// Mixed steps: the decode kernel runs on a second stream of the device while the chunk kernel
 // runs on the caller's, so that the chunk CTAs (tensor-bound, one per SM) take a subset of the
-// SMs while the decode CTAs keep HBM busy on the others.  The stream has the device's highest
-// priority, so its CTAs are dispatched first; events fork it from and join it back into the
+// SMs while the decode CTAs keep HBM busy on the others.  The chunk kernel is launched first,
+// right behind the step's earlier kernels on the caller's stream (programmatic dependent
+// launch), so its CTAs are resident before the decode CTAs arrive and fill the other SMs; in
+// the other order the decode CTAs hold every SM and the chunk CTAs get an SM only when all of
+// its decode CTAs have ended.  Events fork the second stream from and join it back into the
 // caller's stream, which keeps every call stream-ordered (and capturable in a graph).
 constexpr bool kOverlapChunksWithDecode = true;
 
@@ -163,17 +166,17 @@ size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // Tensor maps of a call's Q, output and (cascade) prefix partials for the tcgen05 chunk kernel
 // (head_size 128): Q as {128, Hq, T} bf16 with 128-byte boxes of G heads x 128 / G tokens (one
-// 128-row q-tile half per box, bf16 cache only: FP8 Q is split on the way in), O as
+// 128-row q-tile half per box; with an FP8 cache the kernel splits it in shared memory), O as
 // {128, Hq, T} fp32 and the partials as {128, Hq, T, S} fp32 with boxes of 32 floats x G heads x
 // 32 / G tokens (one warp's rows of one 32-column chunk).  A map whose shape does not fit (G
 // not dividing 128 or 32) is left unused.
 void make_chunk_io(pa::ChunkIo& io, const void* q, float* out, const float* part, int T, int Hq,
-                   int G, int S, bool q_ok) {
+                   int G, int S) {
     std::memset(&io, 0, sizeof(io));
     EncodeTiledFn enc = encode_fn();
     if (!enc || T <= 0) return;
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    if (q_ok && 128 % G == 0) {
+    if (128 % G == 0) {
         cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(Hq), static_cast<cuuint64_t>(T)};
         cuuint64_t strides[2] = {128 * 2, static_cast<cuuint64_t>(Hq) * 128 * 2};
         cuuint32_t box[3] = {64, static_cast<cuuint32_t>(G), static_cast<cuuint32_t>(128 / G)};
@@ -237,6 +240,91 @@ constexpr int kMinChunkSplitBlocks = 16;
 constexpr int kMinChunkSplitTiles = 4;      // a chunk split walks at least four key tiles
 constexpr int kMaxChunkSplitBlocks = 1024;  // chunk kernels stage up to 1024 block ids
 constexpr int kMaxPrefixSplits = pa::kMaxPrefixParts;  // prefix partials a decode row merges
+// Mixed steps: the tcgen05 chunk kernel runs beside the decode kernel on as few SMs as still let
+// it end within the decode kernel's time, each of its CTAs walking a share of the items.  Its
+// time on y CTAs per kv head is estimated at kChunkTileUs per key tile and kChunkItemTiles tiles
+// per item (measured beside the decode kernel on B200: 3.6-4.4 us a tile, about 9 us of set-up
+// and epilogue per item), the decode kernel's at its KV bytes over kDecodeGBs (the decode kernel
+// keeps its bandwidth on the other SMs: it drops by about 1 % with 48 of 148 SMs taken, 3 % with
+// 64, 25 % with 96, half with 128).
+constexpr double kChunkTileUs = 4.2;
+constexpr int kChunkItemTiles = 2;
+constexpr double kDecodeGBsBf16 = 5700.0, kDecodeGBsFp8 = 4100.0;
+
+// The (q-tile pair, split) items of a chunk-kind request with ql queries over ctx keys, each
+// with the key tiles its CTA walks: f(qt, split, tiles) for every item, splits of csb blocks,
+// cta_rows query rows per item, tile_keys keys per tile.
+template <class F>
+void for_each_chunk_item(int ctx, int ql, int G, int bs, int csb, int window, int local_chunk,
+                         int cta_rows, int tile_keys, F&& f) {
+    const int nsplit = pa::ceil_div(pa::ceil_div(ctx, bs), csb);
+    const int nqt = pa::ceil_div(ql * G, cta_rows);
+    for (int qt = 0; qt < nqt; ++qt) {
+        const int last_row = std::min((qt + 1) * cta_rows, ql * G) - 1;
+        const int kmax = ctx - ql + last_row / G;
+        const int lo = pa::first_visible_key(ctx - ql + qt * cta_rows / G, window, local_chunk) / bs * bs;
+        for (int sp = 0; sp < nsplit; ++sp) {
+            const int key_lo = std::max(sp * csb * bs, lo);
+            const int key_hi = std::min(std::min((sp + 1) * csb * bs, ctx), kmax + 1);
+            f(qt, sp, key_hi > key_lo ? pa::ceil_div(key_hi - key_lo, tile_keys) : 0);
+        }
+    }
+}
+
+// Longest-processing-time schedule of the chunk items (tiles, item), most tiles first, over y
+// CTAs: each item goes to the CTA with the least work so far (its tiles plus kChunkItemTiles).
+// Returns the longest CTA's work in tiles; fills cta[c] with CTA c's items when cta is given.
+long long lpt_chunk_ctas(const std::vector<std::pair<int, uint32_t>>& items, int y,
+                         std::vector<std::vector<uint32_t>>* cta) {
+    if (cta) cta->assign(y, {});
+    std::priority_queue<std::pair<long long, int>, std::vector<std::pair<long long, int>>,
+                        std::greater<std::pair<long long, int>>>
+        load;
+    for (int c = 0; c < y; ++c) load.emplace(0, c);
+    long long makespan = 0;
+    for (const auto& it : items) {
+        auto top = load.top();
+        load.pop();
+        if (cta) (*cta)[top.second].push_back(it.second);
+        const long long t = top.first + it.first + kChunkItemTiles;
+        makespan = std::max(makespan, t);
+        load.emplace(t, top.second);
+    }
+    return makespan;
+}
+
+// CTAs per kv head for the chunk kernel beside a decode kernel of decode_us: the fewest whose
+// schedule ends within decode_us, 0 (one CTA per item) when none below the item count does.
+int chunk_ctas_beside_decode(const std::vector<std::pair<int, uint32_t>>& items, int Hkv,
+                             int num_sms, double decode_us) {
+    const int n = static_cast<int>(items.size());
+    if (n < 2 || decode_us <= 0.0) return 0;
+    const double budget = decode_us / kChunkTileUs;  // key tiles
+    long long total = 0;
+    for (const auto& it : items) total += it.first + kChunkItemTiles;
+    if (items.front().first + kChunkItemTiles > budget) return 0;  // the longest item alone
+    const int y_max = std::min(n - 1, num_sms / Hkv);
+    for (int y = std::max(1, static_cast<int>(total / budget)); y <= y_max; ++y)
+        if (lpt_chunk_ctas(items, y, nullptr) <= budget) return y;
+    return 0;
+}
+
+// Lays the chunk items out for y CTAs per kv head that walk the list with stride y: CTA c's
+// k-th item of the schedule above sits at c + k y (kChunkWorkNone where a CTA has fewer
+// items).  False when the layout does not fit the list.
+bool lay_out_chunk_ctas(const std::vector<std::pair<int, uint32_t>>& items, int y,
+                        pa::ChunkWork& work) {
+    static thread_local std::vector<std::vector<uint32_t>> cta;
+    lpt_chunk_ctas(items, y, &cta);
+    size_t longest = 0;
+    for (const auto& c : cta) longest = std::max(longest, c.size());
+    if (longest * static_cast<size_t>(y) > static_cast<size_t>(pa::kMaxChunkWork)) return false;
+    work.count = static_cast<int>(longest) * y;
+    for (size_t k = 0; k < longest; ++k)
+        for (int c = 0; c < y; ++c)
+            work.item[k * y + c] = k < cta[c].size() ? cta[c][k] : pa::kChunkWorkNone;
+    return true;
+}
 
 // Estimated time of the tcgen05 chunk kernel, in key tiles, under KV splits of split_keys keys:
 // its CTAs (one per (q-tile pair, kv head, split), each walking the key tiles of its visible
@@ -477,6 +565,25 @@ int plan_impl(const int32_t* sl, const int32_t* qsl, int B, int T, int Hq, int H
         pl->prefix_splits = pa::ceil_div(pblocks, psb);
         pl->prefix_ctas = qtiles * Hkv * pl->prefix_splits;
         pl->workspace_needed = base + prefix_part_bytes(T, Hq, D, pl->prefix_splits);
+    }
+    if (D == 128 && P == 0 && pl->num_decode_seqs && pl->num_chunk_seqs) {
+        // the tcgen05 chunk kernel beside the decode kernel: as few CTAs as still end with it
+        static thread_local std::vector<std::pair<int, uint32_t>> items;
+        items.clear();
+        for (int r = 0; r < B; ++r) {
+            const int ql = qsl[r + 1] - qsl[r];
+            if (ql <= 0 || pa::is_decode_kind(ql, G)) continue;
+            for_each_chunk_item(sl[r], ql, G, bs, pl->chunk_split_blocks, window, local_chunk,
+                                chunk_cta_rows, chunk_tile_keys,
+                                [&](int, int, int tiles) { items.emplace_back(tiles, 0u); });
+        }
+        std::sort(items.begin(), items.end(),
+                  [](const std::pair<int, uint32_t>& a, const std::pair<int, uint32_t>& b) {
+                      return a.first > b.first;
+                  });
+        const double dec_bytes = static_cast<double>(dec_units) * 2.0 * bs * D * dtype_bytes(kv_dtype);
+        const double gbs = kv_dtype == PA_BF16 ? kDecodeGBsBf16 : kDecodeGBsFp8;
+        pl->chunk_ctas_per_kv_head = chunk_ctas_beside_decode(items, Hkv, num_sms, dec_bytes / gbs / 1e3);
     }
     return PA_OK;
 }
@@ -801,12 +908,12 @@ int pa::attention_call(const pa_cache* cache, const void* q, int num_q_heads,
         static thread_local pa::ChunkIo pio;
         if (cache->head_size == 128)
             make_chunk_io(pio, q, nullptr, pp.part_o, num_tokens, num_q_heads, pp.group,
-                          pl.prefix_splits, cache->kv_dtype == PA_BF16);
+                          pl.prefix_splits);
         else
             std::memset(&pio, 0, sizeof(pio));
         if (ev) record(ev[2], s);
         e = pa::launch_chunk(cache->tmap, cache->tmap_blk, pp, pwork, pio, cache->head_size,
-                             cache->kv_dtype, pl.prefix_splits, s);
+                             cache->kv_dtype, pl.prefix_splits, 0, s);
         if (e != cudaSuccess) return fail_cuda(e);
         if (ev) record(ev[3], s);
     }
@@ -845,20 +952,12 @@ int pa::attention_call(const pa_cache* cache, const void* q, int num_q_heads,
                 fits = false;
                 break;
             }
-            for (int qt = 0; qt < nqt; ++qt) {
-                const int last_row = std::min((qt + 1) * cta_rows, ql * p.group) - 1;
-                const int kmax = ctx - ql + last_row / p.group;
-                const int lo = pa::first_visible_key(ctx - ql + qt * cta_rows / p.group, p.window,
-                                                     p.local_chunk) /
-                               cache->block_size * cache->block_size;
-                for (int sp = 0; sp < nsplit; ++sp) {
-                    const int key_lo = std::max(sp * csb * cache->block_size, lo);
-                    const int key_hi = std::min(std::min((sp + 1) * csb * cache->block_size, ctx), kmax + 1);
-                    const int tiles = key_hi > key_lo ? pa::ceil_div(key_hi - key_lo, tile_keys) : 0;
-                    items.emplace_back(tiles, static_cast<uint32_t>(r) | (static_cast<uint32_t>(qt) << 10) |
-                                                  (static_cast<uint32_t>(sp) << 22));
-                }
-            }
+            for_each_chunk_item(ctx, ql, p.group, cache->block_size, csb, p.window, p.local_chunk,
+                                cta_rows, tile_keys, [&](int qt, int sp, int tiles) {
+                                    items.emplace_back(tiles, static_cast<uint32_t>(r) |
+                                                                  (static_cast<uint32_t>(qt) << 10) |
+                                                                  (static_cast<uint32_t>(sp) << 22));
+                                });
         }
         if (fits) {
             std::stable_sort(items.begin(), items.end(),
@@ -868,7 +967,7 @@ int pa::attention_call(const pa_cache* cache, const void* q, int num_q_heads,
             for (const auto& it : items) work.item[work.count++] = it.second;
         }
     }
-    // a step with both kinds: the chunk kernel on the side stream, forked from this stream after
+    // a step with both kinds: the decode kernel on the side stream, forked from this stream after
     // the counter clear and joined back before the split reduce
     SideStream* side = nullptr;
     std::unique_lock<std::mutex> side_lock;
@@ -882,37 +981,40 @@ int pa::attention_call(const pa_cache* cache, const void* q, int num_q_heads,
             if (e != cudaSuccess) return fail_cuda(e);
         }
     }
-    const cudaStream_t cs = side ? side->stream : s;  // the chunk kernel's stream
+    const cudaStream_t ds = side ? side->stream : s;  // the decode kernel's stream
+    // beside the decode kernel, the tcgen05 chunk kernel keeps to the CTAs the plan chose
+    int chunk_ctas_y = 0;
+    const int y = pl.chunk_ctas_per_kv_head;
+    if (side && y > 0 && y < work.count && lay_out_chunk_ctas(items, y, work)) chunk_ctas_y = y;
     static thread_local pa::ChunkIo io;
     if (pl.num_chunk_seqs && cache->head_size == 128)
         make_chunk_io(io, q, out, pl.chunk_max_splits > 1 ? p.part_o : nullptr, num_tokens,
-                      num_q_heads, p.group, p.max_splits,
-                      cache->kv_dtype == PA_BF16);
+                      num_q_heads, p.group, p.max_splits);
     else
         std::memset(&io, 0, sizeof(io));
     if (pl.num_chunk_seqs && side) {
-        if (ev) record(ev[2], cs);
+        if (ev) record(ev[2], s);
         e = pa::launch_chunk(cache->tmap, cache->tmap_blk, p, work, io, cache->head_size,
-                             cache->kv_dtype, pl.chunk_max_splits, cs);
+                             cache->kv_dtype, pl.chunk_max_splits, chunk_ctas_y, s);
         if (e != cudaSuccess) return fail_cuda(e);
-        if (ev) record(ev[3], cs);
+        if (ev) record(ev[3], s);
     }
     if (pl.num_decode_seqs) {
-        if (ev) record(ev[0], s);
+        if (ev) record(ev[0], ds);
         e = pa::launch_decode(cache->tmap, p, cache->head_size, cache->kv_dtype,
-                              pl.decode_max_splits, s);
+                              pl.decode_max_splits, ds);
         if (e != cudaSuccess) return fail_cuda(e);
-        if (ev) record(ev[1], s);
+        if (ev) record(ev[1], ds);
     }
     if (pl.num_chunk_seqs && !side) {
         if (ev) record(ev[2], s);
         e = pa::launch_chunk(cache->tmap, cache->tmap_blk, p, work, io, cache->head_size,
-                             cache->kv_dtype, pl.chunk_max_splits, s);
+                             cache->kv_dtype, pl.chunk_max_splits, 0, s);
         if (e != cudaSuccess) return fail_cuda(e);
         if (ev) record(ev[3], s);
     }
     if (side) {
-        e = cudaEventRecord(side->join, cs);
+        e = cudaEventRecord(side->join, ds);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(s, side->join, 0);
         if (e != cudaSuccess) return fail_cuda(e);
         side_lock.unlock();

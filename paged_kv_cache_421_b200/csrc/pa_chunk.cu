@@ -368,10 +368,10 @@ cudaError_t launch_chunk_t(const CUtensorMap& tmap, const AttnParams& p, const C
 
 cudaError_t launch_chunk(const CUtensorMap& tmap, const CUtensorMap& tmap_blk, const AttnParams& p,
                          const ChunkWork& work, const ChunkIo& io, int head_size, int kv_dtype,
-                         int max_splits, cudaStream_t stream) {
+                         int max_splits, int ctas_y, cudaStream_t stream) {
     if (head_size == 128)
-        return launch_chunk_tc(tmap, tmap_blk, p, work, io, kv_dtype, max_splits, stream);
-    if (kv_dtype != PA_BF16) return cudaErrorInvalidValue;
+        return launch_chunk_tc(tmap, tmap_blk, p, work, io, kv_dtype, max_splits, ctas_y, stream);
+    if (kv_dtype != PA_BF16 || ctas_y != 0) return cudaErrorInvalidValue;
     if (head_size == 64) return launch_chunk_t<64>(tmap, p, work, max_splits, stream);
     return cudaErrorInvalidValue;
 }

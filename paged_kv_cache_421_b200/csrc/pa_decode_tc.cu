@@ -93,18 +93,6 @@ __device__ __forceinline__ bool softmax_any(bool pred) {
     return out != 0;
 }
 
-// Two probabilities -> two E4M3 terms each, through f16: hi = e4m3(a), lo = e4m3(a - hi) (the
-// remainder is exact in f16); two 8-bit codes per result, a.x in the low byte.
-__device__ __forceinline__ void split_e4m3x2_h(float a, float b, uint32_t& hi, uint32_t& lo) {
-    const __half2 h = __floats2half2_rn(a, b);
-    const __nv_fp8x2_storage_t c1 =
-        __nv_cvt_halfraw2_to_fp8x2(static_cast<__half2_raw>(h), __NV_SATFINITE, __NV_E4M3);
-    const __half2 back = __half2(__nv_cvt_fp8x2_to_halfraw2(c1, __NV_E4M3));
-    const __half2 rem = __hsub2(h, back);
-    hi = c1;
-    lo = __nv_cvt_halfraw2_to_fp8x2(static_cast<__half2_raw>(rem), __NV_SATFINITE, __NV_E4M3);
-}
-
 __global__ void __launch_bounds__(kThreads, 2)
 decode_tc8_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
     pdl_trigger();
@@ -338,8 +326,8 @@ decode_tc8_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) 
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
                 uint32_t h0, l0, h1, l1;
-                split_e4m3x2_h(x[4 * j] * up, x[4 * j + 1] * up, h0, l0);
-                split_e4m3x2_h(x[4 * j + 2] * up, x[4 * j + 3] * up, h1, l1);
+                split_e4m3x2(make_float2(x[4 * j] * up, x[4 * j + 1] * up), h0, l0);
+                split_e4m3x2(make_float2(x[4 * j + 2] * up, x[4 * j + 3] * up), h1, l1);
                 hi[j] = h0 | (h1 << 16);
                 lo[j] = l0 | (l1 << 16);
             }
@@ -468,7 +456,7 @@ decode_tc8_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) 
             }
             uint32_t h[4], l[4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) split_e4m3x2_h(pr[2 * i], pr[2 * i + 1], h[i], l[i]);
+            for (int i = 0; i < 4; ++i) split_e4m3x2(make_float2(pr[2 * i], pr[2 * i + 1]), h[i], l[i]);
             // the P^T buffer is free once the P V of tile t - kPBufs completed
             if (t >= kPBufs && !__all_sync(0xffffffffu, mbar_wait(smem_u32(&bar_pv[t % kPBufs]),
                                                                  ((t / kPBufs) + 1) & 1u, kWaitLimitNs, p.err))) {

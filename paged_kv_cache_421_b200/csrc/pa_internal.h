@@ -105,9 +105,12 @@ struct ChunkList {
 
 // The CTAs of a chunk launch, most key tiles first (longest-processing-time order, so the
 // short CTAs fill in behind the long ones): item = request | q-tile << 10 | split << 22.
-// count == 0 means "derive them from the grid" (x: q-tile and split, z: request).
+// count == 0 means "derive them from the grid" (x: q-tile and split, z: request).  The
+// head_size-128 kernel may run fewer CTAs than items: CTA (kv head, y) then takes items y,
+// y + gridDim.y, y + 2 gridDim.y, ... in turn, and kChunkWorkNone marks an empty place.
 constexpr int kMaxChunkWork = 3072;
 constexpr int kChunkWorkMaxReq = 1 << 10, kChunkWorkMaxQt = 1 << 12, kChunkWorkMaxSplit = 1 << 10;
+constexpr uint32_t kChunkWorkNone = 0xffffffffu;
 struct ChunkWork {
     int count;
     uint32_t item[kMaxChunkWork];
@@ -139,12 +142,13 @@ cudaError_t launch_decode(const CUtensorMap& tmap, const AttnParams& p, int head
 // FP8 E4M3 cache, head_size 128: the tcgen05 decode kernel (pa_decode_tc.cu)
 cudaError_t launch_decode_tc8(const CUtensorMap& tmap, const AttnParams& p, int max_splits,
                               cudaStream_t stream);
+// ctas_y: CTAs per kv head that walk the work list (head_size 128 only; 0: one per item)
 cudaError_t launch_chunk(const CUtensorMap& tmap, const CUtensorMap& tmap_blk, const AttnParams& p,
                          const ChunkWork& work, const ChunkIo& io, int head_size, int kv_dtype,
-                         int max_splits, cudaStream_t stream);
+                         int max_splits, int ctas_y, cudaStream_t stream);
 cudaError_t launch_chunk_tc(const CUtensorMap& tmap, const CUtensorMap& tmap_blk,
                             const AttnParams& p, const ChunkWork& work, const ChunkIo& io,
-                            int kv_dtype, int max_splits, cudaStream_t stream);
+                            int kv_dtype, int max_splits, int ctas_y, cudaStream_t stream);
 cudaError_t launch_reduce(const AttnParams& p, const ChunkList& list, int head_size,
                           cudaStream_t stream);
 cudaError_t launch_zero_counters(int* counters, int n, cudaStream_t stream);

@@ -155,16 +155,19 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
         : "memory");
 }
 
-// Two probabilities -> their two-term E4M3 split: hi = e4m3(a) and lo = e4m3(a - hi) (the
-// remainder is exact in fp32), two 8-bit codes each with a.x in the low byte.
+// Two values -> their two-term E4M3 split: hi = e4m3(a) and lo = e4m3(a - hi), two 8-bit codes
+// each with a.x in the low byte.  Through f16x2: the pair rounds to f16 (11 significant bits,
+// more than the two terms keep), the first term's codes convert back exactly and the f16
+// remainder is exact (the first term lies within a factor of two of the value): four
+// conversions for two values.
 __device__ __forceinline__ void split_e4m3x2(float2 a, uint32_t& hi, uint32_t& lo) {
-    const __nv_fp8x2_storage_t c1 = __nv_cvt_float2_to_fp8x2(a, __NV_SATFINITE, __NV_E4M3);
-    const __half2 h = __half2(__nv_cvt_fp8x2_to_halfraw2(c1, __NV_E4M3));
-    const float2 back = __half22float2(h);
-    const __nv_fp8x2_storage_t c2 = __nv_cvt_float2_to_fp8x2(
-        make_float2(a.x - back.x, a.y - back.y), __NV_SATFINITE, __NV_E4M3);
+    const __half2 h = __floats2half2_rn(a.x, a.y);
+    const __nv_fp8x2_storage_t c1 =
+        __nv_cvt_halfraw2_to_fp8x2(static_cast<__half2_raw>(h), __NV_SATFINITE, __NV_E4M3);
+    const __half2 back = __half2(__nv_cvt_fp8x2_to_halfraw2(c1, __NV_E4M3));
+    const __half2 rem = __hsub2(h, back);
     hi = c1;
-    lo = c2;
+    lo = __nv_cvt_halfraw2_to_fp8x2(static_cast<__half2_raw>(rem), __NV_SATFINITE, __NV_E4M3);
 }
 
 // 3-D tiled load (the Q map: {dim, head, token}).
@@ -235,6 +238,18 @@ __device__ __forceinline__ void fence_proxy_async_all() {
 // Barrier `id` among the first `count` threads of the CTA (whole warps).
 __device__ __forceinline__ void named_barrier_sync(int id, int count) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Barrier `id` among `count` threads (whole warps) that ORs `pred` over them.
+__device__ __forceinline__ bool named_barrier_or(int id, int count, bool pred) {
+    uint32_t out;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(out)
+        : "r"(static_cast<uint32_t>(pred)), "r"(id), "r"(count)
+        : "memory");
+    return out != 0;
 }
 
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {

@@ -338,3 +338,45 @@ def test_plan_random_metadata_stays_inside_the_workspace(lib):
                 ns = -(-int(blocks[r]) // p["chunk_split_blocks"])
                 assert 1 <= ns <= p["chunk_max_splits"]
     assert accepted > 150
+
+
+def _mixed(dec_ctx, chunk_ctx, chunk_ql, hq=32, hkv=8):
+    ctx = np.array(list(dec_ctx) + list(chunk_ctx))
+    ql = np.array([1] * len(dec_ctx) + list(chunk_ql))
+    return ctx, np.concatenate([[0], np.cumsum(ql)])
+
+
+def test_plan_chunk_ctas_beside_decode(lib):
+    """A step with both kinds gives the tcgen05 chunk kernel fewer CTAs than items when their
+    estimated schedule ends within the decode kernel's time, and one CTA per item otherwise:
+    for a step of one kind only, for head_size 64, and when even the longest item outlasts the
+    decodes.  More decode work never asks for more chunk CTAs."""
+    def plan(ctx, qsl, d=128, kv_dtype=0, hq=32, hkv=8):
+        mb = int(max(-(-int(c) // 16) for c in ctx))
+        return B.pa_plan_attention(ctx, qsl, hq, hkv, d, mb, 148, 1 << 30, kv_dtype=kv_dtype)
+
+    for kv_dtype, name in [(W.BF16, "mixed_step"), (W.FP8_E4M3, "mixed_step_fp8")]:
+        wl = W.CONFIGS[name]()
+        p = plan(wl.seq_lens, wl.qsl, kv_dtype=kv_dtype)
+        items = p["chunk_ctas"] // wl.num_kv_heads
+        assert 0 < p["chunk_ctas_per_kv_head"] < items, (name, p)
+    for name in ["prefill_chunks", "llama8b_decode", "long70b_decode"]:  # one kind only
+        wl = W.CONFIGS[name]()
+        assert plan(wl.seq_lens, wl.qsl)["chunk_ctas_per_kv_head"] == 0, name
+    ctx, qsl = _mixed([4000] * 32, [700, 900], [400, 300])
+    assert plan(ctx, qsl, d=64)["chunk_ctas_per_kv_head"] == 0  # the mma.sync chunk kernel
+    # a chunk whose longest item alone outlasts two short decodes: one CTA per item
+    ctx, qsl = _mixed([100, 120], [16000, 900], [2000, 300])
+    assert plan(ctx, qsl)["chunk_ctas_per_kv_head"] == 0
+    # more decode bytes: never more chunk CTAs, and within [1, items)
+    prev = None
+    for n_dec in [16, 32, 64, 128]:
+        ctx, qsl = _mixed([5000] * n_dec, [70, 430, 1033, 250, 764, 90],
+                          [70, 130, 33, 200, 64, 90])
+        p = plan(ctx, qsl)
+        y = p["chunk_ctas_per_kv_head"]
+        if y:
+            assert 1 <= y < p["chunk_ctas"] // 8
+            assert prev is None or prev == 0 or y <= prev, (n_dec, y, prev)
+        prev = y
+    assert prev > 0
