@@ -779,6 +779,13 @@ def run_device_bench(args, rank, world, local):
                           "traffic": None, "peak_kind": tkind,
                           "flops_per_launch": flops,
                           "ms_per_launch": round(chunk_ms, 4)}
+            y = step.plan.get("chunk_ctas_per_kv_head", 0)
+            if y and not step.prefix and step.plan["num_decode_seqs"]:
+                # beside the decode kernel the chunk kernel holds y CTAs (SMs) per kv head only
+                sms = torch.cuda.get_device_properties(device).multi_processor_count
+                held = min(sms, y * wl.num_kv_heads)
+                chunk_roof["sms_held"] = held
+                chunk_roof["frac_of_held_sms"] = round(tflops / (tpeak * held / sms), 4)
             if roof is None:
                 roof = chunk_roof
         result = {

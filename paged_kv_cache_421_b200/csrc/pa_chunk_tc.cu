@@ -857,7 +857,15 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
                             bulk_commit();
                         }
                     }
-                    if (lane == 0) bulk_wait_all();  // the rows are written before the CTA ends
+                    // the staging buffers are free once the stores have read them; the rows
+                    // themselves must have reached memory only where this CTA's split merge
+                    // (below) may read them back: otherwise the kernel's end publishes them
+                    if (lane == 0) {
+                        if (nsplit > 1 && p.chunk_fused_merge && !prefix)
+                            bulk_wait_all();
+                        else
+                            bulk_wait_read0();
+                    }
                     __syncwarp();
                 } else if (all_ok) {
                     // O / l through shared memory (this q-tile's Q region: its last MMA has
@@ -1022,7 +1030,7 @@ chunk_tc_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p,
                             __syncwarp();
                             if (c + ngrp < kD / 32) issue(c + ngrp);
                         }
-                        if (lane == 0) bulk_wait_all();  // the rows are written before the CTA ends
+                        if (lane == 0) bulk_wait_read0();  // the boxes have left shared memory
                         __syncwarp();
                     } else {
                         for (int i0 = 0; i0 < 32; i0 += kMergeRows) {
