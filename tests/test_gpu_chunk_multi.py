@@ -44,6 +44,12 @@ CASES = {
     "fused_split_merge": (_DEC + [1800, 300], [1] * 32 + [64, 100], 32, 8, W.BF16, 0),
     # eight splits: partials merged by the reduce kernel after the chunk kernel
     "reduce_splits": (_DEC + [4000, 300], [1] * 32 + [64, 100], 32, 8, W.BF16, 0),
+    # group 3, which divides no TMA box of 128 rows: Q staged by the softmax warps (bf16) or
+    # loaded and split by them from global memory (FP8), item after item
+    "g3_staged_q_bf16": (_DEC + [70, 430, 1033, 250, 764, 90], [1] * 32 + [70, 130, 33, 200, 64, 90],
+                         24, 8, W.BF16, 0),
+    "g3_staged_q_fp8": (_DEC + [70, 430, 1033, 250, 764, 90], [1] * 32 + [70, 130, 33, 200, 64, 90],
+                        24, 8, W.FP8_E4M3, 0),
     # one kv head, group 8: many small items over many CTAs of the one kv head
     "one_kv_head_many_items": (_decodes(64, 7000, 9000, 11) + [40 + 13 * i for i in range(30)],
                                [1] * 64 + [40] * 30, 8, 1, W.BF16, 0),

@@ -241,6 +241,8 @@ FP8_CHUNK_CASES = {
     "qlen3_g4": ([50, 300], [3, 3], 8, 2),
     "mixed_decodes_and_chunk": ([2000, 3001, 600, 700], [1, 1, 200, 1], 32, 8),
     "ragged_chunk_tails": ([129, 255, 17], [129, 100, 17], 8, 1),
+    # G 3 divides no 128-row TMA box of Q: the softmax warps load and split Q themselves
+    "g3_no_q_map": ([200, 90], [50, 37], 6, 2),
 }
 
 
