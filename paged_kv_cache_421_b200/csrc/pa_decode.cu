@@ -240,6 +240,8 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
         const int mine = (ok && units > warp) ? (units - warp + NW - 1) / NW : 0;
         const int kend = (rb + rn) * kBlockSize;  // first position past this round's blocks
 
+        // each K/V byte of a decode is read once: the L2 evicts these lines first
+        const uint64_t l2_stream = l2_evict_first_policy();
         auto issue = [&](int i, uint32_t n) {
             if (i == skip_i) return;
             const int u0 = (warp + i * NW) * BPU;  // round index of the unit's first block
@@ -254,8 +256,9 @@ decode_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) {
                 const uint32_t dk = dst + h * 2 * C::kTileBytes;
 #pragma unroll
                 for (int b = 0; b < C::kBoxes; ++b) {
-                    tma_load_2d(dk + b * 2048, &tmap, bar, b * C::kBoxElems, rowk);
-                    tma_load_2d(dk + C::kTileBytes + b * 2048, &tmap, bar, b * C::kBoxElems, rowv);
+                    tma_load_2d_hint(dk + b * 2048, &tmap, bar, b * C::kBoxElems, rowk, l2_stream);
+                    tma_load_2d_hint(dk + C::kTileBytes + b * 2048, &tmap, bar, b * C::kBoxElems,
+                                     rowv, l2_stream);
                 }
             }
         };

@@ -226,12 +226,16 @@ decode_tc8_kernel(const __grid_constant__ CUtensorMap tmap, const AttnParams p) 
                     }
                 }
                 const int rowk = blk * kv_rows_per_block + g * kBlockSize;
+                // each K/V byte of a decode is read once: the L2 evicts these lines first
+                const uint64_t l2_stream = l2_evict_first_policy();
                 if (!is_v) {
-                    tma_load_2d(k_s + sl * kTileBytes + lane * kBlockTile, &tmap, bar, 0, rowk);
+                    tma_load_2d_hint(k_s + sl * kTileBytes + lane * kBlockTile, &tmap, bar, 0, rowk,
+                                     l2_stream);
                 } else {
                     const int rowv = rowk + p.num_kv_heads * kBlockSize;
-                    bulk_load(v_s + sl * kTileBytes + lane * kBlockTile,
-                              p.cache + static_cast<int64_t>(rowv) * kD, kBlockTile, bar);
+                    bulk_load_hint(v_s + sl * kTileBytes + lane * kBlockTile,
+                                   p.cache + static_cast<int64_t>(rowv) * kD, kBlockTile, bar,
+                                   l2_stream);
                 }
             }
             __syncwarp();
