@@ -161,7 +161,11 @@ size_t pa_attention_workspace_bytes(int num_tokens, int num_q_heads, int head_si
  *   and with pa_attention_opts.local_chunk = C > 0 only to those from floor(p / C) * C.
  * Requests with q_len * (num_q_heads / num_kv_heads) <= 8 run in the decode kernel, the others
  *   in the chunked-prefill kernel (bf16 or FP8 E4M3 cache; any mix of the two kinds in one
- *   call).
+ *   call).  A call with both kinds (and no common prefix) launches the chunked-prefill kernel
+ *   on `stream` and the decode kernel beside it on a second stream of the device that the
+ *   library creates on first use, forked from and joined back into `stream` by events: the
+ *   call stays ordered on `stream` and capturable in a graph (pa_attention_noalloc keeps both
+ *   kernels on `stream`).
  * out: device fp32 [num_tokens][num_q_heads][head_size].
  * workspace: device scratch of workspace_bytes for split-KV partials (may be NULL/0: then no
  *   request is split).  Its contents are opaque; it must not be shared by calls that

@@ -6,8 +6,9 @@
 // bottom-right causal mask of chunked prefill ("vLLM: from KV Cache to high-throughput
 // serving", article 5 outline) and the online softmax of FlashAttention (article 7 outline).
 //
-// How.  One CTA owns two 128-row query tiles (256 rows of one (request, kv head)) and
-// optionally one KV split; one CTA per SM.  Its warps specialise: warps 0-7 run the softmax
+// How.  A work item is two 128-row query tiles (256 rows of one (request, kv head)) and
+// optionally one KV split; a CTA takes one item, or (beside the decode kernel, on fewer CTAs)
+// several in turn; one CTA per SM.  Its warps specialise: warps 0-7 run the softmax
 // (warps 4q..4q+3 serve q-tile q; thread i of the q-tile owns row i, which is TMEM lane i),
 // warp 8 issues the tensor-core MMAs, warp 9 the TMA loads.  Keys are walked in tiles of 128
 // (eight physical blocks from the block table); each block's K and V tiles arrive by TMA (2-D
