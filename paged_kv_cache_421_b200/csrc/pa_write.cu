@@ -9,7 +9,8 @@
 // One thread moves 16 bytes of bf16 input; consecutive threads cover consecutive bytes of a
 // row, so both the reads of k/v and the writes into the pool are coalesced.  An FP8 pool
 // stores e4m3(x / scale[head]) with an IEEE-rounded fp32 divide and saturating conversion;
-// its V tiles are dim-major, so V bytes are scattered with a 16-byte stride.
+// its V tiles are dim-major: a lane converts one dim of 16 consecutive tokens and writes it as
+// one 16-byte row when they fill one block, else scatters each token's byte (16-byte stride).
 #include <algorithm>
 
 #include "pa_internal.h"
@@ -53,13 +54,15 @@ write_kv_kernel(uint8_t* __restrict__ cache, const uint16_t* __restrict__ k,
     pdl_trigger();
     pdl_wait();
     constexpr int kChunks = D / 8;  // 16-byte pieces of one bf16 row
-    const int64_t total = static_cast<int64_t>(num_tokens) * num_kv_heads * 2 * kChunks;
+    // bf16: K and V rows here; FP8: K rows here, V rows by warps below
+    constexpr int kKinds = FP8 ? 1 : 2;
+    const int64_t total = static_cast<int64_t>(num_tokens) * num_kv_heads * kKinds * kChunks;
     for (int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
          idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const int c = static_cast<int>(idx % kChunks);
         int64_t rest = idx / kChunks;
-        const int kv = static_cast<int>(rest % 2);
-        rest /= 2;
+        const int kv = static_cast<int>(rest % kKinds);
+        rest /= kKinds;
         const int h = static_cast<int>(rest % num_kv_heads);
         const int64_t t = rest / num_kv_heads;
         const int slot = slots[t];
@@ -76,7 +79,7 @@ write_kv_kernel(uint8_t* __restrict__ cache, const uint16_t* __restrict__ k,
         if constexpr (!FP8) {
             *reinterpret_cast<uint4*>(cache + dst * 2) = x;
         } else {
-            const float s = (kv ? v_scale : k_scale)[h];
+            const float s = k_scale[h];
             const uint32_t w[4] = {x.x, x.y, x.z, x.w};
             uint16_t out[4];
 #pragma unroll
@@ -86,18 +89,65 @@ write_kv_kernel(uint8_t* __restrict__ cache, const uint16_t* __restrict__ k,
                 float2 y = make_float2(__fdiv_rn(lo, s), __fdiv_rn(hi, s));
                 out[j] = static_cast<uint16_t>(__nv_cvt_float2_to_fp8x2(y, __NV_SATFINITE, __NV_E4M3));
             }
-            if (kv == 0) {
-                uint2 packed;
-                packed.x = static_cast<uint32_t>(out[0]) | (static_cast<uint32_t>(out[1]) << 16);
-                packed.y = static_cast<uint32_t>(out[2]) | (static_cast<uint32_t>(out[3]) << 16);
-                *reinterpret_cast<uint2*>(cache + dst) = packed;
-            } else {
-                // FP8 V tiles are dim-major: dim d of token o sits at byte d * 16 + o of the tile
-                uint8_t* tile = cache + (dst - (slot % kBlockSize) * D - c * 8);
+            uint2 packed;
+            packed.x = static_cast<uint32_t>(out[0]) | (static_cast<uint32_t>(out[1]) << 16);
+            packed.y = static_cast<uint32_t>(out[2]) | (static_cast<uint32_t>(out[3]) << 16);
+            *reinterpret_cast<uint2*>(cache + dst) = packed;
+        }
+    }
+    if constexpr (FP8) {
+        // V: FP8 V tiles are dim-major (dim d of token o at byte d * 16 + o of the tile).  A warp
+        // takes 16 consecutive tokens of one kv head and 32 of their dims, lane l dim 32 q + l:
+        // the lane converts its dim of the 16 tokens, which is one 16-byte row of the tile.
+        // When the 16 slots fill one block in order (a prefill chunk's tokens) the row is written
+        // with one 16-byte store (a warp writes 512 contiguous bytes); otherwise (decode tokens,
+        // partly filled blocks) each token's byte goes on its own.
+        const unsigned kFull = 0xffffffffu;
+        const int lane = threadIdx.x & 31;
+        constexpr int kQuarters = D / 32;
+        const int64_t nwarps = static_cast<int64_t>(gridDim.x) * (blockDim.x / 32);
+        const int64_t units =
+            static_cast<int64_t>(ceil_div(num_tokens, kBlockSize)) * num_kv_heads * kQuarters;
+        for (int64_t u = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) / 32; u < units;
+             u += nwarps) {
+            const int d = static_cast<int>(u % kQuarters) * 32 + lane;
+            const int64_t rest = u / kQuarters;
+            const int h = static_cast<int>(rest % num_kv_heads);
+            const int64_t t0 = (rest / num_kv_heads) * kBlockSize;
+            const int s = (lane < kBlockSize && t0 + lane < num_tokens) ? slots[t0 + lane] : -1;
+            const int s0 = __shfl_sync(kFull, s, 0);
+            const bool whole = __all_sync(kFull, lane >= kBlockSize ||
+                                                     (s0 >= 0 && s0 % kBlockSize == 0 &&
+                                                      s0 + kBlockSize <= num_slots && s == s0 + lane));
+            const float sc = v_scale[h];
+            uint32_t row[4] = {0u, 0u, 0u, 0u};  // byte i: the code of token t0 + i
 #pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    tile[(c * 8 + j) * kBlockSize + slot % kBlockSize] =
-                        static_cast<uint8_t>(out[j >> 1] >> (8 * (j & 1)));
+            for (int i = 0; i < kBlockSize; i += 2) {
+                float x0 = 0.f, x1 = 0.f;
+                if (t0 + i < num_tokens)
+                    x0 = __uint_as_float(static_cast<uint32_t>(v[((t0 + i) * num_kv_heads + h) * D + d]) << 16);
+                if (t0 + i + 1 < num_tokens)
+                    x1 = __uint_as_float(static_cast<uint32_t>(v[((t0 + i + 1) * num_kv_heads + h) * D + d]) << 16);
+                const uint32_t pair = __nv_cvt_float2_to_fp8x2(
+                    make_float2(__fdiv_rn(x0, sc), __fdiv_rn(x1, sc)), __NV_SATFINITE, __NV_E4M3);
+                row[i / 4] |= pair << (8 * (i % 4));
+            }
+            if (whole) {
+                uint8_t* tile = cache + ((static_cast<int64_t>(s0 / kBlockSize) * 2 + 1) * num_kv_heads + h) *
+                                            kBlockSize * D;
+                *reinterpret_cast<uint4*>(tile + d * kBlockSize) = make_uint4(row[0], row[1], row[2], row[3]);
+            } else {
+                for (int i = 0; i < kBlockSize; ++i) {
+                    const int si = __shfl_sync(kFull, s, i);
+                    if (si < 0) continue;
+                    if (si >= num_slots) {
+                        if (lane == 0) raise_error(err, kErrBadSlotMeta);
+                        continue;
+                    }
+                    uint8_t* tile = cache + ((static_cast<int64_t>(si / kBlockSize) * 2 + 1) * num_kv_heads + h) *
+                                                kBlockSize * D;
+                    tile[d * kBlockSize + si % kBlockSize] = static_cast<uint8_t>(row[i / 4] >> (8 * (i % 4)));
+                }
             }
         }
     }
@@ -149,6 +199,8 @@ __global__ void validate_slots_kernel(const int32_t* __restrict__ slots, int num
 template <int D, bool FP8>
 cudaError_t launch_write_t(const pa_cache& c, const void* k, const void* v, const int32_t* slots,
                            int num_tokens, int* err, cudaStream_t stream) {
+    // one thread per 16-byte piece of a K or V row (FP8: of a K row, and one warp per 16 tokens
+    // and 32 dims of a kv head for V: the thread count covers both)
     const int64_t total = static_cast<int64_t>(num_tokens) * c.num_kv_heads * 2 * (D / 8);
     const int threads = 256;
     const int64_t blocks = (total + threads - 1) / threads;
