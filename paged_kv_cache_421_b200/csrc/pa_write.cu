@@ -120,14 +120,19 @@ write_kv_kernel(uint8_t* __restrict__ cache, const uint16_t* __restrict__ k,
                                                      (s0 >= 0 && s0 % kBlockSize == 0 &&
                                                       s0 + kBlockSize <= num_slots && s == s0 + lane));
             const float sc = v_scale[h];
+            // all 16 loads first (clamped to the last token, masked below), so that their
+            // latencies overlap instead of queueing behind each divide
+            uint32_t raw[kBlockSize];
+#pragma unroll
+            for (int i = 0; i < kBlockSize; ++i) {
+                const int64_t t = min(t0 + i, static_cast<int64_t>(num_tokens) - 1);
+                raw[i] = __ldg(v + (t * num_kv_heads + h) * D + d);
+            }
             uint32_t row[4] = {0u, 0u, 0u, 0u};  // byte i: the code of token t0 + i
 #pragma unroll
             for (int i = 0; i < kBlockSize; i += 2) {
-                float x0 = 0.f, x1 = 0.f;
-                if (t0 + i < num_tokens)
-                    x0 = __uint_as_float(static_cast<uint32_t>(v[((t0 + i) * num_kv_heads + h) * D + d]) << 16);
-                if (t0 + i + 1 < num_tokens)
-                    x1 = __uint_as_float(static_cast<uint32_t>(v[((t0 + i + 1) * num_kv_heads + h) * D + d]) << 16);
+                const float x0 = t0 + i < num_tokens ? __uint_as_float(raw[i] << 16) : 0.f;
+                const float x1 = t0 + i + 1 < num_tokens ? __uint_as_float(raw[i + 1] << 16) : 0.f;
                 const uint32_t pair = __nv_cvt_float2_to_fp8x2(
                     make_float2(__fdiv_rn(x0, sc), __fdiv_rn(x1, sc)), __NV_SATFINITE, __NV_E4M3);
                 row[i / 4] |= pair << (8 * (i % 4));
